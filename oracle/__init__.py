@@ -1,0 +1,117 @@
+"""ctypes wrapper around the fp64 sequential oracle (``ssd_oracle.c``).
+
+TEST INFRASTRUCTURE ONLY.  This package may be imported by ``tests/``, by the
+package's ``smoke()`` check and by the CPU-baseline leg of ``bench.py``, and by
+nothing else.  It shares no code with the CUDA library: both sides only see the
+same seeded inputs.
+
+All arrays are numpy, C-contiguous; real data is float64 and complex data is
+complex128 (interleaved re/im doubles, the layout the C file reads).  Inputs
+that were bf16 on the GPU side are passed here widened to float64 exactly.
+
+Reference: "Mamba-3-Lite" README (the recurrence section) and "Block Anatomy,
+Numerical Stability & Scaling" (Numerical Stability, section 4); the C file
+header lists the readings taken.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB = os.path.join(_HERE, "libssd_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_L = ctypes.c_long
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (-O2, no fast-math: fp64 semantics kept)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-std=c99", "-O2", "-fPIC", "-shared",
+                               "-fno-fast-math", "-o", tmp, src, "-lm"])
+        os.replace(tmp, out)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building first if needed) and declare the oracle's entry points."""
+    global _lib
+    if path is None:
+        with _lock:
+            if _lib is None:
+                _lib = _declare(ctypes.CDLL(build()))
+            return _lib
+    return _declare(ctypes.CDLL(path))
+
+
+def _declare(lib):
+    scan_args = [_D, _D, _D, _D, _D, _D, _D, _D, _D, _L, _L, _L, _L, _L, _L]
+    upd_args = [_D, _D, _D, _D, _D, _D, _D, _D, _L, _L, _L, _L, _L]
+    for name in ("oracle_scan_real", "oracle_scan_complex"):
+        getattr(lib, name).argtypes = scan_args
+        getattr(lib, name).restype = ctypes.c_int
+    for name in ("oracle_state_update_real", "oracle_state_update_complex"):
+        getattr(lib, name).argtypes = upd_args
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+def _ptr(a, dtype):
+    if a is None:
+        return None
+    assert a.dtype == dtype and a.flags["C_CONTIGUOUS"], (a.dtype, a.flags)
+    return a.ctypes.data_as(_D)
+
+
+def scan(x, dt, A, B, C, D=None, init_state=None, ngroups=None, lib=None):
+    """Run the sequential scan.  Complex variant when A is complex.
+
+    x [b,T,H,P] float64, dt [b,T,H] float64, A [H] (float64 or complex128),
+    B, C [b,T,G,N] (float64 or complex128), D [H] float64 or None,
+    init_state [b,H,P,N] (float64 or complex128) or None.
+    Returns (y [b,T,H,P] float64, final_state [b,H,P,N]).
+    """
+    lib = lib or load()
+    cplx = np.iscomplexobj(A)
+    sdt = np.complex128 if cplx else np.float64
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.zeros((b, T, H, P), np.float64)
+    fs = np.zeros((b, H, P, N), sdt)
+    fn = lib.oracle_scan_complex if cplx else lib.oracle_scan_real
+    rc = fn(_ptr(x, np.float64), _ptr(dt, np.float64), _ptr(A, sdt), _ptr(B, sdt),
+            _ptr(C, sdt), _ptr(D, np.float64), _ptr(init_state, sdt),
+            _ptr(y, np.float64), _ptr(fs, sdt), b, T, H, P, G, N)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return y, fs
+
+
+def state_update(state, x, dt, A, B, C, D=None, lib=None):
+    """One decoding step.  Returns (y [b,H,P], new state); the input is not modified.
+
+    state [b,H,P,N], x [b,H,P], dt [b,H], A [H], B, C [b,G,N], D [H] or None.
+    """
+    lib = lib or load()
+    cplx = np.iscomplexobj(A)
+    sdt = np.complex128 if cplx else np.float64
+    st = np.array(state, dtype=sdt, copy=True, order="C")
+    b, H, P, N = st.shape
+    G = B.shape[1]
+    y = np.zeros((b, H, P), np.float64)
+    fn = lib.oracle_state_update_complex if cplx else lib.oracle_state_update_real
+    rc = fn(_ptr(st, sdt), _ptr(x, np.float64), _ptr(dt, np.float64), _ptr(A, sdt),
+            _ptr(B, sdt), _ptr(C, sdt), _ptr(D, np.float64), _ptr(y, np.float64),
+            b, H, P, G, N)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return y, st
