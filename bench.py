@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Throughput of the chunked SSD scan on B200, one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+A step is one ``ssd_scan_fwd`` call over one batch of the workload, i.e. the
+whole scan (cumulative decay, segsum decay, diagonal block, chunk states,
+inter-chunk state passing, off-diagonal output, D skip).  The default workload
+is the Mamba-2 BitMamba-1B layer shape (batch 2, T 2048, 64 heads, head dim 64,
+d_state 128, one group, chunk 256, bf16 x/B/C/y, float32 dt/A/D/state).
+
+Timing: inputs are resident in HBM; the K timed steps are bracketed by a
+barrier and a device synchronize; each step is timed with CUDA events on the
+launching stream and L2 is flushed (a 512 MiB write) between steps, outside the
+event pairs; the reported time is the max over ranks.  Under torchrun every
+rank scans its own copy of the workload (independent sequences: weak scaling,
+no collective on the data path).
+
+``--impl reference`` times the fp64 CPU oracle (the program the GPU results are
+checked against) on the host cores instead, each step a bounded sample of the
+same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "SSD scan tokens/s at Mamba-2 1B layer shape; % of roofline (TC or HBM)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_FLUSH_BYTES = 512 << 20
+
+
+# ----------------------------------------------------------------- ranks
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+    return rank, world
+
+
+def dist_barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def dist_max(value: float, device=None) -> float:
+    """Max of a host float over all ranks (identity on one rank)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------- algorithmic work
+def algorithmic_bytes(shape) -> int:
+    """Each input read once and each output written once; chunk states count zero."""
+    io = 4 if (shape.io_dtype == "f32" or shape.complex) else 2
+    bc = 8 if shape.complex else io
+    st = 8 if shape.complex else 4
+    b, T, H, P, G, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups, shape.dstate
+    n = 2 * b * T * H * P * io            # x in, y out
+    n += b * T * H * 4                     # dt
+    n += 2 * b * T * G * N * bc            # B, C
+    n += H * (8 if shape.complex else 4) + H * 4  # A, D
+    n += b * H * P * N * st                # final state out
+    if shape.init_state:
+        n += b * H * P * N * st
+    return n
+
+
+def algorithmic_flops(shape) -> int:
+    """2 flops per MAC; causal half of each intra-chunk product; exps not counted."""
+    b, T, H, P, G, N, Q = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups,
+                           shape.dstate, shape.chunk)
+    total = 0
+    for c0 in range(0, T, Q):
+        q = min(Q, T - c0)
+        tri = q * (q + 1) // 2
+        per_head = 2 * tri * P + 2 * q * N * P + 2 * q * N * P   # diag, chunk state, off-diagonal
+        per_group = 2 * tri * N                                  # C B^T
+        if shape.complex:
+            # Re(M) x is real; the chunk state is a complex MAC (8 flops); the
+            # off-diagonal readout keeps only the real part (4 flops per MAC)
+            per_head = 2 * tri * P + 8 * q * N * P + 4 * q * N * P
+            per_group = 8 * tri * N
+        total += b * (H * per_head + G * per_group)
+    return total
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+def kernel_source_sha(path: str) -> str:
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def lookup_traffic(kernel: str, source: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it is for this source."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    sha = kernel_source_sha(source)
+    for row in table.get("entries", []):
+        if row.get("kernel") == kernel and row.get("workload") == workload and row.get("source_sha") == sha:
+            return row.get("dram_bytes_per_launch")
+    return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Polls NVML for the SM clock and the clock-event reasons in a thread."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self.ok = False
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # no NVML: report clocks as unavailable
+            self.err = repr(exc)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except Exception:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        win = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not win:  # a very short region: take the samples nearest to it
+            win = sorted(self.samples, key=lambda s: min(abs(s[0] - t0), abs(s[0] - t1)))[:3]
+        reasons = set()
+        for _, _, rs in win:
+            for bit, name in self.REASONS.items():
+                if rs & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s[1] for s in win) if win else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(reasons), "samples": len(win)}
+
+
+# ------------------------------------------------------------ CPU oracle
+def oracle_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_oracle_units(w: dict, units, threads: int) -> float:
+    """Oracle over the given (batch, head) sequences, one per thread; seconds."""
+    import numpy as np
+
+    import oracle
+
+    lib = oracle.load()
+    G = w["B"].shape[2]
+    c = np.ascontiguousarray
+
+    def one(unit):
+        b, h = unit
+        g = 0 if G == 1 else h
+        oracle.scan(c(w["x"][b:b + 1, :, h:h + 1]), c(w["dt"][b:b + 1, :, h:h + 1]), c(w["A"][h:h + 1]),
+                    c(w["B"][b:b + 1, :, g:g + 1]), c(w["C"][b:b + 1, :, g:g + 1]),
+                    None if w["D"] is None else c(w["D"][h:h + 1]),
+                    None if w["init_state"] is None else c(w["init_state"][b:b + 1, h:h + 1]), lib=lib)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, units))
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(shape, max_updates: float = 4e9):
+    """The oracle as it stands, timed on this host's cores on a bounded sample:
+    the first (batch, head) sequences of the workload, up to ~max_updates state
+    element updates (the whole workload when it fits)."""
+    from selective_state_space_22_b200 import inputs
+
+    threads = oracle_threads()
+    w = inputs.widen_all(inputs.scan_inputs(shape))
+    total = shape.batch * shape.nheads
+    per_unit = shape.seqlen * shape.headdim * shape.dstate
+    n = max(1, min(total, int(max_updates // per_unit)))
+    units = [(i // shape.nheads, i % shape.nheads) for i in range(n)]
+    secs = run_oracle_units(w, units, threads)
+    tokens = shape.seqlen * n / shape.nheads
+    return {"value": tokens / secs, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
+            "sample": f"{n} of {total} (batch, head) sequences of {shape.name} (T={shape.seqlen}); "
+                      f"fp64 sequential recurrence, one sequence per thread; tokens/s counts "
+                      f"sequences/nheads x T",
+            "seconds": secs}
+
+
+# ------------------------------------------------------------------ arms
+def bench_reference(args, shape):
+    rank, world = dist_init("gloo")
+    if rank != 0:
+        return 0
+    from selective_state_space_22_b200 import inputs
+
+    threads = oracle_threads()
+    inp = inputs.scan_inputs(shape)
+    w = inputs.widen_all(inp)
+    n_heads = min(shape.nheads, max(threads, 1))
+    heads = list(range(n_heads))
+    units = [(0, h) for h in heads]
+    for _ in range(args.warmup):
+        run_oracle_units(w, units[:1], 1)
+    times = [run_oracle_units(w, units, threads) for _ in range(args.steps)]
+    secs = sum(times)
+    tokens = shape.seqlen * n_heads / shape.nheads * args.steps
+    value = tokens / secs
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
+                   "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
+                   "dstate": shape.dstate, "chunk": shape.chunk},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(threads, n_heads),
+                         "kind": "oracle",
+                         "sample": f"per step {n_heads} of {shape.nheads} heads of batch 0 "
+                                   f"(T={shape.seqlen}), one sequence per thread"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def bench_ours(args, shape):
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device for --impl ours")
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+
+    # inputs resident in HBM
+    inp = inputs.scan_inputs(shape)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    cplx = shape.complex
+    io = ssd.SSD_F32 if (cplx or shape.io_dtype == "f32") else ssd.SSD_BF16
+    y = torch.empty_like(d["x"])
+    fs = torch.empty((shape.batch, shape.nheads, shape.headdim, shape.dstate),
+                     dtype=torch.complex64 if cplx else torch.float32, device=dev)
+    nbytes = ssd.ssd_scan_workspace_size(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                                         shape.ngroups, shape.dstate, shape.chunk, cplx, io)
+    ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    fn = ssd.ssd_scan_fwd_complex if cplx else ssd.ssd_scan_fwd
+    launches = ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                                            shape.ngroups, shape.dstate, shape.chunk, cplx, io)
+
+    def step():
+        fn(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], chunk_size=shape.chunk,
+           y=y, final_state=fs, workspace=ws)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    ssd.ssd_get_device_status()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    local_s = sum(per_step_ms) / 1e3
+    total_s = dist_max(local_s, dev)
+    tokens = shape.tokens * world * args.steps
+    value = tokens / total_s
+    ms_per_step = 1e3 * total_s / args.steps
+
+    # roofline of the dominant kernel (the whole call when it is one launch)
+    peaks = load_peaks()
+    abytes = algorithmic_bytes(shape)
+    aflops = algorithmic_flops(shape)
+    t_launch = statistics.median(per_step_ms) / 1e3 if launches == 1 else sum(per_step_ms) / len(per_step_ms) / 1e3
+    hbm_t = abytes / (peaks["hbm_gbs"] * 1e9)
+    tc_t = aflops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if hbm_t >= tc_t else "tensor"
+    if bound == "hbm":
+        achieved, peak, unit = abytes / t_launch / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = aflops / t_launch / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
+    kernel = "ssd_scan_tc_kernel" if tc_path else "chunk_state+state_pass+chunk_scan (3 kernels)"
+    src = os.path.join(ROOT, "selective_state_space_22_b200", "csrc",
+                       "scan_tc.cu" if tc_path else "scan_generic.cu")
+    traffic = lookup_traffic(kernel, src, shape.name)
+    roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
+                "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
+                if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
+                "roofline_time_us": 1e6 * max(hbm_t, tc_t), "kernel_time_us": 1e6 * t_launch,
+                "frac_of_roofline_time": max(hbm_t, tc_t) / t_launch}
+
+    # end to end through the public API: pinned host inputs in, results back out
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
+        yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        fh = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
+        d2h = yh.numel() * yh.element_size() + fh.numel() * fh.element_size()
+        k_e2e = max(3, min(args.steps, 30))
+
+        def e2e_step():
+            for k, v in hin.items():
+                if v is not None:
+                    d[k].copy_(v, non_blocking=True)
+            step()
+            yh.copy_(y, non_blocking=True)
+            fh.copy_(fs, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist_barrier()
+        torch.cuda.synchronize()
+        es.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize()
+        dist_barrier()
+        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
+        e2e = {"value": shape.tokens * world * k_e2e / e2e_s, "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
+               "ms_per_step": 1e3 * e2e_s / k_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(shape)
+        cpu.pop("seconds", None)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if tc_path else "f32",
+        "data": "synthetic",
+        "impl": "ours",
+        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
+                   "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
+                   "dstate": shape.dstate, "chunk": shape.chunk, "io_dtype": shape.io_dtype,
+                   "state_dtype": "f32", "l2": "flushed between timed steps (512 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "clocks": sampler.summary(t0, t1),
+        "gpu_launches": launches * args.steps,
+        "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0] if len(per_step_ms) > 1 else per_step_ms[0],
+                                statistics.median(per_step_ms),
+                                statistics.quantiles(per_step_ms, n=10)[-1] if len(per_step_ms) > 1 else per_step_ms[0]],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2-bitmamba1b-layer-bf16")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    from selective_state_space_22_b200 import inputs
+
+    shape = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return bench_reference(args, shape)
+    return bench_ours(args, shape)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

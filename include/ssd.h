@@ -1,0 +1,172 @@
+/*
+ * ssd.h -- C ABI of the B200 selective state-space (SSD) scan library, libssd.so.
+ *
+ * The operation (all three entry points evaluate the same recurrence):
+ *
+ *   h_t = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T          (state P x N per head)
+ *   y_t = Re( h_t C_t ) + D_h * x_t                             (output P per head)
+ *
+ * Sources: "Mamba-3-Lite" README, the section on the classical (real) Mamba-2
+ * recurrence and its complex promotion; "Block Anatomy, Numerical Stability &
+ * Scaling" -- Block Anatomy section 3 (the interface: (B,T,H,D)-shaped inputs in,
+ * a (B,T,H,D) real output out), section 4.3 (x and dt stay float32, B and C are
+ * complex64), section 4.4 (one complex A per head, decay exp(softplus(dt) A)),
+ * section 6 (the real part of the output leaves the scan; the state starts at
+ * zero); Numerical Stability section 4 (the chunkwise form: within-chunk decay
+ * exp(segsum(dt A)) and the inter-chunk propagation).  "BitMamba 1B" (Portuguese
+ * edition, "Contexto") gives the Mamba-2 layer shape: 64 heads, d_state 128,
+ * d_inner 4096 (head dim 64), one real A per head.
+ *
+ * Conventions shared by every entry point
+ *  - Every tensor pointer is a DEVICE pointer to contiguous row-major memory,
+ *    16-byte aligned.  The caller owns all memory; nothing is allocated, freed
+ *    or retained by the library.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is the
+ *    legacy default stream) and is asynchronous: a returned SSD_OK means the
+ *    launch was accepted, not that it finished.
+ *  - Arguments are validated on the host before any launch; on a non-OK status
+ *    nothing was launched and ssd_last_error() describes why.
+ *  - dt is the step size AFTER softplus and dt_bias (the library applies no
+ *    softplus).  Head h reads group h / (nheads / ngroups) of B and C.
+ *  - The input is injected as dt_t * x_t B_t^T and the output reads the state
+ *    after that step's update.
+ *  - Complex tensors are interleaved (re, im) float pairs, the memory layout of
+ *    a complex64 tensor.  The complex output is the real part only.
+ *  - Outputs never alias inputs, except: final_state may equal init_state, and
+ *    ssd_state_update updates `state` in place.
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size; nothing launched */
+    SSD_ERR_UNSUPPORTED = 2,   /* valid arguments this build has no kernel for */
+    SSD_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch or query) */
+    SSD_ERR_TIMEOUT = 4,       /* a bounded inter-block wait gave up (device-side) */
+    SSD_ERR_WORKSPACE = 5      /* workspace NULL or smaller than ssd_scan_workspace_size */
+} ssd_status;
+
+typedef enum {
+    SSD_F32 = 0,   /* float32 */
+    SSD_BF16 = 1   /* bfloat16 */
+} ssd_dtype;
+
+/*
+ * Workspace bytes that ssd_scan_fwd / ssd_scan_fwd_complex need for these sizes.
+ * Returns 0 when the sizes are invalid.  The workspace must be ZERO-FILLED once
+ * after it is allocated; after that it needs no clearing between calls (the
+ * kernels leave it reusable).  One workspace may not be used by two calls that
+ * can run at the same time (different streams): they would race.
+ */
+size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
+                               int ngroups, int dstate, int chunk_size,
+                               int is_complex, ssd_dtype io_dtype);
+
+/*
+ * Number of kernels that one ssd_scan_fwd / ssd_scan_fwd_complex call with these
+ * sizes enqueues when seqlen > 0 (0 for invalid sizes).  For capture planning
+ * and launch accounting; it launches nothing.
+ */
+int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int ngroups,
+                             int dstate, int chunk_size, int is_complex, ssd_dtype io_dtype);
+
+/*
+ * Real chunked scan (Mamba-2 layout, one real A per head).
+ *
+ *  x           [batch, seqlen, nheads, headdim]  io_dtype
+ *  dt          [batch, seqlen, nheads]           float32, > 0 (post-softplus)
+ *  A           [nheads]                          float32, expected <= 0
+ *  B, C        [batch, seqlen, ngroups, dstate]  io_dtype
+ *  D           [nheads] float32, or NULL for no skip term
+ *  init_state  [batch, nheads, headdim, dstate] float32, or NULL for zeros
+ *  final_state [batch, nheads, headdim, dstate] float32, or NULL to skip
+ *  y           [batch, seqlen, nheads, headdim]  io_dtype (output)
+ *  chunk_size  chunk length of the chunkwise evaluation: 64, 128 or 256.  The
+ *              result does not depend on it beyond rounding.
+ *  workspace   device scratch of at least ssd_scan_workspace_size(...) bytes,
+ *              zero-filled once after allocation.
+ *
+ * seqlen may be 0 (then y is empty and final_state = init_state, or zeros) and
+ * need not be a multiple of chunk_size.  io_dtype SSD_BF16 runs the tcgen05
+ * tensor-core kernel when headdim == 64 and dstate is 64 or 128; every other
+ * combination runs the float32 CUDA-core kernels.  State and accumulation are
+ * float32 in both.
+ */
+ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A,
+                        const void *B, const void *C, const float *D,
+                        const float *init_state, float *final_state, void *y,
+                        ssd_dtype io_dtype, int batch, int seqlen, int nheads,
+                        int headdim, int ngroups, int dstate, int chunk_size,
+                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Complex chunked scan (Mamba-3-Lite layout, one complex A per head).
+ *
+ *  x           [batch, seqlen, nheads, headdim]       float32 (real)
+ *  dt          [batch, seqlen, nheads]                float32
+ *  A           [nheads] complex (float pairs), Re A expected <= 0
+ *  B, C        [batch, seqlen, ngroups, dstate] complex
+ *  D           [nheads] float32 or NULL
+ *  init_state  [batch, nheads, headdim, dstate] complex, or NULL for zeros
+ *  final_state [batch, nheads, headdim, dstate] complex, or NULL
+ *  y           [batch, seqlen, nheads, headdim] float32 = Re(h_t C_t) + D x_t
+ *
+ * Runs in float32 (complex64) throughout.  Other arguments as ssd_scan_fwd.
+ */
+ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A,
+                                const float *B, const float *C, const float *D,
+                                const float *init_state, float *final_state, float *y,
+                                int batch, int seqlen, int nheads, int headdim,
+                                int ngroups, int dstate, int chunk_size,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One recurrent decoding step, in place on the state (real variant):
+ *   state <- exp(dt A) state + dt x B^T ;  y = state C + D x
+ *
+ *  state [batch, nheads, headdim, dstate] float32, read and overwritten
+ *  x     [batch, nheads, headdim]  io_dtype
+ *  dt    [batch, nheads]           float32
+ *  A     [nheads] float32;  B, C [batch, ngroups, dstate] io_dtype
+ *  D     [nheads] float32 or NULL;  y [batch, nheads, headdim] io_dtype (output)
+ *
+ * Needs no workspace.  "batch" is the number of sequences decoded together.
+ */
+ssd_status ssd_state_update(float *state, const void *x, const float *dt,
+                            const float *A, const void *B, const void *C,
+                            const float *D, void *y, ssd_dtype io_dtype, int batch,
+                            int nheads, int headdim, int ngroups, int dstate,
+                            void *stream);
+
+/* The complex decoding step: state, A, B, C complex; x, dt, D, y float32. */
+ssd_status ssd_state_update_complex(float *state, const float *x, const float *dt,
+                                    const float *A, const float *B, const float *C,
+                                    const float *D, float *y, int batch, int nheads,
+                                    int headdim, int ngroups, int dstate, void *stream);
+
+/*
+ * Waits for `stream`, then reports and clears an error that a kernel raised on
+ * the device since the last call on this device (SSD_ERR_TIMEOUT when a bounded
+ * inter-block wait gave up; the outputs of that call are then invalid), or a
+ * CUDA error from the stream.  SSD_OK when there was none.
+ */
+ssd_status ssd_get_device_status(void *stream);
+
+/* Message for the last non-OK status returned on the calling host thread. */
+const char *ssd_last_error(void);
+
+/* Library version string. */
+const char *ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SSD_B200_H */

@@ -1,0 +1,280 @@
+// ssd_api.cu -- the C ABI of libssd (declared in include/ssd.h).
+//
+// Host-side argument validation, workspace sizing, kernel selection and the
+// device error word.  Every check happens before the first launch, so a
+// non-OK status means nothing was enqueued.
+#include <stdarg.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "../../include/ssd.h"
+#include "ssd_internal.cuh"
+
+// First device-side error raised by a kernel of this library on this device
+// (a bounded wait that gave up).  Read and cleared by ssd_get_device_status.
+__device__ int g_ssd_device_error = 0;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+ssd_status fail(ssd_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+ssd_status fail(ssd_status s, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+ssd_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(SSD_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int *device_error_ptr(ssd_status *st) {
+    static int *cache[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *st = cuda_fail(e, "cudaGetDevice");
+        return nullptr;
+    }
+    if (!cache[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_ssd_device_error);
+        if (e != cudaSuccess) {
+            *st = cuda_fail(e, "cudaGetSymbolAddress(device error word)");
+            return nullptr;
+        }
+        cache[dev] = static_cast<int *>(p);
+    }
+    return cache[dev];
+}
+
+constexpr int kMaxHeaddim = 256;
+constexpr int kMaxDstate = 256;
+
+// Shape checks shared by the scans.
+ssd_status check_scan_dims(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                           int chunk) {
+    if (batch < 0 || seqlen < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch (%d) and seqlen (%d) must be >= 0", batch, seqlen);
+    if (nheads <= 0 || headdim <= 0 || ngroups <= 0 || dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "nheads (%d), headdim (%d), ngroups (%d), dstate (%d) must be > 0", nheads,
+                    headdim, ngroups, dstate);
+    if (nheads % ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "ngroups (%d) must divide nheads (%d)", ngroups, nheads);
+    if (chunk != 64 && chunk != 128 && chunk != 256)
+        return fail(SSD_ERR_INVALID_ARG, "chunk_size must be 64, 128 or 256 (got %d)", chunk);
+    if (headdim > kMaxHeaddim || dstate > kMaxDstate)
+        return fail(SSD_ERR_UNSUPPORTED, "headdim (%d) and dstate (%d) must be <= %d and %d",
+                    headdim, dstate, kMaxHeaddim, kMaxDstate);
+    if (nheads > 65535 || batch > 2048 || (long long)batch * seqlen > (1LL << 31))
+        return fail(SSD_ERR_UNSUPPORTED, "sizes beyond the supported grid (batch <= 2048, "
+                    "nheads <= 65535, batch*seqlen <= 2^31)");
+    return SSD_OK;
+}
+
+struct Plan {
+    bool tc;  // tcgen05 tensor-core kernel
+    size_t ws;
+    int launches;
+};
+
+Plan plan_scan(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate, int chunk,
+               bool cplx, bool bf16) {
+    Plan p{false, 0, 0};
+    const int nchunks = seqlen > 0 ? (seqlen + chunk - 1) / chunk : 0;
+    if (!cplx && bf16 && ssd::tc_supported(headdim, dstate, chunk)) {
+        p.tc = true;
+        p.ws = ssd::tc_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk);
+        p.launches = ssd::tc_kernel_launches();
+        return p;
+    }
+    p.ws = ssd::generic_workspace_bytes(batch, nheads, headdim, dstate, chunk, nchunks, cplx);
+    p.launches = 3;
+    return p;
+}
+
+ssd_status run_scan(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                    const float *D, const float *init_state, float *final_state, void *y, bool cplx,
+                    bool bf16, int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                    int chunk, void *workspace, size_t workspace_bytes, void *stream) {
+    ssd_status s = check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk);
+    if (s != SSD_OK) return s;
+    const size_t state_floats = (size_t)batch * nheads * headdim * dstate * (cplx ? 2 : 1);
+    const bool any_tokens = (size_t)batch * seqlen > 0;
+    if (any_tokens) {
+        if (!x || !dt || !A || !B || !C || !y)
+            return fail(SSD_ERR_INVALID_ARG, "x, dt, A, B, C and y must be non-null");
+        const void *ptrs[] = {x, dt, A, B, C, y, D, init_state, final_state};
+        for (const void *p : ptrs)
+            if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    } else {
+        if ((init_state && !aligned16(init_state)) || (final_state && !aligned16(final_state)))
+            return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!any_tokens) {
+        // No tokens: the final state is the initial one (or zeros).
+        if (final_state && final_state != init_state) {
+            cudaError_t e = ssd::launch_copy_or_zero_state(init_state, final_state, state_floats, st);
+            if (e != cudaSuccess) return cuda_fail(e, "state copy launch");
+        }
+        return SSD_OK;
+    }
+    Plan pl = plan_scan(batch, seqlen, nheads, headdim, ngroups, dstate, chunk, cplx, bf16);
+    if (pl.ws > 0) {
+        if (!workspace)
+            return fail(SSD_ERR_WORKSPACE, "workspace is NULL; %zu bytes are needed", pl.ws);
+        if (workspace_bytes < pl.ws)
+            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes is too small; %zu are needed",
+                        workspace_bytes, pl.ws);
+        if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    }
+    int *dev_err = device_error_ptr(&s);
+    if (!dev_err) return s;
+
+    ssd::ScanArgs a;
+    a.x = x;
+    a.dt = dt;
+    a.A = A;
+    a.B = B;
+    a.C = C;
+    a.D = D;
+    a.init_state = init_state;
+    a.final_state = final_state;
+    a.y = y;
+    a.batch = batch;
+    a.seqlen = seqlen;
+    a.nheads = nheads;
+    a.headdim = headdim;
+    a.ngroups = ngroups;
+    a.dstate = dstate;
+    a.chunk = chunk;
+    a.nchunks = (seqlen + chunk - 1) / chunk;
+    a.dev_error = dev_err;
+    cudaError_t e = pl.tc ? ssd::launch_tc_scan(a, workspace, st)
+                          : ssd::launch_generic_scan(a, cplx, bf16, workspace, st);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return SSD_OK;
+}
+
+ssd_status run_update(float *state, const void *x, const float *dt, const float *A, const void *B,
+                      const void *C, const float *D, void *y, bool bf16, bool cplx, int batch,
+                      int nheads, int headdim, int ngroups, int dstate, void *stream) {
+    if (batch < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch (%d) must be >= 0", batch);
+    if (nheads <= 0 || headdim <= 0 || ngroups <= 0 || dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG,
+                    "nheads (%d), headdim (%d), ngroups (%d), dstate (%d) must be > 0", nheads,
+                    headdim, ngroups, dstate);
+    if (nheads % ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "ngroups (%d) must divide nheads (%d)", ngroups, nheads);
+    if ((long long)batch * nheads * headdim > (1LL << 36))
+        return fail(SSD_ERR_UNSUPPORTED, "batch * nheads * headdim too large");
+    if (batch == 0) return SSD_OK;
+    if (!state || !x || !dt || !A || !B || !C || !y)
+        return fail(SSD_ERR_INVALID_ARG, "state, x, dt, A, B, C and y must be non-null");
+    const void *ptrs[] = {state, x, dt, A, B, C, y, D};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = ssd::launch_state_update(state, x, dt, A, B, C, D, y, bf16, cplx, batch, nheads,
+                                             headdim, ngroups, dstate, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "state update launch");
+    return SSD_OK;
+}
+
+bool valid_dtype(ssd_dtype d) { return d == SSD_F32 || d == SSD_BF16; }
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,
+                               int dstate, int chunk_size, int is_complex, ssd_dtype io_dtype) {
+    if (!valid_dtype(io_dtype)) return 0;
+    if (check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size) != SSD_OK)
+        return 0;
+    Plan pl = plan_scan(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size, is_complex != 0,
+                        io_dtype == SSD_BF16);
+    return pl.ws;
+}
+
+int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate,
+                             int chunk_size, int is_complex, ssd_dtype io_dtype) {
+    if (!valid_dtype(io_dtype)) return 0;
+    if (check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size) != SSD_OK)
+        return 0;
+    return plan_scan(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size, is_complex != 0,
+                     io_dtype == SSD_BF16)
+        .launches;
+}
+
+ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A, const void *B,
+                        const void *C, const float *D, const float *init_state, float *final_state,
+                        void *y, ssd_dtype io_dtype, int batch, int seqlen, int nheads, int headdim,
+                        int ngroups, int dstate, int chunk_size, void *workspace,
+                        size_t workspace_bytes, void *stream) {
+    if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    return run_scan(x, dt, A, B, C, D, init_state, final_state, y, false, io_dtype == SSD_BF16, batch,
+                    seqlen, nheads, headdim, ngroups, dstate, chunk_size, workspace, workspace_bytes,
+                    stream);
+}
+
+ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A, const float *B,
+                                const float *C, const float *D, const float *init_state,
+                                float *final_state, float *y, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate, int chunk_size, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    return run_scan(x, dt, A, B, C, D, init_state, final_state, y, true, false, batch, seqlen, nheads,
+                    headdim, ngroups, dstate, chunk_size, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_state_update(float *state, const void *x, const float *dt, const float *A,
+                            const void *B, const void *C, const float *D, void *y,
+                            ssd_dtype io_dtype, int batch, int nheads, int headdim, int ngroups,
+                            int dstate, void *stream) {
+    if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    return run_update(state, x, dt, A, B, C, D, y, io_dtype == SSD_BF16, false, batch, nheads, headdim,
+                      ngroups, dstate, stream);
+}
+
+ssd_status ssd_state_update_complex(float *state, const float *x, const float *dt, const float *A,
+                                    const float *B, const float *C, const float *D, float *y,
+                                    int batch, int nheads, int headdim, int ngroups, int dstate,
+                                    void *stream) {
+    return run_update(state, x, dt, A, B, C, D, y, false, true, batch, nheads, headdim, ngroups,
+                      dstate, stream);
+}
+
+ssd_status ssd_get_device_status(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int code = 0;
+    e = cudaMemcpyFromSymbol(&code, g_ssd_device_error, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (code == 0) return SSD_OK;
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_ssd_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    if (code == ssd::DEV_TIMEOUT)
+        return fail(SSD_ERR_TIMEOUT, "a bounded inter-block wait gave up on the device; the "
+                    "outputs of the call that raised it are invalid");
+    return fail(SSD_ERR_CUDA, "device error code %d", code);
+}
+
+const char *ssd_last_error(void) { return g_last_error.c_str(); }
+
+const char *ssd_version(void) { return "ssd-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,91 @@
+// ssd_internal.cuh -- types and helpers shared by the CUDA kernels of libssd.
+//
+// Nothing here is part of the public ABI (include/ssd.h is).  All kernels run
+// on the stream the caller passes and read/write caller-owned device memory.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// ----------------------------------------------------------------- io types
+template <typename T> __device__ __forceinline__ float ld_f32(const T *p);
+template <> __device__ __forceinline__ float ld_f32<float>(const float *p) { return *p; }
+template <> __device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16 *p) {
+    return __bfloat162float(*p);
+}
+template <typename T> __device__ __forceinline__ void st_f32(T *p, float v);
+template <> __device__ __forceinline__ void st_f32<float>(float *p, float v) { *p = v; }
+template <> __device__ __forceinline__ void st_f32<__nv_bfloat16>(__nv_bfloat16 *p, float v) {
+    *p = __float2bfloat16_rn(v);
+}
+
+// ------------------------------------------------------------ complex floats
+// Interleaved (re, im) pairs, the memory layout of complex64.
+struct cf {
+    float re, im;
+};
+__device__ __forceinline__ cf cmul(cf a, cf b) {
+    return {fmaf(a.re, b.re, -a.im * b.im), fmaf(a.re, b.im, a.im * b.re)};
+}
+__device__ __forceinline__ cf cfma(cf a, cf b, cf c) {  // a*b + c
+    return {fmaf(a.re, b.re, fmaf(-a.im, b.im, c.re)), fmaf(a.re, b.im, fmaf(a.im, b.re, c.im))};
+}
+__device__ __forceinline__ cf cscale(cf a, float s) { return {a.re * s, a.im * s}; }
+__device__ __forceinline__ cf cadd(cf a, cf b) { return {a.re + b.re, a.im + b.im}; }
+
+// exp(z) for a complex exponent z = (a, w) given in double: e^a (cos w, sin w).
+__device__ __forceinline__ cf cexp_d(double a, double w) {
+    float r = (float)exp(a);
+    float s, c;
+    sincosf((float)w, &s, &c);
+    return {r * c, r * s};
+}
+
+// -------------------------------------------------------------- arguments
+// One scan call as the kernels see it.  For the complex variant the complex
+// tensors (A, B, C, states) are float pairs.
+struct ScanArgs {
+    const void *x;
+    const float *dt;
+    const float *A;
+    const void *B;
+    const void *C;
+    const float *D;
+    const float *init_state;
+    float *final_state;
+    void *y;
+    int batch, seqlen, nheads, headdim, ngroups, dstate, chunk;
+    int nchunks;
+    int *dev_error;  // device error word (see ssd_get_device_status)
+};
+
+// Device error codes written to *dev_error (first writer wins).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
+
+// --------------------------------------------------------- kernel launchers
+// Each returns cudaSuccess or the launch error; none synchronises.
+size_t generic_workspace_bytes(int batch, int nheads, int headdim, int dstate, int chunk,
+                               int nchunks, bool cplx);
+cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *ws,
+                                cudaStream_t st);
+
+// tcgen05 tensor-core scan (bf16 io, real A).
+bool tc_supported(int headdim, int dstate, int chunk);
+size_t tc_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate, int chunk);
+cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st);
+int tc_kernel_launches();
+
+cudaError_t launch_state_update(float *state, const void *x, const float *dt, const float *A,
+                                const void *B, const void *C, const float *D, void *y,
+                                bool bf16, bool cplx, int batch, int nheads, int headdim,
+                                int ngroups, int dstate, cudaStream_t st);
+
+cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_state,
+                                      size_t nfloats, cudaStream_t st);
+
+static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace ssd
