@@ -60,10 +60,10 @@ typedef enum {
 
 /*
  * Workspace bytes that ssd_scan_fwd / ssd_scan_fwd_complex need for these sizes.
- * Returns 0 when the sizes are invalid.  The workspace must be ZERO-FILLED once
- * after it is allocated; after that it needs no clearing between calls (the
- * kernels leave it reusable).  One workspace may not be used by two calls that
- * can run at the same time (different streams): they would race.
+ * Returns 0 when the sizes are invalid.  The workspace needs no initialisation:
+ * each call clears, on its stream, whatever it needs cleared.  One workspace may
+ * not be used by two calls that can run at the same time (different streams):
+ * they would race.
  */
 size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
                                int ngroups, int dstate, int chunk_size,
@@ -90,14 +90,17 @@ int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int
  *  y           [batch, seqlen, nheads, headdim]  io_dtype (output)
  *  chunk_size  chunk length of the chunkwise evaluation: 64, 128 or 256.  The
  *              result does not depend on it beyond rounding.
- *  workspace   device scratch of at least ssd_scan_workspace_size(...) bytes,
- *              zero-filled once after allocation.
+ *  workspace   device scratch of at least ssd_scan_workspace_size(...) bytes.
  *
  * seqlen may be 0 (then y is empty and final_state = init_state, or zeros) and
- * need not be a multiple of chunk_size.  io_dtype SSD_BF16 runs the tcgen05
- * tensor-core kernel when headdim == 64 and dstate is 64 or 128; every other
- * combination runs the float32 CUDA-core kernels.  State and accumulation are
- * float32 in both.
+ * need not be a multiple of chunk_size.  io_dtype SSD_BF16 with headdim 64,
+ * dstate 128 and seqlen >= 128 runs the tcgen05 tensor-core kernel (one launch,
+ * plus a small memset of its workspace flags); it evaluates 128-token chunks
+ * (its MMA tile height) whatever chunk_size says, and its results are
+ * reproducible to rounding but not bitwise (the inter-chunk look-back may add
+ * the same terms in a different order).  Every other combination runs the
+ * float32 CUDA-core kernels (three launches), which honour chunk_size.  State
+ * and accumulation are float32 in both.
  */
 ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A,
                         const void *B, const void *C, const float *D,

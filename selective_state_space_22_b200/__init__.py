@@ -119,7 +119,7 @@ _ws_cache: dict = {}
 
 
 def _workspace(device, nbytes: int):
-    """A zero-filled, cached per-device workspace of at least nbytes."""
+    """A cached per-device workspace of at least nbytes (no initialisation needed)."""
     if nbytes == 0:
         return None
     key = device.index
@@ -149,7 +149,7 @@ def ssd_scan_fwd(x, dt, A, B, C, D=None, init_state=None, *, chunk_size=256, y=N
     """Real chunked scan.  Returns (y, final_state or None).
 
     x [b,T,H,P] and B, C [b,T,G,N] bf16 or float32 (same dtype); dt [b,T,H], A [H],
-    D [H], init_state [b,H,P,N] float32.  ``workspace`` is an optional zero-filled
+    D [H], init_state [b,H,P,N] float32.  ``workspace`` is an optional
     uint8 CUDA tensor (a cached one is used otherwise).
     """
     lib = load_library()

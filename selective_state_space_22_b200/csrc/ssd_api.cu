@@ -93,9 +93,9 @@ Plan plan_scan(int batch, int seqlen, int nheads, int headdim, int ngroups, int 
                bool cplx, bool bf16) {
     Plan p{false, 0, 0};
     const int nchunks = seqlen > 0 ? (seqlen + chunk - 1) / chunk : 0;
-    if (!cplx && bf16 && ssd::tc_supported(headdim, dstate, chunk)) {
+    if (!cplx && bf16 && ssd::tc_supported(headdim, dstate, seqlen)) {
         p.tc = true;
-        p.ws = ssd::tc_workspace_bytes(batch, seqlen, nheads, headdim, dstate, chunk);
+        p.ws = ssd::tc_workspace_bytes(batch, nheads);
         p.launches = ssd::tc_kernel_launches();
         return p;
     }

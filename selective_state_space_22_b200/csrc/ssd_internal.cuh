@@ -73,8 +73,8 @@ cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *w
                                 cudaStream_t st);
 
 // tcgen05 tensor-core scan (bf16 io, real A).
-bool tc_supported(int headdim, int dstate, int chunk);
-size_t tc_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate, int chunk);
+bool tc_supported(int headdim, int dstate, int seqlen);
+size_t tc_workspace_bytes(int batch, int nheads);
 cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st);
 int tc_kernel_launches();
 

@@ -117,12 +117,31 @@ def test_no_D_no_final_state():
 
 
 def test_repeated_calls_reuse_workspace():
+    """Calls on one workspace agree; the look-back may sum the same terms in a
+    different order from call to call, so agreement is to rounding, not bitwise."""
     shape = small("rep", 2, 700, 4, 64, 1, 128, 256, "bf16", init=True)
     inp = inputs.scan_inputs(shape)
     y0, f0 = gpu_scan(inp, 256, False)
     for _ in range(3):
         y1, f1 = gpu_scan(inp, 256, False)
-        assert torch.equal(y0, y1) and torch.equal(f0, f1)
+        assert rel_err(y1.numpy(), y0.numpy()) <= 1e-2
+        assert rel_err(f1.numpy(), f0.numpy()) <= 1e-5
+
+
+def _tc(shape):
+    return ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                                        shape.ngroups, shape.dstate, shape.chunk, False,
+                                        ssd.SSD_BF16) == 1
+
+
+@pytest.mark.parametrize("T", [128, 129, 256, 1000, 128 * 20 + 5])
+@pytest.mark.parametrize("H,G", [(1, 1), (4, 2), (6, 6)])
+def test_tcgen05_path(T, H, G):
+    """The tensor-core kernel: one chunk, ragged tails, more chunks than ring slots
+    (slot reuse), several groups."""
+    shape = small("tc", 2, T, H, 64, G, 128, 256, "bf16", init=(H != 1), seed=T + H)
+    assert _tc(shape), "expected the tcgen05 kernel for this shape"
+    check_full(shape, TOL_BF16)
 
 
 # --------------------------------------------------------- full-size, sampled
@@ -138,6 +157,7 @@ def _sampled(shape, samples, tol):
 
 
 def test_mamba2_1b_layer_sampled():
+    assert _tc(inputs.MAMBA2_1B)
     _sampled(inputs.MAMBA2_1B, [(0, 0), (0, 37), (1, 5), (1, 63)], TOL_BF16)
 
 
@@ -146,4 +166,5 @@ def test_mamba3_complex_layer_sampled():
 
 
 def test_long_sequence_sampled():
+    assert _tc(inputs.LONG)
     _sampled(inputs.LONG, [(0, 3), (0, 60)], TOL_BF16)
