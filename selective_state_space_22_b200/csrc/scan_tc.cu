@@ -49,29 +49,40 @@ using namespace ptx;
 constexpr int QT = 128;   // tokens per tile (tcgen05 M)
 constexpr int PD = 64;    // head dim
 constexpr int ND = 128;   // state dim
-constexpr int NTH = 128;  // threads per CTA: 4 warps, one per TMEM lane quadrant
 constexpr int RING = 8;   // published-state slots per sequence
-constexpr int DEPTH = 3;  // look-back reads at most this many predecessors
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int DEPTH = 2;  // look-back reads at most this many predecessors
+
+// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 "math" warpgroup (decay, W,
+// M, y), 6-9 "state" warpgroup (look-back, publication, h_in).  A warpgroup's
+// warp w reaches TMEM lanes 32*(w%4)..+31, so each covers all 128 lanes.
+constexpr int NTH = 320;
+constexpr int MATH_W0 = 2, STATE_W0 = 6;
+constexpr uint32_t BAR_MATH = 1;  // named barrier of the math warpgroup (128 threads)
+
+// TMEM: two column sets of 256 (tiles alternate between them).
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M in place (bf16 pairs, 64 cols)
 constexpr uint32_t COL_YD = 128; // M X                       (64 cols)
 constexpr uint32_t COL_S = 192;  // chunk state, then C h^T   (64 cols)
-constexpr uint32_t LOAD_BYTES = 2 * (QT * ND * 2) + QT * PD * 2;
 
-// Shared memory (offsets from a 1024-byte aligned base; every operand tile is
-// rows of 128 bytes in the 128-byte swizzle pattern TMA writes).
-constexpr int OFF_C = 0;          // C   [128 l][128 n]  two 64-column panels
-constexpr int OFF_B = 32768;      // B   [128 s][128 n]  two panels
-constexpr int OFF_X = 65536;      // X   [128 s][64 p];  later h_in^T bf16 [64 p][128 n]
-constexpr int OFF_W = 81920;      // W = diag(w) X;      later the y tile
-constexpr int OFF_MISC = 98304;   // cs, dt, column factors, warp sums, mbarriers, TMEM base
-constexpr int MISC_BYTES = 3 * QT * 4 + 16 + 5 * 8 + 8;
+// Shared memory: two input stages {C, B, X} and two W / y buffers.
+constexpr int STAGE_BYTES = 81920;
+constexpr int OFF_C = 0, OFF_B = 32768, OFF_X = 65536;  // within a stage
+constexpr int OFF_W = 2 * STAGE_BYTES;                  // 2 x 16 KB
+constexpr int OFF_MISC = OFF_W + 2 * 16384;
+constexpr uint32_t LOAD_BYTES = 2 * (QT * ND * 2) + QT * PD * 2;
+enum {
+    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_YD = 8, B_YO = 10,         // count 1
+    B_CS = 12, B_W = 14, B_M = 16, B_H = 18, B_FREE = 20, NBARS = 22         // count 128
+};
+// misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], wtot[4], bars, tmem base
+constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
 constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 1, 1);    // B^T (MN-major) x W (MN-major)
 constexpr uint32_t IDESC_YD = idesc_bf16_f32(128, 64, 0, 1);   // M (TMEM) x X (MN-major)
-constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 0);   // C (K-major) x h (K-major)
+constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C (K-major) x h^T (MN-major)
 
 enum : uint32_t { ST_AGG = 1, ST_PREFIX = 2 };
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on every wait
@@ -84,11 +95,27 @@ struct TcParams {
     float *final_state;
     uint32_t *flags;  // [bH][RING][4 warps]  (chunk << 2) | status
     float *lam;       // [bH][RING][4 warps]  log-decay of the chunk in the slot
-    float *agg;       // [bH][RING][PD][ND]
-    float *pre;       // [bH][RING][PD][ND]
+    float *agg;       // [bH][RING][ND][PD]   chunk state from a zero start
+    float *pre;       // [bH][RING][ND][PD]   state after the chunk
     int seqlen, nheads, ngroups, nchunks, ntiles, bH;
     int *dev_error;
 };
+
+struct Tile {
+    int c, bh, b, h, g, t0, valid;
+};
+__device__ __forceinline__ Tile decode_tile(const TcParams &p, int k) {
+    Tile t;
+    const int tile = blockIdx.x + k * gridDim.x;
+    t.c = tile / p.bH;
+    t.bh = tile % p.bH;
+    t.b = t.bh / p.nheads;
+    t.h = t.bh % p.nheads;
+    t.g = t.h / (p.nheads / p.ngroups);
+    t.t0 = t.c * QT;
+    t.valid = min(QT, p.seqlen - t.t0);
+    return t;
+}
 
 __device__ __forceinline__ unsigned long long now_ns() {
     unsigned long long t;
@@ -98,17 +125,16 @@ __device__ __forceinline__ unsigned long long now_ns() {
 
 __device__ __forceinline__ void report_timeout(int *err) { atomicCAS(err, 0, DEV_TIMEOUT); }
 
-// Bounded wait on an mbarrier phase; false (and the device error set) on timeout.
-__device__ bool mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait on an mbarrier phase (the device error is set on timeout).
+__device__ void mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
+    if (mbar_try_wait(bar, parity)) return;
     const unsigned long long t0 = now_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (now_ns() - t0 > WAIT_NS) {
             report_timeout(err);
-            return false;
+            return;
         }
     }
-    return true;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -116,16 +142,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Lane 0 of a warp waits until *f satisfies `ready`; the value is broadcast.
+// Lane 0 of a warp waits until *f satisfies `ready`; the value is broadcast
+// (0 after a timeout, which is also reported).
 template <typename Pred>
-__device__ uint32_t warp_wait_flag(const uint32_t *f, Pred ready, int *err, bool &ok) {
+__device__ uint32_t warp_wait_flag(const uint32_t *f, Pred ready, int *err) {
     uint32_t v = 0;
     if ((threadIdx.x & 31) == 0) {
         v = ld_acquire_u32(f);
         if (!ready(v)) {
             const unsigned long long t0 = now_ns();
             while (true) {
-                __nanosleep(64);
+                __nanosleep(32);
                 v = ld_acquire_u32(f);
                 if (ready(v)) break;
                 if (now_ns() - t0 > WAIT_NS) {
@@ -136,39 +163,46 @@ __device__ uint32_t warp_wait_flag(const uint32_t *f, Pred ready, int *err, bool
             }
         }
     }
-    v = __shfl_sync(0xffffffffu, v, 0);
-    if (v == 0) ok = false;
-    return v;
+    return __shfl_sync(0xffffffffu, v, 0);
 }
 
-// State entering chunk c of sequence bh for this warp's 32 state rows (n), and
-// publication of this chunk's aggregate and prefix.  s[] is the chunk state
-// S[n][p] of this thread's row n; hp[] receives h_in[p][n].
-__device__ void lookback(const TcParams &p, int bh, int c, int warp, int lane, float lam,
-                         const float (&s)[PD], float (&hp)[PD], bool &ok) {
-    const int n = warp * 32 + lane;
-    const size_t ring0 = (size_t)bh * RING;
-    const int slot = c % RING;
-    uint32_t *flag = p.flags + (ring0 + slot) * 4 + warp;
-    float *aggp = p.agg + (ring0 + slot) * (PD * ND) + n;
-    float *prep = p.pre + (ring0 + slot) * (PD * ND) + n;
+__device__ __forceinline__ void ld_row64(const float *src, float (&v)[PD]) {
+#pragma unroll
+    for (int q = 0; q < PD; q += 4) {
+        const float4 f = ld_cg_f4(src + q);
+        v[q] = f.x; v[q + 1] = f.y; v[q + 2] = f.z; v[q + 3] = f.w;
+    }
+}
+__device__ __forceinline__ void st_row64(float *dst, const float (&v)[PD]) {
+#pragma unroll
+    for (int q = 0; q < PD; q += 4) *reinterpret_cast<float4 *>(dst + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
+}
 
-    // Reuse of this slot: the chunk that last used it (c - RING) and the chunks
-    // that may still read it (up to c - RING + DEPTH) must all have published
-    // their prefixes (a later chunk in their slot also proves it).
-    if (c >= RING) {
+// State entering chunk c of sequence bh for this warp's 32 state rows (n = row),
+// and publication of this chunk's prefix (and, when its predecessor's prefix is
+// not there yet, first its aggregate).  s[] is S[n][:] of this thread's row;
+// hp[] receives h_in[:][n].  Slot layout [n][p]: a row is 256 contiguous bytes.
+__device__ void lookback(const TcParams &p, const Tile &t, int quad, int lane, float lam,
+                         const float (&s)[PD], float (&hp)[PD]) {
+    const int n = quad * 32 + lane;
+    const int c = t.c;
+    const size_t ring0 = (size_t)t.bh * RING;
+    const int slot = c % RING;
+    uint32_t *flag = p.flags + (ring0 + slot) * 4 + quad;
+    const size_t row = (size_t)n * PD;
+
+    if (c >= RING) {  // slot reuse: its last user and possible readers have published prefixes
         for (int k = 0; k <= DEPTH; ++k) {
             const int j = c - RING + k;
-            const uint32_t *f = p.flags + (ring0 + j % RING) * 4 + warp;
-            warp_wait_flag(f, [j](uint32_t v) {
+            warp_wait_flag(p.flags + (ring0 + j % RING) * 4 + quad, [j](uint32_t v) {
                 return (int)(v >> 2) > j || ((int)(v >> 2) == j && (v & 3u) == ST_PREFIX);
-            }, p.dev_error, ok);
+            }, p.dev_error);
         }
     }
 
     if (c == 0) {
         if (p.init_state) {
-            const float *h0 = p.init_state + (size_t)bh * PD * ND + n;
+            const float *h0 = p.init_state + (size_t)t.bh * PD * ND + n;
 #pragma unroll
             for (int q = 0; q < PD; ++q) hp[q] = h0[q * ND];
         } else {
@@ -176,64 +210,76 @@ __device__ void lookback(const TcParams &p, int bh, int c, int warp, int lane, f
             for (int q = 0; q < PD; ++q) hp[q] = 0.f;
         }
     } else {
+        const uint32_t *fprev = p.flags + (ring0 + (c - 1) % RING) * 4 + quad;
+        uint32_t v0 = (lane == 0) ? ld_acquire_u32(fprev) : 0u;
+        v0 = __shfl_sync(0xffffffffu, v0, 0);
+        if (v0 == (((uint32_t)(c - 1) << 2) | ST_PREFIX)) {
+            ld_row64(p.pre + (ring0 + (c - 1) % RING) * (ND * PD) + row, hp);  // fast path
+        } else {
+            st_row64(p.agg + (ring0 + slot) * (ND * PD) + row, s);
+            if (lane == 0) p.lam[(ring0 + slot) * 4 + quad] = lam;
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release_u32(flag, ((uint32_t)c << 2) | ST_AGG);
 #pragma unroll
-        for (int q = 0; q < PD; ++q) aggp[q * ND] = s[q];
-        if (lane == 0) p.lam[(ring0 + slot) * 4 + warp] = lam;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) st_release_u32(flag, ((uint32_t)c << 2) | ST_AGG);
-
+            for (int q = 0; q < PD; ++q) hp[q] = 0.f;
+            float dec = 0.f;
+            for (int j = c - 1; j >= 0; --j) {
+                const int sj = j % RING;
+                const bool need_prefix = (j == c - DEPTH) || (j == 0);
+                const uint32_t v = warp_wait_flag(p.flags + (ring0 + sj) * 4 + quad, [j, need_prefix](uint32_t v) {
+                    return (int)(v >> 2) == j && ((v & 3u) == ST_PREFIX || (!need_prefix && (v & 3u) == ST_AGG));
+                }, p.dev_error);
+                const bool is_prefix = (v & 3u) == ST_PREFIX || v == 0;
+                const float fd = __expf(dec);
+                const float *src = (is_prefix ? p.pre : p.agg) + (ring0 + sj) * (ND * PD) + row;
 #pragma unroll
-        for (int q = 0; q < PD; ++q) hp[q] = 0.f;
-        float dec = 0.f;
-        for (int j = c - 1; j >= 0; --j) {
-            const int sj = j % RING;
-            const uint32_t *f = p.flags + (ring0 + sj) * 4 + warp;
-            const bool need_prefix = (j == c - DEPTH) || (j == 0);
-            const uint32_t v = warp_wait_flag(f, [j, need_prefix](uint32_t v) {
-                return (int)(v >> 2) == j && ((v & 3u) == ST_PREFIX || (!need_prefix && (v & 3u) == ST_AGG));
-            }, p.dev_error, ok);
-            const bool is_prefix = (v & 3u) == ST_PREFIX || v == 0;
-            const float fd = __expf(dec);
-            const float *src = (is_prefix ? p.pre : p.agg) + (ring0 + sj) * (PD * ND) + n;
-#pragma unroll
-            for (int q = 0; q < PD; ++q) hp[q] = fmaf(fd, __ldcg(src + q * ND), hp[q]);
-            if (is_prefix) break;
-            dec += __ldcg(p.lam + (ring0 + sj) * 4 + warp);
+                for (int q = 0; q < PD; q += 4) {
+                    const float4 f = ld_cg_f4(src + q);
+                    hp[q] = fmaf(fd, f.x, hp[q]);
+                    hp[q + 1] = fmaf(fd, f.y, hp[q + 1]);
+                    hp[q + 2] = fmaf(fd, f.z, hp[q + 2]);
+                    hp[q + 3] = fmaf(fd, f.w, hp[q + 3]);
+                }
+                if (is_prefix) break;
+                dec += __ldcg(p.lam + (ring0 + sj) * 4 + quad);
+            }
         }
     }
 
     const float el = __expf(lam);
-    const bool last = (c == p.nchunks - 1) && p.final_state;
-    float *fin = last ? p.final_state + (size_t)bh * PD * ND + n : nullptr;
+    float hc[PD];
 #pragma unroll
-    for (int q = 0; q < PD; ++q) {
-        const float hc = fmaf(el, hp[q], s[q]);
-        prep[q * ND] = hc;
-        if (last) fin[q * ND] = hc;
+    for (int q = 0; q < PD; ++q) hc[q] = fmaf(el, hp[q], s[q]);
+    st_row64(p.pre + (ring0 + slot) * (ND * PD) + row, hc);
+    if ((c == p.nchunks - 1) && p.final_state) {
+        float *fin = p.final_state + (size_t)t.bh * PD * ND + n;
+#pragma unroll
+        for (int q = 0; q < PD; ++q) fin[q * ND] = hc[q];
     }
     __threadfence();
     __syncwarp();
     if (lane == 0) st_release_u32(flag, ((uint32_t)c << 2) | ST_PREFIX);
 }
 
-__global__ void __launch_bounds__(NTH, 2)
+__global__ void __launch_bounds__(NTH, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
                        const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t *sC = sm + OFF_C, *sB = sm + OFF_B, *sX = sm + OFF_X, *sW = sm + OFF_W;
-    float *cs = reinterpret_cast<float *>(sm + OFF_MISC);
-    float *dtv = cs + QT;
-    float *bfac = dtv + QT;
-    float *wtot = bfac + QT;
+    float *cs = reinterpret_cast<float *>(sm + OFF_MISC);  // [2][128]
+    float *dtv = cs + 2 * QT;                              // [2][128]
+    float *bfac = dtv + 2 * QT;                            // [2][128]
+    float *lam_s = bfac + 2 * QT;                          // [2]
+    float *wtot = lam_s + 2;                               // [4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 4);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 5);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < 5; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], 1);
+        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -244,189 +290,92 @@ __global__ void __launch_bounds__(NTH, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lane quadrant
+    const int ntl = (blockIdx.x < p.ntiles) ? (p.ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const uint32_t sbase = smem_u32(sm);
+    int *err = p.dev_error;
 
-    const int T = p.seqlen, H = p.nheads, hpg = p.nheads / p.ngroups;
-    const uint32_t aC = smem_u32(sC), aB = smem_u32(sB), aX = smem_u32(sX), aW = smem_u32(sW);
-    uint32_t ph = 0;
-    bool ok = true;
-
-    for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x) {
-        const int c = tile / p.bH, bh = tile % p.bH;
-        const int b = bh / H, h = bh % H, g = h / hpg;
-        const int t0 = c * QT, valid = min(QT, T - t0);
-
-        if (tid == 0) bulk_wait_group_read0();  // the previous y store has read sW
-        if (!__syncthreads_and(ok)) break;      // a timed-out wait ends the CTA's work
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&bars[0], LOAD_BYTES);
-            tma_load_4d(sC, &tm_c, &bars[0], 0, g, t0, b);
-            tma_load_4d(sC + 16384, &tm_c, &bars[0], 64, g, t0, b);
-            tma_load_4d(sB, &tm_b, &bars[0], 0, g, t0, b);
-            tma_load_4d(sB + 16384, &tm_b, &bars[0], 64, g, t0, b);
-            tma_load_4d(sX, &tm_x, &bars[0], 0, h, t0, b);
-        }
-
-        // dt, dA = dt*A, inclusive cumulative sum over the chunk (row s = tid)
-        const float d = (tid < valid) ? p.dt[((size_t)b * T + t0 + tid) * H + h] : 0.f;
-        float v = d * p.A[h];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float y = __shfl_up_sync(0xffffffffu, v, o);
-            if (lane >= o) v += y;
-        }
-        if (lane == 31) wtot[warp] = v;
-        __syncthreads();
-        for (int w = 0; w < warp; ++w) v += wtot[w];
-        cs[tid] = v;
-        dtv[tid] = d;
-        __syncthreads();
-        const float lam = cs[QT - 1];
-        // exp(A_cs[r] - A_cs[s]) dt_s with r the first row of s's 32-row block
-        bfac[tid] = __expf(cs[tid & ~31] - v) * d;
-
-        if (!mbar_wait(&bars[0], ph, p.dev_error)) ok = false;
-
-        if (tid == 0) {  // G = C B^T
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t off = (k >> 2) * 16384 + (k & 3) * 32;
-                mma_ss(tmem + COL_G, smem_desc_sw128(aC + off, 16, 1024), smem_desc_sw128(aB + off, 16, 1024),
-                       IDESC_G, k > 0);
+    if (warp == 0) {
+        // ------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            for (int k = 0; k < ntl; ++k) {
+                const Tile t = decode_tile(p, k);
+                const int s = k & 1;
+                mbar_wait(&bars[B_EMPTY + s], ((k >> 1) & 1) ^ 1, err);
+                uint8_t *st = sm + s * STAGE_BYTES;
+                mbar_arrive_expect_tx(&bars[B_FULL + s], LOAD_BYTES);
+                tma_load_4d(st + OFF_C, &tm_c, &bars[B_FULL + s], 0, t.g, t.t0, t.b);
+                tma_load_4d(st + OFF_C + 16384, &tm_c, &bars[B_FULL + s], 64, t.g, t.t0, t.b);
+                tma_load_4d(st + OFF_B, &tm_b, &bars[B_FULL + s], 0, t.g, t.t0, t.b);
+                tma_load_4d(st + OFF_B + 16384, &tm_b, &bars[B_FULL + s], 64, t.g, t.t0, t.b);
+                tma_load_4d(st + OFF_X, &tm_x, &bars[B_FULL + s], 0, t.h, t.t0, t.b);
             }
-            mma_commit(&bars[1]);
         }
-
-        {  // W row s = exp(lam - A_cs[s]) dt_s x_s  (rows keep their swizzled 16-byte chunks)
-            const float w = __expf(lam - v) * d;
-            const uint4 *src = reinterpret_cast<const uint4 *>(sX + tid * 128);
-            uint4 *dst = reinterpret_cast<uint4 *>(sW + tid * 128);
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            auto issue_yo = [&](int j) {
+                const int s = j & 1;
+                const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s;
+                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aH = sbase + s * STAGE_BYTES + OFF_X;
+                mbar_wait(&bars[B_H + s], par, err);
+                tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                uint4 q = src[j];
-                uint32_t *u = reinterpret_cast<uint32_t *>(&q);
+                for (int k = 0; k < 8; ++k)
+                    mma_ss(tm + COL_S, smem_desc_sw128(aC + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
+                           smem_desc_sw128(aH + k * 2048, 8192, 1024), IDESC_YO, k > 0);
+                mma_commit(&bars[B_YO + s]);
+                mma_commit(&bars[B_EMPTY + s]);
+            };
+            for (int k = 0; k < ntl; ++k) {
+                const int s = k & 1;
+                const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
+                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aB = sbase + s * STAGE_BYTES + OFF_B;
+                const uint32_t aX = sbase + s * STAGE_BYTES + OFF_X, aW = sbase + OFF_W + s * 16384;
+                mbar_wait(&bars[B_FULL + s], par, err);
+                mbar_wait(&bars[B_FREE + s], par ^ 1, err);
+                tc_fence_after();
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    __nv_bfloat162 pr = *reinterpret_cast<__nv_bfloat162 *>(&u[e]);
-                    float2 f = __bfloat1622float2(pr);
-                    u[e] = pack_bf16x2(f.x * w, f.y * w);
+                for (int kk = 0; kk < 8; ++kk) {  // G = C B^T
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tm + COL_G, smem_desc_sw128(aC + off, 16, 1024), smem_desc_sw128(aB + off, 16, 1024),
+                           IDESC_G, kk > 0);
                 }
-                dst[j] = q;
+                mma_commit(&bars[B_G + s]);
+                mbar_wait(&bars[B_W + s], par, err);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // S = B^T W
+                    mma_ss(tm + COL_S, smem_desc_sw128(aB + kk * 2048, 16384, 1024),
+                           smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
+                mma_commit(&bars[B_S + s]);
+                mbar_wait(&bars[B_M + s], par, err);
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)  // Y = M X
+                    mma_ts(tm + COL_YD, tm + COL_G + 8 * kk, smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD,
+                           kk > 0);
+                mma_commit(&bars[B_YD + s]);
+                if (k > 0) issue_yo(k - 1);
             }
+            if (ntl > 0) issue_yo(ntl - 1);
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-
-        if (tid == 0) {  // S = B^T W (chunk state, rows n)
+    } else if (warp < STATE_W0) {
+        // ------------------------------------------------ math warpgroup
+        const int quad = warp & 3, row = quad * 32 + lane, mt = tid - MATH_W0 * 32;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        auto epilogue = [&](int j) {  // y = Y + exp(A_cs[l]) Y_off  -> TMA store
+            const Tile t = decode_tile(p, j);
+            const int s = j & 1;
+            const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s + lane_off;
+            uint8_t *sy = sm + OFF_W + s * 16384;
+            mbar_wait(&bars[B_YO + s], par, err);
             tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_ss(tmem + COL_S, smem_desc_sw128(aB + k * 2048, 16384, 1024),
-                       smem_desc_sw128(aW + k * 2048, 8192, 1024), IDESC_S, k > 0);
-            mma_commit(&bars[2]);
-        }
-
-        // M = G o L o dt (+ D on the diagonal), bf16, in place in TMEM
-        if (!mbar_wait(&bars[1], ph, p.dev_error)) ok = false;
-        tc_fence_after();
-        {
-            const int l = tid;
-            const float csl = v;
-            const float Dh = p.D ? p.D[h] : 0.f;
-#pragma unroll 1
-            for (int j = 0; j < 4; ++j) {
-                uint32_t packed[16];
-                if (j > warp) {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = 0u;
-                } else {
-                    uint32_t gr[32];
-                    tmem_ld32(trow + COL_G + 32 * j, gr);
-                    const int r = 32 * j;
-                    const bool direct = fabsf(cs[r] - cs[r + 31]) > 80.f;
-                    const float a = __expf(csl - cs[r]);
-                    float m[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int s = r + i;
-                        const float L = direct ? __expf(csl - cs[s]) * dtv[s] : a * bfac[s];
-                        float mv = (s <= l) ? __uint_as_float(gr[i]) * L : 0.f;
-                        if (s == l) mv += Dh;
-                        m[i] = mv;
-                    }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(m[2 * i], m[2 * i + 1]);
-                }
-                tmem_st16(trow + COL_G + 16 * j, packed);
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-
-        if (tid == 0) {  // Y = M X
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_ts(tmem + COL_YD, tmem + COL_G + 8 * k, smem_desc_sw128(aX + k * 2048, 8192, 1024), IDESC_YD,
-                       k > 0);
-            mma_commit(&bars[3]);
-        }
-
-        // chunk state -> look-back -> state entering the chunk
-        if (!mbar_wait(&bars[2], ph, p.dev_error)) ok = false;
-        tc_fence_after();
-        float s_reg[PD];
-        {
-            uint32_t r[32];
-            tmem_ld32(trow + COL_S, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s_reg[i] = __uint_as_float(r[i]);
-            tmem_ld32(trow + COL_S + 32, r);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) s_reg[32 + i] = __uint_as_float(r[i]);
-        }
-        float hp[PD];
-        lookback(p, bh, c, warp, lane, lam, s_reg, hp, ok);
-
-        // h_in^T as bf16 (K-major, rows p, 128-byte swizzle) over X, once M X is done
-        if (!mbar_wait(&bars[3], ph, p.dev_error)) ok = false;
-        {
-            const int n = tid;
-            const uint32_t base = (n >> 6) * 8192 + (n & 7) * 2;
-            const uint32_t chunk = (n & 63) >> 3;
-#pragma unroll
-            for (int q = 0; q < PD; ++q) {
-                const uint32_t off = base + q * 128 + ((chunk ^ (q & 7)) << 4);
-                *reinterpret_cast<__nv_bfloat16 *>(sX + off) = __float2bfloat16_rn(hp[q]);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-
-        if (tid == 0) {  // Y_off = C h_in^T
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint32_t aoff = (k >> 2) * 16384 + (k & 3) * 32;
-                const uint32_t boff = (k >> 2) * 8192 + (k & 3) * 32;
-                mma_ss(tmem + COL_S, smem_desc_sw128(aC + aoff, 16, 1024), smem_desc_sw128(aX + boff, 16, 1024),
-                       IDESC_YO, k > 0);
-            }
-            mma_commit(&bars[4]);
-        }
-        if (!mbar_wait(&bars[4], ph, p.dev_error)) ok = false;
-        tc_fence_after();
-
-        {  // y = Y + exp(A_cs[l]) Y_off -> bf16 -> y tile (rows l, 128-byte swizzle)
-            const float e = __expf(v);
+            const float e = __expf(cs[s * QT + row]);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t yd[32], yo[32];
-                tmem_ld32(trow + COL_YD + 32 * half, yd);
-                tmem_ld32(trow + COL_S + 32 * half, yo);
+                tmem_ld32(tm + COL_YD + 32 * half, yd);
+                tmem_ld32(tm + COL_S + 32 * half, yo);
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -434,24 +383,147 @@ __global__ void __launch_bounds__(NTH, 2)
                                         fmaf(e, __uint_as_float(yo[2 * i + 1]), __uint_as_float(yd[2 * i + 1])));
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int chunk = 4 * half + q;
-                    const int phys = chunk ^ (tid & 7);
-                    *reinterpret_cast<uint4 *>(sW + tid * 128 + phys * 16) =
+                    const int phys = (4 * half + q) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) =
                         make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
                 }
             }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar_sync(BAR_MATH, 128);
+            if (mt == 0) {
+                tma_store_4d(&tm_y, sy, 0, t.h, t.t0, t.b);
+                bulk_commit_group();
+            }
+            mbar_arrive(&bars[B_FREE + s]);
+        };
+        for (int k = 0; k < ntl; ++k) {
+            const Tile t = decode_tile(p, k);
+            const int s = k & 1;
+            const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
+            float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
+            uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W + s * 16384;
+            const float d = (row < t.valid) ? p.dt[((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h] : 0.f;
+            const float Ah = p.A[t.h];
+            // the stage's data is here, and (through the stage handshake) the
+            // state warpgroup is done with this set's decay values of tile k-2
+            mbar_wait(&bars[B_FULL + s], par, err);
+            if (mt == 0) bulk_wait_group_read0();  // the y store of tile k-2 has read sw
+            float v = d * Ah;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += y;
+            }
+            if (lane == 31) wtot[quad] = v;
+            named_bar_sync(BAR_MATH, 128);
+            for (int w = 0; w < quad; ++w) v += wtot[w];
+            csk[row] = v;
+            dtk[row] = d;
+            named_bar_sync(BAR_MATH, 128);
+            const float lam = csk[QT - 1];
+            if (mt == 0) lam_s[s] = lam;
+            bfk[row] = __expf(csk[row & ~31] - v) * d;
+            mbar_arrive(&bars[B_CS + s]);
+            {  // W row = exp(lam - A_cs[row]) dt x_row (swizzled 16-byte chunks keep their places)
+                const float w = __expf(lam - v) * d;
+                const uint4 *src = reinterpret_cast<const uint4 *>(sx + row * 128);
+                uint4 *dst = reinterpret_cast<uint4 *>(sw + row * 128);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint4 q = src[j];
+                    uint32_t *u = reinterpret_cast<uint32_t *>(&q);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u[e]));
+                        u[e] = pack_bf16x2(f.x * w, f.y * w);
+                    }
+                    dst[j] = q;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bars[B_W + s]);
+            named_bar_sync(BAR_MATH, 128);  // bfac of every row written
+            // M = G o L o dt (+ D on the diagonal), bf16 pairs, in place in TMEM
+            mbar_wait(&bars[B_G + s], par, err);
+            tc_fence_after();
+            {
+                const float csl = v;
+                const float Dh = p.D ? p.D[t.h] : 0.f;
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t packed[16];
+                    if (j > quad) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) packed[i] = 0u;
+                    } else {
+                        uint32_t gr[32];
+                        tmem_ld32(tm + COL_G + 32 * j, gr);
+                        const int r = 32 * j;
+                        const bool direct = fabsf(csk[r] - csk[r + 31]) > 80.f;
+                        const float a = __expf(csl - csk[r]);
+                        float m[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            const int sidx = r + i;
+                            const float L = direct ? __expf(csl - csk[sidx]) * dtk[sidx] : a * bfk[sidx];
+                            float mv = (sidx <= row) ? __uint_as_float(gr[i]) * L : 0.f;
+                            if (sidx == row) mv += Dh;
+                            m[i] = mv;
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(m[2 * i], m[2 * i + 1]);
+                    }
+                    tmem_st16(tm + COL_G + 16 * j, packed);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[B_M + s]);
+            if (k > 0) epilogue(k - 1);
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tma_store_4d(&tm_y, sW, 0, h, t0, b);
-            bulk_commit_group();
+        if (ntl > 0) epilogue(ntl - 1);
+        if (mt == 0) bulk_wait_group0();
+    } else {
+        // ----------------------------------------------- state warpgroup
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        for (int k = 0; k < ntl; ++k) {
+            const Tile t = decode_tile(p, k);
+            const int s = k & 1;
+            const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
+            mbar_wait(&bars[B_CS + s], par, err);
+            const float lam = lam_s[s];
+            mbar_wait(&bars[B_S + s], par, err);
+            tc_fence_after();
+            float sv[PD];
+            {
+                uint32_t r[32];
+                tmem_ld32(tm + COL_S, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r[i]);
+                tmem_ld32(tm + COL_S + 32, r);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r[i]);
+            }
+            float hp[PD];
+            lookback(p, t, quad, lane, lam, sv, hp);
+            // h_in^T (rows n, bf16, 128-byte swizzle) over X, once M X has read X
+            mbar_wait(&bars[B_YD + s], par, err);
+            uint8_t *sh = sm + s * STAGE_BYTES + OFF_X;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int phys = q ^ (row & 7);
+                *reinterpret_cast<uint4 *>(sh + row * 128 + phys * 16) =
+                    make_uint4(pack_bf16x2(hp[8 * q], hp[8 * q + 1]), pack_bf16x2(hp[8 * q + 2], hp[8 * q + 3]),
+                               pack_bf16x2(hp[8 * q + 4], hp[8 * q + 5]), pack_bf16x2(hp[8 * q + 6], hp[8 * q + 7]));
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_H + s]);
         }
-        ph ^= 1;
     }
 
-    if (tid == 0) bulk_wait_group0();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -578,7 +650,7 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
     p.bH = bH;
     p.dev_error = a.dev_error;
 
-    const int grid = std::min(p.ntiles, di.per_sm * di.sms);
+    const int grid = std::min(p.ntiles, di.per_sm * di.sms);  // one CTA per SM
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NTH);
