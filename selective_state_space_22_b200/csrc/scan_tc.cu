@@ -49,17 +49,17 @@ using namespace ptx;
 constexpr int QT = 128;   // tokens per tile (tcgen05 M)
 constexpr int PD = 64;    // head dim
 constexpr int ND = 128;   // state dim
-constexpr int RING = 8;   // published-state slots per sequence
+constexpr int RING = 8;   // published-state slots per sequence (chunk-parallel mode)
 constexpr int DEPTH = 2;  // look-back reads at most this many predecessors
 
-// Warp roles: 0 TMA producer, 1 MMA issuer, 2-5 "math" warpgroup (decay, W,
-// M, y), 6-9 "state" warpgroup (look-back, publication, h_in).  A warpgroup's
-// warp w reaches TMEM lanes 32*(w%4)..+31, so each covers all 128 lanes.
+// Warp roles: 0 TMA producer, 1 MMA issuer (G, S, M X), 2-5 "math" warpgroup
+// (decay, W, M, y), 6-9 "state" warpgroup (inter-chunk state, h_in, C h_in^T).
+// A warpgroup's warp w reaches TMEM lanes 32*(w%4)..+31, so each covers all 128.
 constexpr int NTH = 320;
 constexpr int MATH_W0 = 2, STATE_W0 = 6;
-constexpr uint32_t BAR_MATH = 1;  // named barrier of the math warpgroup (128 threads)
+constexpr uint32_t BAR_MATH = 1, BAR_STATE = 2;  // named barriers (128 threads each)
 
-// TMEM: two column sets of 256 (tiles alternate between them).
+// TMEM: two column sets of 256 (consecutive tiles alternate).
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M in place (bf16 pairs, 64 cols)
 constexpr uint32_t COL_YD = 128; // M X                       (64 cols)
@@ -72,8 +72,8 @@ constexpr int OFF_W = 2 * STAGE_BYTES;                  // 2 x 16 KB
 constexpr int OFF_MISC = OFF_W + 2 * 16384;
 constexpr uint32_t LOAD_BYTES = 2 * (QT * ND * 2) + QT * PD * 2;
 enum {
-    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_YD = 8, B_YO = 10,         // count 1
-    B_CS = 12, B_W = 14, B_M = 16, B_H = 18, B_FREE = 20, NBARS = 22         // count 128
+    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_YD = 8, B_YO = 10,   // count 1 (TMA / commit)
+    B_CS = 12, B_W = 14, B_M = 16, B_FREE = 18, NBARS = 20            // count 128 (warpgroup)
 };
 // misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], wtot[4], bars, tmem base
 constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
@@ -93,28 +93,44 @@ struct TcParams {
     const float *D;
     const float *init_state;
     float *final_state;
-    uint32_t *flags;  // [bH][RING][4 warps]  (chunk << 2) | status
-    float *lam;       // [bH][RING][4 warps]  log-decay of the chunk in the slot
+    uint32_t *flags;  // [bH][RING][ND]  (chunk << 2) | status, one per state row
+    float *lam;       // [bH][RING][ND]  log-decay of the chunk in the slot
     float *agg;       // [bH][RING][ND][PD]   chunk state from a zero start
     float *pre;       // [bH][RING][ND][PD]   state after the chunk
     int seqlen, nheads, ngroups, nchunks, ntiles, bH;
+    int resident;     // 1: each CTA owns whole sequences (state stays on chip)
     int *dev_error;
 };
 
+// Tile order.  Sequence-resident: CTA i takes sequences i, i+G, ... and walks
+// each one's chunks in order.  Chunk-parallel: tiles are numbered chunk-major
+// and dealt round-robin, so every wait is on a smaller tile number.
 struct Tile {
     int c, bh, b, h, g, t0, valid;
 };
 __device__ __forceinline__ Tile decode_tile(const TcParams &p, int k) {
     Tile t;
-    const int tile = blockIdx.x + k * gridDim.x;
-    t.c = tile / p.bH;
-    t.bh = tile % p.bH;
+    if (p.resident) {
+        t.c = k % p.nchunks;
+        t.bh = blockIdx.x + (k / p.nchunks) * gridDim.x;
+    } else {
+        const int tile = blockIdx.x + k * gridDim.x;
+        t.c = tile / p.bH;
+        t.bh = tile % p.bH;
+    }
     t.b = t.bh / p.nheads;
     t.h = t.bh % p.nheads;
     t.g = t.h / (p.nheads / p.ngroups);
     t.t0 = t.c * QT;
     t.valid = min(QT, p.seqlen - t.t0);
     return t;
+}
+__device__ __forceinline__ int local_tiles(const TcParams &p) {
+    if (p.resident) {
+        const int nseq = (blockIdx.x < p.bH) ? (p.bH - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+        return nseq * p.nchunks;
+    }
+    return (blockIdx.x < p.ntiles) ? (p.ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
 }
 
 __device__ __forceinline__ unsigned long long now_ns() {
@@ -142,59 +158,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// Lane 0 of a warp waits until *f satisfies `ready`; the value is broadcast
-// (0 after a timeout, which is also reported).
+// This thread waits until its own flag *f satisfies `ready` (0 after a timeout).
 template <typename Pred>
-__device__ uint32_t warp_wait_flag(const uint32_t *f, Pred ready, int *err) {
-    uint32_t v = 0;
-    if ((threadIdx.x & 31) == 0) {
+__device__ __forceinline__ uint32_t wait_flag(const uint32_t *f, Pred ready, int *err) {
+    uint32_t v = ld_acquire_u32(f);
+    if (ready(v)) return v;
+    const unsigned long long t0 = now_ns();
+    while (true) {
+        __nanosleep(32);
         v = ld_acquire_u32(f);
-        if (!ready(v)) {
-            const unsigned long long t0 = now_ns();
-            while (true) {
-                __nanosleep(32);
-                v = ld_acquire_u32(f);
-                if (ready(v)) break;
-                if (now_ns() - t0 > WAIT_NS) {
-                    report_timeout(err);
-                    v = 0;
-                    break;
-                }
-            }
+        if (ready(v)) return v;
+        if (now_ns() - t0 > WAIT_NS) {
+            report_timeout(err);
+            return 0;
         }
     }
-    return __shfl_sync(0xffffffffu, v, 0);
 }
 
-__device__ __forceinline__ void ld_row64(const float *src, float (&v)[PD]) {
-#pragma unroll
-    for (int q = 0; q < PD; q += 4) {
-        const float4 f = ld_cg_f4(src + q);
-        v[q] = f.x; v[q + 1] = f.y; v[q + 2] = f.z; v[q + 3] = f.w;
-    }
-}
-__device__ __forceinline__ void st_row64(float *dst, const float (&v)[PD]) {
-#pragma unroll
-    for (int q = 0; q < PD; q += 4) *reinterpret_cast<float4 *>(dst + q) = make_float4(v[q], v[q + 1], v[q + 2], v[q + 3]);
-}
-
-// State entering chunk c of sequence bh for this warp's 32 state rows (n = row),
-// and publication of this chunk's prefix (and, when its predecessor's prefix is
-// not there yet, first its aggregate).  s[] is S[n][:] of this thread's row;
-// hp[] receives h_in[:][n].  Slot layout [n][p]: a row is 256 contiguous bytes.
-__device__ void lookback(const TcParams &p, const Tile &t, int quad, int lane, float lam,
-                         const float (&s)[PD], float (&hp)[PD]) {
-    const int n = quad * 32 + lane;
+// Chunk-parallel mode: the state entering chunk c for this thread's state row
+// n, by a decoupled look-back that each row runs on its own (rows are
+// independent: every flag, decay and 256-byte slot row belongs to one thread,
+// and a release store orders the thread's own data before its flag).  On entry
+// h holds S[n][:] of this chunk; on exit h holds h_in[:][n] and the chunk's
+// prefix h_c = exp(lam) h_in + S has been published.
+__device__ void lookback_row(const TcParams &p, const Tile &t, int n, float lam, float (&h)[PD],
+                             float (&hin)[PD]) {
     const int c = t.c;
     const size_t ring0 = (size_t)t.bh * RING;
     const int slot = c % RING;
-    uint32_t *flag = p.flags + (ring0 + slot) * 4 + quad;
-    const size_t row = (size_t)n * PD;
+    const size_t fl = (ring0 + slot) * ND + n;  // this row's flag / lam index in the slot
+    float *prow = p.pre + fl * PD;
 
     if (c >= RING) {  // slot reuse: its last user and possible readers have published prefixes
+#pragma unroll
         for (int k = 0; k <= DEPTH; ++k) {
             const int j = c - RING + k;
-            warp_wait_flag(p.flags + (ring0 + j % RING) * 4 + quad, [j](uint32_t v) {
+            wait_flag(p.flags + (ring0 + j % RING) * ND + n, [j](uint32_t v) {
                 return (int)(v >> 2) > j || ((int)(v >> 2) == j && (v & 3u) == ST_PREFIX);
             }, p.dev_error);
         }
@@ -204,62 +203,58 @@ __device__ void lookback(const TcParams &p, const Tile &t, int quad, int lane, f
         if (p.init_state) {
             const float *h0 = p.init_state + (size_t)t.bh * PD * ND + n;
 #pragma unroll
-            for (int q = 0; q < PD; ++q) hp[q] = h0[q * ND];
+            for (int q = 0; q < PD; ++q) hin[q] = h0[q * ND];
         } else {
 #pragma unroll
-            for (int q = 0; q < PD; ++q) hp[q] = 0.f;
+            for (int q = 0; q < PD; ++q) hin[q] = 0.f;
         }
     } else {
-        const uint32_t *fprev = p.flags + (ring0 + (c - 1) % RING) * 4 + quad;
-        uint32_t v0 = (lane == 0) ? ld_acquire_u32(fprev) : 0u;
-        v0 = __shfl_sync(0xffffffffu, v0, 0);
-        if (v0 == (((uint32_t)(c - 1) << 2) | ST_PREFIX)) {
-            ld_row64(p.pre + (ring0 + (c - 1) % RING) * (ND * PD) + row, hp);  // fast path
-        } else {
-            st_row64(p.agg + (ring0 + slot) * (ND * PD) + row, s);
-            if (lane == 0) p.lam[(ring0 + slot) * 4 + quad] = lam;
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) st_release_u32(flag, ((uint32_t)c << 2) | ST_AGG);
+        const size_t fp = (ring0 + (c - 1) % RING) * ND + n;
+        const uint32_t v0 = ld_acquire_u32(p.flags + fp);
+        if (v0 == (((uint32_t)(c - 1) << 2) | ST_PREFIX)) {  // predecessor done: no aggregate needed
+            const float *src = p.pre + fp * PD;
 #pragma unroll
-            for (int q = 0; q < PD; ++q) hp[q] = 0.f;
+            for (int q = 0; q < PD; q += 4) {
+                const float4 f = ld_cg_f4(src + q);
+                hin[q] = f.x; hin[q + 1] = f.y; hin[q + 2] = f.z; hin[q + 3] = f.w;
+            }
+        } else {
+            float *arow = p.agg + fl * PD;
+#pragma unroll
+            for (int q = 0; q < PD; q += 4) *reinterpret_cast<float4 *>(arow + q) = make_float4(h[q], h[q + 1], h[q + 2], h[q + 3]);
+            p.lam[fl] = lam;
+            st_release_u32(p.flags + fl, ((uint32_t)c << 2) | ST_AGG);
+#pragma unroll
+            for (int q = 0; q < PD; ++q) hin[q] = 0.f;
             float dec = 0.f;
             for (int j = c - 1; j >= 0; --j) {
-                const int sj = j % RING;
+                const size_t fj = (ring0 + j % RING) * ND + n;
                 const bool need_prefix = (j == c - DEPTH) || (j == 0);
-                const uint32_t v = warp_wait_flag(p.flags + (ring0 + sj) * 4 + quad, [j, need_prefix](uint32_t v) {
+                const uint32_t v = wait_flag(p.flags + fj, [j, need_prefix](uint32_t v) {
                     return (int)(v >> 2) == j && ((v & 3u) == ST_PREFIX || (!need_prefix && (v & 3u) == ST_AGG));
                 }, p.dev_error);
                 const bool is_prefix = (v & 3u) == ST_PREFIX || v == 0;
                 const float fd = __expf(dec);
-                const float *src = (is_prefix ? p.pre : p.agg) + (ring0 + sj) * (ND * PD) + row;
+                const float *src = (is_prefix ? p.pre : p.agg) + fj * PD;
 #pragma unroll
                 for (int q = 0; q < PD; q += 4) {
                     const float4 f = ld_cg_f4(src + q);
-                    hp[q] = fmaf(fd, f.x, hp[q]);
-                    hp[q + 1] = fmaf(fd, f.y, hp[q + 1]);
-                    hp[q + 2] = fmaf(fd, f.z, hp[q + 2]);
-                    hp[q + 3] = fmaf(fd, f.w, hp[q + 3]);
+                    hin[q] = fmaf(fd, f.x, hin[q]);
+                    hin[q + 1] = fmaf(fd, f.y, hin[q + 1]);
+                    hin[q + 2] = fmaf(fd, f.z, hin[q + 2]);
+                    hin[q + 3] = fmaf(fd, f.w, hin[q + 3]);
                 }
                 if (is_prefix) break;
-                dec += __ldcg(p.lam + (ring0 + sj) * 4 + quad);
+                dec += __ldcg(p.lam + fj);
             }
         }
     }
-
     const float el = __expf(lam);
-    float hc[PD];
 #pragma unroll
-    for (int q = 0; q < PD; ++q) hc[q] = fmaf(el, hp[q], s[q]);
-    st_row64(p.pre + (ring0 + slot) * (ND * PD) + row, hc);
-    if ((c == p.nchunks - 1) && p.final_state) {
-        float *fin = p.final_state + (size_t)t.bh * PD * ND + n;
+    for (int q = 0; q < PD; ++q) h[q] = fmaf(el, hin[q], h[q]);
 #pragma unroll
-        for (int q = 0; q < PD; ++q) fin[q * ND] = hc[q];
-    }
-    __threadfence();
-    __syncwarp();
-    if (lane == 0) st_release_u32(flag, ((uint32_t)c << 2) | ST_PREFIX);
+    for (int q = 0; q < PD; q += 4) *reinterpret_cast<float4 *>(prow + q) = make_float4(h[q], h[q + 1], h[q + 2], h[q + 3]);
+    st_release_u32(p.flags + fl, ((uint32_t)c << 2) | ST_PREFIX);
 }
 
 __global__ void __launch_bounds__(NTH, 1)
@@ -290,7 +285,7 @@ __global__ void __launch_bounds__(NTH, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const int ntl = (blockIdx.x < p.ntiles) ? (p.ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int ntl = local_tiles(p);
     const uint32_t sbase = smem_u32(sm);
     int *err = p.dev_error;
 
@@ -311,21 +306,8 @@ __global__ void __launch_bounds__(NTH, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+        // ------------------------------------------- MMA issuer: G, S, M X
         if (lane == 0) {
-            auto issue_yo = [&](int j) {
-                const int s = j & 1;
-                const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s;
-                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aH = sbase + s * STAGE_BYTES + OFF_X;
-                mbar_wait(&bars[B_H + s], par, err);
-                tc_fence_after();
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    mma_ss(tm + COL_S, smem_desc_sw128(aC + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024),
-                           smem_desc_sw128(aH + k * 2048, 8192, 1024), IDESC_YO, k > 0);
-                mma_commit(&bars[B_YO + s]);
-                mma_commit(&bars[B_EMPTY + s]);
-            };
             for (int k = 0; k < ntl; ++k) {
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
@@ -355,9 +337,7 @@ __global__ void __launch_bounds__(NTH, 1)
                     mma_ts(tm + COL_YD, tm + COL_G + 8 * kk, smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD,
                            kk > 0);
                 mma_commit(&bars[B_YD + s]);
-                if (k > 0) issue_yo(k - 1);
             }
-            if (ntl > 0) issue_yo(ntl - 1);
         }
     } else if (warp < STATE_W0) {
         // ------------------------------------------------ math warpgroup
@@ -376,16 +356,17 @@ __global__ void __launch_bounds__(NTH, 1)
                 uint32_t yd[32], yo[32];
                 tmem_ld32(tm + COL_YD + 32 * half, yd);
                 tmem_ld32(tm + COL_S + 32 * half, yo);
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[2 * i]), __uint_as_float(yd[2 * i])),
-                                        fmaf(e, __uint_as_float(yo[2 * i + 1]), __uint_as_float(yd[2 * i + 1])));
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int e0 = 8 * q + 2 * i;
+                        pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
+                                            fmaf(e, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
+                    }
                     const int phys = (4 * half + q) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) =
-                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                 }
             }
             fence_proxy_async_smem();
@@ -405,11 +386,12 @@ __global__ void __launch_bounds__(NTH, 1)
             uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W + s * 16384;
             const float d = (row < t.valid) ? p.dt[((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h] : 0.f;
             const float Ah = p.A[t.h];
-            // the stage's data is here, and (through the stage handshake) the
-            // state warpgroup is done with this set's decay values of tile k-2
+            const float Dh = p.D ? p.D[t.h] : 0.f;
+            // The stage's data is here; through the stage handshake, the state
+            // warpgroup is also done with this buffer set's decay values of tile k-2.
             mbar_wait(&bars[B_FULL + s], par, err);
             if (mt == 0) bulk_wait_group_read0();  // the y store of tile k-2 has read sw
-            float v = d * Ah;
+            float v = d * Ah;                       // inclusive cumsum of dt*A over the chunk
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, v, o);
@@ -423,21 +405,18 @@ __global__ void __launch_bounds__(NTH, 1)
             named_bar_sync(BAR_MATH, 128);
             const float lam = csk[QT - 1];
             if (mt == 0) lam_s[s] = lam;
-            bfk[row] = __expf(csk[row & ~31] - v) * d;
+            bfk[row] = __expf(csk[row & ~31] - v) * d;  // exp(A_cs[r] - A_cs[s]) dt_s, r = s's 32-block start
             mbar_arrive(&bars[B_CS + s]);
             {  // W row = exp(lam - A_cs[row]) dt x_row (swizzled 16-byte chunks keep their places)
-                const float w = __expf(lam - v) * d;
+                const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(lam - v) * d);
                 const uint4 *src = reinterpret_cast<const uint4 *>(sx + row * 128);
                 uint4 *dst = reinterpret_cast<uint4 *>(sw + row * 128);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     uint4 q = src[j];
-                    uint32_t *u = reinterpret_cast<uint32_t *>(&q);
+                    __nv_bfloat162 *u = reinterpret_cast<__nv_bfloat162 *>(&q);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162 *>(&u[e]));
-                        u[e] = pack_bf16x2(f.x * w, f.y * w);
-                    }
+                    for (int e = 0; e < 4; ++e) u[e] = __hmul2(u[e], w2);
                     dst[j] = q;
                 }
             }
@@ -449,7 +428,6 @@ __global__ void __launch_bounds__(NTH, 1)
             tc_fence_after();
             {
                 const float csl = v;
-                const float Dh = p.D ? p.D[t.h] : 0.f;
 #pragma unroll 1
                 for (int j = 0; j < 4; ++j) {
                     uint32_t packed[16];
@@ -460,16 +438,34 @@ __global__ void __launch_bounds__(NTH, 1)
                         uint32_t gr[32];
                         tmem_ld32(tm + COL_G + 32 * j, gr);
                         const int r = 32 * j;
-                        const bool direct = fabsf(csk[r] - csk[r + 31]) > 80.f;
-                        const float a = __expf(csl - csk[r]);
+                        const int lim = (j == quad) ? lane : 31;  // causal mask on the diagonal block
+                        float L[32];
+                        if (fabsf(csk[r] - csk[r + 31]) <= 80.f) {
+                            // L[l, s] = exp(A_cs[l] - A_cs[r]) * (exp(A_cs[r] - A_cs[s]) dt_s): one exp per row
+                            const float a = __expf(csl - csk[r]);
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4) {
+                                const float4 b4 = *reinterpret_cast<const float4 *>(bfk + r + i);
+                                L[i] = a * b4.x; L[i + 1] = a * b4.y; L[i + 2] = a * b4.z; L[i + 3] = a * b4.w;
+                            }
+                        } else {  // a wide decay range in this block: one exp per element
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4) {
+                                const float4 c4 = *reinterpret_cast<const float4 *>(csk + r + i);
+                                const float4 d4 = *reinterpret_cast<const float4 *>(dtk + r + i);
+                                L[i] = __expf(fminf(csl - c4.x, 0.f)) * d4.x;
+                                L[i + 1] = __expf(fminf(csl - c4.y, 0.f)) * d4.y;
+                                L[i + 2] = __expf(fminf(csl - c4.z, 0.f)) * d4.z;
+                                L[i + 3] = __expf(fminf(csl - c4.w, 0.f)) * d4.w;
+                            }
+                        }
                         float m[32];
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            const int sidx = r + i;
-                            const float L = direct ? __expf(csl - csk[sidx]) * dtk[sidx] : a * bfk[sidx];
-                            float mv = (sidx <= row) ? __uint_as_float(gr[i]) * L : 0.f;
-                            if (sidx == row) mv += Dh;
-                            m[i] = mv;
+                        for (int i = 0; i < 32; ++i) m[i] = (i <= lim) ? __uint_as_float(gr[i]) * L[i] : 0.f;
+                        if (j == quad) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i == lane) m[i] += Dh;
                         }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(m[2 * i], m[2 * i + 1]);
@@ -486,8 +482,9 @@ __global__ void __launch_bounds__(NTH, 1)
         if (mt == 0) bulk_wait_group0();
     } else {
         // ----------------------------------------------- state warpgroup
-        const int quad = warp & 3, row = quad * 32 + lane;
+        const int quad = warp & 3, row = quad * 32 + lane, st_t = tid - STATE_W0 * 32;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        float hcar[PD];  // sequence-resident mode: the state carried from chunk to chunk (row n)
         for (int k = 0; k < ntl; ++k) {
             const Tile t = decode_tile(p, k);
             const int s = k & 1;
@@ -506,8 +503,34 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r[i]);
             }
-            float hp[PD];
-            lookback(p, t, quad, lane, lam, sv, hp);
+            float hin[PD];
+            if (p.resident) {
+                if (t.c == 0) {
+                    if (p.init_state) {
+                        const float *h0 = p.init_state + (size_t)t.bh * PD * ND + row;
+#pragma unroll
+                        for (int q = 0; q < PD; ++q) hcar[q] = h0[q * ND];
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < PD; ++q) hcar[q] = 0.f;
+                    }
+                }
+                const float el = __expf(lam);
+#pragma unroll
+                for (int q = 0; q < PD; ++q) {
+                    hin[q] = hcar[q];
+                    hcar[q] = fmaf(el, hcar[q], sv[q]);
+                }
+            } else {
+                lookback_row(p, t, row, lam, sv, hin);
+#pragma unroll
+                for (int q = 0; q < PD; ++q) hcar[q] = sv[q];
+            }
+            if (t.c == p.nchunks - 1 && p.final_state) {
+                float *fin = p.final_state + (size_t)t.bh * PD * ND + row;
+#pragma unroll
+                for (int q = 0; q < PD; ++q) fin[q * ND] = hcar[q];
+            }
             // h_in^T (rows n, bf16, 128-byte swizzle) over X, once M X has read X
             mbar_wait(&bars[B_YD + s], par, err);
             uint8_t *sh = sm + s * STAGE_BYTES + OFF_X;
@@ -515,12 +538,23 @@ __global__ void __launch_bounds__(NTH, 1)
             for (int q = 0; q < 8; ++q) {
                 const int phys = q ^ (row & 7);
                 *reinterpret_cast<uint4 *>(sh + row * 128 + phys * 16) =
-                    make_uint4(pack_bf16x2(hp[8 * q], hp[8 * q + 1]), pack_bf16x2(hp[8 * q + 2], hp[8 * q + 3]),
-                               pack_bf16x2(hp[8 * q + 4], hp[8 * q + 5]), pack_bf16x2(hp[8 * q + 6], hp[8 * q + 7]));
+                    make_uint4(pack_bf16x2(hin[8 * q], hin[8 * q + 1]), pack_bf16x2(hin[8 * q + 2], hin[8 * q + 3]),
+                               pack_bf16x2(hin[8 * q + 4], hin[8 * q + 5]), pack_bf16x2(hin[8 * q + 6], hin[8 * q + 7]));
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bars[B_H + s]);
+            named_bar_sync(BAR_STATE, 128);
+            if (st_t == 0) {  // Y_off = C h_in^T, then the stage is free
+                tc_fence_after();
+                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aH = sbase + s * STAGE_BYTES + OFF_X;
+                const uint32_t tmo = tmem + 256 * s;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ss(tmo + COL_S, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                           smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
+                mma_commit(&bars[B_YO + s]);
+                mma_commit(&bars[B_EMPTY + s]);
+            }
         }
     }
 
@@ -566,11 +600,11 @@ struct TcWs {
 TcWs carve_tc(void *ws, int bH) {
     TcWs w;
     char *p = static_cast<char *>(ws);
-    w.flag_bytes = (size_t)bH * RING * 4 * sizeof(uint32_t);
+    w.flag_bytes = (size_t)bH * RING * ND * sizeof(uint32_t);
     w.flags = reinterpret_cast<uint32_t *>(p);
     p += align_up(w.flag_bytes, 256);
     w.lam = reinterpret_cast<float *>(p);
-    p += align_up((size_t)bH * RING * 4 * sizeof(float), 256);
+    p += align_up((size_t)bH * RING * ND * sizeof(float), 256);
     w.agg = reinterpret_cast<float *>(p);
     p += align_up((size_t)bH * RING * PD * ND * sizeof(float), 256);
     w.pre = reinterpret_cast<float *>(p);
@@ -592,7 +626,7 @@ bool tc_supported(int headdim, int dstate, int seqlen) {
 
 size_t tc_workspace_bytes(int batch, int nheads) {
     const size_t bH = (size_t)batch * nheads;
-    return align_up(bH * RING * 4 * sizeof(uint32_t), 256) + align_up(bH * RING * 4 * sizeof(float), 256) +
+    return align_up(bH * RING * ND * sizeof(uint32_t), 256) + align_up(bH * RING * ND * sizeof(float), 256) +
            2 * align_up(bH * RING * PD * ND * sizeof(float), 256);
 }
 
@@ -629,8 +663,11 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
 
     const int bH = a.batch * a.nheads;
     TcWs w = carve_tc(ws, bH);
-    // The look-back protocol starts from empty slot flags.
-    if ((e = cudaMemsetAsync(w.flags, 0, w.flag_bytes, st)) != cudaSuccess) return e;
+    // With at least ~3/4 as many sequences as SMs, each CTA owns whole sequences
+    // and keeps the state on chip; otherwise chunks are spread over all SMs and
+    // the state passes through the look-back slots, which start empty.
+    const bool resident = 4 * bH >= 3 * di.sms;
+    if (!resident && (e = cudaMemsetAsync(w.flags, 0, w.flag_bytes, st)) != cudaSuccess) return e;
 
     TcParams p;
     p.dt = a.dt;
@@ -648,9 +685,10 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
     p.nchunks = (a.seqlen + QT - 1) / QT;
     p.ntiles = p.nchunks * bH;
     p.bH = bH;
+    p.resident = resident ? 1 : 0;
     p.dev_error = a.dev_error;
 
-    const int grid = std::min(p.ntiles, di.per_sm * di.sms);  // one CTA per SM
+    const int grid = std::min(resident ? bH : p.ntiles, di.per_sm * di.sms);  // one CTA per SM
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NTH);
