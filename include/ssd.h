@@ -162,6 +162,42 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
  */
 ssd_status ssd_get_device_status(void *stream);
 
+/*
+ * Size of the fixed scratch array behind ssd_scan_fwd_noalloc (16 MiB).  Every
+ * GPU that loads this library holds it until the process exits.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * ssd_scan_fwd_noalloc -- the real scan for callers that cannot allocate.
+ *
+ * (The pages have no counterpart to this entry point.)  Some callers cannot call
+ * cudaMalloc or hand over a workspace: a plugin inside a host application that
+ * owns all device memory, a path where an allocation's latency or implicit
+ * synchronisation is not acceptable.  This variant takes the same arguments as
+ * ssd_scan_fwd minus the workspace, and keeps its scratch in a fixed device
+ * array of SSD_NOALLOC_SCRATCH_BYTES inside the library.  It allocates and frees
+ * nothing, ever.
+ *
+ *  - It runs the float32 CUDA-core scan (for bf16 or float32 io).  Sizes whose
+ *    scratch exceeds SSD_NOALLOC_SCRATCH_BYTES are rejected with
+ *    SSD_ERR_WORKSPACE before anything is launched; the scratch grows with
+ *    batch * nheads * ceil(seqlen / chunk_size) * (headdim * dstate * 4 +
+ *    chunk_size * 8) bytes.  batch and seqlen must be > 0.
+ *  - The first call on a device looks up the array's device address (once, with
+ *    that device current); make that first call before any stream capture.
+ *  - All calls share the one array, and each call overwrites it: calls whose
+ *    work can overlap on the GPU (other streams, other host threads) race and
+ *    give wrong results.  Serialise them.
+ *  - Errors are reported by the return status and ssd_last_error().
+ */
+ssd_status ssd_scan_fwd_noalloc(const void *x, const float *dt, const float *A,
+                                const void *B, const void *C, const float *D,
+                                const float *init_state, float *final_state, void *y,
+                                ssd_dtype io_dtype, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate, int chunk_size,
+                                void *stream);
+
 /* Message for the last non-OK status returned on the calling host thread. */
 const char *ssd_last_error(void);
 

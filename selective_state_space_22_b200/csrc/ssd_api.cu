@@ -197,6 +197,10 @@ bool valid_dtype(ssd_dtype d) { return d == SSD_F32 || d == SSD_BF16; }
 
 }  // namespace
 
+namespace ssd {
+void set_last_error(const char *msg) { g_last_error = msg; }
+}  // namespace ssd
+
 extern "C" {
 
 size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,

@@ -86,6 +86,9 @@ cudaError_t launch_state_update(float *state, const void *x, const float *dt, co
 cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_state,
                                       size_t nfloats, cudaStream_t st);
 
+// Sets the message ssd_last_error() returns on this host thread.
+void set_last_error(const char *msg);
+
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 }  // namespace ssd
