@@ -11,28 +11,30 @@
 //   M    = G o L o dt (+ D on the diagonal),  L[l,s] = exp(A_cs[l] - A_cs[s]), s <= l,
 //          rewritten in place in TMEM as bf16                     (CUDA cores)
 //   S    = B^T (exp(A_cs[last] - A_cs[s]) dt_s x_s)               (tcgen05: chunk state)
-//   Y    = M X                            (D x enters through M's diagonal)
-//   h_in = the state entering the chunk;   h_out = exp(A_cs[last]) h_in + S
-//   y    = Y + exp(A_cs[l]) C h_in^T                              (tcgen05)
+//   y    = M X + (diag(exp(A_cs)) C) h_in^T                       (tcgen05, one accumulator)
+//   h_out = exp(A_cs[last]) h_in + S
 //
-// Operands reach shared memory by TMA (128-byte swizzle, zero fill past the end
-// of the sequence) and y leaves by a TMA store, which clips the ragged tail.
+// D x enters through M's diagonal, and the row factor exp(A_cs[l]) of the
+// off-diagonal term is applied to C in shared memory once G has read it, so both
+// products of y accumulate into the same TMEM columns.  Operands reach shared
+// memory by TMA (128-byte swizzle, zero fill past the end of the sequence) and y
+// leaves by a TMA store, which clips the ragged tail.
 //
 // Inter-chunk state passing.  The pages carry chunk c's end state into a later
 // chunk z with exp(CD[z-1] - CD[c]) (a strict lower-triangular "decay_chunk"
 // product).  Here the same quantity is a running state: h_out of one chunk is
 // h_in of the next, updated in registers by the CTA that owns the sequence, so
-// no state leaves the chip between chunks.  When there are fewer sequences than
-// SMs, each sequence is cut into R runs of consecutive chunks and run r gets its
-// own CTA.  That CTA first streams the chunks before its run through a
-// state-only pass (W and the S MMA; no G, M or Y) to obtain its entering state,
-// then scans its run in full.  CTAs never wait for one another, and the result
-// does not depend on timing.
+// no state leaves the chip between chunks, and h_in of a chunk is ready before
+// its data arrives.  When there are fewer sequences than SMs, each sequence is
+// cut into R runs of consecutive chunks and run r gets its own CTA.  That CTA
+// first streams the chunks before its run through a state-only pass (W and the
+// S MMA; no G, M or y) to obtain its entering state, then scans its run in full.
+// CTAs never wait for one another, and the result does not depend on timing.
 //
-// Warp roles (10 warps): 0 TMA producer; 1 MMA issuer (G, S, M X); 2-5 "math"
-// warpgroup (decay, W, M); 6-9 "state" warpgroup (state update, h_in^T, the
-// C h_in^T MMA, the y epilogue).  Two input stages and two TMEM column sets let
-// consecutive tiles overlap.
+// Warp roles (10 warps): 0 TMA producer; 1 MMA issuer; 2-5 "math" warpgroup
+// (decay, W, the first half of M, the scaled C); 6-9 "state" warpgroup (the
+// second half of M, state update, h_in^T, the y epilogue).  Two input stages and two TMEM column sets let consecutive tiles
+// overlap.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -52,27 +54,29 @@ constexpr int ND = 128;  // state dim
 constexpr int MAX_RUNS = 16;
 
 constexpr int NTH = 320;
-constexpr int STATE_W0 = 6;  // warps 2-5 are the math warpgroup
+constexpr int STATE_W0 = 6;  // warps 2-5 are the math warpgroup, 6-9 the state warpgroup
 constexpr uint32_t BAR_MATH = 1, BAR_STATE = 2;  // named barriers (128 threads each)
 
 // TMEM: two column sets of 256 (consecutive tiles alternate).
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M in place (bf16 pairs, 64 cols)
-constexpr uint32_t COL_YD = 128; // M X                       (64 cols)
-constexpr uint32_t COL_S = 192;  // chunk state, then C h^T   (64 cols)
+constexpr uint32_t COL_Y = 128;  // y accumulator (64 cols)
+constexpr uint32_t COL_S = 192;  // chunk state (64 cols)
 
-// Shared memory: two input stages {C, B, X} and two W buffers.  Within a stage,
-// X later holds h_in^T (once M X has read X) and C the y tile (once C h^T has
-// read C).
+// Shared memory: two input stages {C, B, X}; one W, one h_in^T and one y buffer.
 constexpr int STAGE_BYTES = 81920;
 constexpr int OFF_C = 0, OFF_B = 32768, OFF_X = 65536;
 constexpr int OFF_W = 2 * STAGE_BYTES;
-constexpr int OFF_MISC = OFF_W + 2 * 16384;
+constexpr int OFF_H = OFF_W + 16384;
+constexpr int OFF_Y = OFF_H + 16384;
+constexpr int OFF_MISC = OFF_Y + 16384;
 constexpr uint32_t LOAD_FULL = 2 * (QT * ND * 2) + QT * PD * 2;  // C, B, X
 constexpr uint32_t LOAD_STATE = QT * ND * 2 + QT * PD * 2;       // B, X
 enum {
-    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_YD = 8, B_YO = 10,   // count 1 (TMA / commit / elected)
-    B_CS = 12, B_W = 14, B_M = 16, B_FREE = 18, NBARS = 20            // count 128 (a warpgroup)
+    // count 1 (TMA bytes or an MMA commit)
+    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8,
+    // count 128 (a whole warpgroup arrives; B_M: both warpgroups, 256)
+    B_CS = 10, B_W = 12, B_M = 14, B_C = 16, B_H = 18, B_FREE = 20, NBARS = 22
 };
 // misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], wtot[4], bars, tmem base
 constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
@@ -81,7 +85,7 @@ constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 1, 1);    // B^T (MN-major) x W (MN-major)
 constexpr uint32_t IDESC_YD = idesc_bf16_f32(128, 64, 0, 1);   // M (TMEM) x X (MN-major)
-constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C (K-major) x h^T (MN-major)
+constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C' (K-major) x h^T (MN-major)
 
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on every wait
 
@@ -155,43 +159,147 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-// M for one 32-column block j of this thread's row (G block in gr): the causal
-// mask on the diagonal block, D on the diagonal.
-__device__ __forceinline__ void m_block(const uint32_t (&gr)[32], int j, int quad, int lane, float csl,
-                                        const float *csk, const float *dtk, const float *bfk, float Dh,
-                                        uint32_t (&packed)[16]) {
+// Decay factors of one 32-column block j for this thread's row l:
+// L[s] = exp(A_cs[l] - A_cs[s]) dt_s, as pairs.
+__device__ __forceinline__ void block_decay(int j, float csl, const float *csk, const float *dtk, const float *bfk,
+                                           float2 (&L)[16]) {
     const int r = 32 * j;
-    const int lim = (j == quad) ? lane : 31;
-    float L[32];
     if (fabsf(csk[r] - csk[r + 31]) <= 80.f) {
-        // L[l, s] = exp(A_cs[l] - A_cs[r]) * (exp(A_cs[r] - A_cs[s]) dt_s): one exp per row
+        // exp(A_cs[l] - A_cs[r]) * (exp(A_cs[r] - A_cs[s]) dt_s): one exp per row
         const float a = __expf(csl - csk[r]);
+        const float2 a2 = make_float2(a, a);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(bfk + r + i);
-            L[i] = a * b4.x; L[i + 1] = a * b4.y; L[i + 2] = a * b4.z; L[i + 3] = a * b4.w;
+        for (int i = 0; i < 8; ++i) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(bfk + r + 4 * i);
+            L[2 * i] = fmul2(a2, make_float2(b4.x, b4.y));
+            L[2 * i + 1] = fmul2(a2, make_float2(b4.z, b4.w));
         }
     } else {  // a wide decay range inside this block: one exp per element
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            const float4 c4 = *reinterpret_cast<const float4 *>(csk + r + i);
-            const float4 d4 = *reinterpret_cast<const float4 *>(dtk + r + i);
-            L[i] = __expf(fminf(csl - c4.x, 0.f)) * d4.x;
-            L[i + 1] = __expf(fminf(csl - c4.y, 0.f)) * d4.y;
-            L[i + 2] = __expf(fminf(csl - c4.z, 0.f)) * d4.z;
-            L[i + 3] = __expf(fminf(csl - c4.w, 0.f)) * d4.w;
+        for (int i = 0; i < 8; ++i) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(csk + r + 4 * i);
+            const float4 d4 = *reinterpret_cast<const float4 *>(dtk + r + 4 * i);
+            L[2 * i] = make_float2(__expf(fminf(csl - c4.x, 0.f)) * d4.x, __expf(fminf(csl - c4.y, 0.f)) * d4.y);
+            L[2 * i + 1] = make_float2(__expf(fminf(csl - c4.z, 0.f)) * d4.z, __expf(fminf(csl - c4.w, 0.f)) * d4.w);
         }
     }
-    float m[32];
+}
+
+// M = G o L for one block (G block in gr), bf16 pairs; on the diagonal block
+// only s <= l is kept and D is added at s == l.
+__device__ __forceinline__ void block_apply(const uint32_t (&gr)[32], const float2 (&L)[16], bool diag, int lane,
+                                            float Dh, uint32_t (&packed)[16]) {
+    if (!diag) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) m[i] = (i <= lim) ? __uint_as_float(gr[i]) * L[i] : 0.f;
-    if (j == quad) {
+        for (int i = 0; i < 16; ++i) {
+            const float2 m = fmul2(make_float2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1])), L[i]);
+            packed[i] = pack_bf16x2(m.x, m.y);
+        }
+    } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            if (i == lane) m[i] += Dh;
+        for (int i = 0; i < 16; ++i) {
+            float2 m = fmul2(make_float2(__uint_as_float(gr[2 * i]), __uint_as_float(gr[2 * i + 1])), L[i]);
+            m.x = (2 * i < lane) ? m.x : (2 * i == lane ? m.x + Dh : 0.f);
+            m.y = (2 * i + 1 < lane) ? m.y : (2 * i + 1 == lane ? m.y + Dh : 0.f);
+            packed[i] = pack_bf16x2(m.x, m.y);
+        }
+    }
+}
+
+// One M block: TMEM load of G, decay factors computed while it is in flight,
+// then M (bf16 pairs, 16 columns) written over G columns this block's own
+// warpgroup has already read: blocks 0, 1 (math warpgroup) to columns 0-31,
+// blocks 2, 3 (state warpgroup) to columns 64-95.  The two warpgroups thus never
+// write a column the other still reads.
+__host__ __device__ constexpr uint32_t m_col(int j) { return 16 * j + (j >= 2 ? 32 : 0); }
+__device__ __forceinline__ void m_block(uint32_t tm, int j, int quad, int lane, float csl, const float *csk,
+                                        const float *dtk, const float *bfk, float Dh) {
+    uint32_t pk[16];
+    if (j > quad) {  // above the diagonal
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = 0u;
+    } else {
+        uint32_t g[32];
+        float2 L[16];
+        tmem_ld32_nowait(tm + 32 * j, g);
+        block_decay(j, csl, csk, dtk, bfk, L);
+        tmem_wait_ld(g);
+        block_apply(g, L, j == quad, lane, Dh, pk);
+    }
+    tmem_st16(tm + m_col(j), pk);
+}
+
+// Row scaling of a 128-byte swizzled shared-memory row (eight 16-byte chunks),
+// src -> dst (may be the same row).  The factor is the same for the whole row,
+// so the chunks are visited as j ^ key (key = row % 8): the eight rows a
+// quarter-warp touches then fall on eight different bank groups.
+__device__ __forceinline__ void scale_row(const uint8_t *src, uint8_t *dst, int key, __nv_bfloat162 f) {
+    uint4 q[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) q[j] = reinterpret_cast<const uint4 *>(src)[j ^ key];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        __nv_bfloat162 *u = reinterpret_cast<__nv_bfloat162 *>(&q[j]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) u[e] = __hmul2(u[e], f);
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(m[2 * i], m[2 * i + 1]);
+    for (int j = 0; j < 8; ++j) reinterpret_cast<uint4 *>(dst)[j ^ key] = q[j];
+}
+
+// The same M block in two 16-column halves (fewer live registers, for the
+// warpgroup that also carries the state).
+__device__ __forceinline__ void m_block_halves(uint32_t tm, int j, int quad, int lane, float csl, const float *csk,
+                                               const float *dtk, const float *bfk, float Dh) {
+    const uint32_t dst = tm + m_col(j);
+    if (j > quad) {
+        uint32_t z[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) z[i] = 0u;
+        tmem_st8(dst, z);
+        tmem_st8(dst + 8, z);
+        return;
+    }
+    const int r = 32 * j;
+    const bool direct = fabsf(csk[r] - csk[r + 31]) > 80.f;
+    const float a = __expf(csl - csk[r]);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint32_t g[16];
+        tmem_ld16_nowait(tm + r + 16 * half, g);
+        float2 L[8];
+        const int c0 = r + 16 * half;
+        if (!direct) {
+            const float2 a2 = make_float2(a, a);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(bfk + c0 + 4 * i);
+                L[2 * i] = fmul2(a2, make_float2(b4.x, b4.y));
+                L[2 * i + 1] = fmul2(a2, make_float2(b4.z, b4.w));
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 c4 = *reinterpret_cast<const float4 *>(csk + c0 + 4 * i);
+                const float4 d4 = *reinterpret_cast<const float4 *>(dtk + c0 + 4 * i);
+                L[2 * i] = make_float2(__expf(fminf(csl - c4.x, 0.f)) * d4.x, __expf(fminf(csl - c4.y, 0.f)) * d4.y);
+                L[2 * i + 1] = make_float2(__expf(fminf(csl - c4.z, 0.f)) * d4.z, __expf(fminf(csl - c4.w, 0.f)) * d4.w);
+            }
+        }
+        tmem_wait_ld16(g);
+        uint32_t pk[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float2 m = fmul2(make_float2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1])), L[i]);
+            if (j == quad) {
+                const int s0 = 16 * half + 2 * i;
+                m.x = (s0 < lane) ? m.x : (s0 == lane ? m.x + Dh : 0.f);
+                m.y = (s0 + 1 < lane) ? m.y : (s0 + 1 == lane ? m.y + Dh : 0.f);
+            }
+            pk[i] = pack_bf16x2(m.x, m.y);
+        }
+        tmem_st8(dst + 8 * half, pk);
+    }
 }
 
 __global__ void __launch_bounds__(NTH, 1)
@@ -211,7 +319,7 @@ __global__ void __launch_bounds__(NTH, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], 1);
-        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
+        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], (i == B_M || i == B_M + 1) ? 256 : 128);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -246,14 +354,15 @@ __global__ void __launch_bounds__(NTH, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------- MMA issuer: G, S, M X
+        // ------------------------------------------------------- MMA issuer
         if (lane == 0) {
+            const uint32_t aW = sbase + OFF_W, aH = sbase + OFF_H;
             for (int k = 0; k < ntl; ++k) {
                 const bool so = decode_tile(p, k).state_only;
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aB = sbase + s * STAGE_BYTES + OFF_B;
-                const uint32_t aX = sbase + s * STAGE_BYTES + OFF_X, aW = sbase + OFF_W + s * 16384;
+                const uint32_t aX = sbase + s * STAGE_BYTES + OFF_X;
                 mbar_wait(&bars[B_FULL + s], par, err);
                 mbar_wait(&bars[B_FREE + s], par ^ 1, err);
                 tc_fence_after();
@@ -273,15 +382,25 @@ __global__ void __launch_bounds__(NTH, 1)
                     mma_ss(tm + COL_S, smem_desc_sw128(aB + kk * 2048, 16384, 1024),
                            smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
                 mma_commit(&bars[B_S + s]);
+                mbar_wait(&bars[B_C + s], par, err);
+                mbar_wait(&bars[B_H + s], par, err);
+                tc_fence_after();
+                if (!so) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)  // y = C' h_in^T
+                        mma_ss(tm + COL_Y, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                               smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
+                }
                 mbar_wait(&bars[B_M + s], par, err);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // Y = M X
-                        mma_ts(tm + COL_YD, tm + COL_G + 8 * kk, smem_desc_sw128(aX + kk * 2048, 8192, 1024),
-                               IDESC_YD, kk > 0);
+                    for (int kk = 0; kk < 8; ++kk)  // y += M X
+                        mma_ts(tm + COL_Y, tm + COL_G + m_col(kk >> 1) + 8 * (kk & 1),
+                               smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD, 1);
                 }
-                mma_commit(&bars[B_YD + s]);
+                mma_commit(&bars[B_Y + s]);
+                mma_commit(&bars[B_EMPTY + s]);
             }
         }
     } else if (warp < STATE_W0) {
@@ -300,7 +419,7 @@ __global__ void __launch_bounds__(NTH, 1)
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
             float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
-            uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W + s * 16384;
+            uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W;
             const float Ah = p.A[t.h];
             const float Dh = p.D ? p.D[t.h] : 0.f;
             // The stage's data is here; through the stage handshake, the state
@@ -322,78 +441,39 @@ __global__ void __launch_bounds__(NTH, 1)
             if (row == 0) lam_s[s] = lam;
             bfk[row] = __expf(csk[row & ~31] - v) * d;  // exp(A_cs[r] - A_cs[s]) dt_s, r = s's 32-block start
             mbar_arrive(&bars[B_CS + s]);
-            {  // W row = exp(lam - A_cs[row]) dt x_row (swizzled 16-byte chunks keep their places)
-                const __nv_bfloat162 w2 = __float2bfloat162_rn(__expf(lam - v) * d);
-                const uint4 *src = reinterpret_cast<const uint4 *>(sx + row * 128);
-                uint4 *dst = reinterpret_cast<uint4 *>(sw + row * 128);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    uint4 q = src[j];
-                    __nv_bfloat162 *u = reinterpret_cast<__nv_bfloat162 *>(&q);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) u[e] = __hmul2(u[e], w2);
-                    dst[j] = q;
-                }
-            }
+            // W (one buffer): the previous tile's S must have read it
+            if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
+            // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk places)
+            scale_row(sx + row * 128, sw + row * 128, row & 7, __float2bfloat162_rn(__expf(lam - v) * d));
             fence_proxy_async_smem();
             mbar_arrive(&bars[B_W + s]);
-            // Every role waits on every phase of every barrier it watches, state-only
-            // tiles included, so no waiter ever runs a phase ahead of a barrier.
-            mbar_wait(&bars[B_G + s], par, err);
-            if (t.state_only) {  // no M for a state-only tile
-                mbar_arrive(&bars[B_M + s]);
-                continue;
-            }
             named_bar_sync(BAR_MATH, 128);  // bfac of every row written
-            // M = G o L o dt (+ D on the diagonal), bf16 pairs, in place in TMEM.
-            // Blocks above the diagonal are zero; the others load two at a time.
+            mbar_wait(&bars[B_G + s], par, err);
             tc_fence_after();
-            {
-                uint32_t pk[16];
-                uint32_t g0[32], g1[32];
-                if (quad >= 1) {
-                    tmem_ld32x2(tm + COL_G, tm + COL_G + 32, g0, g1);
-                    m_block(g0, 0, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G, pk);
-                    m_block(g1, 1, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G + 16, pk);
-                } else {
-                    tmem_ld32(tm + COL_G, g0);
-                    m_block(g0, 0, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G, pk);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                    tmem_st16(tm + COL_G + 16, pk);
-                }
-                if (quad == 3) {
-                    tmem_ld32x2(tm + COL_G + 64, tm + COL_G + 96, g0, g1);
-                    m_block(g0, 2, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G + 32, pk);
-                    m_block(g1, 3, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G + 48, pk);
-                } else if (quad == 2) {
-                    tmem_ld32(tm + COL_G + 64, g0);
-                    m_block(g0, 2, quad, lane, v, csk, dtk, bfk, Dh, pk);
-                    tmem_st16(tm + COL_G + 32, pk);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                    tmem_st16(tm + COL_G + 48, pk);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                    tmem_st16(tm + COL_G + 32, pk);
-                    tmem_st16(tm + COL_G + 48, pk);
-                }
+            if (!t.state_only) {
+                // M = G o L o dt (+ D on the diagonal): this warpgroup builds column
+                // blocks 0 and 1 (s < 64), the state warpgroup blocks 2 and 3.
+                m_block(tm + COL_G, 0, quad, lane, v, csk, dtk, bfk, Dh);
+                m_block(tm + COL_G, 1, quad, lane, v, csk, dtk, bfk, Dh);
                 tmem_wait_st();
             }
             tc_fence_before();
             mbar_arrive(&bars[B_M + s]);
+            if (!t.state_only) {  // C' row l = exp(A_cs[l]) C row l, in place (G has read C)
+                uint8_t *sc = sm + s * STAGE_BYTES + OFF_C;
+                const __nv_bfloat162 e2 = __float2bfloat162_rn(__expf(v));
+                scale_row(sc + row * 128, sc + row * 128, row & 7, e2);
+                scale_row(sc + 16384 + row * 128, sc + 16384 + row * 128, row & 7, e2);
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(&bars[B_C + s]);
         }
     } else {
         // ----------------------------------------------- state warpgroup
         const int quad = warp & 3, row = quad * 32 + lane;
         const bool elected = (tid == STATE_W0 * 32);
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        uint8_t *sh = sm + OFF_H, *sy = sm + OFF_Y;
         float h[PD];  // the state carried from chunk to chunk: h[p] for state row n = row
         for (int k = 0; k < ntl; ++k) {
             const Tile t = decode_tile(p, k);
@@ -409,91 +489,77 @@ __global__ void __launch_bounds__(NTH, 1)
                     for (int q = 0; q < PD; ++q) h[q] = 0.f;
                 }
             }
+            // h_in^T of this tile (rows n, bf16, 128-byte swizzle).  The previous
+            // tile's C' h^T product has read the buffer: its B_Y was waited for.
+            if (!t.state_only) {
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int phys = q ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(sh + row * 128 + phys * 16) =
+                        make_uint4(pack_bf16x2(h[8 * q], h[8 * q + 1]), pack_bf16x2(h[8 * q + 2], h[8 * q + 3]),
+                                   pack_bf16x2(h[8 * q + 4], h[8 * q + 5]), pack_bf16x2(h[8 * q + 6], h[8 * q + 7]));
+                }
+                fence_proxy_async_smem();
+            }
+            mbar_arrive(&bars[B_H + s]);
             mbar_wait(&bars[B_CS + s], par, err);
             const float lam = lam_s[s];
-            mbar_wait(&bars[B_S + s], par, err);
-            // M X has read X once B_YD completes; X then takes h_in^T.
-            mbar_wait(&bars[B_YD + s], par, err);
+            mbar_wait(&bars[B_G + s], par, err);
             tc_fence_after();
-            {  // h_in^T (rows n, bf16, 128-byte swizzle) and h_out = exp(lam) h_in + S, 32 columns at a time
-                uint8_t *sh = sm + s * STAGE_BYTES + OFF_X;
+            if (!t.state_only) {  // M column blocks 2 and 3
+                const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
+                const float Dh = p.D ? p.D[t.h] : 0.f;
+                m_block_halves(tm + COL_G, 2, quad, lane, csk[row], csk, dtk, bfk, Dh);
+                m_block_halves(tm + COL_G, 3, quad, lane, csk[row], csk, dtk, bfk, Dh);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[B_M + s]);
+            mbar_wait(&bars[B_S + s], par, err);
+            tc_fence_after();
+            {  // h_out = exp(lam) h_in + S, 32 columns at a time
                 const float el = __expf(lam);
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t r[32];
                     tmem_ld32(tm + COL_S + 32 * half, r);
-                    if (!t.state_only) {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int b0 = 32 * half + 8 * q;
-                            const int phys = (4 * half + q) ^ (row & 7);
-                            *reinterpret_cast<uint4 *>(sh + row * 128 + phys * 16) =
-                                make_uint4(pack_bf16x2(h[b0], h[b0 + 1]), pack_bf16x2(h[b0 + 2], h[b0 + 3]),
-                                           pack_bf16x2(h[b0 + 4], h[b0 + 5]), pack_bf16x2(h[b0 + 6], h[b0 + 7]));
-                        }
-                    }
 #pragma unroll
                     for (int q = 0; q < 32; ++q) h[32 * half + q] = fmaf(el, h[32 * half + q], __uint_as_float(r[q]));
                 }
-            }
-            if (t.state_only) {  // no C h^T and no y: release the TMEM set and the stage
-                tc_fence_before();
-                if (elected) mbar_arrive(&bars[B_YO + s]);
-                mbar_wait(&bars[B_YO + s], par, err);
-                mbar_arrive(&bars[B_FREE + s]);
-                if (elected) mbar_arrive(&bars[B_EMPTY + s]);
-                continue;
             }
             if (t.c == p.nchunks - 1 && p.final_state) {
                 float *fin = p.final_state + (size_t)t.bh * PD * ND + row;
 #pragma unroll
                 for (int q = 0; q < PD; ++q) fin[q * ND] = h[q];
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            named_bar_sync(BAR_STATE, 128);
-            const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aH = sbase + s * STAGE_BYTES + OFF_X;
-            if (elected) {  // Y_off = C h_in^T
-                tc_fence_after();
-                const uint32_t tmo = tmem + 256 * s;
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ss(tmo + COL_S, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                           smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
-                mma_commit(&bars[B_YO + s]);
-            }
-            // y = Y + exp(A_cs[l]) Y_off -> bf16 -> y tile over C -> TMA store
-            mbar_wait(&bars[B_YO + s], par, err);
+            mbar_wait(&bars[B_Y + s], par, err);
             tc_fence_after();
-            uint8_t *sy = sm + s * STAGE_BYTES + OFF_C;
-            const float e = __expf(cs[s * QT + row]);
+            if (!t.state_only) {  // y tile: accumulator -> bf16 -> y buffer -> TMA store
+                if (elected) bulk_wait_group_read0();  // the previous y store has read the buffer
+                named_bar_sync(BAR_STATE, 128);
+                uint32_t yv[32], yw[32];
+                tmem_ld32x2(tm + COL_Y, tm + COL_Y + 32, yv, yw);
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t yd[32], yo[32];
-                tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_S + 32 * half, yd, yo);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int e0 = 8 * q + 2 * i;
-                        pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
-                                            fmaf(e, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
-                    }
-                    const int phys = (4 * half + q) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                for (int q = 0; q < 8; ++q) {
+                    const uint32_t *src = (q < 4) ? &yv[8 * q] : &yw[8 * (q - 4)];
+                    const int phys = q ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) = make_uint4(
+                        pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+                        pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+                        pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+                        pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
                 }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                named_bar_sync(BAR_STATE, 128);
+                if (elected) {
+                    tma_store_4d(&tm_y, sy, 0, t.h, t.t0, t.b);
+                    bulk_commit_group();
+                }
+            } else {
+                tc_fence_before();
             }
-            fence_proxy_async_smem();
-            tc_fence_before();
             mbar_arrive(&bars[B_FREE + s]);
-            named_bar_sync(BAR_STATE, 128);
-            if (elected) {
-                tma_store_4d(&tm_y, sy, 0, t.h, t.t0, t.b);
-                bulk_commit_group();
-                bulk_wait_group_read0();  // the y tile has left the stage
-                mbar_arrive(&bars[B_EMPTY + s]);
-            }
         }
         if (elected) bulk_wait_group0();
     }
