@@ -58,12 +58,16 @@ typedef enum {
     SSD_BF16 = 1   /* bfloat16 */
 } ssd_dtype;
 
+/* Returned by ssd_scan_workspace_size for sizes that no scan accepts. */
+#define SSD_WORKSPACE_INVALID ((size_t)-1)
+
 /*
- * Workspace bytes that ssd_scan_fwd / ssd_scan_fwd_complex need for these sizes.
- * Returns 0 when the sizes are invalid.  The workspace needs no initialisation:
- * each call clears, on its stream, whatever it needs cleared.  One workspace may
- * not be used by two calls that can run at the same time (different streams):
- * they would race.
+ * Workspace bytes that ssd_scan_fwd / ssd_scan_fwd_complex need for these sizes:
+ * 0 when the selected kernel needs none (then the workspace argument may be
+ * NULL), SSD_WORKSPACE_INVALID when the sizes are invalid.  The workspace needs
+ * no initialisation: every value is written before it is read.  One workspace
+ * may not be used by two calls that can run at the same time (different
+ * streams): they would race.
  */
 size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
                                int ngroups, int dstate, int chunk_size,
@@ -94,13 +98,11 @@ int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int
  *
  * seqlen may be 0 (then y is empty and final_state = init_state, or zeros) and
  * need not be a multiple of chunk_size.  io_dtype SSD_BF16 with headdim 64,
- * dstate 128 and seqlen >= 128 runs the tcgen05 tensor-core kernel (one launch,
- * plus a small memset of its workspace flags); it evaluates 128-token chunks
- * (its MMA tile height) whatever chunk_size says, and its results are
- * reproducible to rounding but not bitwise (the inter-chunk look-back may add
- * the same terms in a different order).  Every other combination runs the
- * float32 CUDA-core kernels (three launches), which honour chunk_size.  State
- * and accumulation are float32 in both.
+ * dstate 128 and seqlen >= 128 runs the tcgen05 tensor-core kernel: one launch,
+ * no workspace, bitwise reproducible.  It evaluates 128-token chunks (its MMA
+ * tile height) whatever chunk_size says.  Every other combination runs the
+ * float32 CUDA-core kernels (three launches, a workspace), which honour
+ * chunk_size.  State and accumulation are float32 in both.
  */
 ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A,
                         const void *B, const void *C, const float *D,

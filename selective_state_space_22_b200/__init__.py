@@ -130,8 +130,12 @@ def _workspace(device, nbytes: int):
     return buf
 
 
+SSD_WORKSPACE_INVALID = (1 << 64) - 1  # (size_t)-1: sizes that no scan accepts
+
+
 def ssd_scan_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size,
                             is_complex=False, io_dtype=SSD_BF16) -> int:
+    """Workspace bytes the scan needs (0: none); SSD_WORKSPACE_INVALID for invalid sizes."""
     return int(load_library().ssd_scan_workspace_size(batch, seqlen, nheads, headdim, ngroups,
                                                       dstate, chunk_size, int(bool(is_complex)),
                                                       io_dtype))

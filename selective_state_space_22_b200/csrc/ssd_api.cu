@@ -205,9 +205,9 @@ extern "C" {
 
 size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,
                                int dstate, int chunk_size, int is_complex, ssd_dtype io_dtype) {
-    if (!valid_dtype(io_dtype)) return 0;
+    if (!valid_dtype(io_dtype)) return SSD_WORKSPACE_INVALID;
     if (check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size) != SSD_OK)
-        return 0;
+        return SSD_WORKSPACE_INVALID;
     Plan pl = plan_scan(batch, seqlen, nheads, headdim, ngroups, dstate, chunk_size, is_complex != 0,
                         io_dtype == SSD_BF16);
     return pl.ws;

@@ -47,12 +47,15 @@ def test_version(lib):
 
 
 def test_workspace_size(lib):
-    n = ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 1, 128, 256, False, ssd.SSD_BF16)
-    assert n > 0
-    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 3, 128, 256, False, ssd.SSD_BF16) == 0
-    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 1, 128, 100, False, ssd.SSD_BF16) == 0
-    assert ssd.ssd_scan_workspace_size(-1, 2048, 64, 64, 1, 128, 256, False, ssd.SSD_BF16) == 0
+    bad = ssd.SSD_WORKSPACE_INVALID
+    # the tensor-core kernel (bf16, headdim 64, dstate 128) needs none
+    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 1, 128, 256, False, ssd.SSD_BF16) == 0
+    # the CUDA-core kernels keep per-chunk decays and states
+    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 1, 128, 256, False, ssd.SSD_F32) > 0
     assert ssd.ssd_scan_workspace_size(1, 256, 16, 64, 16, 64, 256, True, ssd.SSD_F32) > 0
+    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 3, 128, 256, False, ssd.SSD_BF16) == bad
+    assert ssd.ssd_scan_workspace_size(2, 2048, 64, 64, 1, 128, 100, False, ssd.SSD_BF16) == bad
+    assert ssd.ssd_scan_workspace_size(-1, 2048, 64, 64, 1, 128, 256, False, ssd.SSD_BF16) == bad
 
 
 FAKE = ctypes.c_void_p(1 << 20)  # 16-byte aligned, never dereferenced: validation fails first
