@@ -11,14 +11,12 @@
 //   M    = G o L o dt (+ D on the diagonal),  L[l,s] = exp(A_cs[l] - A_cs[s]), s <= l,
 //          rewritten in place in TMEM as bf16                     (CUDA cores)
 //   S    = B^T (exp(A_cs[last] - A_cs[s]) dt_s x_s)               (tcgen05: chunk state)
-//   y    = M X + (diag(exp(A_cs)) C) h_in^T                       (tcgen05, one accumulator)
+//   y    = M X + exp(A_cs[l]) C h_in^T                            (tcgen05)
 //   h_out = exp(A_cs[last]) h_in + S
 //
-// D x enters through M's diagonal, and the row factor exp(A_cs[l]) of the
-// off-diagonal term is applied to C in shared memory once G has read it, so both
-// products of y accumulate into the same TMEM columns.  Operands reach shared
-// memory by TMA (128-byte swizzle, zero fill past the end of the sequence) and y
-// leaves by a TMA store, which clips the ragged tail.
+// D x enters through M's diagonal.  Operands reach shared memory by TMA
+// (128-byte swizzle, zero fill past the end of the sequence); y is written from
+// registers, rows past the end of the sequence skipped.
 //
 // Inter-chunk state passing.  The pages carry chunk c's end state into a later
 // chunk z with exp(CD[z-1] - CD[c]) (a strict lower-triangular "decay_chunk"
@@ -31,10 +29,12 @@
 // S MMA; no G, M or y) to obtain its entering state, then scans its run in full.
 // CTAs never wait for one another, and the result does not depend on timing.
 //
-// Warp roles (10 warps): 0 TMA producer; 1 MMA issuer; 2-5 "math" warpgroup
-// (decay, W, the first half of M, the scaled C); 6-9 "state" warpgroup (the
-// second half of M, state update, h_in^T, the y epilogue).  Two input stages and two TMEM column sets let consecutive tiles
-// overlap.
+// Warp roles (15 warps): 0 TMA producer; 1 MMA issuer for G and S; 14 MMA
+// issuer for the two products of y; 2-5 "math" warpgroup (decay, W, M);
+// 6-9 "state" warpgroup (h_in^T, the state update); 10-13 epilogue warpgroup
+// (y).  Hot loops are kept rolled: four roles share each SM sub-partition's
+// instruction cache.  Two input stages and two TMEM column
+// sets let consecutive tiles overlap; a set is released as soon as its y is out.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -53,43 +53,45 @@ constexpr int PD = 64;   // head dim
 constexpr int ND = 128;  // state dim
 constexpr int MAX_RUNS = 16;
 
-constexpr int NTH = 320;
-constexpr int STATE_W0 = 6;  // warps 2-5 are the math warpgroup, 6-9 the state warpgroup
-constexpr uint32_t BAR_MATH = 1, BAR_STATE = 2;  // named barriers (128 threads each)
+constexpr int NTH = 480;
+constexpr int STATE_W0 = 6;     // warps 2-5: math warpgroup; 6-9: state warpgroup
+constexpr int EPI_W0 = 10;      // warps 10-13: epilogue warpgroup
+constexpr int Y_MMA_WARP = 14;  // issues the two products of y
+constexpr uint32_t BAR_MATH = 1;  // named barrier of the math warpgroup (128 threads)
 
 // TMEM: two column sets of 256 (consecutive tiles alternate).
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M in place (bf16 pairs, 64 cols)
-constexpr uint32_t COL_Y = 128;  // y accumulator (64 cols)
-constexpr uint32_t COL_S = 192;  // chunk state (64 cols)
+constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M (bf16 pairs) in columns 0-63
+constexpr uint32_t COL_YD = 128; // M X                                       (64 cols)
+constexpr uint32_t COL_S = 192;  // chunk state, then C h_in^T once it is read  (64 cols)
 
-// Shared memory: two input stages {C, B, X}; one W, one h_in^T and one y buffer.
+// Shared memory: two input stages {C, B, X}; one W buffer; two h_in^T buffers.
 constexpr int STAGE_BYTES = 81920;
 constexpr int OFF_C = 0, OFF_B = 32768, OFF_X = 65536;
 constexpr int OFF_W = 2 * STAGE_BYTES;
-constexpr int OFF_H = OFF_W + 16384;
-constexpr int OFF_Y = OFF_H + 16384;
-constexpr int OFF_MISC = OFF_Y + 16384;
+constexpr int OFF_H = OFF_W + 16384;  // [2][16 KB]
+constexpr int OFF_MISC = OFF_H + 2 * 16384;
 constexpr uint32_t LOAD_FULL = 2 * (QT * ND * 2) + QT * PD * 2;  // C, B, X
 constexpr uint32_t LOAD_STATE = QT * ND * 2 + QT * PD * 2;       // B, X
 enum {
     // count 1 (TMA bytes or an MMA commit)
     B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8,
-    // count 128 (a whole warpgroup arrives; B_M: both warpgroups, 256)
-    B_CS = 10, B_W = 12, B_M = 14, B_C = 16, B_H = 18, B_FREE = 20, NBARS = 22
+    // count 128 (one warpgroup)
+    B_CS = 10, B_W = 12, B_M = 14, B_H = 16, B_FREE = 18, NBARS = 20
 };
-// misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], wtot[4], bars, tmem base
-constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
+// misc: cs[2][128], dtv[2][128], bfac[2][128], ebuf[2][128] floats, lam[2], wtot[4], bars, tmem base
+constexpr int MISC_BYTES = 4 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
 constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
 constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 1, 1);    // B^T (MN-major) x W (MN-major)
 constexpr uint32_t IDESC_YD = idesc_bf16_f32(128, 64, 0, 1);   // M (TMEM) x X (MN-major)
-constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C' (K-major) x h^T (MN-major)
+constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C (K-major) x h^T (MN-major)
 
 constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on every wait
 
 struct TcParams {
+    __nv_bfloat16 *y;
     const float *dt;
     const float *A;
     const float *D;
@@ -207,11 +209,9 @@ __device__ __forceinline__ void block_apply(const uint32_t (&gr)[32], const floa
 }
 
 // One M block: TMEM load of G, decay factors computed while it is in flight,
-// then M (bf16 pairs, 16 columns) written over G columns this block's own
-// warpgroup has already read: blocks 0, 1 (math warpgroup) to columns 0-31,
-// blocks 2, 3 (state warpgroup) to columns 64-95.  The two warpgroups thus never
-// write a column the other still reads.
-__host__ __device__ constexpr uint32_t m_col(int j) { return 16 * j + (j >= 2 ? 32 : 0); }
+// then M (bf16 pairs, 16 columns) written to columns 16j..16j+15.  The blocks of
+// a row are built in order by the one thread that owns the row, and block j's
+// columns belong to G blocks <= j, which that thread has already read.
 __device__ __forceinline__ void m_block(uint32_t tm, int j, int quad, int lane, float csl, const float *csk,
                                         const float *dtk, const float *bfk, float Dh) {
     uint32_t pk[16];
@@ -226,7 +226,7 @@ __device__ __forceinline__ void m_block(uint32_t tm, int j, int quad, int lane, 
         tmem_wait_ld(g);
         block_apply(g, L, j == quad, lane, Dh, pk);
     }
-    tmem_st16(tm + m_col(j), pk);
+    tmem_st16(tm + 16 * j, pk);
 }
 
 // Row scaling of a 128-byte swizzled shared-memory row (eight 16-byte chunks),
@@ -247,71 +247,16 @@ __device__ __forceinline__ void scale_row(const uint8_t *src, uint8_t *dst, int 
     for (int j = 0; j < 8; ++j) reinterpret_cast<uint4 *>(dst)[j ^ key] = q[j];
 }
 
-// The same M block in two 16-column halves (fewer live registers, for the
-// warpgroup that also carries the state).
-__device__ __forceinline__ void m_block_halves(uint32_t tm, int j, int quad, int lane, float csl, const float *csk,
-                                               const float *dtk, const float *bfk, float Dh) {
-    const uint32_t dst = tm + m_col(j);
-    if (j > quad) {
-        uint32_t z[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) z[i] = 0u;
-        tmem_st8(dst, z);
-        tmem_st8(dst + 8, z);
-        return;
-    }
-    const int r = 32 * j;
-    const bool direct = fabsf(csk[r] - csk[r + 31]) > 80.f;
-    const float a = __expf(csl - csk[r]);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint32_t g[16];
-        tmem_ld16_nowait(tm + r + 16 * half, g);
-        float2 L[8];
-        const int c0 = r + 16 * half;
-        if (!direct) {
-            const float2 a2 = make_float2(a, a);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(bfk + c0 + 4 * i);
-                L[2 * i] = fmul2(a2, make_float2(b4.x, b4.y));
-                L[2 * i + 1] = fmul2(a2, make_float2(b4.z, b4.w));
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float4 c4 = *reinterpret_cast<const float4 *>(csk + c0 + 4 * i);
-                const float4 d4 = *reinterpret_cast<const float4 *>(dtk + c0 + 4 * i);
-                L[2 * i] = make_float2(__expf(fminf(csl - c4.x, 0.f)) * d4.x, __expf(fminf(csl - c4.y, 0.f)) * d4.y);
-                L[2 * i + 1] = make_float2(__expf(fminf(csl - c4.z, 0.f)) * d4.z, __expf(fminf(csl - c4.w, 0.f)) * d4.w);
-            }
-        }
-        tmem_wait_ld16(g);
-        uint32_t pk[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float2 m = fmul2(make_float2(__uint_as_float(g[2 * i]), __uint_as_float(g[2 * i + 1])), L[i]);
-            if (j == quad) {
-                const int s0 = 16 * half + 2 * i;
-                m.x = (s0 < lane) ? m.x : (s0 == lane ? m.x + Dh : 0.f);
-                m.y = (s0 + 1 < lane) ? m.y : (s0 + 1 == lane ? m.y + Dh : 0.f);
-            }
-            pk[i] = pack_bf16x2(m.x, m.y);
-        }
-        tmem_st8(dst + 8 * half, pk);
-    }
-}
-
 __global__ void __launch_bounds__(NTH, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                       const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                       const TcParams p) {
+                       const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float *cs = reinterpret_cast<float *>(sm + OFF_MISC);  // [2][128]
     float *dtv = cs + 2 * QT;                              // [2][128]
     float *bfac = dtv + 2 * QT;                            // [2][128]
-    float *lam_s = bfac + 2 * QT;                          // [2]
+    float *ebuf = bfac + 2 * QT;                           // [2][128] exp(A_cs) for the epilogue
+    float *lam_s = ebuf + 2 * QT;                          // [2]
     float *wtot = lam_s + 2;                               // [4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
@@ -319,7 +264,7 @@ __global__ void __launch_bounds__(NTH, 1)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], 1);
-        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], (i == B_M || i == B_M + 1) ? 256 : 128);
+        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -354,20 +299,19 @@ __global__ void __launch_bounds__(NTH, 1)
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------- MMA issuer
+        // ------------------------------------------- MMA issuer: G and S
         if (lane == 0) {
-            const uint32_t aW = sbase + OFF_W, aH = sbase + OFF_H;
+            const uint32_t aW = sbase + OFF_W;
             for (int k = 0; k < ntl; ++k) {
                 const bool so = decode_tile(p, k).state_only;
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aB = sbase + s * STAGE_BYTES + OFF_B;
-                const uint32_t aX = sbase + s * STAGE_BYTES + OFF_X;
                 mbar_wait(&bars[B_FULL + s], par, err);
                 mbar_wait(&bars[B_FREE + s], par ^ 1, err);
                 tc_fence_after();
                 if (!so) {
-#pragma unroll
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk) {  // G = C B^T
                         const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
                         mma_ss(tm + COL_G, smem_desc_sw128(aC + off, 16, 1024), smem_desc_sw128(aB + off, 16, 1024),
@@ -377,28 +321,41 @@ __global__ void __launch_bounds__(NTH, 1)
                 mma_commit(&bars[B_G + s]);
                 mbar_wait(&bars[B_W + s], par, err);
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)  // S = B^T W
                     mma_ss(tm + COL_S, smem_desc_sw128(aB + kk * 2048, 16384, 1024),
                            smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
                 mma_commit(&bars[B_S + s]);
-                mbar_wait(&bars[B_C + s], par, err);
-                mbar_wait(&bars[B_H + s], par, err);
-                tc_fence_after();
-                if (!so) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // y = C' h_in^T
-                        mma_ss(tm + COL_Y, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                               smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
-                }
+            }
+        }
+    } else if (warp == Y_MMA_WARP) {
+        // --------------------------------- MMA issuer: M X and C h_in^T
+        if (lane == 0) {
+            for (int k = 0; k < ntl; ++k) {
+                const bool so = decode_tile(p, k).state_only;
+                const int s = k & 1;
+                const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
+                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aX = sbase + s * STAGE_BYTES + OFF_X;
+                const uint32_t aH = sbase + OFF_H + s * 16384;
                 mbar_wait(&bars[B_M + s], par, err);
                 tc_fence_after();
                 if (!so) {
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)  // y += M X
-                        mma_ts(tm + COL_Y, tm + COL_G + m_col(kk >> 1) + 8 * (kk & 1),
-                               smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD, 1);
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)  // Y = M X
+                        mma_ts(tm + COL_YD, tm + COL_G + 8 * kk,
+                               smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD, kk > 0);
                 }
+                // h_in^T is written and the chunk state has been read out of COL_S
+                mbar_wait(&bars[B_H + s], par, err);
+                tc_fence_after();
+                if (!so) {
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)  // Y_off = C h_in^T
+                        mma_ss(tm + COL_S, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                               smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
+                }
+                // G and S of this tile completed before B_M and B_H could arrive, so
+                // once these commits fire the whole stage and TMEM set are read.
                 mma_commit(&bars[B_Y + s]);
                 mma_commit(&bars[B_EMPTY + s]);
             }
@@ -422,8 +379,8 @@ __global__ void __launch_bounds__(NTH, 1)
             uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W;
             const float Ah = p.A[t.h];
             const float Dh = p.D ? p.D[t.h] : 0.f;
-            // The stage's data is here; through the stage handshake, the state
-            // warpgroup is also done with this buffer set's values of tile k-2.
+            // The stage's data is here.  The stage was released only after tile
+            // k-2's M was built, so both warpgroups are done with its decays.
             mbar_wait(&bars[B_FULL + s], par, err);
             float v = d * Ah;  // inclusive cumsum of dt*A over the chunk
 #pragma unroll
@@ -450,35 +407,33 @@ __global__ void __launch_bounds__(NTH, 1)
             named_bar_sync(BAR_MATH, 128);  // bfac of every row written
             mbar_wait(&bars[B_G + s], par, err);
             tc_fence_after();
+            // exp(A_cs[row]) for the epilogue warpgroup.  G of this tile was issued
+            // after tile k-2's epilogue released the set, so that epilogue is done
+            // with this slot.
+            ebuf[s * QT + row] = __expf(v);
             if (!t.state_only) {
-                // M = G o L o dt (+ D on the diagonal): this warpgroup builds column
-                // blocks 0 and 1 (s < 64), the state warpgroup blocks 2 and 3.
-                m_block(tm + COL_G, 0, quad, lane, v, csk, dtk, bfk, Dh);
-                m_block(tm + COL_G, 1, quad, lane, v, csk, dtk, bfk, Dh);
+                // M = G o L o dt (+ D on the diagonal), column blocks in order
+#pragma unroll 1
+                for (int j = 0; j < 4; ++j) m_block(tm + COL_G, j, quad, lane, v, csk, dtk, bfk, Dh);
                 tmem_wait_st();
             }
             tc_fence_before();
             mbar_arrive(&bars[B_M + s]);
-            if (!t.state_only) {  // C' row l = exp(A_cs[l]) C row l, in place (G has read C)
-                uint8_t *sc = sm + s * STAGE_BYTES + OFF_C;
-                const __nv_bfloat162 e2 = __float2bfloat162_rn(__expf(v));
-                scale_row(sc + row * 128, sc + row * 128, row & 7, e2);
-                scale_row(sc + 16384 + row * 128, sc + 16384 + row * 128, row & 7, e2);
-                fence_proxy_async_smem();
-            }
-            mbar_arrive(&bars[B_C + s]);
         }
-    } else {
+    } else if (warp < EPI_W0) {
         // ----------------------------------------------- state warpgroup
         const int quad = warp & 3, row = quad * 32 + lane;
-        const bool elected = (tid == STATE_W0 * 32);
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        uint8_t *sh = sm + OFF_H, *sy = sm + OFF_Y;
         float h[PD];  // the state carried from chunk to chunk: h[p] for state row n = row
         for (int k = 0; k < ntl; ++k) {
             const Tile t = decode_tile(p, k);
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
+            mbar_wait(&bars[B_CS + s], par, err);
+            const float lam = lam_s[s];
+            // G of this tile was issued after tile k-2's epilogue, so the C h^T
+            // product of tile k-2 is done with this tile's h_in^T buffer.
+            mbar_wait(&bars[B_G + s], par, err);
             if (t.c == 0) {
                 if (p.init_state) {
                     const float *h0 = p.init_state + (size_t)t.bh * PD * ND + row;
@@ -489,9 +444,9 @@ __global__ void __launch_bounds__(NTH, 1)
                     for (int q = 0; q < PD; ++q) h[q] = 0.f;
                 }
             }
-            // h_in^T of this tile (rows n, bf16, 128-byte swizzle).  The previous
-            // tile's C' h^T product has read the buffer: its B_Y was waited for.
-            if (!t.state_only) {
+            if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle); its buffer was
+                                  // last read by the C h^T product of tile k-2
+                uint8_t *sh = sm + OFF_H + s * 16384;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int phys = q ^ (row & 7);
@@ -501,20 +456,6 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 fence_proxy_async_smem();
             }
-            mbar_arrive(&bars[B_H + s]);
-            mbar_wait(&bars[B_CS + s], par, err);
-            const float lam = lam_s[s];
-            mbar_wait(&bars[B_G + s], par, err);
-            tc_fence_after();
-            if (!t.state_only) {  // M column blocks 2 and 3
-                const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
-                const float Dh = p.D ? p.D[t.h] : 0.f;
-                m_block_halves(tm + COL_G, 2, quad, lane, csk[row], csk, dtk, bfk, Dh);
-                m_block_halves(tm + COL_G, 3, quad, lane, csk[row], csk, dtk, bfk, Dh);
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[B_M + s]);
             mbar_wait(&bars[B_S + s], par, err);
             tc_fence_after();
             {  // h_out = exp(lam) h_in + S, 32 columns at a time
@@ -527,41 +468,51 @@ __global__ void __launch_bounds__(NTH, 1)
                     for (int q = 0; q < 32; ++q) h[32 * half + q] = fmaf(el, h[32 * half + q], __uint_as_float(r[q]));
                 }
             }
+            tc_fence_before();
+            mbar_arrive(&bars[B_H + s]);  // h_in^T written, chunk state read: C h_in^T may go
             if (t.c == p.nchunks - 1 && p.final_state) {
                 float *fin = p.final_state + (size_t)t.bh * PD * ND + row;
 #pragma unroll
                 for (int q = 0; q < PD; ++q) fin[q * ND] = h[q];
             }
+        }
+    } else if (warp < Y_MMA_WARP) {
+        // -------------------------------------------- epilogue warpgroup
+        // y = M X + exp(A_cs[l]) C h_in^T, straight from TMEM to global memory.
+        const int quad = warp & 3, row = quad * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        for (int k = 0; k < ntl; ++k) {
+            const Tile t = decode_tile(p, k);
+            const int s = k & 1;
+            const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
+            mbar_wait(&bars[B_M + s], par, err);  // orders the ebuf write before this read
+            const float e = ebuf[s * QT + row];
             mbar_wait(&bars[B_Y + s], par, err);
             tc_fence_after();
-            if (!t.state_only) {  // y tile: accumulator -> bf16 -> y buffer -> TMA store
-                if (elected) bulk_wait_group_read0();  // the previous y store has read the buffer
-                named_bar_sync(BAR_STATE, 128);
-                uint32_t yv[32], yw[32];
-                tmem_ld32x2(tm + COL_Y, tm + COL_Y + 32, yv, yw);
+            if (!t.state_only) {
+                __nv_bfloat16 *yrow = p.y + (((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h) * PD;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t yd[32], yo[32];
+                    tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_S + 32 * half, yd, yo);
+                    if (row < t.valid) {
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t *src = (q < 4) ? &yv[8 * q] : &yw[8 * (q - 4)];
-                    const int phys = q ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(sy + row * 128 + phys * 16) = make_uint4(
-                        pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
-                        pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
-                        pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
-                        pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                const int e0 = 8 * q + 2 * i;
+                                pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
+                                                    fmaf(e, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
+                            }
+                            *reinterpret_cast<uint4 *>(yrow + 32 * half + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
                 }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                named_bar_sync(BAR_STATE, 128);
-                if (elected) {
-                    tma_store_4d(&tm_y, sy, 0, t.h, t.t0, t.b);
-                    bulk_commit_group();
-                }
-            } else {
-                tc_fence_before();
             }
+            tc_fence_before();
             mbar_arrive(&bars[B_FREE + s]);
         }
-        if (elected) bulk_wait_group0();
     }
 
     tc_fence_before();
@@ -657,13 +608,13 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     }
     const DevInfo &di = g_dev[dev];
 
-    CUtensorMap mx, mb, mc, my;
+    CUtensorMap mx, mb, mc;
     if ((e = make_map(&mx, a.x, a.headdim, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = make_map(&mb, a.B, a.dstate, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = make_map(&mc, a.C, a.dstate, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
-    if ((e = make_map(&my, a.y, a.headdim, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
 
     TcParams p;
+    p.y = static_cast<__nv_bfloat16 *>(a.y);
     p.dt = a.dt;
     p.A = a.A;
     p.D = a.D;
@@ -689,7 +640,7 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = SMEM_ALLOC;
     cfg.stream = st;
-    return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel, mx, mb, mc, my, p);
+    return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel, mx, mb, mc, p);
 }
 
 }  // namespace ssd
