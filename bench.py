@@ -17,6 +17,11 @@ event pairs; the reported time is the max over ranks.  Under torchrun every
 rank scans its own copy of the workload (independent sequences: weak scaling,
 no collective on the data path).
 
+``--workload decode-bitmamba1b-256seq`` times the one-step decode update
+instead: a step is one ``ssd_state_update`` call that advances 256 sequences by
+one token each (the float32 state, 537 MB, is streamed through HBM every step,
+so L2 holds nothing from one step to the next).
+
 ``--impl reference`` times the fp64 CPU oracle (the program the GPU results are
 checked against) on the host cores instead, each step a bounded sample of the
 same workload; under torchrun only rank 0 runs it.
@@ -266,6 +271,192 @@ def cpu_baseline(shape, max_updates: float = 4e9):
             "seconds": secs}
 
 
+# ---------------------------------------------------------------- decode
+DECODE_POOL = 8  # distinct per-step inputs resident on the device, used in turn
+
+
+def decode_bytes(shape) -> int:
+    """Per step: the state read and written once, x in, y out, dt, B, C, A, D."""
+    io = 4 if shape.io_dtype == "f32" else 2
+    b, H, P, G, N = shape.batch, shape.nheads, shape.headdim, shape.ngroups, shape.dstate
+    return 2 * b * H * P * N * 4 + 2 * b * H * P * io + b * H * 4 + 2 * b * G * N * io + 2 * H * 4
+
+
+def decode_cpu_baseline(shape, seqs: int = 16, steps: int = 8):
+    """The oracle's one-step update on the first ``seqs`` sequences, one
+    sequence per thread, ``steps`` steps; tokens/s = sequences x steps / s."""
+    import numpy as np
+
+    import oracle
+    from selective_state_space_22_b200 import inputs
+
+    threads = oracle_threads()
+    lib = oracle.load()
+    gen, const = inputs.decode_setup(shape)
+    st = inputs.widen(const["state"][:seqs])
+    A, D = inputs.widen(const["A"]), inputs.widen(const["D"])
+    step_inp = [inputs.widen_all(inputs.decode_step_inputs(gen, shape)) for _ in range(steps)]
+    c = np.ascontiguousarray
+    states = [c(st[i:i + 1]) for i in range(seqs)]
+
+    def one(i, w):
+        _, states[i] = oracle.state_update(states[i], c(w["x"][i:i + 1]), c(w["dt"][i:i + 1]), A,
+                                           c(w["B"][i:i + 1]), c(w["C"][i:i + 1]), D, lib=lib)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        for w in step_inp:
+            list(ex.map(lambda i: one(i, w), range(seqs)))
+    secs = time.perf_counter() - t0
+    return {"value": seqs * steps / secs, "unit": "tokens/s", "cores": min(threads, seqs), "kind": "oracle",
+            "sample": f"{seqs} of {shape.batch} sequences x {steps} decode steps of {shape.name}; fp64 "
+                      f"one-step update, one sequence per thread",
+            "seconds": secs}
+
+
+def bench_decode(args, shape):
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device for --impl ours")
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+
+    gen, const = inputs.decode_setup(shape)
+    state = const["state"].to(dev)
+    A, D = const["A"].to(dev), const["D"].to(dev)
+    pool_host = [inputs.decode_step_inputs(gen, shape) for _ in range(DECODE_POOL)]
+    pool = [{k: v.to(dev) for k, v in p.items()} for p in pool_host]
+    y = torch.empty_like(pool[0]["x"])
+
+    def step(i):
+        p = pool[i % DECODE_POOL]
+        ssd.ssd_state_update(state, p["x"], p["dt"], A, p["B"], p["C"], D, y=y)
+
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    ssd.ssd_get_device_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_s = dist_max(sum(per_step_ms) / 1e3, dev)
+    value = shape.batch * world * args.steps / total_s
+    peaks = load_peaks()
+    abytes = decode_bytes(shape)
+    t_launch = statistics.median(per_step_ms) / 1e3
+    kernel = "update_real_vec" if shape.dstate % 128 == 0 else "update_generic"
+    src = os.path.join(ROOT, "selective_state_space_22_b200", "csrc", "decode.cu")
+    roofline = {"bound": "hbm", "achieved": abytes / t_launch / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": abytes / t_launch / 1e9 / peaks["hbm_gbs"],
+                "traffic": lookup_traffic(kernel, src, shape.name), "kernel": kernel,
+                "algorithmic_bytes_per_launch": abytes,
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
+                if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
+                "roofline_time_us": 1e6 * abytes / (peaks["hbm_gbs"] * 1e9), "kernel_time_us": 1e6 * t_launch}
+
+    e2e = None
+    if not args.no_e2e:
+        hin = [{k: v.pin_memory() for k, v in p.items()} for p in pool_host]
+        yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in hin[0].values())
+        d2h = yh.numel() * yh.element_size()
+        k_e2e = max(3, min(args.steps, 50))
+
+        def e2e_step(i):
+            src_, dst = hin[i % DECODE_POOL], pool[i % DECODE_POOL]
+            for k in dst:
+                dst[k].copy_(src_[k], non_blocking=True)
+            step(i)
+            yh.copy_(y, non_blocking=True)
+
+        e2e_step(0)
+        torch.cuda.synchronize()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist_barrier()
+        torch.cuda.synchronize()
+        es.record(stream)
+        for i in range(k_e2e):
+            e2e_step(i)
+        ee.record(stream)
+        torch.cuda.synchronize()
+        dist_barrier()
+        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
+        e2e = {"value": shape.batch * world * k_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(shape)
+        cpu.pop("seconds", None)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
+        "config": {"workload": shape.name, "batch": shape.batch, "nheads": shape.nheads,
+                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
+                   "io_dtype": shape.io_dtype, "state_dtype": "f32",
+                   "l2": "state (537 MB) larger than L2, streamed every step",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
+        "gpu_launches": args.steps,
+        "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0], statistics.median(per_step_ms),
+                                statistics.quantiles(per_step_ms, n=10)[-1]],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_reference_decode(args, shape):
+    rank, world = dist_init("gloo")
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        decode_cpu_baseline(shape, seqs=1, steps=1)
+    res = [decode_cpu_baseline(shape) for _ in range(args.steps)]
+    secs = sum(r["seconds"] for r in res)
+    tokens = sum(r["value"] * r["seconds"] for r in res)
+    value = tokens / secs
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": shape.name, "batch": shape.batch, "nheads": shape.nheads,
+                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res[0]["cores"], "kind": "oracle",
+                         "sample": "per step " + res[0]["sample"]},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ------------------------------------------------------------------ arms
 def bench_reference(args, shape):
     rank, world = dist_init("gloo")
@@ -475,6 +666,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     from selective_state_space_22_b200 import inputs
 
+    if args.workload == inputs.DECODE.name:
+        shape = inputs.DECODE
+        return bench_reference_decode(args, shape) if args.impl == "reference" else bench_decode(args, shape)
     shape = inputs.WORKLOADS[args.workload]
     if args.impl == "reference":
         return bench_reference(args, shape)

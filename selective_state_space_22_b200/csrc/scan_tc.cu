@@ -364,21 +364,28 @@ __global__ void __launch_bounds__(NTH, 1)
         // ------------------------------------------------ math warpgroup
         const int quad = warp & 3, row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+        // The next tile's dt, A and D are loaded while this tile is built, so no
+        // global-memory latency sits on the per-tile path.
         Tile tn = ntl > 0 ? decode_tile(p, 0) : Tile{};
-        float dn = (ntl > 0 && row < tn.valid) ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
+        float dn = 0.f, An = 0.f, Dn = 0.f;
+        if (ntl > 0) {
+            dn = row < tn.valid ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
+            An = p.A[tn.h];
+            Dn = p.D ? p.D[tn.h] : 0.f;
+        }
         for (int k = 0; k < ntl; ++k) {
             const Tile t = tn;
-            const float d = dn;
-            if (k + 1 < ntl) {  // next tile's dt, in flight while this tile is built
+            const float d = dn, Ah = An, Dh = Dn;
+            if (k + 1 < ntl) {
                 tn = decode_tile(p, k + 1);
                 dn = (row < tn.valid) ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
+                An = p.A[tn.h];
+                Dn = p.D ? p.D[tn.h] : 0.f;
             }
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
             float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
             uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W;
-            const float Ah = p.A[t.h];
-            const float Dh = p.D ? p.D[t.h] : 0.f;
             // The stage's data is here.  The stage was released only after tile
             // k-2's M was built, so both warpgroups are done with its decays.
             mbar_wait(&bars[B_FULL + s], par, err);
