@@ -44,69 +44,62 @@ template <> __device__ __forceinline__ float4 ld4<__nv_bfloat16>(const __nv_bflo
     return v;
 }
 
-// Real step, dstate a multiple of 128: lane j holds elements 4j..4j+3 of each
-// 128-wide slice; ROWS independent rows per warp keep enough loads in flight.
+// Real step, dstate a multiple of 128.  One block per (batch, head): its index
+// arithmetic, dt, the decay and D are computed once, and B and C (shared by the
+// head's rows) once per warp.  A warp streams ROWS state rows at a time, lane j
+// holding elements 4j..4j+3 of each 128-wide slice, so ROWS x 512 bytes of loads
+// are in flight per warp before the first use.
 template <typename TIO, int ROWS>
-__global__ void __launch_bounds__(NT) update_real_vec(float *__restrict__ state, const TIO *__restrict__ x,
+__global__ void __launch_bounds__(NT, 4) update_real_vec(float *__restrict__ state, const TIO *__restrict__ x,
                                                       const float *__restrict__ dt, const float *__restrict__ A,
                                                       const TIO *__restrict__ B, const TIO *__restrict__ C,
                                                       const float *__restrict__ D, TIO *__restrict__ y,
-                                                      int batch, int nheads, int headdim, int ngroups,
-                                                      int dstate) {
-    const int lane = threadIdx.x & 31;
-    const long warp = (long)blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
-    const long nrows = (long)batch * nheads * headdim;
-    const long row0 = warp * ROWS;
-    if (row0 >= nrows) return;
-    const int slices = dstate / 128;
-    float yacc[ROWS];
-#pragma unroll
-    for (int r = 0; r < ROWS; ++r) yacc[r] = 0.f;
-    for (int sl = 0; sl < slices; ++sl) {
-        float4 hv[ROWS];
-        float xs[ROWS], dd[ROWS], aa[ROWS];
-        int gi[ROWS];
-        long bb[ROWS];
+                                                      int nheads, int headdim, int ngroups, int dstate) {
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const size_t bh = blockIdx.x;
+    const int h = (int)(bh % (unsigned)nheads);
+    const size_t b = bh / (unsigned)nheads;
+    const int g = h / (nheads / ngroups);
+    const float dtv = dt[bh];
+    const float dec = __expf(dtv * A[h]);
+    const float Dh = D ? D[h] : 0.f;
+    const TIO *Bg = B + (b * ngroups + g) * dstate + lane * 4;
+    const TIO *Cg = C + (b * ngroups + g) * dstate + lane * 4;
+    float *st = state + bh * headdim * dstate + lane * 4;
+    const TIO *xr = x + bh * headdim;
+    TIO *yr = y + bh * headdim;
+    for (int p0 = wib * ROWS; p0 < headdim; p0 += (NT / 32) * ROWS) {
+        float yacc[ROWS], u[ROWS];
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
-            const long row = row0 + r;
-            const long rr = row < nrows ? row : nrows - 1;
-            const long bh = rr / headdim;
-            const int h = (int)(bh % nheads);
-            bb[r] = bh / nheads;
-            gi[r] = h / (nheads / ngroups);
-            hv[r] = ld_stream(reinterpret_cast<const float4 *>(state + rr * dstate + sl * 128) + lane);
-            xs[r] = ld_f32(x + rr);
-            dd[r] = dt[bh];
-            aa[r] = A[h];
+            yacc[r] = 0.f;
+            u[r] = p0 + r < headdim ? dtv * ld_f32(xr + p0 + r) : 0.f;
+        }
+#pragma unroll 1
+        for (int sl = 0; sl < dstate; sl += 128) {
+            float4 hv[ROWS];
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r)
+                if (p0 + r < headdim) hv[r] = ld_stream(reinterpret_cast<const float4 *>(st + (size_t)(p0 + r) * dstate + sl));
+            const float4 bv = ld4(Bg + sl), cv = ld4(Cg + sl);
+#pragma unroll
+            for (int r = 0; r < ROWS; ++r) {
+                if (p0 + r >= headdim) continue;
+                float4 h4 = hv[r];
+                h4.x = fmaf(dec, h4.x, u[r] * bv.x);
+                h4.y = fmaf(dec, h4.y, u[r] * bv.y);
+                h4.z = fmaf(dec, h4.z, u[r] * bv.z);
+                h4.w = fmaf(dec, h4.w, u[r] * bv.w);
+                yacc[r] += h4.x * cv.x + h4.y * cv.y + h4.z * cv.z + h4.w * cv.w;
+                st_stream(reinterpret_cast<float4 *>(st + (size_t)(p0 + r) * dstate + sl), h4);
+            }
         }
 #pragma unroll
         for (int r = 0; r < ROWS; ++r) {
-            const long row = row0 + r;
-            const size_t bgo = ((size_t)bb[r] * ngroups + gi[r]) * dstate + sl * 128 + lane * 4;
-            const float4 bv = ld4(B + bgo), cv = ld4(C + bgo);
-            const float dec = __expf(dd[r] * aa[r]);
-            const float u = dd[r] * xs[r];
-            float4 h4 = hv[r];
-            h4.x = fmaf(dec, h4.x, u * bv.x);
-            h4.y = fmaf(dec, h4.y, u * bv.y);
-            h4.z = fmaf(dec, h4.z, u * bv.z);
-            h4.w = fmaf(dec, h4.w, u * bv.w);
-            yacc[r] += h4.x * cv.x + h4.y * cv.y + h4.z * cv.z + h4.w * cv.w;
-            if (row < nrows)
-                st_stream(reinterpret_cast<float4 *>(state + row * dstate + sl * 128) + lane, h4);
-        }
-    }
+            float part = yacc[r];
 #pragma unroll
-    for (int r = 0; r < ROWS; ++r) {
-        float part = yacc[r];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-        const long row = row0 + r;
-        if (lane == 0 && row < nrows) {
-            const long bh = row / headdim;
-            const float xv = ld_f32(x + row);
-            st_f32(y + row, part + (D ? D[bh % nheads] * xv : 0.f));
+            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+            if (lane == 0 && p0 + r < headdim) st_f32(yr + p0 + r, part + Dh * ld_f32(xr + p0 + r));
         }
     }
 }
@@ -163,12 +156,9 @@ cudaError_t launch_real(float *state, const void *x, const float *dt, const floa
                         int ngroups, int dstate, cudaStream_t st) {
     const long nrows = (long)batch * nheads * headdim;
     if (dstate % 128 == 0) {
-        constexpr int ROWS = 4;
-        const long warps = (nrows + ROWS - 1) / ROWS;
-        const long blocks = (warps + NT / 32 - 1) / (NT / 32);
-        update_real_vec<TIO, ROWS><<<(unsigned)blocks, NT, 0, st>>>(
-            state, (const TIO *)x, dt, A, (const TIO *)B, (const TIO *)C, D, (TIO *)y, batch, nheads,
-            headdim, ngroups, dstate);
+        update_real_vec<TIO, 4><<<(unsigned)((long)batch * nheads), NT, 0, st>>>(
+            state, (const TIO *)x, dt, A, (const TIO *)B, (const TIO *)C, D, (TIO *)y, nheads, headdim,
+            ngroups, dstate);
     } else {
         const long blocks = (nrows + NT / 32 - 1) / (NT / 32);
         update_generic<TIO, false><<<(unsigned)blocks, NT, 0, st>>>(
