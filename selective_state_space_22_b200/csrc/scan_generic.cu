@@ -462,7 +462,7 @@ size_t generic_workspace_bytes(int batch, int nheads, int headdim, int dstate, i
 }
 
 cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *ws, cudaStream_t st) {
-    if (cplx) return launch_typed<true, float>(a, ws, st);
+    if (cplx) return launch_complex_scan(a, ws, st);
     if (bf16) return launch_typed<false, __nv_bfloat16>(a, ws, st);
     return launch_typed<false, float>(a, ws, st);
 }

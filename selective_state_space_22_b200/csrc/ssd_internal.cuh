@@ -69,6 +69,9 @@ enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 // Each returns cudaSuccess or the launch error; none synchronises.
 size_t generic_workspace_bytes(int batch, int nheads, int headdim, int dstate, int chunk,
                                int nchunks, bool cplx);
+// Complex scan on CUDA cores (scan_complex.cu); same workspace layout and size as
+// generic_workspace_bytes(..., cplx = true).
+cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st);
 cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *ws,
                                 cudaStream_t st);
 
