@@ -573,9 +573,13 @@ def bench_ours(args, shape):
     else:
         achieved, peak, unit = aflops / t_launch / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
-    kernel = "ssd_scan_tc_kernel" if tc_path else "chunk_state+state_pass+chunk_scan (3 kernels)"
-    src = os.path.join(ROOT, "selective_state_space_22_b200", "csrc",
-                       "scan_tc.cu" if tc_path else "scan_generic.cu")
+    if tc_path:
+        kernel, src_name = "ssd_scan_tc_kernel", "scan_tc.cu"
+    elif cplx:
+        kernel, src_name = "cplx_chunk_state+cplx_state_pass+cplx_chunk_scan (3 kernels)", "scan_complex.cu"
+    else:
+        kernel, src_name = "chunk_state+state_pass+chunk_scan (3 kernels)", "scan_generic.cu"
+    src = os.path.join(ROOT, "selective_state_space_22_b200", "csrc", src_name)
     traffic = lookup_traffic(kernel, src, shape.name)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
