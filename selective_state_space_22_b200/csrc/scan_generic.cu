@@ -14,14 +14,15 @@
 //     pages' strict-lower-triangular decay_chunk propagation evaluated as a
 //     running product.  The last h_c is the final state.
 //  3. chunk_scan: per (batch, head, chunk, 64-row tile, 64-column tile)
-//        y[l, p] = Re( sum_{s <= l} (C_l . B_s) exp(A_cs[l] - A_cs[s]) dt_s x_s[p]
-//                      + exp(A_cs[l]) C_l . h_in[p, :] ) + D x_l[p].
+//        y[l, p] = sum_{s <= l} (C_l . B_s) exp(A_cs[l] - A_cs[s]) dt_s x_s[p]
+//                  + exp(A_cs[l]) C_l . h_in[p, :] + D x_l[p].
 //
-// The real and complex variants share the code through a "number" type (float
-// or interleaved complex).  A partial last chunk is handled by masking: tokens
-// past seqlen contribute nothing and the final state is the state after the
-// last real token.  Every exponent evaluated is a difference A_cs[l] - A_cs[s]
-// with l >= s (or A_cs[l] itself), so for Re A <= 0 no exp can overflow.
+// These serve the real variant in float32 and every shape the tensor-core
+// kernel does not take (the complex variant has its own kernels).  A partial
+// last chunk is handled by masking: tokens past seqlen contribute nothing and
+// the final state is the state after the last real token.  Every exponent
+// evaluated is a difference A_cs[l] - A_cs[s] with l >= s (or A_cs[l] itself),
+// so for A <= 0 no exp can overflow.
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -35,40 +36,16 @@ constexpr int ST = 64;   // source tokens per diagonal stage
 constexpr int SS = 32;   // tokens per chunk-state stage
 constexpr int OPT = 16;  // chunk-state outputs per thread
 
-template <bool CPLX> struct NumT { using T = float; };
-template <> struct NumT<true> { using T = cf; };
-
-__device__ __forceinline__ float madd(float acc, float a, float b) { return fmaf(a, b, acc); }
-__device__ __forceinline__ cf madd(cf acc, cf a, cf b) { return cfma(a, b, acc); }
-__device__ __forceinline__ float re_mul(float a, float b) { return a * b; }
-__device__ __forceinline__ float re_mul(cf a, cf b) { return fmaf(a.re, b.re, -a.im * b.im); }
-__device__ __forceinline__ float scal(float a, float s) { return a * s; }
-__device__ __forceinline__ cf scal(cf a, float s) { return cscale(a, s); }
-template <typename T> __device__ __forceinline__ T zero_num();
-template <> __device__ __forceinline__ float zero_num<float>() { return 0.f; }
-template <> __device__ __forceinline__ cf zero_num<cf>() { return {0.f, 0.f}; }
-__device__ __forceinline__ float mulnum(float a, float b) { return a * b; }
-__device__ __forceinline__ cf mulnum(cf a, cf b) { return cmul(a, b); }
-
-// B / C element: io dtype for the real variant, complex64 for the complex one.
-template <bool CPLX, typename TIO>
-__device__ __forceinline__ typename NumT<CPLX>::T ld_bc(const void *base, size_t i) {
-    if constexpr (CPLX) {
-        return reinterpret_cast<const cf *>(base)[i];
-    } else {
-        return ld_f32(reinterpret_cast<const TIO *>(base) + i);
-    }
+// B / C element of the io dtype, as float.
+template <typename TIO> __device__ __forceinline__ float ld_bc(const void *base, size_t i) {
+    return ld_f32(reinterpret_cast<const TIO *>(base) + i);
 }
 
-// exp of a (real or complex) log-decay given in double.
-template <bool CPLX> __device__ __forceinline__ typename NumT<CPLX>::T decay(double re, double im);
-template <> __device__ __forceinline__ float decay<false>(double re, double) { return (float)exp(re); }
-template <> __device__ __forceinline__ cf decay<true>(double re, double im) { return cexp_d(re, im); }
-
-// Workspace regions (each 256-byte aligned):
-//   cs  [b][H][nc][K][Q] double   K = 1 (real) or 2 (re block, im block)
+// Workspace regions (each 256-byte aligned; the complex kernels use the same
+// layout with K = 2):
+//   cs  [b][H][nc][K][Q] double   K = 1 here
 //   lam [b][H][nc][K]    double
-//   S   [b][H][nc][P][N] float or complex float
+//   S   [b][H][nc][P][N] float
 struct GenericWs {
     double *cs;
     double *lam;
@@ -108,45 +85,23 @@ __device__ void warp0_inclusive_scan(double *v, int Q) {
 
 // Shared prologue: dt and the cumulative log-decay of one chunk into shared
 // memory.  Tokens past the end of the sequence get dt = 0 (decay 1, no input).
-template <bool CPLX>
-__device__ void load_chunk_decay(const ScanArgs &a, int b, int h, int c, float *dts, double *cs_re,
-                                 double *cs_im) {
+__device__ void load_chunk_decay(const ScanArgs &a, int b, int h, int c, float *dts, double *cs_re) {
     const int Q = a.chunk, t0 = c * Q;
     const int valid = min(Q, a.seqlen - t0);
-    float Ar = CPLX ? a.A[2 * h] : a.A[h];
-    float Ai = CPLX ? a.A[2 * h + 1] : 0.f;
+    const float Ar = a.A[h];
     for (int s = threadIdx.x; s < Q; s += blockDim.x) {
-        float d = (s < valid) ? a.dt[((size_t)b * a.seqlen + t0 + s) * a.nheads + h] : 0.f;
+        const float d = (s < valid) ? a.dt[((size_t)b * a.seqlen + t0 + s) * a.nheads + h] : 0.f;
         dts[s] = d;
         cs_re[s] = (double)d * (double)Ar;
-        if (CPLX) cs_im[s] = (double)d * (double)Ai;
     }
     __syncthreads();
-    if (threadIdx.x < 32) {
-        warp0_inclusive_scan(cs_re, Q);
-    } else if (CPLX && threadIdx.x < 64) {
-        // the second warp scans the phase
-        const int lane = threadIdx.x & 31;
-        double carry = 0.0;
-        for (int base = 0; base < Q; base += 32) {
-            double x = (base + lane < Q) ? cs_im[base + lane] : 0.0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                double y = __shfl_up_sync(0xffffffffu, x, o);
-                if (lane >= o) x += y;
-            }
-            x += carry;
-            if (base + lane < Q) cs_im[base + lane] = x;
-            carry = __shfl_sync(0xffffffffu, x, 31);
-        }
-    }
+    if (threadIdx.x < 32) warp0_inclusive_scan(cs_re, Q);
     __syncthreads();
 }
 
 // ------------------------------------------------------------ 1. chunk state
-template <bool CPLX, typename TIO>
+template <typename TIO>
 __global__ void __launch_bounds__(NT) chunk_state_kernel(ScanArgs a, GenericWs w) {
-    using num = typename NumT<CPLX>::T;
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int PN = P * N;
     const int nsplit = (PN + NT * OPT - 1) / (NT * OPT);
@@ -154,37 +109,34 @@ __global__ void __launch_bounds__(NT) chunk_state_kernel(ScanArgs a, GenericWs w
     const int b = blockIdx.z / nsplit, split = blockIdx.z % nsplit;
     const int g = h / (H / a.ngroups);
     const int t0 = c * Q;
-    const int K = CPLX ? 2 : 1;
+    const int K = 1;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     double *cs_re = reinterpret_cast<double *>(smem_raw);
-    double *cs_im = cs_re + Q;
-    float *dts = reinterpret_cast<float *>(cs_im + Q);
-    num *ws_ = reinterpret_cast<num *>(dts + Q);  // per-token weight exp(Lambda - A_cs[s]) dt_s
-    num *xw = ws_ + Q;                            // [SS][P]
-    num *Bs = xw + SS * P;                        // [SS][N]
+    float *dts = reinterpret_cast<float *>(cs_re + Q);
+    float *ws_ = reinterpret_cast<float *>(dts + Q);  // per-token weight exp(Lambda - A_cs[s]) dt_s
+    float *xw = ws_ + Q;                            // [SS][P]
+    float *Bs = xw + SS * P;                        // [SS][N]
 
-    load_chunk_decay<CPLX>(a, b, h, c, dts, cs_re, cs_im);
-    const double lam_re = cs_re[Q - 1], lam_im = CPLX ? cs_im[Q - 1] : 0.0;
+    load_chunk_decay(a, b, h, c, dts, cs_re);
+    const double lam_re = cs_re[Q - 1];
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c;
     if (split == 0) {
         for (int s = threadIdx.x; s < Q; s += NT) {
             w.cs[(bhc * K) * Q + s] = cs_re[s];
-            if (CPLX) w.cs[(bhc * K + 1) * Q + s] = cs_im[s];
         }
         if (threadIdx.x == 0) {
             w.lam[bhc * K] = lam_re;
-            if (CPLX) w.lam[bhc * K + 1] = lam_im;
         }
     }
     for (int s = threadIdx.x; s < Q; s += NT)
-        ws_[s] = scal(decay<CPLX>(lam_re - cs_re[s], CPLX ? lam_im - cs_im[s] : 0.0), dts[s]);
+        ws_[s] = (float)exp(lam_re - cs_re[s]) * dts[s];
     __syncthreads();
 
     const int o0 = split * NT * OPT;
-    num acc[OPT];
+    float acc[OPT];
 #pragma unroll
-    for (int k = 0; k < OPT; ++k) acc[k] = zero_num<num>();
+    for (int k = 0; k < OPT; ++k) acc[k] = 0.f;
 
     const int valid = min(Q, a.seqlen - t0);
     const TIO *xg = reinterpret_cast<const TIO *>(a.x);
@@ -192,17 +144,17 @@ __global__ void __launch_bounds__(NT) chunk_state_kernel(ScanArgs a, GenericWs w
         const int sc = min(SS, valid - s0);
         for (int i = threadIdx.x; i < SS * P; i += NT) {
             int s = i / P, p = i % P;
-            num v = zero_num<num>();
+            float v = 0.f;
             if (s < sc) {
                 float xv = ld_f32(xg + (((size_t)b * a.seqlen + t0 + s0 + s) * H + h) * P + p);
-                v = scal(ws_[s0 + s], xv);
+                v = ws_[s0 + s] * xv;
             }
             xw[i] = v;
         }
         for (int i = threadIdx.x; i < SS * N; i += NT) {
             int s = i / N, n = i % N;
-            Bs[i] = (s < sc) ? ld_bc<CPLX, TIO>(a.B, (((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + n)
-                             : zero_num<num>();
+            Bs[i] = (s < sc) ? ld_bc<TIO>(a.B, (((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + n)
+                             : 0.f;
         }
         __syncthreads();
 #pragma unroll
@@ -210,14 +162,14 @@ __global__ void __launch_bounds__(NT) chunk_state_kernel(ScanArgs a, GenericWs w
             const int o = o0 + threadIdx.x + k * NT;
             if (o < PN) {
                 const int p = o / N, n = o % N;
-                num v = acc[k];
-                for (int s = 0; s < sc; ++s) v = madd(v, xw[s * P + p], Bs[s * N + n]);
+                float v = acc[k];
+                for (int s = 0; s < sc; ++s) v = fmaf(xw[s * P + p], Bs[s * N + n], v);
                 acc[k] = v;
             }
         }
         __syncthreads();
     }
-    num *S = reinterpret_cast<num *>(w.S) + bhc * PN;
+    float *S = reinterpret_cast<float *>(w.S) + bhc * PN;
 #pragma unroll
     for (int k = 0; k < OPT; ++k) {
         const int o = o0 + threadIdx.x + k * NT;
@@ -226,32 +178,29 @@ __global__ void __launch_bounds__(NT) chunk_state_kernel(ScanArgs a, GenericWs w
 }
 
 // ------------------------------------------------------------ 2. state pass
-template <bool CPLX>
 __global__ void __launch_bounds__(NT) state_pass_kernel(ScanArgs a, GenericWs w) {
-    using num = typename NumT<CPLX>::T;
     const int PN = a.headdim * a.dstate;
     const int e = blockIdx.x * NT + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
     if (e >= PN) return;
-    const int K = CPLX ? 2 : 1;
+    const int K = 1;
     const size_t bh = (size_t)b * a.nheads + h;
-    num run = zero_num<num>();
-    if (a.init_state) run = reinterpret_cast<const num *>(a.init_state)[bh * PN + e];
-    num *S = reinterpret_cast<num *>(w.S);
+    float run = 0.f;
+    if (a.init_state) run = reinterpret_cast<const float *>(a.init_state)[bh * PN + e];
+    float *S = reinterpret_cast<float *>(w.S);
     for (int c = 0; c < a.nchunks; ++c) {
         const size_t bhc = bh * a.nchunks + c;
-        num s = S[bhc * PN + e];
+        float s = S[bhc * PN + e];
         S[bhc * PN + e] = run;  // the state entering chunk c
-        num dec = decay<CPLX>(w.lam[bhc * K], CPLX ? w.lam[bhc * K + 1] : 0.0);
-        run = madd(s, dec, run);
+        const float dec = (float)exp(w.lam[bhc * K]);
+        run = fmaf(dec, run, s);
     }
-    if (a.final_state) reinterpret_cast<num *>(a.final_state)[bh * PN + e] = run;
+    if (a.final_state) reinterpret_cast<float *>(a.final_state)[bh * PN + e] = run;
 }
 
 // ------------------------------------------------------------- 3. chunk scan
-template <bool CPLX, typename TIO>
+template <typename TIO>
 __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w) {
-    using num = typename NumT<CPLX>::T;
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int nrt = (Q + RT - 1) / RT, npt = (P + PT - 1) / PT;
     const int rt = blockIdx.x % nrt, c = blockIdx.x / nrt;
@@ -264,21 +213,19 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
     if (l0 >= valid) return;
     const int rows = min(RT, valid - l0);
     const int p0 = pt * PT;
-    const int K = CPLX ? 2 : 1;
+    const int K = 1;
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c;
 
     extern __shared__ __align__(16) unsigned char smem_raw[];
     double *cs_re = reinterpret_cast<double *>(smem_raw);
-    double *cs_im = cs_re + Q;
-    float *dts = reinterpret_cast<float *>(cs_im + Q);
-    num *At = reinterpret_cast<num *>(dts + Q);  // [KT][RT]
-    num *Bt = At + KT * RT;                      // [KT][64]
+    float *dts = reinterpret_cast<float *>(cs_re + Q);
+    float *At = reinterpret_cast<float *>(dts + Q);  // [KT][RT]
+    float *Bt = At + KT * RT;                      // [KT][64]
     float *Ms = reinterpret_cast<float *>(Bt + KT * 64);  // [ST][RT]
     float *Xs = Ms + ST * RT;                             // [ST][PT]
 
     for (int s = threadIdx.x; s < Q; s += NT) {
         cs_re[s] = w.cs[(bhc * K) * Q + s];
-        if (CPLX) cs_im[s] = w.cs[(bhc * K + 1) * Q + s];
         dts[s] = (s < valid) ? a.dt[((size_t)b * a.seqlen + t0 + s) * H + h] : 0.f;
     }
     __syncthreads();
@@ -295,26 +242,26 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
 
     // Off-diagonal term: exp(A_cs[l]) C_l . h_in[p, :]  (skipped when h_in is 0).
     if (c > 0 || a.init_state) {
-        const num *hin = reinterpret_cast<const num *>(w.S) + bhc * PN;
+        const float *hin = reinterpret_cast<const float *>(w.S) + bhc * PN;
         for (int n0 = 0; n0 < N; n0 += KT) {
             for (int i = threadIdx.x; i < KT * RT; i += NT) {
                 int l = i / KT, k = i % KT;
-                num v = zero_num<num>();
+                float v = 0.f;
                 if (l < rows && n0 + k < N) {
-                    num cv = ld_bc<CPLX, TIO>(a.C, (((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + n0 + k);
-                    v = mulnum(cv, decay<CPLX>(cs_re[l0 + l], CPLX ? cs_im[l0 + l] : 0.0));
+                    float cv = ld_bc<TIO>(a.C, (((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + n0 + k);
+                    v = cv * (float)exp(cs_re[l0 + l]);
                 }
                 At[k * RT + l] = v;
             }
             for (int i = threadIdx.x; i < KT * PT; i += NT) {
                 int p = i / KT, k = i % KT;
                 Bt[k * 64 + p] = (p0 + p < P && n0 + k < N) ? hin[(size_t)(p0 + p) * N + n0 + k]
-                                                            : zero_num<num>();
+                                                            : 0.f;
             }
             __syncthreads();
 #pragma unroll 4
             for (int k = 0; k < KT; ++k) {
-                num av[4], bv[4];
+                float av[4], bv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) av[i] = At[k * RT + li * 4 + i];
 #pragma unroll
@@ -322,7 +269,7 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) acc[i][j] += re_mul(av[i], bv[j]);
+                    for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
             }
             __syncthreads();
         }
@@ -331,28 +278,28 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
     // Diagonal block: sum_{s <= l} Re((C_l . B_s) exp(A_cs[l] - A_cs[s])) dt_s x_s[p].
     const int s_end = l0 + rows;
     for (int s0 = 0; s0 < s_end; s0 += ST) {
-        num gacc[4][4];
+        float gacc[4][4];
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-            for (int j = 0; j < 4; ++j) gacc[i][j] = zero_num<num>();
+            for (int j = 0; j < 4; ++j) gacc[i][j] = 0.f;
         for (int n0 = 0; n0 < N; n0 += KT) {
             for (int i = threadIdx.x; i < KT * RT; i += NT) {
                 int l = i / KT, k = i % KT;
                 At[k * RT + l] = (l < rows && n0 + k < N)
-                    ? ld_bc<CPLX, TIO>(a.C, (((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + n0 + k)
-                    : zero_num<num>();
+                    ? ld_bc<TIO>(a.C, (((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + n0 + k)
+                    : 0.f;
             }
             for (int i = threadIdx.x; i < KT * ST; i += NT) {
                 int s = i / KT, k = i % KT;
                 Bt[k * 64 + s] = (s0 + s < valid && n0 + k < N)
-                    ? ld_bc<CPLX, TIO>(a.B, (((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + n0 + k)
-                    : zero_num<num>();
+                    ? ld_bc<TIO>(a.B, (((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + n0 + k)
+                    : 0.f;
             }
             __syncthreads();
 #pragma unroll 4
             for (int k = 0; k < KT; ++k) {
-                num av[4], bv[4];
+                float av[4], bv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) av[i] = At[k * RT + li * 4 + i];
 #pragma unroll
@@ -360,7 +307,7 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) gacc[i][j] = madd(gacc[i][j], av[i], bv[j]);
+                    for (int j = 0; j < 4; ++j) gacc[i][j] = fmaf(av[i], bv[j], gacc[i][j]);
             }
             __syncthreads();
         }
@@ -373,8 +320,8 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
                 const int l = l0 + li * 4 + i, s = s0 + pi * 4 + j;
                 float m = 0.f;
                 if (s <= l && s < valid && l < valid) {
-                    num L = decay<CPLX>(cs_re[l] - cs_re[s], CPLX ? cs_im[l] - cs_im[s] : 0.0);
-                    m = re_mul(gacc[i][j], L) * dts[s];
+                    const float L = (float)exp(cs_re[l] - cs_re[s]);
+                    m = gacc[i][j] * L * dts[s];
                 }
                 Ms[(pi * 4 + j) * RT + li * 4 + i] = m;
             }
@@ -420,16 +367,15 @@ __global__ void __launch_bounds__(NT) chunk_scan_kernel(ScanArgs a, GenericWs w)
     }
 }
 
-template <bool CPLX, typename TIO>
+template <typename TIO>
 cudaError_t launch_typed(const ScanArgs &a, void *wsp, cudaStream_t st) {
-    using num = typename NumT<CPLX>::T;
-    GenericWs w = carve(wsp, a.batch, a.nheads, a.headdim, a.dstate, a.chunk, a.nchunks, CPLX);
+    GenericWs w = carve(wsp, a.batch, a.nheads, a.headdim, a.dstate, a.chunk, a.nchunks, false);
     const int Q = a.chunk, P = a.headdim, N = a.dstate;
     const int PN = P * N;
     const int nsplit = (PN + NT * OPT - 1) / (NT * OPT);
 
-    size_t sm1 = 2 * Q * sizeof(double) + Q * sizeof(float) + (Q + SS * (P + N)) * sizeof(num);
-    auto k1 = chunk_state_kernel<CPLX, TIO>;
+    size_t sm1 = Q * sizeof(double) + Q * sizeof(float) + (Q + SS * (P + N)) * sizeof(float);
+    auto k1 = chunk_state_kernel<TIO>;
     cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
     if (e != cudaSuccess) return e;
     dim3 g1(a.nchunks, a.nheads, a.batch * nsplit);
@@ -437,12 +383,12 @@ cudaError_t launch_typed(const ScanArgs &a, void *wsp, cudaStream_t st) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     dim3 g2((PN + NT - 1) / NT, a.nheads, a.batch);
-    state_pass_kernel<CPLX><<<g2, NT, 0, st>>>(a, w);
+    state_pass_kernel<<<g2, NT, 0, st>>>(a, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    size_t sm3 = 2 * Q * sizeof(double) + Q * sizeof(float) + (KT * RT + KT * 64) * sizeof(num) +
+    size_t sm3 = Q * sizeof(double) + Q * sizeof(float) + (KT * RT + KT * 64) * sizeof(float) +
                  (ST * RT + ST * PT) * sizeof(float);
-    auto k3 = chunk_scan_kernel<CPLX, TIO>;
+    auto k3 = chunk_scan_kernel<TIO>;
     e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3);
     if (e != cudaSuccess) return e;
     const int nrt = (Q + RT - 1) / RT, npt = (P + PT - 1) / PT;
@@ -463,8 +409,8 @@ size_t generic_workspace_bytes(int batch, int nheads, int headdim, int dstate, i
 
 cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *ws, cudaStream_t st) {
     if (cplx) return launch_complex_scan(a, ws, st);
-    if (bf16) return launch_typed<false, __nv_bfloat16>(a, ws, st);
-    return launch_typed<false, float>(a, ws, st);
+    if (bf16) return launch_typed<__nv_bfloat16>(a, ws, st);
+    return launch_typed<float>(a, ws, st);
 }
 
 }  // namespace ssd
