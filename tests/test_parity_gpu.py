@@ -79,6 +79,13 @@ def test_complex_small_dims():
     check_full(small("cplx2", 1, 129, 2, 16, 2, 8, 64, "f32", cplx=True, init=True), TOL_F32)
 
 
+@pytest.mark.parametrize("P,N,G", [(64, 96, 1), (100, 128, 2), (32, 200, 4)])
+def test_complex_wide_state_and_head_dim(P, N, G):
+    """2N > 128 takes the K-sliced chunk scan and several chunk-state tiles;
+    P > 64 several head-dim tiles."""
+    check_full(small("cplx3", 2, 333, 4, P, G, N, 128, "f32", cplx=True, init=True), TOL_F32)
+
+
 # ------------------------------------------------------------------- edge cases
 def test_empty_sequence_copies_initial_state():
     shape = small("empty", 2, 0, 4, 64, 1, 128, 256, "bf16", init=True)
