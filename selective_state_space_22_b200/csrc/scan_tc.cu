@@ -30,9 +30,9 @@
 // CTAs never wait for one another, and the result does not depend on timing.
 //
 // Warp roles (15 warps): 0 TMA producer; 1 MMA issuer for G and S; 14 MMA
-// issuer for the two products of y; 2-5 "math" warpgroup (decay, W, M);
-// 6-9 "state" warpgroup (h_in^T, the state update); 10-13 epilogue warpgroup
-// (y).  Hot loops are kept rolled: four roles share each SM sub-partition's
+// issuer for the two products of y; 2-5 "math" warpgroup (M); 6-9 "state"
+// warpgroup (h_in^T, the state update); 10-13 "prep/epilogue" warpgroup (the
+// cumulative decay and W of tile k, then y of tile k-1).  Hot loops are kept rolled: four roles share each SM sub-partition's
 // instruction cache.  Two input stages and two TMEM column
 // sets let consecutive tiles overlap; a set is released as soon as its y is out.
 #include <cudaTypedefs.h>
@@ -79,8 +79,8 @@ enum {
     // count 128 (one warpgroup)
     B_CS = 10, B_W = 12, B_M = 14, B_H = 16, B_FREE = 18, NBARS = 20
 };
-// misc: cs[2][128], dtv[2][128], bfac[2][128], ebuf[2][128] floats, lam[2], wtot[4], bars, tmem base
-constexpr int MISC_BYTES = 4 * 2 * QT * 4 + 8 + 16 + NBARS * 8 + 8;
+// misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4], bars, tmem base
+constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + NBARS * 8 + 8;
 constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
@@ -255,9 +255,9 @@ __global__ void __launch_bounds__(NTH, 1)
     float *cs = reinterpret_cast<float *>(sm + OFF_MISC);  // [2][128]
     float *dtv = cs + 2 * QT;                              // [2][128]
     float *bfac = dtv + 2 * QT;                            // [2][128]
-    float *ebuf = bfac + 2 * QT;                           // [2][128] exp(A_cs) for the epilogue
-    float *lam_s = ebuf + 2 * QT;                          // [2]
-    float *wtot = lam_s + 2;                               // [4]
+    float *lam_s = bfac + 2 * QT;                          // [2]
+    float *dh_s = lam_s + 2;                               // [2]
+    float *wtot = dh_s + 2;                                // [4]
     uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 4);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
 
@@ -362,64 +362,20 @@ __global__ void __launch_bounds__(NTH, 1)
         }
     } else if (warp < STATE_W0) {
         // ------------------------------------------------ math warpgroup
+        // Per tile: M = G o L o dt (+ D on the diagonal), the four column blocks in
+        // order, from the decays the prep/epilogue warpgroup put in shared memory.
         const int quad = warp & 3, row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        // The next tile's dt, A and D are loaded while this tile is built, so no
-        // global-memory latency sits on the per-tile path.
-        Tile tn = ntl > 0 ? decode_tile(p, 0) : Tile{};
-        float dn = 0.f, An = 0.f, Dn = 0.f;
-        if (ntl > 0) {
-            dn = row < tn.valid ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
-            An = p.A[tn.h];
-            Dn = p.D ? p.D[tn.h] : 0.f;
-        }
         for (int k = 0; k < ntl; ++k) {
-            const Tile t = tn;
-            const float d = dn, Ah = An, Dh = Dn;
-            if (k + 1 < ntl) {
-                tn = decode_tile(p, k + 1);
-                dn = (row < tn.valid) ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
-                An = p.A[tn.h];
-                Dn = p.D ? p.D[tn.h] : 0.f;
-            }
+            const bool so = decode_tile(p, k).state_only;
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
-            float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
-            uint8_t *sx = sm + s * STAGE_BYTES + OFF_X, *sw = sm + OFF_W;
-            // The stage's data is here.  The stage was released only after tile
-            // k-2's M was built, so both warpgroups are done with its decays.
-            mbar_wait(&bars[B_FULL + s], par, err);
-            float v = d * Ah;  // inclusive cumsum of dt*A over the chunk
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float y = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += y;
-            }
-            if (lane == 31) wtot[quad] = v;
-            named_bar_sync(BAR_MATH, 128);
-            for (int w = 0; w < quad; ++w) v += wtot[w];
-            csk[row] = v;
-            dtk[row] = d;
-            named_bar_sync(BAR_MATH, 128);
-            const float lam = csk[QT - 1];
-            if (row == 0) lam_s[s] = lam;
-            bfk[row] = __expf(csk[row & ~31] - v) * d;  // exp(A_cs[r] - A_cs[s]) dt_s, r = s's 32-block start
-            mbar_arrive(&bars[B_CS + s]);
-            // W (one buffer): the previous tile's S must have read it
-            if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
-            // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk places)
-            scale_row(sx + row * 128, sw + row * 128, row & 7, __float2bfloat162_rn(__expf(lam - v) * d));
-            fence_proxy_async_smem();
-            mbar_arrive(&bars[B_W + s]);
-            named_bar_sync(BAR_MATH, 128);  // bfac of every row written
+            const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
+            mbar_wait(&bars[B_CS + s], par, err);
+            const float v = csk[row], Dh = dh_s[s];
             mbar_wait(&bars[B_G + s], par, err);
             tc_fence_after();
-            // exp(A_cs[row]) for the epilogue warpgroup.  G of this tile was issued
-            // after tile k-2's epilogue released the set, so that epilogue is done
-            // with this slot.
-            ebuf[s * QT + row] = __expf(v);
-            if (!t.state_only) {
-                // M = G o L o dt (+ D on the diagonal), column blocks in order
+            if (!so) {
 #pragma unroll 1
                 for (int j = 0; j < 4; ++j) m_block(tm + COL_G, j, quad, lane, v, csk, dtk, bfk, Dh);
                 tmem_wait_st();
@@ -484,41 +440,100 @@ __global__ void __launch_bounds__(NTH, 1)
             }
         }
     } else if (warp < Y_MMA_WARP) {
-        // -------------------------------------------- epilogue warpgroup
-        // y = M X + exp(A_cs[l]) C h_in^T, straight from TMEM to global memory.
+        // --------------------------------------- prep / epilogue warpgroup
+        // Step k: the cumulative decay and W of tile k, then y of tile k-1:
+        //   y = M X + exp(A_cs[l]) C h_in^T, straight from TMEM to global memory.
+        // Tile k's decays go to slot k % 2, last read for tile k-2: by its M and
+        // its state update, both of which finished before tile k-2's y (waited
+        // for in step k-1).
         const int quad = warp & 3, row = quad * 32 + lane;
         const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-        for (int k = 0; k < ntl; ++k) {
-            const Tile t = decode_tile(p, k);
-            const int s = k & 1;
-            const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
-            mbar_wait(&bars[B_M + s], par, err);  // orders the ebuf write before this read
-            const float e = ebuf[s * QT + row];
-            mbar_wait(&bars[B_Y + s], par, err);
-            tc_fence_after();
-            if (!t.state_only) {
-                __nv_bfloat16 *yrow = p.y + (((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h) * PD;
+        // The next tile's dt, A and D are loaded while this tile is built, so no
+        // global-memory latency sits on the per-tile path.
+        Tile tn = ntl > 0 ? decode_tile(p, 0) : Tile{};
+        float dn = 0.f, An = 0.f, Dn = 0.f;
+        if (ntl > 0) {
+            dn = row < tn.valid ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
+            An = p.A[tn.h];
+            Dn = p.D ? p.D[tn.h] : 0.f;
+        }
+        Tile prev{};  // tile k-1, whose y this step writes
+        for (int k = 0; k <= ntl; ++k) {
+            Tile cur{};
+            if (k < ntl) {
+                cur = tn;
+                const float d = dn, Ah = An, Dh = Dn;
+                if (k + 1 < ntl) {
+                    tn = decode_tile(p, k + 1);
+                    dn = (row < tn.valid) ? p.dt[((size_t)tn.b * p.seqlen + tn.t0 + row) * p.nheads + tn.h] : 0.f;
+                    An = p.A[tn.h];
+                    Dn = p.D ? p.D[tn.h] : 0.f;
+                }
+                const int s = k & 1;
+                const uint32_t par = (k >> 1) & 1;
+                float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
+                float v = d * Ah;  // inclusive cumsum of dt*A over the chunk
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, v, o);
+                    if (lane >= o) v += y;
+                }
+                if (lane == 31) wtot[quad] = v;
+                named_bar_sync(BAR_MATH, 128);
+                for (int w = 0; w < quad; ++w) v += wtot[w];
+                csk[row] = v;
+                dtk[row] = d;
+                named_bar_sync(BAR_MATH, 128);
+                const float lam = csk[QT - 1];
+                if (row == 0) {
+                    lam_s[s] = lam;
+                    dh_s[s] = Dh;
+                }
+                bfk[row] = __expf(csk[row & ~31] - v) * d;  // exp(A_cs[r] - A_cs[s]) dt_s, r = s's 32-block start
+                named_bar_sync(BAR_MATH, 128);  // every row's decays written
+                mbar_arrive(&bars[B_CS + s]);
+                // W (one buffer): the previous tile's S must have read it
+                mbar_wait(&bars[B_FULL + s], par, err);
+                if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
+                // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk places)
+                scale_row(sm + s * STAGE_BYTES + OFF_X + row * 128, sm + OFF_W + row * 128, row & 7,
+                          __float2bfloat162_rn(__expf(lam - v) * d));
+                fence_proxy_async_smem();
+                mbar_arrive(&bars[B_W + s]);
+            }
+            if (k > 0) {  // y of tile k-1
+                const int j = k - 1, s = j & 1;
+                const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s + lane_off;
+                const Tile t = prev;
+                const float e = __expf(cs[s * QT + row]);
+                mbar_wait(&bars[B_Y + s], par, err);
+                tc_fence_after();
+                if (!t.state_only) {
+                    __nv_bfloat16 *yrow = p.y + (((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h) * PD;
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t yd[32], yo[32];
-                    tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_S + 32 * half, yd, yo);
-                    if (row < t.valid) {
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t yd[32], yo[32];
+                        tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_S + 32 * half, yd, yo);
+                        if (row < t.valid) {
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            uint32_t pk[4];
+                            for (int q = 0; q < 4; ++q) {
+                                uint32_t pk[4];
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                const int e0 = 8 * q + 2 * i;
-                                pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
-                                                    fmaf(e, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
+                                for (int i = 0; i < 4; ++i) {
+                                    const int e0 = 8 * q + 2 * i;
+                                    pk[i] = pack_bf16x2(fmaf(e, __uint_as_float(yo[e0]), __uint_as_float(yd[e0])),
+                                                        fmaf(e, __uint_as_float(yo[e0 + 1]), __uint_as_float(yd[e0 + 1])));
+                                }
+                                *reinterpret_cast<uint4 *>(yrow + 32 * half + 8 * q) =
+                                    make_uint4(pk[0], pk[1], pk[2], pk[3]);
                             }
-                            *reinterpret_cast<uint4 *>(yrow + 32 * half + 8 * q) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                         }
                     }
                 }
+                tc_fence_before();
+                mbar_arrive(&bars[B_FREE + s]);
             }
-            tc_fence_before();
-            mbar_arrive(&bars[B_FREE + s]);
+            prev = cur;
         }
     }
 
