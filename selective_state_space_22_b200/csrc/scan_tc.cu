@@ -495,9 +495,16 @@ __global__ void __launch_bounds__(NTH, 1)
                 // W (one buffer): the previous tile's S must have read it
                 mbar_wait(&bars[B_FULL + s], par, err);
                 if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
-                // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk places)
-                scale_row(sm + s * STAGE_BYTES + OFF_X + row * 128, sm + OFF_W + row * 128, row & 7,
-                          __float2bfloat162_rn(__expf(lam - v) * d));
+                // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
+                // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
+                // SM sub-partition also builds the most M blocks, skips it and the warp
+                // of quadrant 0 (the fewest) takes those rows too.
+                auto w_row = [&](int r) {
+                    scale_row(sm + s * STAGE_BYTES + OFF_X + r * 128, sm + OFF_W + r * 128, r & 7,
+                              __float2bfloat162_rn(__expf(lam - csk[r]) * dtk[r]));
+                };
+                if (quad != 3) w_row(row);
+                if (quad == 0) w_row(96 + lane);
                 fence_proxy_async_smem();
                 mbar_arrive(&bars[B_W + s]);
             }
