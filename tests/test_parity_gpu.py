@@ -152,6 +152,39 @@ def test_tcgen05_path(T, H, G):
     check_full(shape, TOL_BF16)
 
 
+@pytest.mark.parametrize("io", ["bf16", "f32"])
+def test_steep_decay(io):
+    """A in [-100, -40] with dt up to 0.1: a 32-token block can span well over 80 of
+    log-decay, so the kernels take their per-element decay path (the factored
+    form's factors would leave the float range).  Nothing may overflow."""
+    shape = small("steep", 2, 700, 4, 64, 1, 128, 256, io, init=True, seed=99)
+    inp = inputs.scan_inputs(shape)
+    inp["A"] = -torch.linspace(40.0, 100.0, shape.nheads)
+    inp["dt"] = (inp["dt"] * 4.0).clamp(max=0.1).contiguous()
+    if io == "bf16":
+        assert _tc(shape)
+    y, fs = gpu_scan(inp, shape.chunk, False)
+    assert torch.isfinite(y).all() and torch.isfinite(fs).all()
+    y_ref, fs_ref = oracle_scan(inp)
+    tol = TOL_BF16 if io == "bf16" else TOL_F32
+    ey, ef = rel_err(y.numpy(), y_ref), rel_err(fs.numpy(), fs_ref)
+    assert ey <= tol and ef <= tol, (ey, ef)
+
+
+def test_steep_decay_complex():
+    """Complex A with real part in [-100, -40]: decays that underflow within a
+    chunk must come out as zeros, never as inf or NaN."""
+    shape = small("steepc", 2, 500, 4, 64, 4, 64, 256, "f32", cplx=True, init=True, seed=98)
+    inp = inputs.scan_inputs(shape)
+    inp["A"] = torch.complex(-torch.linspace(40.0, 100.0, shape.nheads), inp["A"].imag).contiguous()
+    inp["dt"] = (inp["dt"] * 4.0).clamp(max=0.1).contiguous()
+    y, fs = gpu_scan(inp, shape.chunk, True)
+    assert torch.isfinite(y).all() and torch.isfinite(torch.view_as_real(fs)).all()
+    y_ref, fs_ref = oracle_scan(inp)
+    ey, ef = rel_err(y.numpy(), y_ref), rel_err(fs.numpy(), fs_ref)
+    assert ey <= TOL_F32 and ef <= TOL_F32, (ey, ef)
+
+
 # --------------------------------------------------------- full-size, sampled
 def _sampled(shape, samples, tol):
     inp = inputs.scan_inputs(shape)
