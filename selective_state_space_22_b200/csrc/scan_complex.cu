@@ -91,7 +91,9 @@ __device__ void chunk_log_decay(const ScanArgs &a, int b, int h, int c, float *d
 // ------------------------------------------------------------ 1. chunk state
 // S[p, n] = e^{i Theta} sum_s w_s x_s[p] B'_s[n],  w_s = exp(R - r_s) dt_s.
 // Block: one (batch, head, chunk) and a 64 x 128 tile of (p, interleaved n);
-// thread: 4 p x 8 interleaved values.
+// thread: 4 p x 8 interleaved values, columns 4 tj .. 4 tj + 3 and 64 + 4 tj ..
+// 64 + 4 tj + 3 (each 8-thread phase of a 128-bit shared load then reads 128
+// contiguous bytes: no bank conflict).
 __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w, int npt, int njt) {
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int c = blockIdx.x, h = blockIdx.y;
@@ -171,8 +173,8 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
 #pragma unroll 4
         for (int k = 0; k < KS; ++k) {
             const float4 xa = *reinterpret_cast<const float4 *>(Xw + k * TP + 4 * tp);
-            const float4 b0 = *reinterpret_cast<const float4 *>(Bt + k * TJ + 8 * tj);
-            const float4 b1 = *reinterpret_cast<const float4 *>(Bt + k * TJ + 8 * tj + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(Bt + k * TJ + 4 * tj);
+            const float4 b1 = *reinterpret_cast<const float4 *>(Bt + k * TJ + 64 + 4 * tj);
             const float av[4] = {xa.x, xa.y, xa.z, xa.w};
             const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
@@ -191,8 +193,8 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
         const int p = p0 + 4 * tp + i;
         if (p >= P) continue;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const int n = n0 + 4 * tj + m;
+        for (int m = 0; m < 4; ++m) {  // complex columns 2 tj, 2 tj + 1, 32 + 2 tj, 32 + 2 tj + 1
+            const int n = n0 + (m < 2 ? 2 * tj + m : 32 + 2 * tj + (m - 2));
             if (n >= N) continue;
             const float sr = acc[i][2 * m], si = acc[i][2 * m + 1];
             S[(size_t)p * N + n] = {er * sr - ei * si, er * si + ei * sr};
@@ -410,8 +412,15 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
 // The chunk scan for 2N <= 128: the rotated C of the block's 64 rows is staged
 // once, in full K, and reused by the off-diagonal product and every source tile;
 // each source tile stages its rotated B and x in one step.  Tiles in shared
-// memory are [k][64] with rows padded to LD floats.
+// memory are [k][64] with rows padded to LD floats; K holds the real parts in
+// rows 0-63 and the imaginary parts in rows 64-127 (zero past N).  A warp stages
+// 8 state indices x 4 tokens at a time, so its 32 stores fall in 32 banks.
 constexpr int LD = 68;
+__device__ __forceinline__ void stage_index(int i, int &m, int &c) {  // i in [0, 4096) -> (m, c)
+    const int lane = i & 31, blk = i >> 5;
+    m = (blk & 7) * 8 + (lane & 7);
+    c = (blk >> 3) * 4 + (lane >> 3);
+}
 __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, CWs w, int nrt, int npt) {
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int rt = blockIdx.x % nrt, c = blockIdx.x / nrt;
@@ -445,21 +454,23 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
     const cf *Cg = reinterpret_cast<const cf *>(a.C);
     const cf *Bg = reinterpret_cast<const cf *>(a.B);
     const float *xg = reinterpret_cast<const float *>(a.x);
-    constexpr int IT = 64 * 64 / NT;  // staged elements per thread (n fastest: coalesced reads)
+    constexpr int IT = 64 * 64 / NT;  // staged elements per thread
     {
         cf cv[IT];
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
-            const int i = threadIdx.x + it * NT, l = i / 64, m = i % 64;
+            int m, l;
+            stage_index(threadIdx.x + it * NT, m, l);
             cv[it] = (l < rows && m < N) ? Cg[(((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + m]
                                          : cf{0.f, 0.f};
         }
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
-            const int i = threadIdx.x + it * NT, l = i / 64, m = i % 64;
+            int m, l;
+            stage_index(threadIdx.x + it * NT, m, l);
             const float2 e = ph[l0 + l];
-            Ch[(2 * m) * LD + l] = cv[it].re * e.x - cv[it].im * e.y;
-            Ch[(2 * m + 1) * LD + l] = -(cv[it].re * e.y + cv[it].im * e.x);
+            Ch[m * LD + l] = cv[it].re * e.x - cv[it].im * e.y;
+            Ch[(64 + m) * LD + l] = -(cv[it].re * e.y + cv[it].im * e.x);
         }
     }
 
@@ -472,7 +483,7 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
     // acc(l, j) += sum_k Ch[k][l] T[k][j] over the 2N interleaved values
     auto gemm_k = [&](const float *T, float (&o)[4][4]) {
 #pragma unroll 4
-        for (int k = 0; k < 2 * N; ++k) {
+        for (int k = 0; k < 128; ++k) {
             const float4 av = *reinterpret_cast<const float4 *>(Ch + k * LD + 4 * li);
             const float4 bv = *reinterpret_cast<const float4 *>(T + k * LD + 4 * pi);
             const float aa[4] = {av.x, av.y, av.z, av.w}, bb[4] = {bv.x, bv.y, bv.z, bv.w};
@@ -489,14 +500,16 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
         cf hv[IT];
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
-            const int i = threadIdx.x + it * NT, p = i / 64, m = i % 64;
-            hv[it] = (p0 + p < P && m < N) ? hin[(size_t)(p0 + p) * N + m] : cf{0.f, 0.f};
+            int m, q;
+            stage_index(threadIdx.x + it * NT, m, q);
+            hv[it] = (p0 + q < P && m < N) ? hin[(size_t)(p0 + q) * N + m] : cf{0.f, 0.f};
         }
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
-            const int i = threadIdx.x + it * NT, p = i / 64, m = i % 64;
-            Bs[(2 * m) * LD + p] = hv[it].re;
-            Bs[(2 * m + 1) * LD + p] = hv[it].im;
+            int m, q;
+            stage_index(threadIdx.x + it * NT, m, q);
+            Bs[m * LD + q] = hv[it].re;
+            Bs[(64 + m) * LD + q] = hv[it].im;
         }
         __syncthreads();
         gemm_k(Bs, acc);
@@ -517,20 +530,23 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
             float xv[IT];
 #pragma unroll
             for (int it = 0; it < IT; ++it) {
-                const int i = threadIdx.x + it * NT, s = i / 64, m = i % 64;
-                bv[it] = (s0 + s < valid && m < N) ? Bg[(((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + m]
-                                                   : cf{0.f, 0.f};
-                const int p = i % TP;
+                int m, sb;
+                stage_index(threadIdx.x + it * NT, m, sb);
+                bv[it] = (s0 + sb < valid && m < N) ? Bg[(((size_t)b * a.seqlen + t0 + s0 + sb) * a.ngroups + g) * N + m]
+                                                    : cf{0.f, 0.f};
+                const int i = threadIdx.x + it * NT, s = i / TP, p = i % TP;  // x: p fastest
                 xv[it] = (s0 + s < valid && p0 + p < P) ? xg[(((size_t)b * a.seqlen + t0 + s0 + s) * H + h) * P + p0 + p]
                                                         : 0.f;
             }
 #pragma unroll
             for (int it = 0; it < IT; ++it) {
-                const int i = threadIdx.x + it * NT, s = i / 64, m = i % 64;
-                const float2 e = ph[s0 + s];  // rotate by e^{-i theta_s}
-                Bs[(2 * m) * LD + s] = bv[it].re * e.x + bv[it].im * e.y;
-                Bs[(2 * m + 1) * LD + s] = bv[it].im * e.x - bv[it].re * e.y;
-                Xs[s * LD + i % TP] = xv[it];
+                int m, sb;
+                stage_index(threadIdx.x + it * NT, m, sb);
+                const float2 e = ph[s0 + sb];  // rotate by e^{-i theta_s}
+                Bs[m * LD + sb] = bv[it].re * e.x + bv[it].im * e.y;
+                Bs[(64 + m) * LD + sb] = bv[it].im * e.x - bv[it].re * e.y;
+                const int i = threadIdx.x + it * NT;
+                Xs[(i / TP) * LD + i % TP] = xv[it];
             }
         }
         __syncthreads();
