@@ -170,7 +170,7 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
             }
         }
         __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
         for (int k = 0; k < KS; ++k) {
             const float4 xa = *reinterpret_cast<const float4 *>(Xw + k * TP + 4 * tp);
             const float4 b0 = *reinterpret_cast<const float4 *>(Bt + k * TJ + 4 * tj);
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
     // acc(l, j) += sum_k Ch[k][l] T[k][j] over the 2N interleaved values
     auto gemm_k = [&](const float *T, float (&o)[4][4]) {
-#pragma unroll 4
+#pragma unroll 8
         for (int k = 0; k < 128; ++k) {
             const float4 av = *reinterpret_cast<const float4 *>(Ch + k * LD + 4 * li);
             const float4 bv = *reinterpret_cast<const float4 *>(T + k * LD + 4 * pi);
@@ -568,7 +568,7 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
             }
         }
         __syncthreads();
-#pragma unroll 4
+#pragma unroll 8
         for (int s = 0; s < 64; ++s) {
             const float4 mv = *reinterpret_cast<const float4 *>(Ms + s * LD + 4 * li);
             const float4 xv = *reinterpret_cast<const float4 *>(Xs + s * LD + 4 * pi);
