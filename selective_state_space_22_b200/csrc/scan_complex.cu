@@ -556,16 +556,18 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
 #pragma unroll
             for (int j = 0; j < 4; ++j) gacc[i][j] = 0.f;
         gemm_k(Bs, gacc);
-        // M[l, s] = exp(r_l - r_s) dt_s Re(C'_l . B'_s), zero above the diagonal
+        // M[l, s] = exp(r_l - r_s) dt_s Re(C'_l . B'_s), zero above the diagonal;
+        // each source column's 4 rows go out as one float4
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int j = 0; j < 4; ++j) {
+            const int s = s0 + 4 * pi + j;
+            float m4[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int l = l0 + 4 * li + i, s = s0 + 4 * pi + j;
-                float m = 0.f;
-                if (s <= l && s < valid && l < valid) m = gacc[i][j] * expf(rr[l] - rr[s]) * dts[s];
-                Ms[(4 * pi + j) * LD + 4 * li + i] = m;
+            for (int i = 0; i < 4; ++i) {
+                const int l = l0 + 4 * li + i;
+                m4[i] = (s <= l && s < valid && l < valid) ? gacc[i][j] * expf(rr[l] - rr[s]) * dts[s] : 0.f;
             }
+            *reinterpret_cast<float4 *>(Ms + (4 * pi + j) * LD + 4 * li) = make_float4(m4[0], m4[1], m4[2], m4[3]);
         }
         __syncthreads();
 #pragma unroll 8
