@@ -123,7 +123,11 @@ ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A,
  *  final_state [batch, nheads, headdim, dstate] complex, or NULL
  *  y           [batch, seqlen, nheads, headdim] float32 = Re(h_t C_t) + D x_t
  *
- * Runs in float32 (complex64) throughout.  Other arguments as ssd_scan_fwd.
+ * Runs in float32 (complex64) throughout, on CUDA cores: three launches and a
+ * workspace (ssd_scan_workspace_size with is_complex = 1).  Each token's C and B
+ * are rotated by its cumulative phase, which leaves a real decay magnitude, so
+ * every contraction is a real float32 product over the 2 dstate interleaved
+ * values.  Other arguments as ssd_scan_fwd.
  */
 ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A,
                                 const float *B, const float *C, const float *D,
@@ -158,9 +162,10 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
 
 /*
  * Waits for `stream`, then reports and clears an error that a kernel raised on
- * the device since the last call on this device (SSD_ERR_TIMEOUT when a bounded
- * inter-block wait gave up; the outputs of that call are then invalid), or a
- * CUDA error from the stream.  SSD_OK when there was none.
+ * the device since the last call on this device (SSD_ERR_TIMEOUT when one of the
+ * tensor-core kernel's bounded waits between its warp roles gave up after 2 s;
+ * the outputs of that call are then invalid), or a CUDA error from the stream.
+ * SSD_OK when there was none.
  */
 ssd_status ssd_get_device_status(void *stream);
 

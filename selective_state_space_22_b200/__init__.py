@@ -21,7 +21,8 @@ import torch
 
 __all__ = ["SSDError", "ssd_scan_fwd", "ssd_scan_fwd_complex", "ssd_state_update",
            "ssd_state_update_complex", "ssd_scan_workspace_size", "ssd_scan_kernel_launches", "ssd_get_device_status",
-           "ssd_last_error", "ssd_version", "load_library", "LIB_PATH"]
+           "ssd_scan_fwd_noalloc", "ssd_last_error", "ssd_version", "load_library", "LIB_PATH",
+           "SSD_WORKSPACE_INVALID"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -65,6 +66,8 @@ def load_library(path: str | None = None):
         lib.ssd_state_update.restype = _I
         lib.ssd_state_update_complex.argtypes = [_VP] * 8 + [_I] * 5 + [_VP]
         lib.ssd_state_update_complex.restype = _I
+        lib.ssd_scan_fwd_noalloc.argtypes = [_VP] * 9 + [_I] * 8 + [_VP]
+        lib.ssd_scan_fwd_noalloc.restype = _I
         lib.ssd_get_device_status.argtypes = [_VP]
         lib.ssd_get_device_status.restype = _I
         lib.ssd_last_error.argtypes = []
@@ -182,6 +185,39 @@ def ssd_scan_fwd(x, dt, A, B, C, D=None, init_state=None, *, chunk_size=256, y=N
         st = lib.ssd_scan_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
                               _ptr(final_state), _ptr(y), io, b, T, H, P, G, N, chunk_size,
                               _ptr(ws), 0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st)
+    return y, final_state
+
+
+def ssd_scan_fwd_noalloc(x, dt, A, B, C, D=None, init_state=None, *, chunk_size=256, y=None,
+                         final_state=None, return_final_state=True, stream=None):
+    """Real scan with the library's fixed scratch array instead of a workspace
+    (float32 CUDA-core kernels; sizes whose scratch exceeds the array raise).
+    Same tensors and return value as ssd_scan_fwd."""
+    lib = load_library()
+    dev = x.device
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = {torch.bfloat16: SSD_BF16, torch.float32: SSD_F32}.get(x.dtype)
+    if io is None:
+        raise ValueError("x must be bfloat16 or float32")
+    _need(x, "x", x.dtype, dev)
+    _need(dt, "dt", torch.float32, dev, (b, T, H))
+    _need(A, "A", torch.float32, dev, (H,))
+    _need(B, "B", x.dtype, dev, (b, T, G, N))
+    _need(C, "C", x.dtype, dev, (b, T, G, N))
+    _need(D, "D", torch.float32, dev, (H,), allow_none=True)
+    _need(init_state, "init_state", torch.float32, dev, (b, H, P, N), allow_none=True)
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", x.dtype, dev, x.shape)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", torch.float32, dev, (b, H, P, N), allow_none=True)
+    with torch.cuda.device(dev):
+        st = lib.ssd_scan_fwd_noalloc(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                                      _ptr(final_state), _ptr(y), io, b, T, H, P, G, N, chunk_size,
+                                      _stream_handle(stream))
     _check(st)
     return y, final_state
 

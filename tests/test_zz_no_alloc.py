@@ -71,3 +71,16 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(lib):
                                   2, 65536, 64, 64, 1, 128, 256, None)
     assert st == ssd.SSD_ERR_WORKSPACE
     assert "scratch" in ssd.ssd_last_error()
+
+
+def test_noalloc_python_binding_matches_scan():
+    """The Python wrapper of the same name marshals the same call."""
+    shape = inputs.ScanShape("noalloc-py", 1, 200, 2, 64, 1, 128, 64, "f32", init_state=True, seed=92)
+    d = to_dev(inputs.scan_inputs(shape))
+    y_ref, fs_ref = ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                                     chunk_size=shape.chunk)
+    y, fs = ssd.ssd_scan_fwd_noalloc(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                                     chunk_size=shape.chunk)
+    ssd.ssd_get_device_status()
+    assert rel_err(y.cpu().numpy(), y_ref.cpu().numpy()) <= TOL_F32
+    assert rel_err(fs.cpu().numpy(), fs_ref.cpu().numpy()) <= TOL_F32
