@@ -35,6 +35,8 @@
 // cumulative decay and W of tile k, then y of tile k-1).  Hot loops are kept rolled: four roles share each SM sub-partition's
 // instruction cache.  Two input stages and two TMEM column
 // sets let consecutive tiles overlap; a set is released as soon as its y is out.
+// C h_in^T has its own columns, so it runs as soon as h_in^T is written and the
+// stage's C is free without waiting for the tile's state update.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -62,8 +64,9 @@ constexpr uint32_t BAR_MATH = 1;  // named barrier of the math warpgroup (128 th
 // TMEM: two column sets of 256 (consecutive tiles alternate).
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_G = 0;    // G (f32, 128 cols), then M (bf16 pairs) in columns 0-63
-constexpr uint32_t COL_YD = 128; // M X                                       (64 cols)
-constexpr uint32_t COL_S = 192;  // chunk state, then C h_in^T once it is read  (64 cols)
+constexpr uint32_t COL_YD = 64;  // M X, in G's second half once M is built   (64 cols)
+constexpr uint32_t COL_YO = 128; // C h_in^T                                  (64 cols)
+constexpr uint32_t COL_S = 192;  // chunk state                               (64 cols)
 
 // Shared memory: two input stages {C, B, X}; one W buffer; two h_in^T buffers.
 constexpr int STAGE_BYTES = 81920;
@@ -75,9 +78,11 @@ constexpr uint32_t LOAD_FULL = 2 * (QT * ND * 2) + QT * PD * 2;  // C, B, X
 constexpr uint32_t LOAD_STATE = QT * ND * 2 + QT * PD * 2;       // B, X
 enum {
     // count 1 (TMA bytes or an MMA commit)
+    // B_EMPTY: 2 (a commit from each MMA issuer)
     B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8,
     // count 128 (one warpgroup)
-    B_CS = 10, B_W = 12, B_M = 14, B_H = 16, B_FREE = 18, NBARS = 20
+    // B_HW: h_in^T written; B_H: chunk state read by the state update
+    B_CS = 10, B_W = 12, B_M = 14, B_H = 16, B_FREE = 18, B_HW = 20, NBARS = 22
 };
 // misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4], bars, tmem base
 constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + NBARS * 8 + 8;
@@ -263,7 +268,7 @@ __global__ void __launch_bounds__(NTH, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1) ? 2 : 1);
         for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
         fence_mbar_init();
     }
@@ -320,16 +325,19 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 mma_commit(&bars[B_G + s]);
                 mbar_wait(&bars[B_W + s], par, err);
+                // S's columns held the chunk state of tile k-2 until its state update
+                if (k >= 2) mbar_wait(&bars[B_H + s], par ^ 1, err);
                 tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)  // S = B^T W
                     mma_ss(tm + COL_S, smem_desc_sw128(aB + kk * 2048, 16384, 1024),
                            smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
                 mma_commit(&bars[B_S + s]);
+                mma_commit(&bars[B_EMPTY + s]);  // G and S are done with the stage's B and C
             }
         }
     } else if (warp == Y_MMA_WARP) {
-        // --------------------------------- MMA issuer: M X and C h_in^T
+        // --------------------------------- MMA issuer: C h_in^T and M X
         if (lane == 0) {
             for (int k = 0; k < ntl; ++k) {
                 const bool so = decode_tile(p, k).state_only;
@@ -337,27 +345,27 @@ __global__ void __launch_bounds__(NTH, 1)
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aX = sbase + s * STAGE_BYTES + OFF_X;
                 const uint32_t aH = sbase + OFF_H + s * 16384;
+                // G of this tile was issued after tile k-2's epilogue released the
+                // set, so C h^T's columns are free; h_in^T of this tile is written.
+                mbar_wait(&bars[B_G + s], par, err);
+                mbar_wait(&bars[B_HW + s], par, err);
+                tc_fence_after();
+                if (!so) {
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)  // Y_off = C h_in^T
+                        mma_ss(tm + COL_YO, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                               smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
+                }
                 mbar_wait(&bars[B_M + s], par, err);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)  // Y = M X
-                        mma_ts(tm + COL_YD, tm + COL_G + 8 * kk,
-                               smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_YD, kk > 0);
+                        mma_ts(tm + COL_YD, tm + COL_G + 8 * kk, smem_desc_sw128(aX + kk * 2048, 8192, 1024),
+                               IDESC_YD, kk > 0);
                 }
-                // h_in^T is written and the chunk state has been read out of COL_S
-                mbar_wait(&bars[B_H + s], par, err);
-                tc_fence_after();
-                if (!so) {
-#pragma unroll 1
-                    for (int kk = 0; kk < 8; ++kk)  // Y_off = C h_in^T
-                        mma_ss(tm + COL_S, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                               smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
-                }
-                // G and S of this tile completed before B_M and B_H could arrive, so
-                // once these commits fire the whole stage and TMEM set are read.
                 mma_commit(&bars[B_Y + s]);
-                mma_commit(&bars[B_EMPTY + s]);
+                mma_commit(&bars[B_EMPTY + s]);  // C h^T and M X are done with C and X
             }
         }
     } else if (warp < STATE_W0) {
@@ -419,6 +427,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 fence_proxy_async_smem();
             }
+            mbar_arrive(&bars[B_HW + s]);  // C h_in^T may go
             mbar_wait(&bars[B_S + s], par, err);
             tc_fence_after();
             {  // h_out = exp(lam) h_in + S, 32 columns at a time
@@ -432,7 +441,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars[B_H + s]);  // h_in^T written, chunk state read: C h_in^T may go
+            mbar_arrive(&bars[B_H + s]);  // chunk state read: S of tile k+2 may overwrite it
             if (t.c == p.nchunks - 1 && p.final_state) {
                 float *fin = p.final_state + (size_t)t.bh * PD * ND + row;
 #pragma unroll
@@ -520,7 +529,7 @@ __global__ void __launch_bounds__(NTH, 1)
 #pragma unroll 1
                     for (int half = 0; half < 2; ++half) {
                         uint32_t yd[32], yo[32];
-                        tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_S + 32 * half, yd, yo);
+                        tmem_ld32x2(tm + COL_YD + 32 * half, tm + COL_YO + 32 * half, yd, yo);
                         if (row < t.valid) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q) {
