@@ -69,20 +69,27 @@ constexpr uint32_t COL_YO = 128; // C h_in^T                                  (6
 constexpr uint32_t COL_S = 192;  // chunk state                               (64 cols)
 
 // Shared memory: two input stages {C, B, X}; one W buffer; two h_in^T buffers.
-constexpr int STAGE_BYTES = 81920;
-constexpr int OFF_C = 0, OFF_B = 32768, OFF_X = 65536;
-constexpr int OFF_W = 2 * STAGE_BYTES;
-constexpr int OFF_H = OFF_W + 16384;  // [2][16 KB]
-constexpr int OFF_MISC = OFF_H + 2 * 16384;
-constexpr uint32_t LOAD_FULL = 2 * (QT * ND * 2) + QT * PD * 2;  // C, B, X
-constexpr uint32_t LOAD_STATE = QT * ND * 2 + QT * PD * 2;       // B, X
+// C and B (released early, after G, S and C h^T) and X (released after W and
+// M X) live in separate rings: two {C, B} slots of 64 KB and three X slots of
+// 16 KB, so the loads of later tiles do not wait for this tile's M X.
+constexpr int CB_BYTES = 65536;
+constexpr int OFF_C = 0, OFF_B = 32768;           // within a {C, B} slot
+constexpr int OFF_XR = 2 * CB_BYTES;              // X ring [3][16 KB]
+constexpr int X_SLOTS = 3;
+constexpr int OFF_W = OFF_XR + X_SLOTS * 16384;
+constexpr int OFF_H = OFF_W + 16384;              // one h_in^T buffer
+constexpr int OFF_MISC = OFF_H + 16384;
+constexpr uint32_t LOAD_CB = 2 * (QT * ND * 2);   // C, B
+constexpr uint32_t LOAD_B = QT * ND * 2;          // B (state-only tiles)
+constexpr uint32_t LOAD_X = QT * PD * 2;
 enum {
-    // count 1 (TMA bytes or an MMA commit)
-    // B_EMPTY: 2 (a commit from each MMA issuer)
-    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8,
-    // count 128 (one warpgroup)
-    // B_HW: h_in^T written; B_H: chunk state read by the state update
-    B_CS = 10, B_W = 12, B_M = 14, B_H = 16, B_FREE = 18, B_HW = 20, NBARS = 22
+    // count 1 (TMA bytes or an MMA commit); B_EMPTY ({C, B} slot free): 2, a
+    // commit from each MMA issuer
+    B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8, B_YO = 10,
+    // the X ring; B_XEMPTY counts the 128 W threads and M X's commit
+    B_XFULL = 12, B_XEMPTY = 15,
+    // count 128 (one warpgroup).  B_HW: h_in^T written; B_H: chunk state read
+    B_CS = 18, B_W = 20, B_M = 22, B_H = 24, B_FREE = 26, B_HW = 28, NBARS = 30
 };
 // misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4], bars, tmem base
 constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + NBARS * 8 + 8;
@@ -268,7 +275,8 @@ __global__ void __launch_bounds__(NTH, 1)
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int i = 0; i < B_CS; ++i) mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1) ? 2 : 1);
+        for (int i = 0; i < B_CS; ++i)
+            mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1) ? 2 : (i >= B_XEMPTY && i < B_XEMPTY + 3) ? 129 : 1);
         for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
         fence_mbar_init();
     }
@@ -291,16 +299,19 @@ __global__ void __launch_bounds__(NTH, 1)
                 const Tile t = decode_tile(p, k);
                 const int s = k & 1;
                 mbar_wait(&bars[B_EMPTY + s], ((k >> 1) & 1) ^ 1, err);
-                uint8_t *st = sm + s * STAGE_BYTES;
+                uint8_t *st = sm + s * CB_BYTES;
                 uint64_t *full = &bars[B_FULL + s];
-                mbar_arrive_expect_tx(full, t.state_only ? LOAD_STATE : LOAD_FULL);
+                mbar_arrive_expect_tx(full, t.state_only ? LOAD_B : LOAD_CB);
                 if (!t.state_only) {
                     tma_load_4d(st + OFF_C, &tm_c, full, 0, t.g, t.t0, t.b);
                     tma_load_4d(st + OFF_C + 16384, &tm_c, full, 64, t.g, t.t0, t.b);
                 }
                 tma_load_4d(st + OFF_B, &tm_b, full, 0, t.g, t.t0, t.b);
                 tma_load_4d(st + OFF_B + 16384, &tm_b, full, 64, t.g, t.t0, t.b);
-                tma_load_4d(st + OFF_X, &tm_x, full, 0, t.h, t.t0, t.b);
+                const int xs = k % X_SLOTS;
+                mbar_wait(&bars[B_XEMPTY + xs], ((k / X_SLOTS) & 1) ^ 1, err);
+                mbar_arrive_expect_tx(&bars[B_XFULL + xs], LOAD_X);
+                tma_load_4d(sm + OFF_XR + xs * 16384, &tm_x, &bars[B_XFULL + xs], 0, t.h, t.t0, t.b);
             }
         }
     } else if (warp == 1) {
@@ -311,7 +322,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 const bool so = decode_tile(p, k).state_only;
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
-                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aB = sbase + s * STAGE_BYTES + OFF_B;
+                const uint32_t aC = sbase + s * CB_BYTES + OFF_C, aB = sbase + s * CB_BYTES + OFF_B;
                 mbar_wait(&bars[B_FULL + s], par, err);
                 mbar_wait(&bars[B_FREE + s], par ^ 1, err);
                 tc_fence_after();
@@ -343,8 +354,9 @@ __global__ void __launch_bounds__(NTH, 1)
                 const bool so = decode_tile(p, k).state_only;
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
-                const uint32_t aC = sbase + s * STAGE_BYTES + OFF_C, aX = sbase + s * STAGE_BYTES + OFF_X;
-                const uint32_t aH = sbase + OFF_H + s * 16384;
+                const int xs = k % X_SLOTS;
+                const uint32_t aC = sbase + s * CB_BYTES + OFF_C, aX = sbase + OFF_XR + xs * 16384;
+                const uint32_t aH = sbase + OFF_H;
                 // G of this tile was issued after tile k-2's epilogue released the
                 // set, so C h^T's columns are free; h_in^T of this tile is written.
                 mbar_wait(&bars[B_G + s], par, err);
@@ -356,7 +368,10 @@ __global__ void __launch_bounds__(NTH, 1)
                         mma_ss(tm + COL_YO, smem_desc_sw128(aC + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                                smem_desc_sw128(aH + kk * 2048, 8192, 1024), IDESC_YO, kk > 0);
                 }
+                mma_commit(&bars[B_YO + s]);     // done with the h_in^T buffer
+                mma_commit(&bars[B_EMPTY + s]);  // with G and S: done with the {C, B} slot
                 mbar_wait(&bars[B_M + s], par, err);
+                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, err);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(NTH, 1)
                                IDESC_YD, kk > 0);
                 }
                 mma_commit(&bars[B_Y + s]);
-                mma_commit(&bars[B_EMPTY + s]);  // C h^T and M X are done with C and X
+                mma_commit(&bars[B_XEMPTY + xs]);  // with the W threads: done with the X slot
             }
         }
     } else if (warp < STATE_W0) {
@@ -417,7 +432,9 @@ __global__ void __launch_bounds__(NTH, 1)
             }
             if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle); its buffer was
                                   // last read by the C h^T product of tile k-2
-                uint8_t *sh = sm + OFF_H + s * 16384;
+                // the one buffer was last read by C h^T of tile k-1
+                if (k > 0) mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, err);
+                uint8_t *sh = sm + OFF_H;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
                     const int phys = q ^ (row & 7);
@@ -502,20 +519,22 @@ __global__ void __launch_bounds__(NTH, 1)
                 named_bar_sync(BAR_MATH, 128);  // every row's decays written
                 mbar_arrive(&bars[B_CS + s]);
                 // W (one buffer): the previous tile's S must have read it
-                mbar_wait(&bars[B_FULL + s], par, err);
+                const int xs = k % X_SLOTS;
+                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, err);
                 if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
                 // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
                 // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
                 // SM sub-partition also builds the most M blocks, skips it and the warp
                 // of quadrant 0 (the fewest) takes those rows too.
                 auto w_row = [&](int r) {
-                    scale_row(sm + s * STAGE_BYTES + OFF_X + r * 128, sm + OFF_W + r * 128, r & 7,
+                    scale_row(sm + OFF_XR + xs * 16384 + r * 128, sm + OFF_W + r * 128, r & 7,
                               __float2bfloat162_rn(__expf(lam - csk[r]) * dtk[r]));
                 };
                 if (quad != 3) w_row(row);
                 if (quad == 0) w_row(96 + lane);
                 fence_proxy_async_smem();
                 mbar_arrive(&bars[B_W + s]);
+                mbar_arrive(&bars[B_XEMPTY + xs]);  // this thread is done reading the X slot
             }
             if (k > 0) {  // y of tile k-1
                 const int j = k - 1, s = j & 1;
