@@ -417,9 +417,6 @@ __global__ void __launch_bounds__(NTH, 1)
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
             mbar_wait(&bars[B_CS + s], par, err);
             const float lam = lam_s[s];
-            // G of this tile was issued after tile k-2's epilogue, so the C h^T
-            // product of tile k-2 is done with this tile's h_in^T buffer.
-            mbar_wait(&bars[B_G + s], par, err);
             if (t.c == 0) {
                 if (p.init_state) {
                     const float *h0 = p.init_state + (size_t)t.bh * PD * ND + row;
@@ -430,9 +427,9 @@ __global__ void __launch_bounds__(NTH, 1)
                     for (int q = 0; q < PD; ++q) h[q] = 0.f;
                 }
             }
-            if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle); its buffer was
-                                  // last read by the C h^T product of tile k-2
-                // the one buffer was last read by C h^T of tile k-1
+            if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle)
+                // the one buffer was last read by C h^T of tile k-1; waiting for
+                // that (and not for this tile's G) lets C h^T go as early as it can
                 if (k > 0) mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, err);
                 uint8_t *sh = sm + OFF_H;
 #pragma unroll
