@@ -62,6 +62,10 @@ def _declare(lib):
     for name in ("oracle_state_update_real", "oracle_state_update_complex"):
         getattr(lib, name).argtypes = upd_args
         getattr(lib, name).restype = ctypes.c_int
+    bwd_args = [_D] * 16 + [_L] * 6
+    for name in ("oracle_scan_bwd_real", "oracle_scan_bwd_complex"):
+        getattr(lib, name).argtypes = bwd_args
+        getattr(lib, name).restype = ctypes.c_int
     return lib
 
 
@@ -115,3 +119,30 @@ def state_update(state, x, dt, A, B, C, D=None, lib=None):
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return y, st
+
+
+def scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, lib=None):
+    """Gradients of L = sum <dy, y> + Re <dfinal, final_state> through the scan.
+
+    Same inputs as ``scan``; dy [b,T,H,P] float64, dfinal [b,H,P,N] (state
+    dtype) or None.  Returns a dict with dx, ddt, dA, dB, dC, dD and dinit,
+    shaped like x, dt, A, B, C, D [H] and the state.  For complex tensors the
+    gradient of z = u + iv is dL/du + i dL/dv.
+    """
+    lib = lib or load()
+    cplx = np.iscomplexobj(A)
+    sdt = np.complex128 if cplx else np.float64
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    out = dict(dx=np.zeros_like(x), ddt=np.zeros_like(dt), dA=np.zeros(H, sdt),
+               dB=np.zeros((b, T, G, N), sdt), dC=np.zeros((b, T, G, N), sdt),
+               dD=np.zeros(H, np.float64), dinit=np.zeros((b, H, P, N), sdt))
+    fn = lib.oracle_scan_bwd_complex if cplx else lib.oracle_scan_bwd_real
+    rc = fn(_ptr(x, np.float64), _ptr(dt, np.float64), _ptr(A, sdt), _ptr(B, sdt),
+            _ptr(C, sdt), _ptr(D, np.float64), _ptr(init_state, sdt), _ptr(dy, np.float64),
+            _ptr(dfinal, sdt), _ptr(out["dx"], np.float64), _ptr(out["ddt"], np.float64),
+            _ptr(out["dA"], sdt), _ptr(out["dB"], sdt), _ptr(out["dC"], sdt),
+            _ptr(out["dD"], np.float64), _ptr(out["dinit"], sdt), b, T, H, P, G, N)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out

@@ -40,6 +40,10 @@
  *   state [b][h][p][n] (complex: [b][h][p][n][2]), y [b][t][h][p].
  *
  * Every entry point returns 0 on success and -1 on an argument error.
+ *
+ * The gradient entry points (oracle_scan_bwd_*) at the end of the file are the
+ * plain adjoint of the same recurrence; their pins are central finite
+ * differences of the forward entry points.
  */
 #include <complex.h>
 #include <math.h>
@@ -220,5 +224,203 @@ int oracle_state_update_complex(double *state, const double *x, const double *dt
                 y[((size_t)b * nheads + h) * headdim + p] = creal(acc) + (D ? D[h] * xb[p] : 0.0);
             }
         }
+    return 0;
+}
+
+/*
+ * Gradients of the scan (reverse-mode, by the adjoint of the same sequential
+ * recurrence, step by step backwards in time).  The pages train through the
+ * scan: "Block Anatomy, Numerical Stability & Scaling", Numerical Stability
+ * section 5.3 (the backward differentiates the products of exp factors), and
+ * the "Mamba-3-Lite" README's test list (an autograd gradcheck of the kernel's
+ * backward).  They print no backward formula; this is the chain rule through
+ * the recurrence at the top of this file.  The loss is taken as
+ *
+ *   L = sum_t <dy_t, y_t> + Re <dfinal, h_{T-1}>
+ *
+ * so dy [b][t][h][p] and dfinal [b][h][p][n] (nullable: zero) are the upstream
+ * gradients.  Outputs: dx [b][t][h][p], ddt [b][t][h], dA [h], dB and dC
+ * [b][t][g][n] (summed over the heads of a group), dD [h] (nullable), dinit
+ * [b][h][p][n] (nullable).  For complex tensors the gradient of z = u + iv is
+ * dL/du + i dL/dv.
+ *
+ * With G_t the gradient of the state h_t, the backward step is
+ *   G_t  = dfinal (t = T-1, before the readout term) ;
+ *   G_t += conj(C_t) dy_t                                  (readout at step t)
+ *   dC_t += sum_p dy_t[p] conj(h_t[p])
+ *   r_p   = sum_n Re(conj(B_t[n]) G_t[p][n])               (grad of dt_t x_t[p])
+ *   dx_t  = dt_t r + D dy_t ;  dB_t += dt_t sum_p x_t[p] G_t[p]
+ *   g_a   = sum conj(h_{t-1}) G_t                          (grad of a_t = exp(dt_t A))
+ *   ddt_t = sum_p x_t[p] r_p + Re(g_a conj(A a_t)) ;  dA += dt_t conj(a_t) g_a
+ *   G_{t-1} = conj(a_t) G_t ;  dinit = G_{-1}
+ * which is the chain rule through h_t = a_t h_{t-1} + dt_t x_t B_t^T and
+ * y_t = Re(h_t C_t) + D x_t.  The forward states are kept (T+1 of them per
+ * (batch, head)), so this is for the small problems the tests use.
+ */
+int oracle_scan_bwd_real(const double *x, const double *dt, const double *A,
+                         const double *B, const double *C, const double *D,
+                         const double *init_state, const double *dy, const double *dfinal,
+                         double *dx, double *ddt, double *dA, double *dB, double *dC,
+                         double *dD, double *dinit, long batch, long seqlen, long nheads,
+                         long headdim, long ngroups, long dstate) {
+    if (bad_dims(batch, seqlen, nheads, headdim, ngroups, dstate)) return -1;
+    const long hpg = nheads / ngroups;
+    const size_t PN = (size_t)headdim * (size_t)dstate;
+    double *hist = (double *)malloc(sizeof(double) * PN * (size_t)(seqlen + 1));
+    double *Gs = (double *)malloc(sizeof(double) * PN);
+    if (!hist || !Gs) {
+        free(hist); free(Gs);
+        return -1;
+    }
+    memset(dA, 0, sizeof(double) * (size_t)nheads);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)nheads);
+    memset(dB, 0, sizeof(double) * (size_t)batch * seqlen * ngroups * dstate);
+    memset(dC, 0, sizeof(double) * (size_t)batch * seqlen * ngroups * dstate);
+
+    for (long b = 0; b < batch; ++b) {
+        for (long h = 0; h < nheads; ++h) {
+            const long g = h / hpg;
+            const size_t so = (size_t)(b * nheads + h) * PN;
+            /* forward again, keeping every state: hist[t+1] = h_t, hist[0] = h_{-1} */
+            for (size_t i = 0; i < PN; ++i) hist[i] = init_state ? init_state[so + i] : 0.0;
+            for (long t = 0; t < seqlen; ++t) {
+                const double d = dt[((size_t)b * seqlen + t) * nheads + h];
+                const double a = exp(d * A[h]);
+                const double *xt = x + (((size_t)b * seqlen + t) * nheads + h) * headdim;
+                const double *Bt = B + (((size_t)b * seqlen + t) * ngroups + g) * dstate;
+                const double *prev = hist + (size_t)t * PN;
+                double *cur = hist + (size_t)(t + 1) * PN;
+                for (long p = 0; p < headdim; ++p)
+                    for (long n = 0; n < dstate; ++n)
+                        cur[IDX2(p, n, dstate)] = a * prev[IDX2(p, n, dstate)] + d * xt[p] * Bt[n];
+            }
+            /* backward */
+            for (size_t i = 0; i < PN; ++i) Gs[i] = dfinal ? dfinal[so + i] : 0.0;
+            for (long t = seqlen - 1; t >= 0; --t) {
+                const size_t tb = (size_t)b * seqlen + t;
+                const double d = dt[tb * nheads + h];
+                const double a = exp(d * A[h]);
+                const double *xt = x + (tb * nheads + h) * headdim;
+                const double *dyt = dy + (tb * nheads + h) * headdim;
+                const double *Bt = B + (tb * ngroups + g) * dstate;
+                const double *Ct = C + (tb * ngroups + g) * dstate;
+                double *dBt = dB + (tb * ngroups + g) * dstate;
+                double *dCt = dC + (tb * ngroups + g) * dstate;
+                double *dxt = dx + (tb * nheads + h) * headdim;
+                const double *ht = hist + (size_t)(t + 1) * PN, *hp = hist + (size_t)t * PN;
+                for (long p = 0; p < headdim; ++p)
+                    for (long n = 0; n < dstate; ++n) {
+                        Gs[IDX2(p, n, dstate)] += Ct[n] * dyt[p]; /* readout of h_t */
+                        dCt[n] += dyt[p] * ht[IDX2(p, n, dstate)];
+                    }
+                double ga = 0.0, ddt_in = 0.0;
+                for (long p = 0; p < headdim; ++p) {
+                    double rp = 0.0;
+                    for (long n = 0; n < dstate; ++n) {
+                        rp += Bt[n] * Gs[IDX2(p, n, dstate)];
+                        dBt[n] += d * xt[p] * Gs[IDX2(p, n, dstate)];
+                        ga += hp[IDX2(p, n, dstate)] * Gs[IDX2(p, n, dstate)];
+                    }
+                    dxt[p] = d * rp + (D ? D[h] * dyt[p] : 0.0);
+                    ddt_in += xt[p] * rp;
+                    if (dD) dD[h] += dyt[p] * xt[p];
+                }
+                ddt[tb * nheads + h] = ddt_in + ga * A[h] * a; /* d a_t / d dt_t = A a_t */
+                dA[h] += ga * d * a;                          /* d a_t / d A = dt_t a_t */
+                for (size_t i = 0; i < PN; ++i) Gs[i] *= a;    /* gradient of h_{t-1} */
+            }
+            if (dinit)
+                for (size_t i = 0; i < PN; ++i) dinit[so + i] = Gs[i];
+        }
+    }
+    free(hist); free(Gs);
+    return 0;
+}
+
+int oracle_scan_bwd_complex(const double *x, const double *dt, const double *A,
+                            const double *B, const double *C, const double *D,
+                            const double *init_state, const double *dy, const double *dfinal,
+                            double *dx, double *ddt, double *dA, double *dB, double *dC,
+                            double *dD, double *dinit, long batch, long seqlen, long nheads,
+                            long headdim, long ngroups, long dstate) {
+    if (bad_dims(batch, seqlen, nheads, headdim, ngroups, dstate)) return -1;
+    const long hpg = nheads / ngroups;
+    const size_t PN = (size_t)headdim * (size_t)dstate;
+    const double complex *Ac = (const double complex *)A;
+    const double complex *Bc = (const double complex *)B;
+    const double complex *Cc = (const double complex *)C;
+    const double complex *H0 = (const double complex *)init_state;
+    const double complex *GF = (const double complex *)dfinal;
+    double complex *dAc = (double complex *)dA;
+    double complex *dBc = (double complex *)dB;
+    double complex *dCc = (double complex *)dC;
+    double complex *dH0 = (double complex *)dinit;
+    double complex *hist = (double complex *)malloc(sizeof(double complex) * PN * (size_t)(seqlen + 1));
+    double complex *Gs = (double complex *)malloc(sizeof(double complex) * PN);
+    if (!hist || !Gs) {
+        free(hist); free(Gs);
+        return -1;
+    }
+    memset(dA, 0, sizeof(double complex) * (size_t)nheads);
+    if (dD) memset(dD, 0, sizeof(double) * (size_t)nheads);
+    memset(dB, 0, sizeof(double complex) * (size_t)batch * seqlen * ngroups * dstate);
+    memset(dC, 0, sizeof(double complex) * (size_t)batch * seqlen * ngroups * dstate);
+
+    for (long b = 0; b < batch; ++b) {
+        for (long h = 0; h < nheads; ++h) {
+            const long g = h / hpg;
+            const size_t so = (size_t)(b * nheads + h) * PN;
+            for (size_t i = 0; i < PN; ++i) hist[i] = H0 ? H0[so + i] : 0.0;
+            for (long t = 0; t < seqlen; ++t) {
+                const double d = dt[((size_t)b * seqlen + t) * nheads + h];
+                const double complex a = cexp(d * Ac[h]); /* a_t, as in the forward scan */
+                const double *xt = x + (((size_t)b * seqlen + t) * nheads + h) * headdim;
+                const double complex *Bt = Bc + (((size_t)b * seqlen + t) * ngroups + g) * dstate;
+                const double complex *prev = hist + (size_t)t * PN;
+                double complex *cur = hist + (size_t)(t + 1) * PN;
+                for (long p = 0; p < headdim; ++p)
+                    for (long n = 0; n < dstate; ++n)
+                        cur[IDX2(p, n, dstate)] = a * prev[IDX2(p, n, dstate)] + (d * xt[p]) * Bt[n];
+            }
+            for (size_t i = 0; i < PN; ++i) Gs[i] = GF ? GF[so + i] : 0.0;
+            for (long t = seqlen - 1; t >= 0; --t) {
+                const size_t tb = (size_t)b * seqlen + t;
+                const double d = dt[tb * nheads + h];
+                const double complex a = cexp(d * Ac[h]); /* a_t again, going backwards */
+                const double *xt = x + (tb * nheads + h) * headdim;
+                const double *dyt = dy + (tb * nheads + h) * headdim;
+                const double complex *Bt = Bc + (tb * ngroups + g) * dstate;
+                const double complex *Ct = Cc + (tb * ngroups + g) * dstate;
+                double complex *dBt = dBc + (tb * ngroups + g) * dstate;
+                double complex *dCt = dCc + (tb * ngroups + g) * dstate;
+                double *dxt = dx + (tb * nheads + h) * headdim;
+                const double complex *ht = hist + (size_t)(t + 1) * PN, *hp = hist + (size_t)t * PN;
+                for (long p = 0; p < headdim; ++p)
+                    for (long n = 0; n < dstate; ++n) {
+                        Gs[IDX2(p, n, dstate)] += conj(Ct[n]) * dyt[p]; /* readout Re(C h) */
+                        dCt[n] += dyt[p] * conj(ht[IDX2(p, n, dstate)]);
+                    }
+                double complex ga = 0.0;
+                double ddt_in = 0.0;
+                for (long p = 0; p < headdim; ++p) {
+                    double rp = 0.0;
+                    for (long n = 0; n < dstate; ++n) {
+                        rp += creal(conj(Bt[n]) * Gs[IDX2(p, n, dstate)]);
+                        dBt[n] += (d * xt[p]) * Gs[IDX2(p, n, dstate)];
+                        ga += conj(hp[IDX2(p, n, dstate)]) * Gs[IDX2(p, n, dstate)];
+                    }
+                    dxt[p] = d * rp + (D ? D[h] * dyt[p] : 0.0);
+                    ddt_in += xt[p] * rp;
+                    if (dD) dD[h] += dyt[p] * xt[p];
+                }
+                ddt[tb * nheads + h] = ddt_in + creal(ga * conj(Ac[h] * a));
+                dAc[h] += d * conj(a) * ga;
+                for (size_t i = 0; i < PN; ++i) Gs[i] *= conj(a);
+            }
+            if (dH0)
+                for (size_t i = 0; i < PN; ++i) dH0[so + i] = Gs[i];
+        }
+    }
+    free(hist); free(Gs);
     return 0;
 }

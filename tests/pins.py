@@ -295,8 +295,80 @@ def pin_complex_is_rotation_block(lib, seed=10):
     return err
 
 
+def _loss(lib, p, dy, dfinal):
+    y, fs = run(lib, p)
+    return float(np.sum(y * dy)) + float(np.real(np.sum(np.conj(dfinal) * fs)))
+
+
+def _dot(g, v) -> float:
+    """<g, v> over the real parameters: sum Re(conj(g) v)."""
+    return float(np.real(np.sum(np.conj(g) * v)))
+
+
+def pin_gradient_finite_difference(lib, cplx=False, seed=11):
+    """The adjoint (oracle scan_bwd) against central differences of the forward
+    oracle, one random direction per input.  The scan is affine in x, B, C, D and
+    h0 along any one of them, so there the difference quotient is exact up to
+    rounding; dt and A enter through exp, so theirs is Richardson-extrapolated
+    (error O(eps^4)).  dt moves by a relative step so it stays positive.  The
+    error is taken relative to |g| |v|, the bound on the directional derivative,
+    so a direction along which the loss barely moves is not a false alarm."""
+    rng = np.random.default_rng(seed)
+    err = 0.0
+    for (b, T, H, P, G, N) in [(2, 7, 4, 3, 2, 5), (1, 13, 2, 2, 1, 3), (1, 4, 1, 2, 1, 2)]:
+        p = rand_problem(rng, b, T, H, P, G, N, cplx=cplx, init=True, a_range=(0.5, 4.0))
+        dy = rng.standard_normal((b, T, H, P))
+        shp = (b, H, P, N)
+        dfin = rng.standard_normal(shp) + (1j * rng.standard_normal(shp) if cplx else 0)
+        dfin = np.ascontiguousarray(dfin)
+        g = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"], dy, dfin,
+                            lib=lib)
+        for name, gname, exact in [("x", "dx", True), ("B", "dB", True), ("C", "dC", True), ("D", "dD", True),
+                                   ("init_state", "dinit", True), ("dt", "ddt", False), ("A", "dA", False)]:
+            base = p[name]
+            v = rng.standard_normal(base.shape)
+            if np.iscomplexobj(base):
+                v = v + 1j * rng.standard_normal(base.shape)
+            if name == "dt":
+                v = base * rng.uniform(-1.0, 1.0, base.shape)
+
+            def diff(eps):
+                up = _loss(lib, dict(p, **{name: np.ascontiguousarray(base + eps * v)}), dy, dfin)
+                dn = _loss(lib, dict(p, **{name: np.ascontiguousarray(base - eps * v)}), dy, dfin)
+                return (up - dn) / (2 * eps)
+
+            if exact:
+                fd = diff(1e-2)
+            else:
+                eps = 1e-2
+                fd = (4 * diff(eps / 2) - diff(eps)) / 3
+            an = _dot(g[gname], v)
+            # relative to |g| |v|, the largest the directional derivative can be
+            scale = float(np.linalg.norm(g[gname]) * np.linalg.norm(v))
+            err = max(err, abs(fd - an) / max(scale, 1e-300))
+    return err
+
+
+def pin_gradient_empty_and_dfinal(lib, cplx=False, seed=12):
+    """T = 0: every gradient is zero except dinit = dfinal.  And with dy = 0 and
+    a single step, dinit = conj(exp(dt A)) dfinal exactly (the state only decays)."""
+    rng = np.random.default_rng(seed)
+    p = rand_problem(rng, 1, 0, 2, 2, 1, 3, cplx=cplx, init=True)
+    shp = (1, 2, 2, 3)
+    dfin = np.ascontiguousarray(rng.standard_normal(shp) + (1j * rng.standard_normal(shp) if cplx else 0))
+    g = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"],
+                        np.zeros((1, 0, 2, 2)), dfin, lib=lib)
+    err = rel_err(g["dinit"], dfin) + float(np.max(np.abs(g["dA"]))) + float(np.max(np.abs(g["dD"])))
+    p = rand_problem(rng, 1, 1, 2, 2, 1, 3, cplx=cplx, init=True)
+    g = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"],
+                        np.zeros((1, 1, 2, 2)), dfin, lib=lib)
+    a = np.exp(p["dt"][0, 0, :] * p["A"])  # per head
+    return err + rel_err(g["dinit"], np.conj(a)[None, :, None, None] * dfin)
+
+
 REAL_PINS = [pin_brute_force, pin_chunkwise, pin_zero_input, pin_prefix_sum, pin_linearity,
-             pin_continuation, pin_decode_equals_scan, pin_contraction]
+             pin_continuation, pin_decode_equals_scan, pin_contraction,
+             pin_gradient_finite_difference, pin_gradient_empty_and_dfinal]
 COMPLEX_ONLY_PINS = [pin_complex_zero_imag_is_real, pin_complex_is_rotation_block]
 
 

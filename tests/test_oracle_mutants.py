@@ -34,6 +34,20 @@ MUTANTS = {
     "decode_no_dt": ("Sp[n] = a * Sp[n] + d * xb[p] * Bb[n];", "Sp[n] = a * Sp[n] + xb[p] * Bb[n];"),
     "decode_complex_no_decay": ("Sp[n] = a * Sp[n] + (d * xb[p]) * Bb[n];",
                                 "Sp[n] = Sp[n] + (d * xb[p]) * Bb[n];"),
+    # the adjoint (gradient) oracle
+    "bwd_ddt_no_decay_term": ("ddt[tb * nheads + h] = ddt_in + ga * A[h] * a;", "ddt[tb * nheads + h] = ddt_in;"),
+    "bwd_dA_no_dt": ("dA[h] += ga * d * a;", "dA[h] += ga * a;"),
+    "bwd_adjoint_not_decayed": ("Gs[i] *= a;    /* gradient", "Gs[i] *= 1.0;    /* gradient"),
+    "bwd_dC_previous_state": ("dCt[n] += dyt[p] * ht[IDX2(p, n, dstate)];", "dCt[n] += dyt[p] * hp[IDX2(p, n, dstate)];"),
+    "bwd_dB_overwritten": ("dBt[n] += d * xt[p] * Gs[IDX2(p, n, dstate)];", "dBt[n] = d * xt[p] * Gs[IDX2(p, n, dstate)];"),
+    "bwd_complex_decay_not_conjugated": ("Gs[i] *= conj(a);", "Gs[i] *= a;"),
+    "bwd_complex_dA_not_conjugated": ("dAc[h] += d * conj(a) * ga;", "dAc[h] += d * a * ga;"),
+    "bwd_complex_dC_not_conjugated": ("dCt[n] += dyt[p] * conj(ht[IDX2(p, n, dstate)]);",
+                                      "dCt[n] += dyt[p] * ht[IDX2(p, n, dstate)];"),
+    "bwd_complex_readout_not_conjugated": ("Gs[IDX2(p, n, dstate)] += conj(Ct[n]) * dyt[p];",
+                                           "Gs[IDX2(p, n, dstate)] += Ct[n] * dyt[p];"),
+    "bwd_complex_ddt_imag_part": ("creal(ga * conj(Ac[h] * a))", "cimag(ga * conj(Ac[h] * a))"),
+    "bwd_complex_input_grad_imag_part": ("rp += creal(conj(Bt[n]) * Gs", "rp += cimag(conj(Bt[n]) * Gs"),
 }
 
 
