@@ -366,9 +366,103 @@ def pin_gradient_empty_and_dfinal(lib, cplx=False, seed=12):
     return err + rel_err(g["dinit"], np.conj(a)[None, :, None, None] * dfin)
 
 
+def chunked_gradients(p, dy, dfinal, Q):
+    """The gradient of L = sum <dy, y> + Re <dfinal, final> evaluated chunk by
+    chunk, the way a chunked kernel does it (written independently of the
+    sequential adjoint).  Per (batch, head) and chunk, with acs the inclusive
+    within-chunk cumulative sum of dt A, Lam = acs[-1], Lm[l, s] = exp(acs[l] -
+    acs[s]) for l >= s, Gm = C B^T, w_s = exp(Lam - acs[s]) dt_s and Gh the
+    gradient of the chunk's final state:
+      dX  = Re(Mc^T dY) + D dY + Re(conj(w) (conj(B) Gh^T)),  Mc = Gm o Lm o dt
+      dC  = conj((Lm o dt o dY X^T) B + e^{acs} (dY h_in))
+      dB  = conj((Lm o dt o dY X^T)^T C) + conj(w) (X Gh)
+      dh_in = conj(e^{Lam}) Gh + (conj(e^{acs}) dY)^T conj(C)   (Gh of the chunk before)
+    and the decay gradient through acs: with E = Gm o Lm o dt o (dY X^T),
+    dacs = conj(rowsum E - colsum E) + conj(e^{acs} dY.(h_in C)) and, from the
+    final state, conj(H0 + sum K) at the last token and -conj(K_s) at each s;
+    d alpha is the reverse cumulative sum of dacs, ddt += Re(conj(d alpha) A),
+    dA += sum dt d alpha."""
+    x, dt, A, B, C, D, h0 = p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"]
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    cplx = np.iscomplexobj(A)
+    sdt = np.complex128 if cplx else np.float64
+    re = (lambda z: np.real(z)) if cplx else (lambda z: z)
+    Dv = np.zeros(H) if D is None else D
+    out = dict(dx=np.zeros_like(x), ddt=np.zeros_like(dt), dA=np.zeros(H, sdt), dB=np.zeros((b, T, G, N), sdt),
+               dC=np.zeros((b, T, G, N), sdt), dD=np.zeros(H), dinit=np.zeros((b, H, P, N), sdt))
+    hpg = H // G
+    for bi in range(b):
+        for h in range(H):
+            g = h // hpg
+            chunks = [(c0, min(c0 + Q, T)) for c0 in range(0, T, Q)]
+            # forward over chunks: the state entering each chunk
+            hin = []
+            hs = np.zeros((P, N), sdt) if h0 is None else h0[bi, h].astype(sdt)
+            for c0, c1 in chunks:
+                hin.append(hs)
+                d = dt[bi, c0:c1, h]
+                acs = np.cumsum(d * A[h])
+                w = np.exp(acs[-1] - acs) * d
+                hs = np.exp(acs[-1]) * hs + (w[:, None] * x[bi, c0:c1, h]).T @ B[bi, c0:c1, g]
+            Gh = np.zeros((P, N), sdt) if dfinal is None else dfinal[bi, h].astype(sdt)
+            for ci in range(len(chunks) - 1, -1, -1):
+                c0, c1 = chunks[ci]
+                d = dt[bi, c0:c1, h]
+                X, dY = x[bi, c0:c1, h], dy[bi, c0:c1, h]
+                Bc, Cc, hi = B[bi, c0:c1, g], C[bi, c0:c1, g], hin[ci]
+                acs = np.cumsum(d * A[h])
+                lam = acs[-1]
+                Lm = np.tril(np.exp(acs[:, None] - acs[None, :]))
+                Gm = Cc @ Bc.T
+                w = np.exp(lam - acs) * d
+                XdY = dY @ X.T  # [l, s] = dy_l . x_s
+                Mc = Gm * Lm * d[None, :]
+                out["dx"][bi, c0:c1, h] = re(Mc.T @ dY) + Dv[h] * dY + re(np.conj(w)[:, None] * (np.conj(Bc) @ Gh.T))
+                out["dD"][h] += float(np.sum(dY * X))
+                K = Lm * d[None, :] * XdY
+                eacs = np.exp(acs)
+                out["dC"][bi, c0:c1, g] += np.conj(K @ Bc + eacs[:, None] * (dY @ hi))
+                out["dB"][bi, c0:c1, g] += np.conj(K.T @ Cc) + np.conj(w)[:, None] * (X @ Gh)
+                # dt where it multiplies directly (not through the decay)
+                ddt_dir = re(np.sum(Gm * Lm * XdY, axis=0)) + re(np.exp(lam - acs) * np.einsum(
+                    "sp,pn,sn->s", X, np.conj(Gh), Bc))
+                # decay: gradient with respect to acs, then alpha = dt A
+                E = Gm * Lm * d[None, :] * XdY
+                F = eacs * np.einsum("lp,pn,ln->l", dY, hi, Cc)
+                Ks = w * np.einsum("sp,pn,sn->s", X, np.conj(Gh), Bc)
+                H0 = np.exp(lam) * np.sum(np.conj(Gh) * hi)
+                dacs = np.conj(E.sum(axis=1) - E.sum(axis=0)) + np.conj(F) - np.conj(Ks)
+                dacs[-1] += np.conj(H0 + Ks.sum())
+                dalpha = np.cumsum(dacs[::-1])[::-1]
+                out["ddt"][bi, c0:c1, h] = ddt_dir + re(np.conj(dalpha) * A[h])
+                out["dA"][h] += np.sum(d * dalpha)
+                Gh = np.conj(np.exp(lam)) * Gh + (np.conj(eacs)[:, None] * dY).T @ np.conj(Cc)
+            out["dinit"][bi, h] = Gh
+    return out
+
+
+def pin_gradient_chunkwise(lib, cplx=False, seed=13):
+    """The sequential adjoint equals the chunked gradient above for several chunk
+    sizes (1, ragged, one chunk, larger than T)."""
+    rng = np.random.default_rng(seed)
+    err = 0.0
+    for (b, T, H, P, G, N, Qs) in [(2, 23, 4, 3, 2, 5, (1, 4, 7, 23, 40)), (1, 9, 2, 2, 1, 3, (2, 9))]:
+        p = rand_problem(rng, b, T, H, P, G, N, cplx=cplx, init=True)
+        dy = rng.standard_normal((b, T, H, P))
+        shp = (b, H, P, N)
+        dfin = np.ascontiguousarray(rng.standard_normal(shp) + (1j * rng.standard_normal(shp) if cplx else 0))
+        ref = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"], dy, dfin, lib=lib)
+        for Q in Qs:
+            got = chunked_gradients(p, dy, dfin, Q)
+            for k in ref:
+                err = max(err, rel_err(got[k], ref[k]))
+    return err
+
+
 REAL_PINS = [pin_brute_force, pin_chunkwise, pin_zero_input, pin_prefix_sum, pin_linearity,
              pin_continuation, pin_decode_equals_scan, pin_contraction,
-             pin_gradient_finite_difference, pin_gradient_empty_and_dfinal]
+             pin_gradient_finite_difference, pin_gradient_empty_and_dfinal, pin_gradient_chunkwise]
 COMPLEX_ONLY_PINS = [pin_complex_zero_imag_is_real, pin_complex_is_rotation_block]
 
 
