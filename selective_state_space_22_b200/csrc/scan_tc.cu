@@ -32,11 +32,12 @@
 // Warp roles (15 warps): 0 TMA producer; 1 MMA issuer for G and S; 14 MMA
 // issuer for the two products of y; 2-5 "math" warpgroup (M); 6-9 "state"
 // warpgroup (h_in^T, the state update); 10-13 "prep/epilogue" warpgroup (the
-// cumulative decay and W of tile k, then y of tile k-1).  Hot loops are kept rolled: four roles share each SM sub-partition's
-// instruction cache.  Two input stages and two TMEM column
-// sets let consecutive tiles overlap; a set is released as soon as its y is out.
-// C h_in^T has its own columns, so it runs as soon as h_in^T is written and the
-// stage's C is free without waiting for the tile's state update.
+// cumulative decay and W of tile k, then y of tile k-1).  Hot loops are kept
+// rolled: four roles share each SM sub-partition's instruction cache.  Two
+// {C, B} slots, three X slots and two TMEM column sets let consecutive tiles
+// overlap; a column set is released as soon as its y is out.  C h_in^T has its
+// own columns, so it runs as soon as h_in^T is written, without waiting for the
+// tile's state update.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -68,10 +69,10 @@ constexpr uint32_t COL_YD = 64;  // M X, in G's second half once M is built   (6
 constexpr uint32_t COL_YO = 128; // C h_in^T                                  (64 cols)
 constexpr uint32_t COL_S = 192;  // chunk state                               (64 cols)
 
-// Shared memory: two input stages {C, B, X}; one W buffer; two h_in^T buffers.
-// C and B (released early, after G, S and C h^T) and X (released after W and
-// M X) live in separate rings: two {C, B} slots of 64 KB and three X slots of
-// 16 KB, so the loads of later tiles do not wait for this tile's M X.
+// Shared memory: C and B (released after G, S and C h^T) and X (released after W
+// and M X) live in separate rings, two {C, B} slots of 64 KB and three X slots
+// of 16 KB, so the loads of later tiles do not wait for this tile's M X; then
+// one W buffer and one h_in^T buffer.
 constexpr int CB_BYTES = 65536;
 constexpr int OFF_C = 0, OFF_B = 32768;           // within a {C, B} slot
 constexpr int OFF_XR = 2 * CB_BYTES;              // X ring [3][16 KB]
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(NTH, 1)
                     mma_ss(tm + COL_S, smem_desc_sw128(aB + kk * 2048, 16384, 1024),
                            smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
                 mma_commit(&bars[B_S + s]);
-                mma_commit(&bars[B_EMPTY + s]);  // G and S are done with the stage's B and C
+                mma_commit(&bars[B_EMPTY + s]);  // G and S are done with the slot's B and C
             }
         }
     } else if (warp == Y_MMA_WARP) {
@@ -493,7 +494,6 @@ __global__ void __launch_bounds__(NTH, 1)
                     Dn = p.D ? p.D[tn.h] : 0.f;
                 }
                 const int s = k & 1;
-                const uint32_t par = (k >> 1) & 1;
                 float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
                 float v = d * Ah;  // inclusive cumsum of dt*A over the chunk
 #pragma unroll
