@@ -161,6 +161,47 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
                                     int headdim, int ngroups, int dstate, void *stream);
 
 /*
+ * Gradients of the real scan, float32, for training through it.
+ *
+ * The loss is L = sum_t <dy_t, y_t> + <dfinal, final_state>: dy and dfinal are
+ * the gradients arriving at the outputs y and final_state of ssd_scan_fwd.  The
+ * pages train through the scan ("Block Anatomy, Numerical Stability & Scaling",
+ * Numerical Stability section 5.3: the backward differentiates the products of
+ * the exp factors) but print no backward formula; this is the chain rule through
+ * the recurrence above, evaluated in 64-token chunks.
+ *
+ * Inputs (float32, as ssd_scan_fwd with io_dtype SSD_F32):
+ *  x [batch, seqlen, nheads, headdim], dt [batch, seqlen, nheads], A [nheads],
+ *  B, C [batch, seqlen, ngroups, dstate], D [nheads] or NULL,
+ *  init_state [batch, nheads, headdim, dstate] or NULL (zeros),
+ *  dy [batch, seqlen, nheads, headdim], dfinal [batch, nheads, headdim, dstate]
+ *  or NULL (zeros).
+ * Outputs (float32, every element written):
+ *  dx, ddt, dA [nheads], dB and dC [batch, seqlen, ngroups, dstate] (summed over
+ *  the heads of each group), dD [nheads] or NULL (not computed),
+ *  dinit [batch, nheads, headdim, dstate] or NULL (not computed).  dD is the
+ *  gradient for D whether or not D was given.
+ *
+ * Limits: headdim <= 64 and dstate <= 128 (SSD_ERR_UNSUPPORTED otherwise).  Runs
+ * on CUDA cores in six launches.  Sums are taken in a fixed order, so repeated
+ * calls give identical bits.  The workspace (ssd_scan_bwd_workspace_size bytes,
+ * caller-owned, 16-byte aligned, no initialisation needed) holds the chunk
+ * states, the state gradients and per-head partial sums; it grows with
+ * batch * nheads * ceil(seqlen / 64) * headdim * dstate * 12 bytes plus
+ * batch * seqlen * nheads * dstate * 8 bytes.  SSD_ERR_WORKSPACE when it is NULL
+ * or too small.
+ */
+size_t ssd_scan_bwd_workspace_size(int batch, int seqlen, int nheads, int headdim,
+                                   int ngroups, int dstate);
+
+ssd_status ssd_scan_bwd(const float *x, const float *dt, const float *A, const float *B,
+                        const float *C, const float *D, const float *init_state,
+                        const float *dy, const float *dfinal, float *dx, float *ddt,
+                        float *dA, float *dB, float *dC, float *dD, float *dinit,
+                        int batch, int seqlen, int nheads, int headdim, int ngroups,
+                        int dstate, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Waits for `stream`, then reports and clears an error that a kernel raised on
  * the device since the last call on this device (SSD_ERR_TIMEOUT when one of the
  * tensor-core kernel's bounded waits between its warp roles gave up after 2 s;

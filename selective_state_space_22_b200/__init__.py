@@ -22,7 +22,7 @@ import torch
 __all__ = ["SSDError", "ssd_scan_fwd", "ssd_scan_fwd_complex", "ssd_state_update",
            "ssd_state_update_complex", "ssd_scan_workspace_size", "ssd_scan_kernel_launches", "ssd_get_device_status",
            "ssd_scan_fwd_noalloc", "ssd_last_error", "ssd_version", "load_library", "LIB_PATH",
-           "SSD_WORKSPACE_INVALID"]
+           "SSD_WORKSPACE_INVALID", "ssd_scan_bwd", "ssd_scan_bwd_workspace_size"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -68,6 +68,10 @@ def load_library(path: str | None = None):
         lib.ssd_state_update_complex.restype = _I
         lib.ssd_scan_fwd_noalloc.argtypes = [_VP] * 9 + [_I] * 8 + [_VP]
         lib.ssd_scan_fwd_noalloc.restype = _I
+        lib.ssd_scan_bwd_workspace_size.argtypes = [_I] * 6
+        lib.ssd_scan_bwd_workspace_size.restype = _SZ
+        lib.ssd_scan_bwd.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, _SZ, _VP]
+        lib.ssd_scan_bwd.restype = _I
         lib.ssd_get_device_status.argtypes = [_VP]
         lib.ssd_get_device_status.restype = _I
         lib.ssd_last_error.argtypes = []
@@ -304,6 +308,47 @@ def ssd_state_update_complex(state, x, dt, A, B, C, D=None, *, y=None, stream=No
                                           _ptr(D), _ptr(y), b, H, P, G, N, _stream_handle(stream))
     _check(st)
     return y
+
+
+def ssd_scan_bwd_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate) -> int:
+    n = load_library().ssd_scan_bwd_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate)
+    if n == SSD_WORKSPACE_INVALID:
+        raise SSDError(1, "invalid sizes for the backward scan")
+    return n
+
+
+def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=None, stream=None):
+    """Gradients of L = sum <dy, y> + <dfinal, final_state> through the real
+    float32 scan.  Returns a dict with dx, ddt, dA, dB, dC, dD and dinit (dD is
+    None when D is None)."""
+    lib = load_library()
+    dev = x.device
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    f = torch.float32
+    _need(x, "x", f, dev)
+    _need(dt, "dt", f, dev, (b, T, H))
+    _need(A, "A", f, dev, (H,))
+    _need(B, "B", f, dev, (b, T, G, N))
+    _need(C, "C", f, dev, (b, T, G, N))
+    _need(D, "D", f, dev, (H,), allow_none=True)
+    _need(init_state, "init_state", f, dev, (b, H, P, N), allow_none=True)
+    _need(dy, "dy", f, dev, (b, T, H, P))
+    _need(dfinal, "dfinal", f, dev, (b, H, P, N), allow_none=True)
+    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt), dA=torch.empty_like(A),
+               dB=torch.empty_like(B), dC=torch.empty_like(C),
+               dD=None if D is None else torch.empty_like(D),
+               dinit=torch.empty((b, H, P, N), dtype=f, device=dev))
+    nbytes = ssd_scan_bwd_workspace_size(b, T, H, P, G, N)
+    ws = workspace if workspace is not None else _workspace(dev, nbytes)
+    with torch.cuda.device(dev):
+        st = lib.ssd_scan_bwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                              _ptr(dy), _ptr(dfinal), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
+                              _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dinit"]),
+                              b, T, H, P, G, N, _ptr(ws), 0 if ws is None else ws.numel(),
+                              _stream_handle(stream))
+    _check(st)
+    return out
 
 
 def ssd_get_device_status(stream=None) -> None:

@@ -1,0 +1,124 @@
+// scan_bwd.cu -- gradients of the real scan on CUDA cores (fp32), chunk by chunk.
+//
+// The arithmetic is in scan_bwd_body.cuh; this file only launches it.  Six
+// kernels run on the caller's stream:
+//   1. chunk states S_c and the within-chunk cumulative decay      grid (chunks, heads, batch)
+//   2. the state entering each chunk, h_in (a forward pass over chunks)   grid (heads, batch)
+//   3. the readout terms R_c = sum_l exp(acs[l]) dy_l C_l^T         grid (chunks, heads, batch)
+//   4. the gradient of the state leaving each chunk (a backward pass over
+//      chunks), and dinit                                            grid (heads, batch)
+//   5. dx, ddt and each head's dB, dC, dA, dD parts of one chunk    grid (chunks, heads, batch)
+//   6. dB, dC summed over the heads of a group; dA, dD over batch and chunks
+// Sums run in a fixed order, so repeated calls give identical bits.
+#include "scan_bwd_body.cuh"
+#include "ssd_internal.cuh"
+
+namespace ssd {
+namespace {
+
+using namespace bwd;
+
+constexpr size_t SMEM_BYTES = SMEM_FLOATS * sizeof(float);
+
+__global__ void __launch_bounds__(NT) bwd_chunk_state(BwdArgs a) {
+    extern __shared__ float sm[];
+    const Smem m = smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    k1_load(a, c, h, b, tid, m);
+    __syncthreads();
+    k1_cumsum(a, c, h, b, tid, m);
+    __syncthreads();
+    k1_state(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(NT) bwd_state_fwd(BwdArgs a) { k2_pass(a, blockIdx.x, blockIdx.y, threadIdx.x); }
+
+__global__ void __launch_bounds__(NT) bwd_readout(BwdArgs a) {
+    extern __shared__ float sm[];
+    const Smem m = smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    k3_load(a, c, h, b, tid, m);
+    __syncthreads();
+    k3_r(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(NT) bwd_state_bwd(BwdArgs a) { k4_pass(a, blockIdx.x, blockIdx.y, threadIdx.x); }
+
+__global__ void __launch_bounds__(NT) bwd_chunk_grad(BwdArgs a) {
+    extern __shared__ float sm[];
+    const Smem m = smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    k5_load(a, c, h, b, tid, m);
+    __syncthreads();
+    k5_mats(a, tid, m);
+    __syncthreads();
+    k5_tokens(a, tid, m);
+    __syncthreads();
+    k5_decay(a, c, h, b, tid, m);
+    __syncthreads();
+    k5_out(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(NT) bwd_group_sum(BwdArgs a, size_t total) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < total) k6_group(a, i);
+}
+
+__global__ void __launch_bounds__(NT) bwd_head_sum(BwdArgs a) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < a.nheads) k6_head(a, h);
+}
+
+}  // namespace
+
+bool bwd_supported(int headdim, int dstate) {
+    return headdim >= 1 && headdim <= P_MAX && dstate >= 1 && dstate <= N_MAX;
+}
+
+size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate) {
+    const int nchunks = (seqlen + QB - 1) / QB;
+    return ws_floats(batch, seqlen, nheads, headdim, dstate, nchunks) * sizeof(float);
+}
+
+cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
+    BwdArgs a{};
+    a.x = call.x; a.dt = call.dt; a.A = call.A; a.B = call.B; a.C = call.C; a.D = call.D;
+    a.init = call.init_state; a.dy = call.dy; a.dfinal = call.dfinal;
+    a.dx = call.dx; a.ddt = call.ddt; a.dA = call.dA; a.dB = call.dB; a.dC = call.dC;
+    a.dD = call.dD; a.dinit = call.dinit;
+    a.batch = call.batch; a.seqlen = call.seqlen; a.nheads = call.nheads; a.headdim = call.headdim;
+    a.ngroups = call.ngroups; a.dstate = call.dstate;
+    a.nchunks = (call.seqlen + QB - 1) / QB;
+    carve(a, static_cast<float *>(ws));
+
+    // the shared-memory opt-in is per function and per device
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!attr_set[dev]) {
+        for (const void *f : {(const void *)bwd_chunk_state, (const void *)bwd_readout,
+                              (const void *)bwd_chunk_grad}) {
+            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+        }
+        attr_set[dev] = true;
+    }
+    if (a.batch > 0 && a.nchunks > 0) {
+        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(a.nheads, a.batch);
+        bwd_chunk_state<<<gc, NT, SMEM_BYTES, st>>>(a);
+        bwd_state_fwd<<<gh, NT, 0, st>>>(a);
+        bwd_readout<<<gc, NT, SMEM_BYTES, st>>>(a);
+        bwd_state_bwd<<<gh, NT, 0, st>>>(a);
+        bwd_chunk_grad<<<gc, NT, SMEM_BYTES, st>>>(a);
+        const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;
+        bwd_group_sum<<<(unsigned)((total + NT - 1) / NT), NT, 0, st>>>(a, total);
+    } else if (a.batch > 0) {  // empty sequences: dinit = dfinal (or zero)
+        bwd_state_bwd<<<dim3(a.nheads, a.batch), NT, 0, st>>>(a);
+    }
+    bwd_head_sum<<<(a.nheads + NT - 1) / NT, NT, 0, st>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace ssd

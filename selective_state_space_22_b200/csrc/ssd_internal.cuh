@@ -86,6 +86,16 @@ cudaError_t launch_state_update(float *state, const void *x, const float *dt, co
                                 bool bf16, bool cplx, int batch, int nheads, int headdim,
                                 int ngroups, int dstate, cudaStream_t st);
 
+// Gradients of the real fp32 scan (scan_bwd.cu): headdim <= 64, dstate <= 128.
+struct BwdCall {
+    const float *x, *dt, *A, *B, *C, *D, *init_state, *dy, *dfinal;
+    float *dx, *ddt, *dA, *dB, *dC, *dD, *dinit;
+    int batch, seqlen, nheads, headdim, ngroups, dstate;
+};
+bool bwd_supported(int headdim, int dstate);
+size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate);
+cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st);
+
 cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_state,
                                       size_t nfloats, cudaStream_t st);
 

@@ -1,0 +1,73 @@
+// CPU run of the backward kernels' phases (test infrastructure only).
+//
+// Each block of every kernel is run here thread by thread, phase by phase, with
+// a full barrier between phases -- the same functions the CUDA kernels call
+// between __syncthreads().  Shared memory is filled with NaN before each block
+// so that reading anything the block did not write shows up in the result.
+#include <cmath>
+#include <limits>
+#include <vector>
+
+#include "scan_bwd_body.cuh"
+
+using namespace ssd::bwd;
+
+extern "C" int emulate_scan_bwd(const float *x, const float *dt, const float *A, const float *B,
+                                const float *C, const float *D, const float *init, const float *dy,
+                                const float *dfinal, float *dx, float *ddt, float *dA, float *dB,
+                                float *dC, float *dD, float *dinit, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate) {
+    if (headdim < 1 || headdim > P_MAX || dstate < 1 || dstate > N_MAX || nheads % ngroups) return -1;
+    BwdArgs a{};
+    a.x = x; a.dt = dt; a.A = A; a.B = B; a.C = C; a.D = D; a.init = init; a.dy = dy; a.dfinal = dfinal;
+    a.dx = dx; a.ddt = ddt; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD; a.dinit = dinit;
+    a.batch = batch; a.seqlen = seqlen; a.nheads = nheads; a.headdim = headdim; a.ngroups = ngroups;
+    a.dstate = dstate;
+    a.nchunks = (seqlen + QB - 1) / QB;
+    std::vector<float> ws(ws_floats(batch, seqlen, nheads, headdim, dstate, a.nchunks) + 4,
+                          std::numeric_limits<float>::quiet_NaN());
+    carve(a, ws.data());
+    std::vector<float> sm(SMEM_FLOATS);
+    const Smem m = smem_map(sm.data());
+    auto fresh = [&] { std::fill(sm.begin(), sm.end(), std::numeric_limits<float>::quiet_NaN()); };
+    auto each = [&](auto &&f) { for (int tid = 0; tid < NT; ++tid) f(tid); };
+
+    if (batch > 0 && a.nchunks > 0) {
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h)
+                for (int c = 0; c < a.nchunks; ++c) {
+                    fresh();
+                    each([&](int t) { k1_load(a, c, h, b, t, m); });
+                    each([&](int t) { k1_cumsum(a, c, h, b, t, m); });
+                    each([&](int t) { k1_state(a, c, h, b, t, m); });
+                }
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h) each([&](int t) { k2_pass(a, h, b, t); });
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h)
+                for (int c = 0; c < a.nchunks; ++c) {
+                    fresh();
+                    each([&](int t) { k3_load(a, c, h, b, t, m); });
+                    each([&](int t) { k3_r(a, c, h, b, t, m); });
+                }
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h) each([&](int t) { k4_pass(a, h, b, t); });
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h)
+                for (int c = 0; c < a.nchunks; ++c) {
+                    fresh();
+                    each([&](int t) { k5_load(a, c, h, b, t, m); });
+                    each([&](int t) { k5_mats(a, t, m); });
+                    each([&](int t) { k5_tokens(a, t, m); });
+                    each([&](int t) { k5_decay(a, c, h, b, t, m); });
+                    each([&](int t) { k5_out(a, c, h, b, t, m); });
+                }
+        const size_t total = (size_t)batch * seqlen * ngroups * dstate;
+        for (size_t i = 0; i < total; ++i) k6_group(a, i);
+    } else if (batch > 0) {
+        for (int b = 0; b < batch; ++b)
+            for (int h = 0; h < nheads; ++h) each([&](int t) { k4_pass(a, h, b, t); });
+    }
+    for (int h = 0; h < nheads; ++h) k6_head(a, h);
+    return 0;
+}
