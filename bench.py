@@ -658,6 +658,211 @@ def bench_ours(args, shape):
     return 0
 
 
+# --------------------------------------------------------------- backward
+def bwd_bytes(shape) -> int:
+    """Per call (float32): x and dy read, dx written; dt read, ddt written; B and C
+    read, dB and dC written; init_state and dfinal read, dinit written; A and D
+    read, dA and dD written."""
+    b, T, H, P, G, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups, shape.dstate
+    tok = b * T
+    return 4 * (3 * tok * H * P + 2 * tok * H + 4 * tok * G * N + 3 * b * H * P * N + 4 * H)
+
+
+def bwd_cpu_units(shape, units, threads):
+    """The oracle's gradient over the given (batch, head) sequences, one per
+    thread; returns seconds."""
+    import numpy as np
+
+    import oracle
+    from selective_state_space_22_b200 import inputs
+
+    lib = oracle.load()
+    w = inputs.widen_all(inputs.scan_inputs(shape))
+    up = {k: v.double().numpy() for k, v in inputs.bwd_upstream(shape).items()}
+    c = np.ascontiguousarray
+
+    def one(unit):
+        b, h = unit
+        g = 0 if shape.ngroups == 1 else h * shape.ngroups // shape.nheads
+        oracle.scan_bwd(c(w["x"][b:b + 1, :, h:h + 1]), c(w["dt"][b:b + 1, :, h:h + 1]), c(w["A"][h:h + 1]),
+                        c(w["B"][b:b + 1, :, g:g + 1]), c(w["C"][b:b + 1, :, g:g + 1]),
+                        None if w["D"] is None else c(w["D"][h:h + 1]),
+                        None if w["init_state"] is None else c(w["init_state"][b:b + 1, h:h + 1]),
+                        c(up["dy"][b:b + 1, :, h:h + 1]), c(up["dfinal"][b:b + 1, h:h + 1]), lib=lib)
+
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(one, units))
+    return time.perf_counter() - t0
+
+
+def bwd_cpu_baseline(shape, max_units: int = 16):
+    threads = oracle_threads()
+    total = shape.batch * shape.nheads
+    n = max(1, min(total, max_units, threads))
+    units = [(i // shape.nheads, i % shape.nheads) for i in range(n)]
+    secs = bwd_cpu_units(shape, units, threads)
+    return {"value": shape.seqlen * n / shape.nheads / secs, "unit": "tokens/s", "cores": min(threads, n),
+            "kind": "oracle",
+            "sample": f"{n} of {total} (batch, head) sequences of {shape.name} (T={shape.seqlen}); fp64 "
+                      f"sequential adjoint, one sequence per thread; tokens/s counts sequences/nheads x T",
+            "seconds": secs}
+
+
+def bench_bwd(args, shape):
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device for --impl ours")
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+
+    inp = inputs.scan_inputs(shape)
+    up = inputs.bwd_upstream(shape)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    u = {k: v.to(dev) for k, v in up.items()}
+    nbytes = ssd.ssd_scan_bwd_workspace_size(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                                             shape.ngroups, shape.dstate)
+    ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    out = {}
+
+    def step():
+        out.update(ssd.ssd_scan_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                                    u["dy"], u["dfinal"], workspace=ws))
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize()
+    ssd.ssd_get_device_status()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_s = dist_max(sum(per_step_ms) / 1e3, dev)
+    value = shape.tokens * world * args.steps / total_s
+    peaks = load_peaks()
+    abytes = bwd_bytes(shape)
+    t_call = statistics.median(per_step_ms) / 1e3
+    roofline = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                "kernel": "ssd_scan_bwd (6 CUDA-core kernels, timed as one call)",
+                "algorithmic_bytes_per_launch": abytes,
+                "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
+                if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
+                "roofline_time_us": 1e6 * abytes / (peaks["hbm_gbs"] * 1e9), "kernel_time_us": 1e6 * t_call}
+
+    e2e = None
+    if not args.no_e2e:
+        hin = {k: v.pin_memory() for k, v in list(inp.items()) + list(up.items()) if v is not None}
+        dst = {k: (d[k] if k in d else u[k]) for k in hin}
+        step()
+        torch.cuda.synchronize()
+        hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items() if v is not None}
+        h2d = sum(v.numel() * v.element_size() for v in hin.values())
+        d2h = sum(v.numel() * v.element_size() for v in hout.values())
+        k_e2e = max(3, min(args.steps, 20))
+
+        def e2e_step():
+            for k, v in hin.items():
+                dst[k].copy_(v, non_blocking=True)
+            step()
+            for k, v in hout.items():
+                v.copy_(out[k], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        dist_barrier()
+        torch.cuda.synchronize()
+        es.record(stream)
+        for _ in range(k_e2e):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize()
+        dist_barrier()
+        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
+        e2e = {"value": shape.tokens * world * k_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = bwd_cpu_baseline(shape)
+        cpu.pop("seconds", None)
+    line = {
+        "metric": "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
+        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads,
+                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
+                   "chunk": 64, "io_dtype": "f32", "l2": "flushed between timed steps (512 MiB write)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
+        "gpu_launches": 7 * args.steps,
+        "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0], statistics.median(per_step_ms),
+                                statistics.quantiles(per_step_ms, n=10)[-1]],
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def bench_reference_bwd(args, shape):
+    """The oracle's gradient on the host cores, a bounded sample per step."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    threads = oracle_threads()
+    n = max(1, min(shape.batch * shape.nheads, 16, threads))
+    units = [(i // shape.nheads, i % shape.nheads) for i in range(n)]
+    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
+        pass  # the oracle has no warm-up state; warm-up steps are not timed work
+    secs = [bwd_cpu_units(shape, units, threads) for _ in range(args.steps)]
+    tokens = shape.seqlen * n / shape.nheads
+    value = tokens * args.steps / sum(secs)
+    cpu = {"value": value, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
+           "sample": f"{n} of {shape.batch * shape.nheads} (batch, head) sequences per step of {shape.name}"}
+    line = {"metric": "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * sum(secs) / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
+                       "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
+                       "dstate": shape.dstate, "io_dtype": "f32"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -670,6 +875,9 @@ def main(argv=None):
     args = ap.parse_args(argv)
     from selective_state_space_22_b200 import inputs
 
+    if args.workload == inputs.BWD.name:
+        shape = inputs.BWD
+        return bench_reference_bwd(args, shape) if args.impl == "reference" else bench_bwd(args, shape)
     if args.workload == inputs.DECODE.name:
         shape = inputs.DECODE
         return bench_reference_decode(args, shape) if args.impl == "reference" else bench_decode(args, shape)

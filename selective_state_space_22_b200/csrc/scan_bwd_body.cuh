@@ -40,6 +40,9 @@ constexpr int QB = 64;       // tokens per chunk
 constexpr int NT = 256;      // threads per block
 constexpr int P_MAX = 64;    // head dim
 constexpr int N_MAX = 128;   // state dim
+// Shared-memory row strides, one float longer than a row, so that lanes walking
+// down a column hit 32 different banks.
+constexpr int PS = P_MAX + 1, NS = N_MAX + 1, QS = QB + 1;
 
 struct BwdArgs {
     const float *x, *dt, *A, *B, *C, *D, *init, *dy, *dfinal;
@@ -98,18 +101,18 @@ __host__ __device__ inline size_t ix_pn(const BwdArgs &a, int b, int h, int c) {
 __host__ __device__ inline int group_of(const BwdArgs &a, int h) { return h / (a.nheads / a.ngroups); }
 
 // ------------------------------------------------ shared-memory layout
-// One layout serves every chunk kernel (fixed strides P_MAX, N_MAX, QB).
+// One layout serves every chunk kernel (fixed row strides PS, NS, QS).
 struct Smem {
     float *d, *acs, *e, *w;           // [QB]
-    float *X, *dY;                    // [QB][P_MAX]
-    float *Bs, *Cs;                   // [QB][N_MAX]
-    float *Hin, *Gh;                  // [P_MAX][N_MAX]
-    float *GL, *XY, *K;               // [QB][QB]
+    float *X, *dY;                    // [QB][PS]
+    float *Bs, *Cs;                   // [QB][NS]
+    float *Hin, *Gh;                  // [P_MAX][NS]
+    float *GL, *XY, *K;               // [QB][QS]
     float *rowE, *colG, *F, *Ksr;     // [QB]
     float *red;                       // [2 * QB]
     float *misc;                      // [4]: lam, ...
 };
-constexpr size_t SMEM_FLOATS = 4 * QB + 2 * QB * P_MAX + 2 * QB * N_MAX + 2 * P_MAX * N_MAX + 3 * QB * QB +
+constexpr size_t SMEM_FLOATS = 4 * QB + 2 * QB * PS + 2 * QB * NS + 2 * P_MAX * NS + 3 * QB * QS +
                                4 * QB + 2 * QB + 4;
 __host__ __device__ inline Smem smem_map(float *s) {
     Smem m;
@@ -117,15 +120,15 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.acs = s; s += QB;
     m.e = s; s += QB;
     m.w = s; s += QB;
-    m.X = s; s += QB * P_MAX;
-    m.dY = s; s += QB * P_MAX;
-    m.Bs = s; s += QB * N_MAX;
-    m.Cs = s; s += QB * N_MAX;
-    m.Hin = s; s += P_MAX * N_MAX;
-    m.Gh = s; s += P_MAX * N_MAX;
-    m.GL = s; s += QB * QB;
-    m.XY = s; s += QB * QB;
-    m.K = s; s += QB * QB;
+    m.X = s; s += QB * PS;
+    m.dY = s; s += QB * PS;
+    m.Bs = s; s += QB * NS;
+    m.Cs = s; s += QB * NS;
+    m.Hin = s; s += P_MAX * NS;
+    m.Gh = s; s += P_MAX * NS;
+    m.GL = s; s += QB * QS;
+    m.XY = s; s += QB * QS;
+    m.K = s; s += QB * QS;
     m.rowE = s; s += QB;
     m.colG = s; s += QB;
     m.F = s; s += QB;
@@ -147,20 +150,20 @@ __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, 
                                             float *dst) {
     for (int i = tid; i < QB * a.headdim; i += NT) {
         const int s = i / a.headdim, p = i % a.headdim, t = c * QB + s;
-        dst[s * P_MAX + p] = t < a.seqlen ? src[ix_x(a, b, t, h, p)] : 0.f;
+        dst[s * PS + p] = t < a.seqlen ? src[ix_x(a, b, t, h, p)] : 0.f;
     }
 }
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
     for (int i = tid; i < QB * a.dstate; i += NT) {
         const int s = i / a.dstate, n = i % a.dstate, t = c * QB + s;
-        dst[s * N_MAX + n] = t < a.seqlen ? src[ix_bc(a, b, t, g, n)] : 0.f;
+        dst[s * NS + n] = t < a.seqlen ? src[ix_bc(a, b, t, g, n)] : 0.f;
     }
 }
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
     for (int i = tid; i < a.headdim * a.dstate; i += NT) {
         const int p = i / a.dstate, n = i % a.dstate;
-        dst[p * N_MAX + n] = src[i];
+        dst[p * NS + n] = src[i];
     }
 }
 
@@ -191,7 +194,7 @@ __host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, 
     for (int i = tid; i < a.headdim * a.dstate; i += NT) {
         const int p = i / a.dstate, n = i % a.dstate;
         float acc = 0.f;
-        for (int s = 0; s < QB; ++s) acc += m.w[s] * m.X[s * P_MAX + p] * m.Bs[s * N_MAX + n];
+        for (int s = 0; s < QB; ++s) acc += m.w[s] * m.X[s * PS + p] * m.Bs[s * NS + n];
         S[i] = acc;
     }
 }
@@ -221,7 +224,7 @@ __host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int 
     for (int i = tid; i < a.headdim * a.dstate; i += NT) {
         const int p = i / a.dstate, n = i % a.dstate;
         float acc = 0.f;
-        for (int l = 0; l < QB; ++l) acc += m.e[l] * m.dY[l * P_MAX + p] * m.Cs[l * N_MAX + n];
+        for (int l = 0; l < QB; ++l) acc += m.e[l] * m.dY[l * PS + p] * m.Cs[l * NS + n];
         R[i] = acc;
     }
 }
@@ -266,16 +269,16 @@ __host__ __device__ inline void k5_mats(const BwdArgs &a, int tid, const Smem &m
     for (int i = tid; i < QB * QB; i += NT) {
         const int l = i / QB, s = i % QB;
         float gm = 0.f, xy = 0.f;
-        for (int n = 0; n < a.dstate; ++n) gm += m.Cs[l * N_MAX + n] * m.Bs[s * N_MAX + n];
-        for (int p = 0; p < a.headdim; ++p) xy += m.dY[l * P_MAX + p] * m.X[s * P_MAX + p];
-        m.XY[i] = xy;
+        for (int n = 0; n < a.dstate; ++n) gm += m.Cs[l * NS + n] * m.Bs[s * NS + n];
+        for (int p = 0; p < a.headdim; ++p) xy += m.dY[l * PS + p] * m.X[s * PS + p];
+        m.XY[l * QS + s] = xy;
         if (l >= s) {
             const float L = expf(m.acs[l] - m.acs[s]);
-            m.GL[i] = gm * L;
-            m.K[i] = L * m.d[s] * xy;
+            m.GL[l * QS + s] = gm * L;
+            m.K[l * QS + s] = L * m.d[s] * xy;
         } else {
-            m.GL[i] = 0.f;
-            m.K[i] = 0.f;
+            m.GL[l * QS + s] = 0.f;
+            m.K[l * QS + s] = 0.f;
         }
     }
 }
@@ -285,8 +288,8 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
     if (tid < QB) {
         const int t = tid;
         float re = 0.f, cg = 0.f;
-        for (int s = 0; s < QB; ++s) re += m.GL[t * QB + s] * m.XY[t * QB + s] * m.d[s];
-        for (int l = 0; l < QB; ++l) cg += m.GL[l * QB + t] * m.XY[l * QB + t];
+        for (int s = 0; s < QB; ++s) re += m.GL[t * QS + s] * m.XY[t * QS + s] * m.d[s];
+        for (int l = 0; l < QB; ++l) cg += m.GL[l * QS + t] * m.XY[l * QS + t];
         m.rowE[t] = re;
         m.colG[t] = cg;
     } else if (tid < 2 * QB) {  // F[t] = e^{acs[t]} dy_t . (h_in C_t)
@@ -294,8 +297,8 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
         float acc = 0.f;
         for (int p = 0; p < a.headdim; ++p) {
             float hc = 0.f;
-            for (int n = 0; n < a.dstate; ++n) hc += m.Hin[p * N_MAX + n] * m.Cs[t * N_MAX + n];
-            acc += m.dY[t * P_MAX + p] * hc;
+            for (int n = 0; n < a.dstate; ++n) hc += m.Hin[p * NS + n] * m.Cs[t * NS + n];
+            acc += m.dY[t * PS + p] * hc;
         }
         m.F[t] = m.e[t] * acc;
     } else if (tid < 3 * QB) {  // Ksr[t] = x_t . (Gh B_t)
@@ -303,8 +306,8 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
         float acc = 0.f;
         for (int p = 0; p < a.headdim; ++p) {
             float gb = 0.f;
-            for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * N_MAX + n] * m.Bs[t * N_MAX + n];
-            acc += m.X[t * P_MAX + p] * gb;
+            for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * NS + n] * m.Bs[t * NS + n];
+            acc += m.X[t * PS + p] * gb;
         }
         m.Ksr[t] = acc;
     } else if (tid < 4 * QB) {
@@ -312,11 +315,11 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
         float h0 = 0.f, dd = 0.f;
         for (int i = r; i < a.headdim * a.dstate; i += QB) {
             const int p = i / a.dstate, n = i % a.dstate;
-            h0 += m.Gh[p * N_MAX + n] * m.Hin[p * N_MAX + n];
+            h0 += m.Gh[p * NS + n] * m.Hin[p * NS + n];
         }
         for (int i = r; i < QB * a.headdim; i += QB) {
             const int s = i / a.headdim, p = i % a.headdim;
-            dd += m.dY[s * P_MAX + p] * m.X[s * P_MAX + p];
+            dd += m.dY[s * PS + p] * m.X[s * PS + p];
         }
         m.red[r] = h0;
         m.red[QB + r] = dd;
@@ -355,19 +358,19 @@ __host__ __device__ inline void k5_out(const BwdArgs &a, int c, int h, int b, in
         const int s = i / a.headdim, p = i % a.headdim, t = c * QB + s;
         if (t >= a.seqlen) continue;
         float acc = 0.f, gb = 0.f;
-        for (int l = s; l < QB; ++l) acc += m.GL[l * QB + s] * m.dY[l * P_MAX + p];
-        for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * N_MAX + n] * m.Bs[s * N_MAX + n];
-        a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * P_MAX + p] + m.w[s] * gb;
+        for (int l = s; l < QB; ++l) acc += m.GL[l * QS + s] * m.dY[l * PS + p];
+        for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * NS + n] * m.Bs[s * NS + n];
+        a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * PS + p] + m.w[s] * gb;
     }
     for (int i = tid; i < QB * a.dstate; i += NT) {
         const int s = i / a.dstate, n = i % a.dstate, t = c * QB + s;
         if (t >= a.seqlen) continue;
         float db = 0.f, dc = 0.f, xg = 0.f, yh = 0.f;
-        for (int l = s; l < QB; ++l) db += m.K[l * QB + s] * m.Cs[l * N_MAX + n];
-        for (int r = 0; r <= s; ++r) dc += m.K[s * QB + r] * m.Bs[r * N_MAX + n];
+        for (int l = s; l < QB; ++l) db += m.K[l * QS + s] * m.Cs[l * NS + n];
+        for (int r = 0; r <= s; ++r) dc += m.K[s * QS + r] * m.Bs[r * NS + n];
         for (int p = 0; p < a.headdim; ++p) {
-            xg += m.X[s * P_MAX + p] * m.Gh[p * N_MAX + n];
-            yh += m.dY[s * P_MAX + p] * m.Hin[p * N_MAX + n];
+            xg += m.X[s * PS + p] * m.Gh[p * NS + n];
+            yh += m.dY[s * PS + p] * m.Hin[p * NS + n];
         }
         const size_t o = (((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n;
         a.dBh[o] = db + m.w[s] * xg;

@@ -77,6 +77,20 @@ DECODE = DecodeShape("decode-bitmamba1b-256seq", 256, 64, 64, 1, 128, 1024)
 
 WORKLOADS = {w.name: w for w in (TINY, MAMBA2_1B, MAMBA3_COMPLEX, LONG)}
 
+# Gradients through the scan at the Mamba-2 layer shape, float32 (the backward
+# takes float32 tensors); dy and dfinal from bwd_upstream.
+BWD = ScanShape("mamba2-bitmamba1b-layer-bwd-f32", 2, 2048, 64, 64, 1, 128, 64, "f32",
+                init_state=True, seed=SEED_BASE + 5)
+
+
+def bwd_upstream(shape: ScanShape) -> dict:
+    """The gradients arriving at y and final_state: dy [b,T,H,P] and dfinal
+    [b,H,P,N], float32 N(0,1), seeded from the workload's seed."""
+    gen = torch.Generator().manual_seed(shape.seed + 1000)
+    b, T, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    return {"dy": torch.randn((b, T, H, P), generator=gen),
+            "dfinal": torch.randn((b, H, P, N), generator=gen)}
+
 
 def _tdtype(name: str) -> torch.dtype:
     return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
