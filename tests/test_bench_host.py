@@ -21,6 +21,14 @@ def test_algorithmic_counts_mamba2_layer():
     assert bench.algorithmic_flops(inputs.MAMBA2_1B) == 13_036_421_120
 
 
+def test_algorithmic_bytes_backward():
+    # float32: x, dy, dx 3 x 67.11 MB; dt, ddt 2 x 1.05 MB; B, C, dB, dC 4 x 1.05 MB;
+    # init_state, dfinal, dinit 3 x 4.19 MB; A, D, dA, dD 4 x 256 B
+    tok = 2 * 2048
+    expect = 3 * tok * 64 * 64 * 4 + 2 * tok * 64 * 4 + 4 * tok * 128 * 4 + 3 * 2 * 64 * 64 * 128 * 4 + 4 * 64 * 4
+    assert bench.bwd_bytes(inputs.BWD) == expect == 224_396_288
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
