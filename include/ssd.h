@@ -202,6 +202,29 @@ ssd_status ssd_scan_bwd(const float *x, const float *dt, const float *A, const f
                         int dstate, void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Gradients of the complex scan (the Mamba-3-Lite variant), float32.
+ *
+ * The loss is L = sum_t <dy_t, y_t> + Re <dfinal, final_state> with
+ * y_t = Re(h_t C_t) + D x_t.  A [nheads], B and C [batch, seqlen, ngroups, dstate],
+ * init_state and dfinal [batch, nheads, headdim, dstate] are complex (interleaved
+ * float pairs), as are the outputs dA, dB, dC and dinit; x, dt, D, dy, dx, ddt
+ * and dD are float32.  For a complex z = u + iv the gradient written is
+ * dL/du + i dL/dv.  Limits: headdim <= 64 and dstate <= 64; the chunk is 32
+ * tokens.  Workspace from ssd_scan_bwd_complex_workspace_size.  Everything else
+ * as ssd_scan_bwd.
+ */
+size_t ssd_scan_bwd_complex_workspace_size(int batch, int seqlen, int nheads, int headdim,
+                                           int ngroups, int dstate);
+
+ssd_status ssd_scan_bwd_complex(const float *x, const float *dt, const float *A,
+                                const float *B, const float *C, const float *D,
+                                const float *init_state, const float *dy, const float *dfinal,
+                                float *dx, float *ddt, float *dA, float *dB, float *dC,
+                                float *dD, float *dinit, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/*
  * Waits for `stream`, then reports and clears an error that a kernel raised on
  * the device since the last call on this device (SSD_ERR_TIMEOUT when one of the
  * tensor-core kernel's bounded waits between its warp roles gave up after 2 s;

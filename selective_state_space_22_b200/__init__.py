@@ -22,7 +22,8 @@ import torch
 __all__ = ["SSDError", "ssd_scan_fwd", "ssd_scan_fwd_complex", "ssd_state_update",
            "ssd_state_update_complex", "ssd_scan_workspace_size", "ssd_scan_kernel_launches", "ssd_get_device_status",
            "ssd_scan_fwd_noalloc", "ssd_last_error", "ssd_version", "load_library", "LIB_PATH",
-           "SSD_WORKSPACE_INVALID", "ssd_scan_bwd", "ssd_scan_bwd_workspace_size"]
+           "SSD_WORKSPACE_INVALID", "ssd_scan_bwd", "ssd_scan_bwd_workspace_size",
+           "ssd_scan_bwd_complex"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -72,6 +73,10 @@ def load_library(path: str | None = None):
         lib.ssd_scan_bwd_workspace_size.restype = _SZ
         lib.ssd_scan_bwd.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, _SZ, _VP]
         lib.ssd_scan_bwd.restype = _I
+        lib.ssd_scan_bwd_complex_workspace_size.argtypes = [_I] * 6
+        lib.ssd_scan_bwd_complex_workspace_size.restype = _SZ
+        lib.ssd_scan_bwd_complex.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, _SZ, _VP]
+        lib.ssd_scan_bwd_complex.restype = _I
         lib.ssd_get_device_status.argtypes = [_VP]
         lib.ssd_get_device_status.restype = _I
         lib.ssd_last_error.argtypes = []
@@ -347,6 +352,43 @@ def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=No
                               _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dinit"]),
                               b, T, H, P, G, N, _ptr(ws), 0 if ws is None else ws.numel(),
                               _stream_handle(stream))
+    _check(st)
+    return out
+
+
+def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=None, stream=None):
+    """Gradients of L = sum <dy, y> + Re <dfinal, final_state> through the complex
+    scan.  A, B, C, init_state, dfinal complex64; x, dt, D, dy float32.  Returns
+    a dict with dx, ddt (float32), dA, dB, dC, dinit (complex64) and dD (float32,
+    None when D is None)."""
+    lib = load_library()
+    dev = x.device
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    f, c = torch.float32, torch.complex64
+    _need(x, "x", f, dev)
+    _need(dt, "dt", f, dev, (b, T, H))
+    _need(A, "A", c, dev, (H,))
+    _need(B, "B", c, dev, (b, T, G, N))
+    _need(C, "C", c, dev, (b, T, G, N))
+    _need(D, "D", f, dev, (H,), allow_none=True)
+    _need(init_state, "init_state", c, dev, (b, H, P, N), allow_none=True)
+    _need(dy, "dy", f, dev, (b, T, H, P))
+    _need(dfinal, "dfinal", c, dev, (b, H, P, N), allow_none=True)
+    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt), dA=torch.empty_like(A),
+               dB=torch.empty_like(B), dC=torch.empty_like(C),
+               dD=None if D is None else torch.empty_like(D),
+               dinit=torch.empty((b, H, P, N), dtype=c, device=dev))
+    n = lib.ssd_scan_bwd_complex_workspace_size(b, T, H, P, G, N)
+    if n == SSD_WORKSPACE_INVALID:
+        raise SSDError(1, "invalid sizes for the complex backward scan")
+    ws = workspace if workspace is not None else _workspace(dev, n)
+    with torch.cuda.device(dev):
+        st = lib.ssd_scan_bwd_complex(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                                      _ptr(dy), _ptr(dfinal), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),
+                                      _ptr(out["dB"]), _ptr(out["dC"]), _ptr(out["dD"]), _ptr(out["dinit"]),
+                                      b, T, H, P, G, N, _ptr(ws), 0 if ws is None else ws.numel(),
+                                      _stream_handle(stream))
     _check(st)
     return out
 

@@ -9,8 +9,10 @@
 //      chunks), and dinit                                            grid (heads, batch)
 //   5. dx, ddt and each head's dB, dC, dA, dD parts of one chunk    grid (chunks, heads, batch)
 //   6. dB, dC summed over the heads of a group; dA, dD over batch and chunks
-// Sums run in a fixed order, so repeated calls give identical bits.
+// Sums run in a fixed order, so repeated calls give identical bits.  The complex
+// variant (scan_bwd_complex_body.cuh) runs the same six steps on 32-token chunks.
 #include "scan_bwd_body.cuh"
+#include "scan_bwd_complex_body.cuh"
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -69,7 +71,118 @@ __global__ void __launch_bounds__(NT) bwd_head_sum(BwdArgs a) {
     if (h < a.nheads) k6_head(a, h);
 }
 
+// ------------------------------------------------------------- complex
+constexpr size_t SMEM_BYTES_C = bwdc::SMEM_FLOATS * sizeof(float);
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_state(bwdc::BwdArgs a) {
+    extern __shared__ float sm[];
+    const bwdc::Smem m = bwdc::smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    bwdc::k1_load(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k1_cumsum(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k1_state(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_state_fwd(bwdc::BwdArgs a) {
+    bwdc::k2_pass(a, blockIdx.x, blockIdx.y, threadIdx.x);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_readout(bwdc::BwdArgs a) {
+    extern __shared__ float sm[];
+    const bwdc::Smem m = bwdc::smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    bwdc::k3_load(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k3_r(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_state_bwd(bwdc::BwdArgs a) {
+    bwdc::k4_pass(a, blockIdx.x, blockIdx.y, threadIdx.x);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_grad(bwdc::BwdArgs a) {
+    extern __shared__ float sm[];
+    const bwdc::Smem m = bwdc::smem_map(sm);
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    bwdc::k5_load(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k5_mats(a, tid, m);
+    __syncthreads();
+    bwdc::k5_tokens(a, tid, m);
+    __syncthreads();
+    bwdc::k5_decay(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k5_out(a, c, h, b, tid, m);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_group_sum(bwdc::BwdArgs a, size_t total) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i < total) bwdc::k6_group(a, i);
+}
+
+__global__ void __launch_bounds__(bwdc::NT) bwdc_head_sum(bwdc::BwdArgs a) {
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h < a.nheads) bwdc::k6_head(a, h);
+}
+
+cudaError_t set_smem_attr(const void *const *fs, int nf, size_t bytes, bool (&done)[64]) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (done[dev]) return cudaSuccess;
+    for (int i = 0; i < nf; ++i) {
+        e = cudaFuncSetAttribute(fs[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+        if (e != cudaSuccess) return e;
+    }
+    done[dev] = true;
+    return cudaSuccess;
+}
+
 }  // namespace
+
+bool bwd_complex_supported(int headdim, int dstate) {
+    return headdim >= 1 && headdim <= bwdc::P_MAX && dstate >= 1 && dstate <= bwdc::N_MAX;
+}
+
+size_t bwd_complex_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate) {
+    const int nchunks = (seqlen + bwdc::QC - 1) / bwdc::QC;
+    return bwdc::ws_floats(batch, seqlen, nheads, headdim, dstate, nchunks) * sizeof(float);
+}
+
+cudaError_t launch_scan_bwd_complex(const BwdCall &call, void *ws, cudaStream_t st) {
+    bwdc::BwdArgs a{};
+    a.x = call.x; a.dt = call.dt; a.A = call.A; a.B = call.B; a.C = call.C; a.D = call.D;
+    a.init = call.init_state; a.dy = call.dy; a.dfinal = call.dfinal;
+    a.dx = call.dx; a.ddt = call.ddt; a.dA = call.dA; a.dB = call.dB; a.dC = call.dC;
+    a.dD = call.dD; a.dinit = call.dinit;
+    a.batch = call.batch; a.seqlen = call.seqlen; a.nheads = call.nheads; a.headdim = call.headdim;
+    a.ngroups = call.ngroups; a.dstate = call.dstate;
+    a.nchunks = (call.seqlen + bwdc::QC - 1) / bwdc::QC;
+    bwdc::carve(a, static_cast<float *>(ws));
+
+    static bool attr_set[64] = {false};  // the shared-memory opt-in is per function and per device
+    const void *fs[3] = {(const void *)bwdc_chunk_state, (const void *)bwdc_readout, (const void *)bwdc_chunk_grad};
+    cudaError_t e = set_smem_attr(fs, 3, SMEM_BYTES_C, attr_set);
+    if (e != cudaSuccess) return e;
+    const int nt = bwdc::NT;
+    if (a.batch > 0 && a.nchunks > 0) {
+        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(a.nheads, a.batch);
+        bwdc_chunk_state<<<gc, nt, SMEM_BYTES_C, st>>>(a);
+        bwdc_state_fwd<<<gh, nt, 0, st>>>(a);
+        bwdc_readout<<<gc, nt, SMEM_BYTES_C, st>>>(a);
+        bwdc_state_bwd<<<gh, nt, 0, st>>>(a);
+        bwdc_chunk_grad<<<gc, nt, SMEM_BYTES_C, st>>>(a);
+        const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;
+        bwdc_group_sum<<<(unsigned)((total + nt - 1) / nt), nt, 0, st>>>(a, total);
+    } else if (a.batch > 0) {  // empty sequences: dinit = dfinal (or zero)
+        bwdc_state_bwd<<<dim3(a.nheads, a.batch), nt, 0, st>>>(a);
+    }
+    bwdc_head_sum<<<(a.nheads + nt - 1) / nt, nt, 0, st>>>(a);
+    return cudaGetLastError();
+}
 
 bool bwd_supported(int headdim, int dstate) {
     return headdim >= 1 && headdim <= P_MAX && dstate >= 1 && dstate <= N_MAX;

@@ -1,0 +1,435 @@
+// scan_bwd_complex_body.cuh -- the phases of the chunked backward scan, complex A.
+//
+// The complex (Mamba-3-Lite) variant of scan_bwd_body.cuh: A, B, C and the state
+// are complex (interleaved float pairs), x, dt, D, y real.  The loss is
+// L = sum_t <dy_t, y_t> + Re <dfinal, h_final> with y_t = Re(h_t C_t) + D x_t, and
+// the gradient of a complex z = u + iv is dL/du + i dL/dv.  With acs the complex
+// inclusive within-chunk cumulative sum of dt A, lam = acs[last], L[l][s] =
+// exp(acs[l] - acs[s]) (l >= s), e_l = exp(acs[l]), w_s = exp(lam - acs[s]) dt_s:
+//   Gh(previous chunk) = conj(exp(lam)) Gh + sum_l conj(e_l) dy_l conj(C_l)^T
+//   dx_s = Re(sum_l (C_l.B_s) L[l][s] dt_s dy_l) + D dy_s + Re(conj(w_s) Gh conj(B_s))
+//   dB_s = conj(sum_l K[l][s] C_l) + conj(w_s) Gh^T x_s ,  K[l][s] = L[l][s] dt_s (dy_l . x_s)
+//   dC_l = conj(sum_s K[l][s] B_s + e_l h_in^T dy_l)
+// and through acs, with E[l][s] = (C_l.B_s) K[l][s]:
+//   dacs[t] = conj(sum_s E[t][s] - sum_l E[l][t] + e_t dy_t.(h_in C_t) - w_t x_t.(conj(Gh) B_t))
+//             (+ conj(exp(lam) <conj(Gh), h_in> + sum_s w_s x_s.(conj(Gh) B_s)) at the last token)
+//   dalpha = reverse cumulative sum of dacs;  ddt += Re(conj(dalpha) A);  dA += sum dt dalpha.
+// (C_l.B_s = sum_n C_l[n] B_s[n], no conjugate, as in the forward readout.)  The
+// chunk is 32 tokens so that the complex tiles fit in shared memory.  As in the
+// real variant, every phase is a __host__ __device__ function of (block, thread).
+#pragma once
+
+#include <math.h>
+#include <stddef.h>
+
+#ifndef __CUDACC__
+#define __host__
+#define __device__
+#endif
+
+namespace ssd {
+namespace bwdc {
+
+constexpr int QC = 32;        // tokens per chunk
+constexpr int NT = 256;       // threads per block
+constexpr int P_MAX = 64;     // head dim
+constexpr int N_MAX = 64;     // complex state dim
+constexpr int RED = 64;       // threads of the block reductions
+// Row strides in floats, odd so that lanes walking down a column spread over banks.
+constexpr int PS = P_MAX + 1, NS = 2 * N_MAX + 1, QS2 = 2 * QC + 1, QS1 = QC + 1;
+
+struct c2 {
+    float re, im;
+};
+__host__ __device__ inline c2 cmk(float r, float i) { return c2{r, i}; }
+__host__ __device__ inline c2 cadd(c2 a, c2 b) { return c2{a.re + b.re, a.im + b.im}; }
+__host__ __device__ inline c2 csub(c2 a, c2 b) { return c2{a.re - b.re, a.im - b.im}; }
+__host__ __device__ inline c2 cmul(c2 a, c2 b) { return c2{a.re * b.re - a.im * b.im, a.re * b.im + a.im * b.re}; }
+__host__ __device__ inline c2 cconj(c2 a) { return c2{a.re, -a.im}; }
+__host__ __device__ inline c2 cscale(c2 a, float s) { return c2{a.re * s, a.im * s}; }
+__host__ __device__ inline c2 cexpc(c2 z) {
+    const float r = expf(z.re);
+    return c2{r * cosf(z.im), r * sinf(z.im)};
+}
+__host__ __device__ inline c2 ld2(const float *p) { return c2{p[0], p[1]}; }
+__host__ __device__ inline void st2(float *p, c2 v) {
+    p[0] = v.re;
+    p[1] = v.im;
+}
+
+struct BwdArgs {
+    const float *x, *dt, *A, *B, *C, *D, *init, *dy, *dfinal;  // A, B, C, init, dfinal: float pairs
+    float *dx, *ddt, *dA, *dB, *dC, *dD, *dinit;              // dA, dB, dC, dinit: float pairs
+    int batch, seqlen, nheads, headdim, ngroups, dstate, nchunks;
+    // workspace (complex regions are float pairs)
+    float *acs;   // [b][h][nchunks * QC][2]
+    float *lam;   // [b][h][nchunks][2]
+    float *st;    // [b][h][nchunks][P*N][2]: chunk states, then the readout terms R
+    float *hin;   // [b][h][nchunks][P*N][2]
+    float *gh;    // [b][h][nchunks][P*N][2]
+    float *dBh;   // [b][T][h][N][2]
+    float *dCh;   // [b][T][h][N][2]
+    float *dAp;   // [b][h][nchunks][2]
+    float *dDp;   // [b][h][nchunks]
+};
+
+__host__ __device__ inline size_t ws_floats(int batch, int seqlen, int nheads, int headdim, int dstate,
+                                            int nchunks) {
+    auto r4 = [](size_t v) { return (v + 3) / 4 * 4; };
+    const size_t bh = (size_t)batch * nheads, pn = (size_t)headdim * dstate;
+    return r4(2 * bh * nchunks * QC) + r4(2 * bh * nchunks) + 3 * r4(2 * bh * nchunks * pn) +
+           2 * r4(2 * (size_t)batch * seqlen * nheads * dstate) + r4(2 * bh * nchunks) + r4(bh * nchunks);
+}
+
+__host__ __device__ inline void carve(BwdArgs &a, float *ws) {
+    auto r4 = [](size_t v) { return (v + 3) / 4 * 4; };
+    const size_t bh = (size_t)a.batch * a.nheads, pn = (size_t)a.headdim * a.dstate;
+    float *p = ws;
+    a.acs = p; p += r4(2 * bh * a.nchunks * QC);
+    a.lam = p; p += r4(2 * bh * a.nchunks);
+    a.st = p; p += r4(2 * bh * a.nchunks * pn);
+    a.hin = p; p += r4(2 * bh * a.nchunks * pn);
+    a.gh = p; p += r4(2 * bh * a.nchunks * pn);
+    a.dBh = p; p += r4(2 * (size_t)a.batch * a.seqlen * a.nheads * a.dstate);
+    a.dCh = p; p += r4(2 * (size_t)a.batch * a.seqlen * a.nheads * a.dstate);
+    a.dAp = p; p += r4(2 * bh * a.nchunks);
+    a.dDp = p;
+}
+
+// ------------------------------------------------------------- indexing
+__host__ __device__ inline size_t ix_x(const BwdArgs &a, int b, int t, int h, int p) {
+    return (((size_t)b * a.seqlen + t) * a.nheads + h) * a.headdim + p;
+}
+__host__ __device__ inline size_t ix_dt(const BwdArgs &a, int b, int t, int h) {
+    return ((size_t)b * a.seqlen + t) * a.nheads + h;
+}
+// complex element index (multiply by 2 for the float offset)
+__host__ __device__ inline size_t ix_bc(const BwdArgs &a, int b, int t, int g, int n) {
+    return (((size_t)b * a.seqlen + t) * a.ngroups + g) * a.dstate + n;
+}
+__host__ __device__ inline size_t ix_bh(const BwdArgs &a, int b, int h) { return (size_t)b * a.nheads + h; }
+__host__ __device__ inline size_t ix_pn(const BwdArgs &a, int b, int h, int c) {  // complex elements
+    return (ix_bh(a, b, h) * a.nchunks + c) * ((size_t)a.headdim * a.dstate);
+}
+__host__ __device__ inline int group_of(const BwdArgs &a, int h) { return h / (a.nheads / a.ngroups); }
+
+// ------------------------------------------------ shared-memory layout
+struct Smem {
+    float *d;                    // [QC]
+    float *acs, *e, *w;          // [QC][2]
+    float *X, *dY;               // [QC][PS]
+    float *Bs, *Cs;              // [QC][NS], complex n at 2n, 2n+1
+    float *Hin, *Gh;             // [P_MAX][NS]
+    float *GL, *K;               // [QC][QS2], complex s at 2s, 2s+1
+    float *XY;                   // [QC][QS1]
+    float *rowE, *colG, *F, *Ksr;  // [QC][2]
+    float *red;                  // [3][RED]: <conj(Gh), h_in> re, im; dy.x
+    float *misc;                 // [4]: lam re, im
+};
+constexpr size_t SMEM_FLOATS = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS + 2 * P_MAX * NS + 2 * QC * QS2 +
+                               QC * QS1 + 4 * 2 * QC + 3 * RED + 4;
+__host__ __device__ inline Smem smem_map(float *s) {
+    Smem m;
+    m.d = s; s += QC;
+    m.acs = s; s += 2 * QC;
+    m.e = s; s += 2 * QC;
+    m.w = s; s += 2 * QC;
+    m.X = s; s += QC * PS;
+    m.dY = s; s += QC * PS;
+    m.Bs = s; s += QC * NS;
+    m.Cs = s; s += QC * NS;
+    m.Hin = s; s += P_MAX * NS;
+    m.Gh = s; s += P_MAX * NS;
+    m.GL = s; s += QC * QS2;
+    m.K = s; s += QC * QS2;
+    m.XY = s; s += QC * QS1;
+    m.rowE = s; s += 2 * QC;
+    m.colG = s; s += 2 * QC;
+    m.F = s; s += 2 * QC;
+    m.Ksr = s; s += 2 * QC;
+    m.red = s; s += 3 * RED;
+    m.misc = s;
+    return m;
+}
+
+// ------------------------------------------------ shared loading phases
+__host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    for (int i = tid; i < QC; i += NT) {
+        const int t = c * QC + i;
+        m.d[i] = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
+    }
+}
+__host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
+                                            float *dst) {
+    for (int i = tid; i < QC * a.headdim; i += NT) {
+        const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
+        dst[s * PS + p] = t < a.seqlen ? src[ix_x(a, b, t, h, p)] : 0.f;
+    }
+}
+// complex rows of B or C: [QC][N] pairs
+__host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
+                                            float *dst) {
+    for (int i = tid; i < QC * 2 * a.dstate; i += NT) {
+        const int s = i / (2 * a.dstate), f = i % (2 * a.dstate), t = c * QC + s;
+        dst[s * NS + f] = t < a.seqlen ? src[2 * ix_bc(a, b, t, g, 0) + f] : 0.f;
+    }
+}
+// a complex [P][N] block
+__host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
+    for (int i = tid; i < a.headdim * 2 * a.dstate; i += NT) {
+        const int p = i / (2 * a.dstate), f = i % (2 * a.dstate);
+        dst[p * NS + f] = src[i];
+    }
+}
+__host__ __device__ inline c2 sm2(const float *row, int k) { return c2{row[2 * k], row[2 * k + 1]}; }
+
+// ---------------------------------------------- 1: chunk states (forward)
+__host__ __device__ inline void k1_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    load_dt(a, c, h, b, tid, m);
+    load_rows_p(a, a.x, c, h, b, tid, m.X);
+    load_rows_n(a, a.B, c, group_of(a, h), b, tid, m.Bs);
+}
+__host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    if (tid != 0) return;
+    const c2 Ah = ld2(a.A + 2 * h);
+    c2 v = cmk(0.f, 0.f);
+    float *acs_g = a.acs + 2 * (ix_bh(a, b, h) * a.nchunks + c) * QC;
+    for (int i = 0; i < QC; ++i) {
+        v = cadd(v, cscale(Ah, m.d[i]));
+        st2(m.acs + 2 * i, v);
+        st2(acs_g + 2 * i, v);
+    }
+    st2(m.misc, v);
+    st2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c), v);
+    for (int i = 0; i < QC; ++i) st2(m.w + 2 * i, cscale(cexpc(csub(v, ld2(m.acs + 2 * i))), m.d[i]));
+}
+// S[p][n] = sum_s w_s x_s[p] B_s[n]
+__host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    float *S = a.st + 2 * ix_pn(a, b, h, c);
+    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
+        const int p = i / a.dstate, n = i % a.dstate;
+        c2 acc = cmk(0.f, 0.f);
+        for (int s = 0; s < QC; ++s)
+            acc = cadd(acc, cscale(cmul(ld2(m.w + 2 * s), sm2(m.Bs + s * NS, n)), m.X[s * PS + p]));
+        st2(S + 2 * i, acc);
+    }
+}
+
+// ------------------------------------- 2: state entering each chunk (forward)
+__host__ __device__ inline void k2_pass(const BwdArgs &a, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate;
+    for (size_t i = tid; i < pn; i += NT) {
+        c2 hv = a.init ? ld2(a.init + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
+        for (int c = 0; c < a.nchunks; ++c) {
+            const size_t o = 2 * (ix_pn(a, b, h, c) + i);
+            st2(a.hin + o, hv);
+            hv = cadd(cmul(cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c))), hv), ld2(a.st + o));
+        }
+    }
+}
+
+// -------------------- 3: readout terms R = sum_l conj(e_l) dy_l conj(C_l)^T
+__host__ __device__ inline void k3_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const float *acs_g = a.acs + 2 * (ix_bh(a, b, h) * a.nchunks + c) * QC;
+    for (int i = tid; i < QC; i += NT) st2(m.e + 2 * i, cexpc(ld2(acs_g + 2 * i)));
+    load_rows_p(a, a.dy, c, h, b, tid, m.dY);
+    load_rows_n(a, a.C, c, group_of(a, h), b, tid, m.Cs);
+}
+__host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    float *R = a.st + 2 * ix_pn(a, b, h, c);  // the chunk states were consumed by pass 2
+    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
+        const int p = i / a.dstate, n = i % a.dstate;
+        c2 acc = cmk(0.f, 0.f);
+        for (int l = 0; l < QC; ++l)
+            acc = cadd(acc, cscale(cconj(cmul(ld2(m.e + 2 * l), sm2(m.Cs + l * NS, n))), m.dY[l * PS + p]));
+        st2(R + 2 * i, acc);
+    }
+}
+
+// --------------------- 4: gradient of the state leaving each chunk (backward)
+__host__ __device__ inline void k4_pass(const BwdArgs &a, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate;
+    for (size_t i = tid; i < pn; i += NT) {
+        c2 gv = a.dfinal ? ld2(a.dfinal + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
+        for (int c = a.nchunks - 1; c >= 0; --c) {
+            const size_t o = 2 * (ix_pn(a, b, h, c) + i);
+            st2(a.gh + o, gv);
+            const c2 el = cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c)));
+            gv = cadd(cmul(cconj(el), gv), ld2(a.st + o));
+        }
+        if (a.dinit) st2(a.dinit + 2 * (ix_bh(a, b, h) * pn + i), gv);
+    }
+}
+
+// ------------------------------------------------ 5: gradients of one chunk
+__host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int g = group_of(a, h);
+    load_dt(a, c, h, b, tid, m);
+    const float *acs_g = a.acs + 2 * (ix_bh(a, b, h) * a.nchunks + c) * QC;
+    const c2 lam = ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c));
+    for (int i = tid; i < QC; i += NT) {
+        const int t = c * QC + i;
+        const float d = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
+        const c2 ac = ld2(acs_g + 2 * i);
+        st2(m.acs + 2 * i, ac);
+        st2(m.e + 2 * i, cexpc(ac));
+        st2(m.w + 2 * i, cscale(cexpc(csub(lam, ac)), d));
+    }
+    if (tid == 0) st2(m.misc, lam);
+    load_rows_p(a, a.x, c, h, b, tid, m.X);
+    load_rows_p(a, a.dy, c, h, b, tid, m.dY);
+    load_rows_n(a, a.B, c, g, b, tid, m.Bs);
+    load_rows_n(a, a.C, c, g, b, tid, m.Cs);
+    load_pn(a, a.hin + 2 * ix_pn(a, b, h, c), tid, m.Hin);
+    load_pn(a, a.gh + 2 * ix_pn(a, b, h, c), tid, m.Gh);
+}
+// GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY.
+__host__ __device__ inline void k5_mats(const BwdArgs &a, int tid, const Smem &m) {
+    for (int i = tid; i < QC * QC; i += NT) {
+        const int l = i / QC, s = i % QC;
+        c2 gm = cmk(0.f, 0.f);
+        float xy = 0.f;
+        for (int n = 0; n < a.dstate; ++n) gm = cadd(gm, cmul(sm2(m.Cs + l * NS, n), sm2(m.Bs + s * NS, n)));
+        for (int p = 0; p < a.headdim; ++p) xy += m.dY[l * PS + p] * m.X[s * PS + p];
+        m.XY[l * QS1 + s] = xy;
+        if (l >= s) {
+            const c2 L = cexpc(csub(ld2(m.acs + 2 * l), ld2(m.acs + 2 * s)));
+            st2(m.GL + l * QS2 + 2 * s, cmul(gm, L));
+            st2(m.K + l * QS2 + 2 * s, cscale(L, m.d[s] * xy));
+        } else {
+            st2(m.GL + l * QS2 + 2 * s, cmk(0.f, 0.f));
+            st2(m.K + l * QS2 + 2 * s, cmk(0.f, 0.f));
+        }
+    }
+}
+__host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem &m) {
+    if (tid < QC) {  // rows of E and columns of GL o XY
+        const int t = tid;
+        c2 re = cmk(0.f, 0.f), cg = cmk(0.f, 0.f);
+        for (int s = 0; s < QC; ++s)
+            re = cadd(re, cscale(ld2(m.GL + t * QS2 + 2 * s), m.XY[t * QS1 + s] * m.d[s]));
+        for (int l = 0; l < QC; ++l) cg = cadd(cg, cscale(ld2(m.GL + l * QS2 + 2 * t), m.XY[l * QS1 + t]));
+        st2(m.rowE + 2 * t, re);
+        st2(m.colG + 2 * t, cg);
+    } else if (tid < 2 * QC) {  // F[t] = e_t dy_t . (h_in C_t)
+        const int t = tid - QC;
+        c2 acc = cmk(0.f, 0.f);
+        for (int p = 0; p < a.headdim; ++p) {
+            c2 hc = cmk(0.f, 0.f);
+            for (int n = 0; n < a.dstate; ++n) hc = cadd(hc, cmul(sm2(m.Hin + p * NS, n), sm2(m.Cs + t * NS, n)));
+            acc = cadd(acc, cscale(hc, m.dY[t * PS + p]));
+        }
+        st2(m.F + 2 * t, cmul(ld2(m.e + 2 * t), acc));
+    } else if (tid < 3 * QC) {  // Ksr[t] = x_t . (conj(Gh) B_t)
+        const int t = tid - 2 * QC;
+        c2 acc = cmk(0.f, 0.f);
+        for (int p = 0; p < a.headdim; ++p) {
+            c2 gb = cmk(0.f, 0.f);
+            for (int n = 0; n < a.dstate; ++n)
+                gb = cadd(gb, cmul(cconj(sm2(m.Gh + p * NS, n)), sm2(m.Bs + t * NS, n)));
+            acc = cadd(acc, cscale(gb, m.X[t * PS + p]));
+        }
+        st2(m.Ksr + 2 * t, acc);
+    } else if (tid < 3 * QC + RED) {  // <conj(Gh), h_in> and dy . x, partial sums
+        const int r = tid - 3 * QC;
+        c2 h0 = cmk(0.f, 0.f);
+        float dd = 0.f;
+        for (int i = r; i < a.headdim * a.dstate; i += RED) {
+            const int p = i / a.dstate, n = i % a.dstate;
+            h0 = cadd(h0, cmul(cconj(sm2(m.Gh + p * NS, n)), sm2(m.Hin + p * NS, n)));
+        }
+        for (int i = r; i < QC * a.headdim; i += RED) {
+            const int s = i / a.headdim, p = i % a.headdim;
+            dd += m.dY[s * PS + p] * m.X[s * PS + p];
+        }
+        m.red[r] = h0.re;
+        m.red[RED + r] = h0.im;
+        m.red[2 * RED + r] = dd;
+    }
+}
+__host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    if (tid != 0) return;
+    const c2 lam = ld2(m.misc), Ah = ld2(a.A + 2 * h);
+    c2 h0 = cmk(0.f, 0.f), ksum = cmk(0.f, 0.f);
+    float dd = 0.f;
+    for (int r = 0; r < RED; ++r) {
+        h0 = cadd(h0, cmk(m.red[r], m.red[RED + r]));
+        dd += m.red[2 * RED + r];
+    }
+    for (int t = 0; t < QC; ++t) ksum = cadd(ksum, cmul(ld2(m.w + 2 * t), ld2(m.Ksr + 2 * t)));
+    h0 = cmul(cexpc(lam), h0);
+    c2 run = cmk(0.f, 0.f), dAp = cmk(0.f, 0.f);
+    for (int t = QC - 1; t >= 0; --t) {
+        // colsum of E = dt_t * colsum of GL o XY
+        c2 inner = csub(ld2(m.rowE + 2 * t), cscale(ld2(m.colG + 2 * t), m.d[t]));
+        inner = cadd(inner, ld2(m.F + 2 * t));
+        inner = csub(inner, cmul(ld2(m.w + 2 * t), ld2(m.Ksr + 2 * t)));
+        if (t == QC - 1) inner = cadd(inner, cadd(h0, ksum));
+        run = cadd(run, cconj(inner));  // dalpha[t] = sum_{t' >= t} dacs[t']
+        const int tg = c * QC + t;
+        if (tg < a.seqlen) {
+            const c2 wlam = cexpc(csub(lam, ld2(m.acs + 2 * t)));
+            a.ddt[ix_dt(a, b, tg, h)] =
+                m.colG[2 * t] + cmul(wlam, ld2(m.Ksr + 2 * t)).re + cmul(cconj(run), Ah).re;
+        }
+        dAp = cadd(dAp, cscale(run, m.d[t]));
+    }
+    st2(a.dAp + 2 * (ix_bh(a, b, h) * a.nchunks + c), dAp);
+    a.dDp[ix_bh(a, b, h) * a.nchunks + c] = dd;
+}
+__host__ __device__ inline void k5_out(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const float Dh = a.D ? a.D[h] : 0.f;
+    for (int i = tid; i < QC * a.headdim; i += NT) {
+        const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
+        if (t >= a.seqlen) continue;
+        float acc = 0.f;
+        c2 gb = cmk(0.f, 0.f);
+        for (int l = s; l < QC; ++l) acc += ld2(m.GL + l * QS2 + 2 * s).re * m.dY[l * PS + p];
+        for (int n = 0; n < a.dstate; ++n) gb = cadd(gb, cmul(cconj(sm2(m.Bs + s * NS, n)), sm2(m.Gh + p * NS, n)));
+        a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * PS + p] + cmul(cconj(ld2(m.w + 2 * s)), gb).re;
+    }
+    for (int i = tid; i < QC * a.dstate; i += NT) {
+        const int s = i / a.dstate, n = i % a.dstate, t = c * QC + s;
+        if (t >= a.seqlen) continue;
+        c2 db = cmk(0.f, 0.f), dc = cmk(0.f, 0.f), xg = cmk(0.f, 0.f), yh = cmk(0.f, 0.f);
+        for (int l = s; l < QC; ++l) db = cadd(db, cmul(ld2(m.K + l * QS2 + 2 * s), sm2(m.Cs + l * NS, n)));
+        for (int r = 0; r <= s; ++r) dc = cadd(dc, cmul(ld2(m.K + s * QS2 + 2 * r), sm2(m.Bs + r * NS, n)));
+        for (int p = 0; p < a.headdim; ++p) {
+            xg = cadd(xg, cscale(sm2(m.Gh + p * NS, n), m.X[s * PS + p]));
+            yh = cadd(yh, cscale(sm2(m.Hin + p * NS, n), m.dY[s * PS + p]));
+        }
+        const size_t o = 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n);
+        st2(a.dBh + o, cadd(cconj(db), cmul(cconj(ld2(m.w + 2 * s)), xg)));
+        st2(a.dCh + o, cconj(cadd(dc, cmul(ld2(m.e + 2 * s), yh))));
+    }
+}
+
+// ---------------------------------------------------- 6: sums over heads
+__host__ __device__ inline void k6_group(const BwdArgs &a, size_t i) {  // i: complex element of dB / dC
+    const size_t per_t = (size_t)a.ngroups * a.dstate;
+    const size_t bt = i / per_t, rem = i % per_t;
+    const int g = (int)(rem / a.dstate), n = (int)(rem % a.dstate);
+    const int hpg = a.nheads / a.ngroups;
+    c2 sb = cmk(0.f, 0.f), sc = cmk(0.f, 0.f);
+    for (int j = 0; j < hpg; ++j) {
+        const size_t o = 2 * ((bt * a.nheads + (size_t)g * hpg + j) * a.dstate + n);
+        sb = cadd(sb, ld2(a.dBh + o));
+        sc = cadd(sc, ld2(a.dCh + o));
+    }
+    st2(a.dB + 2 * i, sb);
+    st2(a.dC + 2 * i, sc);
+}
+__host__ __device__ inline void k6_head(const BwdArgs &a, int h) {
+    c2 sa = cmk(0.f, 0.f);
+    float sd = 0.f;
+    for (int b = 0; b < a.batch; ++b)
+        for (int c = 0; c < a.nchunks; ++c) {
+            sa = cadd(sa, ld2(a.dAp + 2 * (ix_bh(a, b, h) * a.nchunks + c)));
+            sd += a.dDp[ix_bh(a, b, h) * a.nchunks + c];
+        }
+    st2(a.dA + 2 * h, sa);
+    if (a.dD) a.dD[h] = sd;
+}
+
+}  // namespace bwdc
+}  // namespace ssd

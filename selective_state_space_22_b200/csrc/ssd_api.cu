@@ -201,6 +201,46 @@ namespace ssd {
 void set_last_error(const char *msg) { g_last_error = msg; }
 }  // namespace ssd
 
+// The backward scans (real or complex), after validation.
+static ssd_status run_bwd(bool cplx, const float *x, const float *dt, const float *A, const float *B,
+                          const float *C, const float *D, const float *init_state, const float *dy,
+                          const float *dfinal, float *dx, float *ddt, float *dA, float *dB, float *dC,
+                          float *dD, float *dinit, int batch, int seqlen, int nheads, int headdim,
+                          int ngroups, int dstate, void *workspace, size_t workspace_bytes, void *stream) {
+    ssd_status s = check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, 64);
+    if (s != SSD_OK) return s;
+    if (!cplx && !ssd::bwd_supported(headdim, dstate))
+        return fail(SSD_ERR_UNSUPPORTED, "the backward scan takes headdim <= 64 and dstate <= 128 "
+                    "(got %d and %d)", headdim, dstate);
+    if (cplx && !ssd::bwd_complex_supported(headdim, dstate))
+        return fail(SSD_ERR_UNSUPPORTED, "the complex backward scan takes headdim <= 64 and dstate <= 64 "
+                    "(got %d and %d)", headdim, dstate);
+    if (!A || !dA) return fail(SSD_ERR_INVALID_ARG, "A and dA are required");
+    if ((long long)batch * seqlen > 0 && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C, dy, dx, ddt, dB and dC are required");
+    for (const void *p : {(const void *)x, (const void *)dt, (const void *)A, (const void *)B,
+                          (const void *)C, (const void *)D, (const void *)init_state, (const void *)dy,
+                          (const void *)dfinal, (const void *)dx, (const void *)ddt, (const void *)dA,
+                          (const void *)dB, (const void *)dC, (const void *)dD, (const void *)dinit})
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    if ((unsigned long long)batch * seqlen * ngroups * dstate / 256 >= (1ULL << 31))
+        return fail(SSD_ERR_UNSUPPORTED, "batch * seqlen * ngroups * dstate is beyond the supported grid");
+    const size_t need = cplx ? ssd::bwd_complex_workspace_bytes(batch, seqlen, nheads, headdim, dstate)
+                             : ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need)
+            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    }
+    ssd::BwdCall call{x, dt, A, B, C, D, init_state, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit,
+                      batch, seqlen, nheads, headdim, ngroups, dstate};
+    cudaError_t e = cplx ? ssd::launch_scan_bwd_complex(call, workspace, static_cast<cudaStream_t>(stream))
+                         : ssd::launch_scan_bwd(call, workspace, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "launching the backward scan");
+    return SSD_OK;
+}
+
 extern "C" {
 
 size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,
@@ -268,38 +308,31 @@ size_t ssd_scan_bwd_workspace_size(int batch, int seqlen, int nheads, int headdi
     return ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
 }
 
+size_t ssd_scan_bwd_complex_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,
+                                           int dstate) {
+    if (check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, 64) != SSD_OK)
+        return SSD_WORKSPACE_INVALID;
+    if (!ssd::bwd_complex_supported(headdim, dstate)) return SSD_WORKSPACE_INVALID;
+    return ssd::bwd_complex_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
+}
+
 ssd_status ssd_scan_bwd(const float *x, const float *dt, const float *A, const float *B,
                         const float *C, const float *D, const float *init_state, const float *dy,
                         const float *dfinal, float *dx, float *ddt, float *dA, float *dB, float *dC,
                         float *dD, float *dinit, int batch, int seqlen, int nheads, int headdim,
                         int ngroups, int dstate, void *workspace, size_t workspace_bytes, void *stream) {
-    ssd_status s = check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, 64);
-    if (s != SSD_OK) return s;
-    if (!ssd::bwd_supported(headdim, dstate))
-        return fail(SSD_ERR_UNSUPPORTED, "the backward scan takes headdim <= 64 and dstate <= 128 "
-                    "(got %d and %d)", headdim, dstate);
-    if (!A || !dA) return fail(SSD_ERR_INVALID_ARG, "A and dA are required");
-    if ((long long)batch * seqlen > 0 && (!x || !dt || !B || !C || !dy || !dx || !ddt || !dB || !dC))
-        return fail(SSD_ERR_INVALID_ARG, "x, dt, B, C, dy, dx, ddt, dB and dC are required");
-    for (const void *p : {(const void *)x, (const void *)dt, (const void *)A, (const void *)B,
-                          (const void *)C, (const void *)D, (const void *)init_state, (const void *)dy,
-                          (const void *)dfinal, (const void *)dx, (const void *)ddt, (const void *)dA,
-                          (const void *)dB, (const void *)dC, (const void *)dD, (const void *)dinit})
-        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-    if ((unsigned long long)batch * seqlen * ngroups * dstate / 256 >= (1ULL << 31))
-        return fail(SSD_ERR_UNSUPPORTED, "batch * seqlen * ngroups * dstate is beyond the supported grid");
-    const size_t need = ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need)
-            return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
-                        workspace ? workspace_bytes : (size_t)0);
-        if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
-    }
-    ssd::BwdCall call{x, dt, A, B, C, D, init_state, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit,
-                      batch, seqlen, nheads, headdim, ngroups, dstate};
-    cudaError_t e = ssd::launch_scan_bwd(call, workspace, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) return cuda_fail(e, "launching the backward scan");
-    return SSD_OK;
+    return run_bwd(false, x, dt, A, B, C, D, init_state, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit, batch,
+                   seqlen, nheads, headdim, ngroups, dstate, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_scan_bwd_complex(const float *x, const float *dt, const float *A, const float *B,
+                                const float *C, const float *D, const float *init_state, const float *dy,
+                                const float *dfinal, float *dx, float *ddt, float *dA, float *dB,
+                                float *dC, float *dD, float *dinit, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate, void *workspace,
+                                size_t workspace_bytes, void *stream) {
+    return run_bwd(true, x, dt, A, B, C, D, init_state, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit, batch,
+                   seqlen, nheads, headdim, ngroups, dstate, workspace, workspace_bytes, stream);
 }
 
 ssd_status ssd_get_device_status(void *stream) {

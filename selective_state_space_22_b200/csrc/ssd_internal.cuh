@@ -95,6 +95,11 @@ struct BwdCall {
 bool bwd_supported(int headdim, int dstate);
 size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate);
 cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st);
+// Complex variant: A, B, C, init_state, dfinal and dA, dB, dC, dinit are float
+// pairs; headdim <= 64, dstate <= 64.
+bool bwd_complex_supported(int headdim, int dstate);
+size_t bwd_complex_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate);
+cudaError_t launch_scan_bwd_complex(const BwdCall &call, void *ws, cudaStream_t st);
 
 cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_state,
                                       size_t nfloats, cudaStream_t st);

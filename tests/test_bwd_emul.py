@@ -29,8 +29,9 @@ def emul(tmp_path_factory):
     subprocess.check_call(["g++", "-std=c++17", "-O2", "-fPIC", "-shared", "-I", CSRC, "-o", out,
                            os.path.join(HERE, "bwd_emul.cpp")])
     lib = ctypes.CDLL(out)
-    lib.emulate_scan_bwd.argtypes = [F] * 16 + [ctypes.c_int] * 6
-    lib.emulate_scan_bwd.restype = ctypes.c_int
+    for name in ("emulate_scan_bwd_real", "emulate_scan_bwd_complex"):
+        getattr(lib, name).argtypes = [F] * 16 + [ctypes.c_int] * 6
+        getattr(lib, name).restype = ctypes.c_int
     return lib
 
 
@@ -42,24 +43,39 @@ def _p(a):
     return None if a is None else a.ctypes.data_as(F)
 
 
-def run(emul, b, T, H, P, G, N, init=True, use_D=True, use_dfinal=True, seed=0, a_range=(1.0, 16.0)):
+def _c64(a):
+    """complex128 -> interleaved float32 pairs (complex64 memory)."""
+    return None if a is None else np.ascontiguousarray(a, np.complex64).view(np.float32)
+
+
+def run(emul, b, T, H, P, G, N, init=True, use_D=True, use_dfinal=True, seed=0, a_range=(1.0, 16.0),
+        cplx=False):
     rng = np.random.default_rng(seed)
-    p = pins.rand_problem(rng, b, T, H, P, G, N, init=init, a_range=a_range)
+    p = pins.rand_problem(rng, b, T, H, P, G, N, cplx=cplx, init=init, a_range=a_range)
     if not use_D:
         p["D"] = None
-    # float32 values, widened exactly for the oracle
-    p = {k: (None if v is None else _f32(v).astype(np.float64)) for k, v in p.items()}
+    # float32 / complex64 values, widened exactly for the oracle
+    narrow = lambda v: v.astype(np.complex64 if np.iscomplexobj(v) else np.float32)
+    p = {k: (None if v is None else np.ascontiguousarray(narrow(v).astype(
+        np.complex128 if np.iscomplexobj(v) else np.float64))) for k, v in p.items()}
     dy = _f32(rng.standard_normal((b, T, H, P))).astype(np.float64)
-    dfinal = _f32(rng.standard_normal((b, H, P, N))).astype(np.float64) if use_dfinal else None
+    shp = (b, H, P, N)
+    dfinal = None
+    if use_dfinal:
+        dfinal = rng.standard_normal(shp) + (1j * rng.standard_normal(shp) if cplx else 0)
+        dfinal = np.ascontiguousarray(narrow(dfinal).astype(np.complex128 if cplx else np.float64))
     ref = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"], dy, dfinal)
+    sdt = np.complex64 if cplx else np.float32
     out = dict(dx=np.zeros((b, T, H, P), np.float32), ddt=np.zeros((b, T, H), np.float32),
-               dA=np.zeros(H, np.float32), dB=np.zeros((b, T, G, N), np.float32),
-               dC=np.zeros((b, T, G, N), np.float32), dD=np.zeros(H, np.float32),
-               dinit=np.zeros((b, H, P, N), np.float32))
-    args = [_f32(p["x"]), _f32(p["dt"]), _f32(p["A"]), _f32(p["B"]), _f32(p["C"]), _f32(p["D"]),
-            _f32(p["init_state"]), _f32(dy), _f32(dfinal)]
+               dA=np.zeros(H, sdt), dB=np.zeros((b, T, G, N), sdt), dC=np.zeros((b, T, G, N), sdt),
+               dD=np.zeros(H, np.float32), dinit=np.zeros((b, H, P, N), sdt))
+    st = _c64 if cplx else _f32
+    args = [_f32(p["x"]), _f32(p["dt"]), st(p["A"]), st(p["B"]), st(p["C"]), _f32(p["D"]),
+            st(p["init_state"]), _f32(dy), st(dfinal)]
     names = ("dx", "ddt", "dA", "dB", "dC", "dD", "dinit")
-    rc = emul.emulate_scan_bwd(*[_p(a) for a in args], *[_p(out[k]) for k in names], b, T, H, P, G, N)
+    fn = emul.emulate_scan_bwd_complex if cplx else emul.emulate_scan_bwd_real
+    outp = [(out[k].view(np.float32) if out[k].dtype == np.complex64 else out[k]) for k in names]
+    rc = fn(*[_p(a) for a in args], *[_p(o) for o in outp], b, T, H, P, G, N)
     assert rc == 0
     return {k: pins.rel_err(out[k], ref[k]) for k in names}
 
@@ -96,4 +112,24 @@ def test_empty_sequence(emul):
 def test_steep_decay(emul):
     """A in [-100, -40]: per-step decays far below one; nothing may overflow."""
     errs = run(emul, 1, 150, 2, 4, 1, 8, seed=23, a_range=(40.0, 100.0))
+    assert max(errs.values()) <= TOL, errs
+
+
+# ------------------------------------------------------------------ complex
+@pytest.mark.parametrize("T", [1, 31, 32, 33, 100])
+def test_complex_ragged_and_multi_chunk(emul, T):
+    errs = run(emul, 2, T, 4, 8, 2, 16, init=(T % 2 == 1), seed=40 + T, cplx=True)
+    assert max(errs.values()) <= TOL, errs
+
+
+def test_complex_mamba3lite_head_shape(emul):
+    """Head dim 64 and complex d_state 64 (the Mamba-3-Lite head), one group per head."""
+    errs = run(emul, 1, 70, 2, 64, 2, 64, seed=50, cplx=True)
+    assert max(errs.values()) <= TOL, errs
+
+
+def test_complex_optional_inputs_absent_and_empty(emul):
+    errs = run(emul, 2, 50, 2, 4, 1, 8, init=False, use_D=False, use_dfinal=False, seed=51, cplx=True)
+    assert max(errs.values()) <= TOL, errs
+    errs = run(emul, 2, 0, 3, 4, 1, 8, seed=52, cplx=True)
     assert max(errs.values()) <= TOL, errs
