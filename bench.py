@@ -22,6 +22,10 @@ instead: a step is one ``ssd_state_update`` call that advances 256 sequences by
 one token each (the float32 state, 537 MB, is streamed through HBM every step,
 so L2 holds nothing from one step to the next).
 
+``--workload mamba2-bitmamba1b-layer-bwd-f32`` times the backward instead: a
+step is one ``ssd_scan_bwd`` call (all seven gradients of the float32 scan at
+the layer shape, given seeded dy and dfinal), timed and flushed as above.
+
 ``--impl reference`` times the fp64 CPU oracle (the program the GPU results are
 checked against) on the host cores instead, each step a bounded sample of the
 same workload; under torchrun only rank 0 runs it.
