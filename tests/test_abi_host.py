@@ -108,3 +108,47 @@ def test_binding_rejects_cpu_tensors(lib):
     with pytest.raises(ValueError):
         ssd.ssd_scan_fwd(x, torch.zeros(1, 8, 2), torch.zeros(2), x.new_zeros(1, 8, 1, 128),
                          x.new_zeros(1, 8, 1, 128))
+
+
+def test_bwd_workspace_size(lib):
+    bad = ssd.SSD_WORKSPACE_INVALID
+    assert ssd.ssd_scan_bwd_workspace_size(2, 2048, 64, 64, 1, 128) > 0
+    assert lib.ssd_scan_bwd_workspace_size(2, 2048, 64, 65, 1, 128) == bad      # headdim > 64
+    assert lib.ssd_scan_bwd_workspace_size(2, 2048, 64, 64, 3, 128) == bad      # groups must divide heads
+    assert lib.ssd_scan_bwd_complex_workspace_size(4, 2048, 16, 64, 16, 64) > 0
+    assert lib.ssd_scan_bwd_complex_workspace_size(4, 2048, 16, 64, 16, 128) == bad  # complex dstate > 64
+
+
+def bwd_call(lib, fn="ssd_scan_bwd", **over):
+    args = dict(x=FAKE, dt=FAKE, A=FAKE, B=FAKE, C=FAKE, D=None, init=None, dy=FAKE, dfinal=None,
+                dx=FAKE, ddt=FAKE, dA=FAKE, dB=FAKE, dC=FAKE, dD=None, dinit=None,
+                b=1, T=16, H=2, P=64, G=1, N=64, ws=FAKE, wsb=1 << 30, stream=None)
+    args.update(over)
+    a = args
+    return getattr(lib, fn)(a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["init"], a["dy"], a["dfinal"],
+                            a["dx"], a["ddt"], a["dA"], a["dB"], a["dC"], a["dD"], a["dinit"],
+                            a["b"], a["T"], a["H"], a["P"], a["G"], a["N"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("fn", ["ssd_scan_bwd", "ssd_scan_bwd_complex"])
+@pytest.mark.parametrize("over,status,msg", [
+    (dict(x=None), ssd.SSD_ERR_INVALID_ARG, "required"),
+    (dict(dy=None), ssd.SSD_ERR_INVALID_ARG, "required"),
+    (dict(dA=None), ssd.SSD_ERR_INVALID_ARG, "required"),
+    (dict(P=65), ssd.SSD_ERR_UNSUPPORTED, "headdim <= 64"),
+    (dict(G=3), ssd.SSD_ERR_INVALID_ARG, "divide"),
+    (dict(T=-1), ssd.SSD_ERR_INVALID_ARG, ">= 0"),
+    (dict(dB=ctypes.c_void_p((1 << 20) + 4)), ssd.SSD_ERR_INVALID_ARG, "aligned"),
+    (dict(ws=None), ssd.SSD_ERR_WORKSPACE, "needed"),
+    (dict(wsb=16), ssd.SSD_ERR_WORKSPACE, "needed"),
+])
+def test_bwd_validation(lib, fn, over, status, msg):
+    assert bwd_call(lib, fn, **over) == status
+    assert msg in ssd.ssd_last_error()
+
+
+def test_bwd_dstate_limits(lib):
+    assert bwd_call(lib, "ssd_scan_bwd", N=129) == ssd.SSD_ERR_UNSUPPORTED
+    assert "dstate <= 128" in ssd.ssd_last_error()
+    assert bwd_call(lib, "ssd_scan_bwd_complex", N=65) == ssd.SSD_ERR_UNSUPPORTED
+    assert "dstate <= 64" in ssd.ssd_last_error()
