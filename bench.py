@@ -24,7 +24,9 @@ so L2 holds nothing from one step to the next).
 
 ``--workload mamba2-bitmamba1b-layer-bwd-f32`` times the backward instead: a
 step is one ``ssd_scan_bwd`` call (all seven gradients of the float32 scan at
-the layer shape, given seeded dy and dfinal), timed and flushed as above.
+the layer shape, given seeded dy and dfinal), timed and flushed as above;
+``--workload mamba3lite-complex-bwd-f32`` does the same for the complex scan
+(``ssd_scan_bwd_complex``) at the Mamba-3-Lite layer shape.
 
 ``--impl reference`` times the fp64 CPU oracle (the program the GPU results are
 checked against) on the host cores instead, each step a bounded sample of the
@@ -663,26 +665,34 @@ def bench_ours(args, shape):
 
 
 # --------------------------------------------------------------- backward
+BWD_METRIC = {False: "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
+              True: "SSD complex scan backward tokens/s at Mamba-3-Lite layer shape (float32); % of HBM roofline"}
+
+
 def bwd_bytes(shape) -> int:
-    """Per call (float32): x and dy read, dx written; dt read, ddt written; B and C
-    read, dB and dC written; init_state and dfinal read, dinit written; A and D
-    read, dA and dD written."""
+    """Per call: x and dy read, dx written; dt read, ddt written; B and C read, dB
+    and dC written; init_state and dfinal read, dinit written; A and D read, dA
+    and dD written.  Float32, with the complex tensors (A, B, C, states and their
+    gradients) at 8 bytes an element for a complex workload."""
     b, T, H, P, G, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups, shape.dstate
     tok = b * T
-    return 4 * (3 * tok * H * P + 2 * tok * H + 4 * tok * G * N + 3 * b * H * P * N + 4 * H)
+    z = 8 if shape.complex else 4
+    return 4 * (3 * tok * H * P + 2 * tok * H + 2 * H) + z * (4 * tok * G * N + 3 * b * H * P * N + 2 * H)
 
 
 def bwd_cpu_units(shape, units, threads):
     """The oracle's gradient over the given (batch, head) sequences, one per
     thread; returns seconds."""
     import numpy as np
+    import torch
 
     import oracle
     from selective_state_space_22_b200 import inputs
 
     lib = oracle.load()
     w = inputs.widen_all(inputs.scan_inputs(shape))
-    up = {k: v.double().numpy() for k, v in inputs.bwd_upstream(shape).items()}
+    up = {k: (v.to(torch.complex128) if v.is_complex() else v.double()).numpy()
+          for k, v in inputs.bwd_upstream(shape).items()}
     c = np.ascontiguousarray
 
     def one(unit):
@@ -731,14 +741,16 @@ def bench_bwd(args, shape):
     up = inputs.bwd_upstream(shape)
     d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
     u = {k: v.to(dev) for k, v in up.items()}
-    nbytes = ssd.ssd_scan_bwd_workspace_size(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
-                                             shape.ngroups, shape.dstate)
+    size_fn = ssd.ssd_scan_bwd_complex_workspace_size if shape.complex else ssd.ssd_scan_bwd_workspace_size
+    nbytes = size_fn(shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups, shape.dstate)
     ws = torch.zeros(max(nbytes, 16), dtype=torch.uint8, device=dev)
     out = {}
 
+    fn = ssd.ssd_scan_bwd_complex if shape.complex else ssd.ssd_scan_bwd
+
     def step():
-        out.update(ssd.ssd_scan_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
-                                    u["dy"], u["dfinal"], workspace=ws))
+        out.update(fn(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                      u["dy"], u["dfinal"], workspace=ws))
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
@@ -772,7 +784,8 @@ def bench_bwd(args, shape):
     t_call = statistics.median(per_step_ms) / 1e3
     roofline = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"], "traffic": None,
-                "kernel": "ssd_scan_bwd (6 CUDA-core kernels, timed as one call)",
+                "kernel": ("ssd_scan_bwd_complex" if shape.complex else "ssd_scan_bwd")
+                + " (6 CUDA-core kernels, timed as one call)",
                 "algorithmic_bytes_per_launch": abytes,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
                 if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
@@ -816,13 +829,14 @@ def bench_bwd(args, shape):
         cpu = bwd_cpu_baseline(shape)
         cpu.pop("seconds", None)
     line = {
-        "metric": "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
+        "metric": BWD_METRIC[shape.complex],
         "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
         "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads,
                    "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
-                   "chunk": 64, "io_dtype": "f32", "l2": "flushed between timed steps (512 MiB write)",
+                   "chunk": shape.chunk, "io_dtype": "f32", "complex": shape.complex,
+                   "l2": "flushed between timed steps (512 MiB write)",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
         "gpu_launches": 7 * args.steps,
@@ -846,14 +860,12 @@ def bench_reference_bwd(args, shape):
     threads = oracle_threads()
     n = max(1, min(shape.batch * shape.nheads, 16, threads))
     units = [(i // shape.nheads, i % shape.nheads) for i in range(n)]
-    for _ in range(max(args.warmup, 3) if args.warmup > 0 else 0):
-        pass  # the oracle has no warm-up state; warm-up steps are not timed work
     secs = [bwd_cpu_units(shape, units, threads) for _ in range(args.steps)]
     tokens = shape.seqlen * n / shape.nheads
     value = tokens * args.steps / sum(secs)
     cpu = {"value": value, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
            "sample": f"{n} of {shape.batch * shape.nheads} (batch, head) sequences per step of {shape.name}"}
-    line = {"metric": "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
+    line = {"metric": BWD_METRIC[shape.complex],
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * sum(secs) / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -879,8 +891,8 @@ def main(argv=None):
     args = ap.parse_args(argv)
     from selective_state_space_22_b200 import inputs
 
-    if args.workload == inputs.BWD.name:
-        shape = inputs.BWD
+    if args.workload in inputs.BWD_WORKLOADS:
+        shape = inputs.BWD_WORKLOADS[args.workload]
         return bench_reference_bwd(args, shape) if args.impl == "reference" else bench_bwd(args, shape)
     if args.workload == inputs.DECODE.name:
         shape = inputs.DECODE

@@ -23,7 +23,7 @@ __all__ = ["SSDError", "ssd_scan_fwd", "ssd_scan_fwd_complex", "ssd_state_update
            "ssd_state_update_complex", "ssd_scan_workspace_size", "ssd_scan_kernel_launches", "ssd_get_device_status",
            "ssd_scan_fwd_noalloc", "ssd_last_error", "ssd_version", "load_library", "LIB_PATH",
            "SSD_WORKSPACE_INVALID", "ssd_scan_bwd", "ssd_scan_bwd_workspace_size",
-           "ssd_scan_bwd_complex"]
+           "ssd_scan_bwd_complex", "ssd_scan_bwd_complex_workspace_size"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -356,6 +356,13 @@ def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=No
     return out
 
 
+def ssd_scan_bwd_complex_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate) -> int:
+    n = load_library().ssd_scan_bwd_complex_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate)
+    if n == SSD_WORKSPACE_INVALID:
+        raise SSDError(1, "invalid sizes for the complex backward scan")
+    return n
+
+
 def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=None, stream=None):
     """Gradients of L = sum <dy, y> + Re <dfinal, final_state> through the complex
     scan.  A, B, C, init_state, dfinal complex64; x, dt, D, dy float32.  Returns
@@ -379,10 +386,7 @@ def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, work
                dB=torch.empty_like(B), dC=torch.empty_like(C),
                dD=None if D is None else torch.empty_like(D),
                dinit=torch.empty((b, H, P, N), dtype=c, device=dev))
-    n = lib.ssd_scan_bwd_complex_workspace_size(b, T, H, P, G, N)
-    if n == SSD_WORKSPACE_INVALID:
-        raise SSDError(1, "invalid sizes for the complex backward scan")
-    ws = workspace if workspace is not None else _workspace(dev, n)
+    ws = workspace if workspace is not None else _workspace(dev, ssd_scan_bwd_complex_workspace_size(b, T, H, P, G, N))
     with torch.cuda.device(dev):
         st = lib.ssd_scan_bwd_complex(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
                                       _ptr(dy), _ptr(dfinal), _ptr(out["dx"]), _ptr(out["ddt"]), _ptr(out["dA"]),

@@ -83,13 +83,24 @@ BWD = ScanShape("mamba2-bitmamba1b-layer-bwd-f32", 2, 2048, 64, 64, 1, 128, 64, 
                 init_state=True, seed=SEED_BASE + 5)
 
 
+# The same at the Mamba-3-Lite complex layer shape (32-token chunks).
+BWD_COMPLEX = ScanShape("mamba3lite-complex-bwd-f32", 4, 2048, 16, 64, 16, 64, 32, "f32",
+                        complex=True, init_state=True, seed=SEED_BASE + 6)
+BWD_WORKLOADS = {w.name: w for w in (BWD, BWD_COMPLEX)}
+
+
 def bwd_upstream(shape: ScanShape) -> dict:
-    """The gradients arriving at y and final_state: dy [b,T,H,P] and dfinal
-    [b,H,P,N], float32 N(0,1), seeded from the workload's seed."""
+    """The gradients arriving at y and final_state: dy [b,T,H,P] float32 N(0,1)
+    and dfinal [b,H,P,N] (float32 N(0,1), or complex64 with re/im N(0,1/2) for a
+    complex workload), seeded from the workload's seed."""
     gen = torch.Generator().manual_seed(shape.seed + 1000)
     b, T, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
-    return {"dy": torch.randn((b, T, H, P), generator=gen),
-            "dfinal": torch.randn((b, H, P, N), generator=gen)}
+    dy = torch.randn((b, T, H, P), generator=gen)
+    if shape.complex:
+        re = torch.randn((b, H, P, N), generator=gen) * 0.5 ** 0.5
+        im = torch.randn((b, H, P, N), generator=gen) * 0.5 ** 0.5
+        return {"dy": dy, "dfinal": torch.complex(re, im)}
+    return {"dy": dy, "dfinal": torch.randn((b, H, P, N), generator=gen)}
 
 
 def _tdtype(name: str) -> torch.dtype:
