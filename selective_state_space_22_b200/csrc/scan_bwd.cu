@@ -1,7 +1,7 @@
 // scan_bwd.cu -- gradients of the real scan on CUDA cores (fp32), chunk by chunk.
 //
 // The arithmetic is in scan_bwd_body.cuh; this file only launches it.  Six
-// kernels run on the caller's stream:
+// steps, seven launches, run on the caller's stream:
 //   1. chunk states S_c and the within-chunk cumulative decay      grid (chunks, heads, batch)
 //   2. the state entering each chunk, h_in (a forward pass over chunks)   grid (heads, batch)
 //   3. the readout terms R_c = sum_l exp(acs[l]) dy_l C_l^T         grid (chunks, heads, batch)
@@ -9,6 +9,7 @@
 //      chunks), and dinit                                            grid (heads, batch)
 //   5. dx, ddt and each head's dB, dC, dA, dD parts of one chunk    grid (chunks, heads, batch)
 //   6. dB, dC summed over the heads of a group; dA, dD over batch and chunks
+//      (two kernels)
 // Sums run in a fixed order, so repeated calls give identical bits.  The complex
 // variant (scan_bwd_complex_body.cuh) runs the same six steps on 32-token chunks.
 #include "scan_bwd_body.cuh"
