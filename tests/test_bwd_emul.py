@@ -133,3 +133,55 @@ def test_complex_optional_inputs_absent_and_empty(emul):
     assert max(errs.values()) <= TOL, errs
     errs = run(emul, 2, 0, 3, 4, 1, 8, seed=52, cplx=True)
     assert max(errs.values()) <= TOL, errs
+
+
+def _run_custom(emul, p, dy, dfinal, cplx=False):
+    """Run the phases on a given float32/complex64-exact problem and return the errors."""
+    ref = oracle.scan_bwd(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"], dy, dfinal)
+    b, T, H, P = p["x"].shape
+    G, N = p["B"].shape[2], p["B"].shape[3]
+    sdt = np.complex64 if cplx else np.float32
+    out = dict(dx=np.zeros((b, T, H, P), np.float32), ddt=np.zeros((b, T, H), np.float32),
+               dA=np.zeros(H, sdt), dB=np.zeros((b, T, G, N), sdt), dC=np.zeros((b, T, G, N), sdt),
+               dD=np.zeros(H, np.float32), dinit=np.zeros((b, H, P, N), sdt))
+    st = _c64 if cplx else _f32
+    args = [_f32(p["x"]), _f32(p["dt"]), st(p["A"]), st(p["B"]), st(p["C"]), _f32(p["D"]),
+            st(p["init_state"]), _f32(dy), st(dfinal)]
+    names = ("dx", "ddt", "dA", "dB", "dC", "dD", "dinit")
+    fn = emul.emulate_scan_bwd_complex if cplx else emul.emulate_scan_bwd_real
+    outp = [(out[k].view(np.float32) if out[k].dtype == np.complex64 else out[k]) for k in names]
+    assert fn(*[_p(a) for a in args], *[_p(o) for o in outp], b, T, H, P, G, N) == 0
+    return {k: pins.rel_err(out[k], ref[k]) for k in names}
+
+
+def _exact(p):
+    narrow = lambda v: v.astype(np.complex64 if np.iscomplexobj(v) else np.float32)
+    return {k: (None if v is None else np.ascontiguousarray(narrow(v).astype(
+        np.complex128 if np.iscomplexobj(v) else np.float64))) for k, v in p.items()}
+
+
+@pytest.mark.parametrize("cplx", [False, True])
+def test_zero_dt_tokens_inside_the_sequence(emul, cplx):
+    """dt = 0 on some valid tokens: no decay and no input there, but D x still
+    reaches y, so dx keeps its D dy part."""
+    rng = np.random.default_rng(60)
+    p = pins.rand_problem(rng, 1, 90, 2, 4, 1, 8, cplx=cplx, init=True)
+    p["dt"][0, ::7, :] = 0.0
+    p = _exact(p)
+    dy = rng.standard_normal((1, 90, 2, 4)).astype(np.float32).astype(np.float64)
+    dfinal = rng.standard_normal((1, 2, 4, 8)) + (1j * rng.standard_normal((1, 2, 4, 8)) if cplx else 0)
+    dfinal = _exact({"d": dfinal})["d"]
+    errs = _run_custom(emul, p, dy, dfinal, cplx)
+    assert max(errs.values()) <= TOL, errs
+
+
+@pytest.mark.parametrize("cplx", [False, True])
+def test_no_decay(emul, cplx):
+    """A = 0 (real part 0 for complex: a pure rotation): the state never decays."""
+    rng = np.random.default_rng(61)
+    p = pins.rand_problem(rng, 1, 80, 2, 4, 1, 8, cplx=cplx, init=True)
+    p["A"] = (1j * p["A"].imag) if cplx else np.zeros_like(p["A"])
+    p = _exact(p)
+    dy = rng.standard_normal((1, 80, 2, 4)).astype(np.float32).astype(np.float64)
+    errs = _run_custom(emul, p, dy, None, cplx)
+    assert max(errs.values()) <= TOL, errs
