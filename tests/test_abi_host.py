@@ -152,3 +152,17 @@ def test_bwd_dstate_limits(lib):
     assert "dstate <= 128" in ssd.ssd_last_error()
     assert bwd_call(lib, "ssd_scan_bwd_complex", N=65) == ssd.SSD_ERR_UNSUPPORTED
     assert "dstate <= 64" in ssd.ssd_last_error()
+
+
+@pytest.mark.parametrize("lang,std", [("c", "c99"), ("c++", "c++17")])
+def test_header_compiles_as_c_and_cpp(tmp_path, lang, std):
+    """include/ssd.h is a C ABI: it must compile, pedantically, as C and as C++,
+    with no CUDA include."""
+    import subprocess
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "ssd.h"\n'
+                   "int main(void) { return ssd_scan_bwd_workspace_size(1, 1, 1, 1, 1, 1) == 0 "
+                   "&& ssd_scan_workspace_size(1, 1, 1, 1, 1, 1, 64, 0, SSD_F32) == 0; }\n")
+    cc = "gcc" if lang == "c" else "g++"
+    subprocess.check_call([cc, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                           "-x", lang, "-I", os.path.join(ROOT, "include"), str(src)])
