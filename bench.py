@@ -109,10 +109,12 @@ def algorithmic_bytes(shape) -> int:
     return n
 
 
-def algorithmic_flops(shape) -> int:
-    """2 flops per MAC; causal half of each intra-chunk product; exps not counted."""
-    b, T, H, P, G, N, Q = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups,
-                           shape.dstate, shape.chunk)
+def algorithmic_flops(shape, chunk=None) -> int:
+    """2 flops per MAC; causal half of each intra-chunk product; exps not counted.
+    ``chunk`` is the chunk length the kernel evaluates (default: the shape's)."""
+    b, T, H, P, G, N = (shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.ngroups,
+                        shape.dstate)
+    Q = chunk or shape.chunk
     total = 0
     for c0 in range(0, T, Q):
         q = min(Q, T - c0)
@@ -156,6 +158,87 @@ def lookup_traffic(kernel: str, source: str, workload: str):
         if row.get("kernel") == kernel and row.get("workload") == workload and row.get("source_sha") == sha:
             return row.get("dram_bytes_per_launch")
     return None
+
+
+# ------------------------------------------------------------ configs
+# Both arms (ours and the oracle) print the same config dict for a workload.
+def scan_config(shape, world: int) -> dict:
+    return {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
+            "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
+            "dstate": shape.dstate, "chunk": shape.chunk, "complex": shape.complex,
+            "io_dtype": "f32" if shape.complex else shape.io_dtype,
+            "state_dtype": "c64" if shape.complex else "f32", "init_state": shape.init_state,
+            "l2": "flushed between timed steps (512 MiB write)",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
+def decode_config(shape, world: int) -> dict:
+    return {"workload": shape.name, "batch": shape.batch, "nheads": shape.nheads,
+            "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
+            "io_dtype": shape.io_dtype, "state_dtype": "f32",
+            "l2": "state (537 MB) larger than L2, streamed every step",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
+def bwd_config(shape, world: int) -> dict:
+    return {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads,
+            "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
+            "chunk": shape.chunk, "io_dtype": "f32", "complex": shape.complex,
+            "l2": "flushed between timed steps (512 MiB write)",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
+MIN_TIMED_S = 0.12  # default step count: at least this much timed device work
+
+
+def pick_steps(args, warm_ms: list) -> int:
+    """--steps when given, else enough steps for MIN_TIMED_S of timed device time."""
+    if args.steps is not None:
+        return args.steps
+    t = max(statistics.median(warm_ms), 1e-3)
+    return int(min(20000, max(100, -(-MIN_TIMED_S * 1e3 // t))))
+
+
+def e2e_overlapped(hin: dict, dsets: list, run, douts: list, hout: list, k: int):
+    """End-to-end time of k steps through the public API with host buffers.
+
+    Two device buffer sets alternate.  Step i copies its inputs host -> device
+    on one stream, runs on a second and copies its outputs device -> host on a
+    third, so that step i's results travel back while step i+1's inputs come in
+    and step i+1 runs.  Events order each buffer's reuse.  Returns seconds from
+    the first input copy to the last output copy (device events)."""
+    import torch
+
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done, cmp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(s_in)
+    for i in range(k):
+        j = i & 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(cmp_done[j])     # step i-2 has read this set's inputs
+            for name, v in hin.items():
+                dsets[j][name].copy_(v, non_blocking=True)
+            in_done[j].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(in_done[j])
+            if i >= 2:
+                s_cmp.wait_event(out_done[j])    # step i-2's outputs have left this set
+            run(j)
+            cmp_done[j].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(cmp_done[j])
+            for name, v in hout[j].items():
+                v.copy_(douts[j][name], non_blocking=True)
+            out_done[j].record(s_out)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_cmp)
+    end.record(s_out)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1e3
 
 
 # ----------------------------------------------------------------- clocks
@@ -347,17 +430,23 @@ def bench_decode(args, shape):
 
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(local).start()
+    warm_ms = []
     for i in range(max(args.warmup, 3)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         step(i)
-    torch.cuda.synchronize()
+        b.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b))
     ssd.ssd_get_device_status()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     dist_barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
-    for i in range(args.steps):
+    for i in range(steps):
         starts[i].record(stream)
         step(i)
         ends[i].record(stream)
@@ -368,7 +457,7 @@ def bench_decode(args, shape):
     ssd.ssd_get_device_status()
     per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_s = dist_max(sum(per_step_ms) / 1e3, dev)
-    value = shape.batch * world * args.steps / total_s
+    value = shape.batch * world * steps / total_s
     peaks = load_peaks()
     abytes = decode_bytes(shape)
     t_launch = statistics.median(per_step_ms) / 1e3
@@ -384,49 +473,39 @@ def bench_decode(args, shape):
 
     e2e = None
     if not args.no_e2e:
-        hin = [{k: v.pin_memory() for k, v in p.items()} for p in pool_host]
-        yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in hin[0].values())
-        d2h = yh.numel() * yh.element_size()
-        k_e2e = max(3, min(args.steps, 50))
+        # per step: that step's x, dt, B, C in from pinned host memory, y back out
+        # (the state stays resident: decoding updates it in place on the device)
+        hin = {k: v.pin_memory() for k, v in pool_host[0].items()}
+        dsets = [{k: torch.empty_like(v) for k, v in pool[0].items()} for _ in range(2)]
+        douts = [{"y": torch.empty_like(y)} for _ in range(2)]
+        hout = [{"y": torch.empty(y.shape, dtype=y.dtype).pin_memory()} for _ in range(2)]
+        h2d = sum(v.numel() * v.element_size() for v in hin.values())
+        d2h = hout[0]["y"].numel() * hout[0]["y"].element_size()
+        k_e2e = max(4, min(steps, 64))
 
-        def e2e_step(i):
-            src_, dst = hin[i % DECODE_POOL], pool[i % DECODE_POOL]
-            for k in dst:
-                dst[k].copy_(src_[k], non_blocking=True)
-            step(i)
-            yh.copy_(y, non_blocking=True)
+        def run(j):
+            p = dsets[j]
+            ssd.ssd_state_update(state, p["x"], p["dt"], A, p["B"], p["C"], D, y=douts[j]["y"])
 
-        e2e_step(0)
-        torch.cuda.synchronize()
-        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_overlapped(hin, dsets, run, douts, hout, 2)
         dist_barrier()
-        torch.cuda.synchronize()
-        es.record(stream)
-        for i in range(k_e2e):
-            e2e_step(i)
-        ee.record(stream)
-        torch.cuda.synchronize()
+        e2e_s = dist_max(e2e_overlapped(hin, dsets, run, douts, hout, k_e2e), dev)
         dist_barrier()
-        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
         e2e = {"value": shape.batch * world * k_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e}
+               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e,
+               "how": "two device buffer sets; H2D, compute and D2H on three streams, overlapped"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = decode_cpu_baseline(shape)
         cpu.pop("seconds", None)
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
-        "config": {"workload": shape.name, "batch": shape.batch, "nheads": shape.nheads,
-                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
-                   "io_dtype": shape.io_dtype, "state_dtype": "f32",
-                   "l2": "state (537 MB) larger than L2, streamed every step",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "config": decode_config(shape, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
-        "gpu_launches": args.steps,
+        "gpu_launches": steps,
         "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0], statistics.median(per_step_ms),
                                 statistics.quantiles(per_step_ms, n=10)[-1]],
     }
@@ -445,16 +524,16 @@ def bench_reference_decode(args, shape):
         return 0
     for _ in range(args.warmup):
         decode_cpu_baseline(shape, seqs=1, steps=1)
-    res = [decode_cpu_baseline(shape) for _ in range(args.steps)]
+    steps = args.steps if args.steps is not None else 3
+    res = [decode_cpu_baseline(shape) for _ in range(steps)]
     secs = sum(r["seconds"] for r in res)
     tokens = sum(r["value"] * r["seconds"] for r in res)
     value = tokens / secs
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-        "config": {"workload": shape.name, "batch": shape.batch, "nheads": shape.nheads,
-                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate},
+        "config": decode_config(shape, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": res[0]["cores"], "kind": "oracle",
                          "sample": "per step " + res[0]["sample"]},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -478,18 +557,17 @@ def bench_reference(args, shape):
     units = [(0, h) for h in heads]
     for _ in range(args.warmup):
         run_oracle_units(w, units[:1], 1)
-    times = [run_oracle_units(w, units, threads) for _ in range(args.steps)]
+    steps = args.steps if args.steps is not None else 3
+    times = [run_oracle_units(w, units, threads) for _ in range(steps)]
     secs = sum(times)
-    tokens = shape.seqlen * n_heads / shape.nheads * args.steps
+    tokens = shape.seqlen * n_heads / shape.nheads * steps
     value = tokens / secs
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * secs / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "impl": "reference",
-        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
-                   "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
-                   "dstate": shape.dstate, "chunk": shape.chunk},
+        "config": scan_config(shape, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": min(threads, n_heads),
                          "kind": "oracle",
                          "sample": f"per step {n_heads} of {shape.nheads} heads of batch 0 "
@@ -528,28 +606,36 @@ def bench_ours(args, shape):
     fn = ssd.ssd_scan_fwd_complex if cplx else ssd.ssd_scan_fwd
     launches = ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
                                             shape.ngroups, shape.dstate, shape.chunk, cplx, io)
+    tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
+    kernel_chunk = 128 if tc_path else shape.chunk  # the tensor-core kernel tiles 128 tokens
 
-    def step():
-        fn(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], chunk_size=shape.chunk,
-           y=y, final_state=fs, workspace=ws)
+    def step(dd=d, yy=y, ff=fs, w=ws):
+        fn(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["init_state"], chunk_size=shape.chunk,
+           y=yy, final_state=ff, workspace=w)
 
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(local).start()
 
+    warm_ms = []
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         step()
-    torch.cuda.synchronize()
+        b.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b))
     ssd.ssd_get_device_status()
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))  # every rank the same K
 
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     dist_barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
         step()
@@ -559,17 +645,17 @@ def bench_ours(args, shape):
     dist_barrier()
     sampler.stop()
     ssd.ssd_get_device_status()
-    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    per_step_ms = [s_.elapsed_time(e_) for s_, e_ in zip(starts, ends)]
     local_s = sum(per_step_ms) / 1e3
     total_s = dist_max(local_s, dev)
-    tokens = shape.tokens * world * args.steps
+    tokens = shape.tokens * world * steps
     value = tokens / total_s
-    ms_per_step = 1e3 * total_s / args.steps
+    ms_per_step = 1e3 * total_s / steps
 
     # roofline of the dominant kernel (the whole call when it is one launch)
     peaks = load_peaks()
     abytes = algorithmic_bytes(shape)
-    aflops = algorithmic_flops(shape)
+    aflops = algorithmic_flops(shape, kernel_chunk)
     t_launch = statistics.median(per_step_ms) / 1e3 if launches == 1 else sum(per_step_ms) / len(per_step_ms) / 1e3
     hbm_t = abytes / (peaks["hbm_gbs"] * 1e9)
     tc_t = aflops / (peaks["bf16_tflops"] * 1e12)
@@ -578,7 +664,6 @@ def bench_ours(args, shape):
         achieved, peak, unit = abytes / t_launch / 1e9, peaks["hbm_gbs"], "GB/s"
     else:
         achieved, peak, unit = aflops / t_launch / 1e12, peaks["bf16_tflops"], "TFLOP/s"
-    tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
     if tc_path:
         kernel, src_name = "ssd_scan_tc_kernel", "scan_tc.cu"
     elif cplx:
@@ -589,6 +674,7 @@ def bench_ours(args, shape):
     traffic = lookup_traffic(kernel, src, shape.name)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
+                "kernel_chunk": kernel_chunk,
                 "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
                 if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
@@ -598,36 +684,26 @@ def bench_ours(args, shape):
     # end to end through the public API: pinned host inputs in, results back out
     e2e = None
     if not args.no_e2e:
-        hin = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
-        yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        fh = torch.empty(fs.shape, dtype=fs.dtype).pin_memory()
-        h2d = sum(v.numel() * v.element_size() for v in hin.values() if v is not None)
-        d2h = yh.numel() * yh.element_size() + fh.numel() * fh.element_size()
-        k_e2e = max(3, min(args.steps, 30))
+        hin = {k: v.pin_memory() for k, v in inp.items() if v is not None}
+        dsets = [{k: d[k] for k in hin}, {k: torch.empty_like(d[k]) for k in hin}]
+        douts = [{"y": y, "final_state": fs}, {"y": torch.empty_like(y), "final_state": torch.empty_like(fs)}]
+        hout = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in o.items()} for o in douts]
+        h2d = sum(v.numel() * v.element_size() for v in hin.values())
+        d2h = sum(v.numel() * v.element_size() for v in hout[0].values())
+        k_e2e = max(4, min(steps, 40))
+        full = lambda j: dict(dsets[j], **{k: None for k in d if k not in hin})
 
-        def e2e_step():
-            for k, v in hin.items():
-                if v is not None:
-                    d[k].copy_(v, non_blocking=True)
-            step()
-            yh.copy_(y, non_blocking=True)
-            fh.copy_(fs, non_blocking=True)
+        def run(j):
+            step(full(j), douts[j]["y"], douts[j]["final_state"])
 
-        e2e_step()
-        torch.cuda.synchronize()
-        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_overlapped(hin, dsets, run, douts, hout, 2)  # warm-up
         dist_barrier()
-        torch.cuda.synchronize()
-        es.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        ee.record(stream)
-        torch.cuda.synchronize()
+        e2e_s = dist_max(e2e_overlapped(hin, dsets, run, douts, hout, k_e2e), dev)
         dist_barrier()
-        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
         e2e = {"value": shape.tokens * world * k_e2e / e2e_s, "unit": "tokens/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": k_e2e,
-               "ms_per_step": 1e3 * e2e_s / k_e2e}
+               "ms_per_step": 1e3 * e2e_s / k_e2e,
+               "how": "two device buffer sets; H2D, compute and D2H on three streams, overlapped"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -635,22 +711,18 @@ def bench_ours(args, shape):
         cpu.pop("seconds", None)
 
     line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if tc_path else "f32",
         "data": "synthetic",
         "impl": "ours",
-        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
-                   "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
-                   "dstate": shape.dstate, "chunk": shape.chunk, "io_dtype": shape.io_dtype,
-                   "state_dtype": "f32", "l2": "flushed between timed steps (512 MiB write)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "config": scan_config(shape, world),
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "clocks": sampler.summary(t0, t1),
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": launches * steps,
         "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0] if len(per_step_ms) > 1 else per_step_ms[0],
                                 statistics.median(per_step_ms),
                                 statistics.quantiles(per_step_ms, n=10)[-1] if len(per_step_ms) > 1 else per_step_ms[0]],
@@ -755,18 +827,24 @@ def bench_bwd(args, shape):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
     sampler = ClockSampler(local).start()
+    warm_ms = []
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         step()
-    torch.cuda.synchronize()
+        b.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b))
     ssd.ssd_get_device_status()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     dist_barrier()
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     torch.cuda._sleep(20_000_000)  # let the host queue run ahead of the device
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         starts[i].record(stream)
         step()
@@ -778,7 +856,7 @@ def bench_bwd(args, shape):
     ssd.ssd_get_device_status()
     per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
     total_s = dist_max(sum(per_step_ms) / 1e3, dev)
-    value = shape.tokens * world * args.steps / total_s
+    value = shape.tokens * world * steps / total_s
     peaks = load_peaks()
     abytes = bwd_bytes(shape)
     t_call = statistics.median(per_step_ms) / 1e3
@@ -794,35 +872,30 @@ def bench_bwd(args, shape):
     e2e = None
     if not args.no_e2e:
         hin = {k: v.pin_memory() for k, v in list(inp.items()) + list(up.items()) if v is not None}
-        dst = {k: (d[k] if k in d else u[k]) for k in hin}
+        dsets = [{k: (d[k] if k in d else u[k]) for k in hin}, {k: torch.empty_like(v) for k, v in hin.items()}]
         step()
         torch.cuda.synchronize()
-        hout = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in out.items() if v is not None}
+        douts = [{k: v for k, v in out.items() if v is not None}, {}]
+        douts[1] = {k: torch.empty_like(v) for k, v in douts[0].items()}
+        hout = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in o.items()} for o in douts]
         h2d = sum(v.numel() * v.element_size() for v in hin.values())
-        d2h = sum(v.numel() * v.element_size() for v in hout.values())
-        k_e2e = max(3, min(args.steps, 20))
+        d2h = sum(v.numel() * v.element_size() for v in hout[0].values())
+        k_e2e = max(4, min(steps, 20))
+        size_ws = ws.numel()
+        ws2 = [ws, torch.zeros(size_ws, dtype=torch.uint8, device=dev)]
 
-        def e2e_step():
-            for k, v in hin.items():
-                dst[k].copy_(v, non_blocking=True)
-            step()
-            for k, v in hout.items():
-                v.copy_(out[k], non_blocking=True)
+        def run(j):
+            q = dsets[j]
+            fn(q["x"], q["dt"], q["A"], q["B"], q["C"], q.get("D"), q.get("init_state"), q["dy"], q["dfinal"],
+               out=dict(douts[j]), workspace=ws2[j])
 
-        e2e_step()
-        torch.cuda.synchronize()
-        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_overlapped(hin, dsets, run, douts, hout, 2)
         dist_barrier()
-        torch.cuda.synchronize()
-        es.record(stream)
-        for _ in range(k_e2e):
-            e2e_step()
-        ee.record(stream)
-        torch.cuda.synchronize()
+        e2e_s = dist_max(e2e_overlapped(hin, dsets, run, douts, hout, k_e2e), dev)
         dist_barrier()
-        e2e_s = dist_max(es.elapsed_time(ee) / 1e3, dev)
         e2e = {"value": shape.tokens * world * k_e2e / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e}
+               "d2h_bytes_per_step": d2h, "steps": k_e2e, "ms_per_step": 1e3 * e2e_s / k_e2e,
+               "how": "two device buffer sets; H2D, compute and D2H on three streams, overlapped"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -830,16 +903,12 @@ def bench_bwd(args, shape):
         cpu.pop("seconds", None)
     line = {
         "metric": BWD_METRIC[shape.complex],
-        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+        "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
-        "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen, "nheads": shape.nheads,
-                   "headdim": shape.headdim, "ngroups": shape.ngroups, "dstate": shape.dstate,
-                   "chunk": shape.chunk, "io_dtype": "f32", "complex": shape.complex,
-                   "l2": "flushed between timed steps (512 MiB write)",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "config": bwd_config(shape, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
-        "gpu_launches": 7 * args.steps,
+        "gpu_launches": 7 * steps,
         "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0], statistics.median(per_step_ms),
                                 statistics.quantiles(per_step_ms, n=10)[-1]],
     }
@@ -860,19 +929,18 @@ def bench_reference_bwd(args, shape):
     threads = oracle_threads()
     n = max(1, min(shape.batch * shape.nheads, 16, threads))
     units = [(i // shape.nheads, i % shape.nheads) for i in range(n)]
-    secs = [bwd_cpu_units(shape, units, threads) for _ in range(args.steps)]
+    steps = args.steps if args.steps is not None else 3
+    secs = [bwd_cpu_units(shape, units, threads) for _ in range(steps)]
     tokens = shape.seqlen * n / shape.nheads
-    value = tokens * args.steps / sum(secs)
+    value = tokens * steps / sum(secs)
     cpu = {"value": value, "unit": "tokens/s", "cores": min(threads, n), "kind": "oracle",
            "sample": f"{n} of {shape.batch * shape.nheads} (batch, head) sequences per step of {shape.name}"}
     line = {"metric": BWD_METRIC[shape.complex],
-            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * sum(secs) / args.steps,
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * sum(secs) / steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": shape.name, "batch": shape.batch, "seqlen": shape.seqlen,
-                       "nheads": shape.nheads, "headdim": shape.headdim, "ngroups": shape.ngroups,
-                       "dstate": shape.dstate, "io_dtype": "f32"},
+            "config": bwd_config(shape, world),
             "cpu_baseline": cpu,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -882,7 +950,8 @@ def bench_reference_bwd(args, shape):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for ~0.12 s of timed device work, >= 100)")
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mamba2-bitmamba1b-layer-bf16")

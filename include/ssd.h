@@ -34,6 +34,10 @@
  *    a complex64 tensor.  The complex output is the real part only.
  *  - Outputs never alias inputs, except: final_state may equal init_state, and
  *    ssd_state_update updates `state` in place.
+ *  - Device addresses the library caches (its error word, the no-alloc scratch)
+ *    and kernel attributes are kept per (device, current CUDA context) and looked
+ *    up again when the context changes.  Work enqueued before a cudaDeviceReset
+ *    must not be waited on with ssd_get_device_status afterwards.
  */
 #ifndef SSD_B200_H
 #define SSD_B200_H
@@ -227,8 +231,9 @@ ssd_status ssd_scan_bwd_complex(const float *x, const float *dt, const float *A,
 /*
  * Waits for `stream`, then reports and clears an error that a kernel raised on
  * the device since the last call on this device (SSD_ERR_TIMEOUT when one of the
- * tensor-core kernel's bounded waits between its warp roles gave up after 2 s;
- * the outputs of that call are then invalid), or a CUDA error from the stream.
+ * tensor-core kernel's bounded waits between its warp roles gave up after 1 s;
+ * the kernel then stops at once and the outputs of that call are invalid), or a
+ * CUDA error from the stream.
  * SSD_OK when there was none.
  */
 ssd_status ssd_get_device_status(void *stream);
@@ -252,11 +257,13 @@ ssd_status ssd_get_device_status(void *stream);
  *
  *  - It runs the float32 CUDA-core scan (for bf16 or float32 io).  Sizes whose
  *    scratch exceeds SSD_NOALLOC_SCRATCH_BYTES are rejected with
- *    SSD_ERR_WORKSPACE before anything is launched; the scratch grows with
+ *    SSD_ERR_WORKSPACE before anything is launched.  The scratch needed is
  *    batch * nheads * ceil(seqlen / chunk_size) * (headdim * dstate * 4 +
- *    chunk_size * 8) bytes.  batch and seqlen must be > 0.
- *  - The first call on a device looks up the array's device address (once, with
- *    that device current); make that first call before any stream capture.
+ *    chunk_size * 8 + 8) bytes plus up to 768 bytes of alignment padding.
+ *    batch and seqlen must be > 0.
+ *  - The first call on a device (and the first after the current CUDA context
+ *    changed, e.g. after cudaDeviceReset) looks up the array's device address,
+ *    with that device current; make that first call before any stream capture.
  *  - All calls share the one array, and each call overwrites it: calls whose
  *    work can overlap on the GPU (other streams, other host threads) race and
  *    give wrong results.  Serialise them.
@@ -268,6 +275,22 @@ ssd_status ssd_scan_fwd_noalloc(const void *x, const float *dt, const float *A,
                                 ssd_dtype io_dtype, int batch, int seqlen, int nheads,
                                 int headdim, int ngroups, int dstate, int chunk_size,
                                 void *stream);
+
+/*
+ * Test hook for the failure path (not for production use).  The pages have no
+ * counterpart: it exists so that a test can make the tensor-core kernel's
+ * bounded waits run out without faulting anything.
+ *
+ * With withhold_first_load != 0, every tensor-core scan launched afterwards (on
+ * any thread) has its load producer issue no load at all; every other role of
+ * the kernel then waits for data that never comes, gives up after
+ * wait_limit_ns nanoseconds (0: the default bound of 1 s), and the kernel
+ * leaves at once.  Its outputs are then invalid and the next
+ * ssd_get_device_status reports SSD_ERR_TIMEOUT.  withhold_first_load = 0
+ * restores normal operation; wait_limit_ns then still bounds each wait (0: the
+ * default).  Always returns SSD_OK.
+ */
+ssd_status ssd_debug_inject_stall(int withhold_first_load, unsigned long long wait_limit_ns);
 
 /* Message for the last non-OK status returned on the calling host thread. */
 const char *ssd_last_error(void);

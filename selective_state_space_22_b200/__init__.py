@@ -77,6 +77,8 @@ def load_library(path: str | None = None):
         lib.ssd_scan_bwd_complex_workspace_size.restype = _SZ
         lib.ssd_scan_bwd_complex.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, _SZ, _VP]
         lib.ssd_scan_bwd_complex.restype = _I
+        lib.ssd_debug_inject_stall.argtypes = [_I, ctypes.c_ulonglong]
+        lib.ssd_debug_inject_stall.restype = _I
         lib.ssd_get_device_status.argtypes = [_VP]
         lib.ssd_get_device_status.restype = _I
         lib.ssd_last_error.argtypes = []
@@ -322,10 +324,23 @@ def ssd_scan_bwd_workspace_size(batch, seqlen, nheads, headdim, ngroups, dstate)
     return n
 
 
-def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=None, stream=None):
+def _bwd_outputs(out, like, dev):
+    """The gradient tensors: ``out`` (a dict of preallocated tensors, checked)
+    or fresh ones shaped like the inputs."""
+    if out is None:
+        return {k: (None if v is None else torch.empty(v[0], dtype=v[1], device=dev)) for k, v in like.items()}
+    for k, v in like.items():
+        if v is None:
+            out.setdefault(k, None)
+            continue
+        _need(out.get(k), k, v[1], dev, v[0])
+    return out
+
+
+def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, out=None, workspace=None, stream=None):
     """Gradients of L = sum <dy, y> + <dfinal, final_state> through the real
     float32 scan.  Returns a dict with dx, ddt, dA, dB, dC, dD and dinit (dD is
-    None when D is None)."""
+    None when D is None); ``out`` may pass that dict preallocated."""
     lib = load_library()
     dev = x.device
     b, T, H, P = x.shape
@@ -340,10 +355,9 @@ def ssd_scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=No
     _need(init_state, "init_state", f, dev, (b, H, P, N), allow_none=True)
     _need(dy, "dy", f, dev, (b, T, H, P))
     _need(dfinal, "dfinal", f, dev, (b, H, P, N), allow_none=True)
-    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt), dA=torch.empty_like(A),
-               dB=torch.empty_like(B), dC=torch.empty_like(C),
-               dD=None if D is None else torch.empty_like(D),
-               dinit=torch.empty((b, H, P, N), dtype=f, device=dev))
+    out = _bwd_outputs(out, dict(dx=(x.shape, f), ddt=(dt.shape, f), dA=(A.shape, f), dB=(B.shape, f),
+                                 dC=(C.shape, f), dD=None if D is None else (D.shape, f),
+                                 dinit=((b, H, P, N), f)), dev)
     nbytes = ssd_scan_bwd_workspace_size(b, T, H, P, G, N)
     ws = workspace if workspace is not None else _workspace(dev, nbytes)
     with torch.cuda.device(dev):
@@ -363,7 +377,8 @@ def ssd_scan_bwd_complex_workspace_size(batch, seqlen, nheads, headdim, ngroups,
     return n
 
 
-def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, workspace=None, stream=None):
+def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, out=None, workspace=None,
+                         stream=None):
     """Gradients of L = sum <dy, y> + Re <dfinal, final_state> through the complex
     scan.  A, B, C, init_state, dfinal complex64; x, dt, D, dy float32.  Returns
     a dict with dx, ddt (float32), dA, dB, dC, dinit (complex64) and dD (float32,
@@ -382,10 +397,9 @@ def ssd_scan_bwd_complex(x, dt, A, B, C, D, init_state, dy, dfinal=None, *, work
     _need(init_state, "init_state", c, dev, (b, H, P, N), allow_none=True)
     _need(dy, "dy", f, dev, (b, T, H, P))
     _need(dfinal, "dfinal", c, dev, (b, H, P, N), allow_none=True)
-    out = dict(dx=torch.empty_like(x), ddt=torch.empty_like(dt), dA=torch.empty_like(A),
-               dB=torch.empty_like(B), dC=torch.empty_like(C),
-               dD=None if D is None else torch.empty_like(D),
-               dinit=torch.empty((b, H, P, N), dtype=c, device=dev))
+    out = _bwd_outputs(out, dict(dx=(x.shape, f), ddt=(dt.shape, f), dA=(A.shape, c), dB=(B.shape, c),
+                                 dC=(C.shape, c), dD=None if D is None else (D.shape, f),
+                                 dinit=((b, H, P, N), c)), dev)
     ws = workspace if workspace is not None else _workspace(dev, ssd_scan_bwd_complex_workspace_size(b, T, H, P, G, N))
     with torch.cuda.device(dev):
         st = lib.ssd_scan_bwd_complex(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),

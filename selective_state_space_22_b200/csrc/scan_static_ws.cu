@@ -45,10 +45,11 @@ ssd_status set_msg(ssd_status s, const char *fmt, ...) {
     return s;
 }
 
-// Device addresses of the two device globals, looked up once per device with
-// that device current.  In host code the symbols themselves are host-side
-// stand-ins and must never be handed to a kernel.
+// Device addresses of the two device globals, looked up once per (device,
+// context) with that device current.  In host code the symbols themselves are
+// host-side stand-ins and must never be handed to a kernel.
 struct DevPtrs {
+    void *ctx = nullptr;
     void *scratch = nullptr;
     int *err = nullptr;
 };
@@ -60,8 +61,9 @@ ssd_status device_ptrs(DevPtrs *out) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return set_msg(SSD_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
     if (dev < 0 || dev >= 64) return set_msg(SSD_ERR_UNSUPPORTED, "device index %d out of range", dev);
+    void *ctx = ssd::current_context();
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_ptrs[dev].scratch) {
+    if (!g_ptrs[dev].scratch || g_ptrs[dev].ctx != ctx) {
         void *s = nullptr, *er = nullptr;
         e = cudaGetSymbolAddress(&s, g_noalloc_scratch);
         if (e != cudaSuccess)
@@ -69,6 +71,7 @@ ssd_status device_ptrs(DevPtrs *out) {
         e = cudaGetSymbolAddress(&er, g_noalloc_error);
         if (e != cudaSuccess)
             return set_msg(SSD_ERR_CUDA, "cudaGetSymbolAddress(error word): %s", cudaGetErrorString(e));
+        g_ptrs[dev].ctx = ctx;
         g_ptrs[dev].scratch = s;
         g_ptrs[dev].err = static_cast<int *>(er);
     }

@@ -41,6 +41,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "ssd_internal.cuh"
@@ -90,10 +91,14 @@ enum {
     // the X ring; B_XEMPTY counts the 128 W threads and M X's commit
     B_XFULL = 12, B_XEMPTY = 15,
     // count 128 (one warpgroup).  B_HW: h_in^T written; B_H: chunk state read
-    B_CS = 18, B_W = 20, B_M = 22, B_H = 24, B_FREE = 26, B_HW = 28, NBARS = 30
+    B_CS = 18, B_W = 20, B_M = 22, B_H = 24, B_FREE = 26, B_HW = 28,
+    // count 1: a final commit of each MMA issuer, so that it can wait for its own
+    // MMAs before the CTA exits after an abort
+    B_DRAIN = 30, NBARS = 32
 };
-// misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4], bars, tmem base
-constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + NBARS * 8 + 8;
+// misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4],
+// abort word + 4 votes (8 ints), bars, tmem base
+constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + 32 + NBARS * 8 + 8;
 constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C (K-major) x B (K-major)
@@ -101,7 +106,7 @@ constexpr uint32_t IDESC_S = idesc_bf16_f32(128, 64, 1, 1);    // B^T (MN-major)
 constexpr uint32_t IDESC_YD = idesc_bf16_f32(128, 64, 0, 1);   // M (TMEM) x X (MN-major)
 constexpr uint32_t IDESC_YO = idesc_bf16_f32(128, 64, 0, 1);   // C (K-major) x h^T (MN-major)
 
-constexpr unsigned long long WAIT_NS = 2000000000ull;  // 2 s bound on every wait
+constexpr unsigned long long WAIT_NS = 1000000000ull;  // 1 s bound on every wait
 
 struct TcParams {
     __nv_bfloat16 *y;
@@ -114,6 +119,8 @@ struct TcParams {
     int runs;                    // runs per sequence (1: whole sequences)
     int run_start[MAX_RUNS + 1]; // first chunk of each run; run_start[runs] = nchunks
     int *dev_error;
+    unsigned long long wait_ns;  // bound on every wait (WAIT_NS unless a test shortens it)
+    int withhold;                // test only: the producer issues no load, so every wait runs out
 };
 
 // CTA-local tile k -> (sequence, chunk, state-only?).  CTA i owns work items
@@ -157,17 +164,37 @@ __device__ __forceinline__ unsigned long long now_ns() {
     return t;
 }
 
-// Bounded wait on an mbarrier phase (the device error word is set on timeout).
-__device__ void mbar_wait(uint64_t *bar, uint32_t parity, int *err) {
-    if (mbar_try_wait(bar, parity)) return;
+// Bounded wait on an mbarrier phase.  Returns false, without waiting further,
+// once the CTA's abort word is set; sets the device error word and the abort
+// word when the bound runs out.  A role that gets false stops issuing work and
+// leaves its tile loop (warps decide together: warp_ok).
+__device__ bool mbar_wait(uint64_t *bar, uint32_t parity, const TcParams &p, volatile int *abort_s) {
+    if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = now_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (now_ns() - t0 > WAIT_NS) {
-            atomicCAS(err, 0, DEV_TIMEOUT);
+        if (*abort_s) return false;
+        if (now_ns() - t0 > p.wait_ns) {
+            atomicCAS(p.dev_error, 0, DEV_TIMEOUT);
+            *abort_s = 1;
+            return false;
+        }
+    }
+    return true;
+}
+// The same without the abort shortcut: how a role waits for its own TMA loads
+// or MMAs to finish before the CTA exits (still bounded).
+__device__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, const TcParams &p, volatile int *abort_s) {
+    const unsigned long long t0 = now_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (now_ns() - t0 > p.wait_ns) {
+            atomicCAS(p.dev_error, 0, DEV_TIMEOUT);
+            *abort_s = 1;
             return;
         }
     }
 }
+// A warp goes on only if every lane's wait succeeded.
+__device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
@@ -271,14 +298,19 @@ __global__ void __launch_bounds__(NTH, 1)
     float *lam_s = bfac + 2 * QT;                          // [2]
     float *dh_s = lam_s + 2;                               // [2]
     float *wtot = dh_s + 2;                                // [4]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 4);
+    volatile int *abort_s = reinterpret_cast<volatile int *>(wtot + 4);  // [1], then votes [4]
+    volatile int *votes = abort_s + 4;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 12);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < B_CS; ++i)
             mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1) ? 2 : (i >= B_XEMPTY && i < B_XEMPTY + 3) ? 129 : 1);
-        for (int i = B_CS; i < NBARS; ++i) mbar_init(&bars[i], 128);
+        for (int i = B_CS; i < B_DRAIN; ++i) mbar_init(&bars[i], 128);
+        mbar_init(&bars[B_DRAIN], 1);
+        mbar_init(&bars[B_DRAIN + 1], 1);
+        *abort_s = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -291,15 +323,15 @@ __global__ void __launch_bounds__(NTH, 1)
     const uint32_t tmem = *tmem_slot;
     const int ntl = local_tiles(p);
     const uint32_t sbase = smem_u32(sm);
-    int *err = p.dev_error;
 
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
-        if (lane == 0) {
+        if (lane == 0 && !p.withhold) {
+            int last_cb[2] = {-1, -1}, last_x[X_SLOTS] = {-1, -1, -1};  // last tile loaded per slot
             for (int k = 0; k < ntl; ++k) {
                 const Tile t = decode_tile(p, k);
                 const int s = k & 1;
-                mbar_wait(&bars[B_EMPTY + s], ((k >> 1) & 1) ^ 1, err);
+                if (!mbar_wait(&bars[B_EMPTY + s], ((k >> 1) & 1) ^ 1, p, abort_s)) break;
                 uint8_t *st = sm + s * CB_BYTES;
                 uint64_t *full = &bars[B_FULL + s];
                 mbar_arrive_expect_tx(full, t.state_only ? LOAD_B : LOAD_CB);
@@ -309,11 +341,19 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 tma_load_4d(st + OFF_B, &tm_b, full, 0, t.g, t.t0, t.b);
                 tma_load_4d(st + OFF_B + 16384, &tm_b, full, 64, t.g, t.t0, t.b);
+                last_cb[s] = k;
                 const int xs = k % X_SLOTS;
-                mbar_wait(&bars[B_XEMPTY + xs], ((k / X_SLOTS) & 1) ^ 1, err);
+                if (!mbar_wait(&bars[B_XEMPTY + xs], ((k / X_SLOTS) & 1) ^ 1, p, abort_s)) break;
                 mbar_arrive_expect_tx(&bars[B_XFULL + xs], LOAD_X);
                 tma_load_4d(sm + OFF_XR + xs * 16384, &tm_x, &bars[B_XFULL + xs], 0, t.h, t.t0, t.b);
+                last_x[xs] = k;
             }
+            // Every load issued must have landed before the CTA's shared memory
+            // is released (after an abort its consumer may never have waited).
+            for (int s = 0; s < 2; ++s)
+                if (last_cb[s] >= 0) mbar_wait_drain(&bars[B_FULL + s], (last_cb[s] >> 1) & 1, p, abort_s);
+            for (int xs = 0; xs < X_SLOTS; ++xs)
+                if (last_x[xs] >= 0) mbar_wait_drain(&bars[B_XFULL + xs], (last_x[xs] / X_SLOTS) & 1, p, abort_s);
         }
     } else if (warp == 1) {
         // ------------------------------------------- MMA issuer: G and S
@@ -324,8 +364,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * CB_BYTES + OFF_C, aB = sbase + s * CB_BYTES + OFF_B;
-                mbar_wait(&bars[B_FULL + s], par, err);
-                mbar_wait(&bars[B_FREE + s], par ^ 1, err);
+                if (!mbar_wait(&bars[B_FULL + s], par, p, abort_s)) break;
+                if (!mbar_wait(&bars[B_FREE + s], par ^ 1, p, abort_s)) break;
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -336,9 +376,9 @@ __global__ void __launch_bounds__(NTH, 1)
                     }
                 }
                 mma_commit(&bars[B_G + s]);
-                mbar_wait(&bars[B_W + s], par, err);
+                if (!mbar_wait(&bars[B_W + s], par, p, abort_s)) break;
                 // S's columns held the chunk state of tile k-2 until its state update
-                if (k >= 2) mbar_wait(&bars[B_H + s], par ^ 1, err);
+                if (k >= 2 && !mbar_wait(&bars[B_H + s], par ^ 1, p, abort_s)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)  // S = B^T W
@@ -347,6 +387,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 mma_commit(&bars[B_S + s]);
                 mma_commit(&bars[B_EMPTY + s]);  // G and S are done with the slot's B and C
             }
+            mma_commit(&bars[B_DRAIN]);  // this thread's MMAs are done before the CTA exits
+            mbar_wait_drain(&bars[B_DRAIN], 0, p, abort_s);
         }
     } else if (warp == Y_MMA_WARP) {
         // --------------------------------- MMA issuer: C h_in^T and M X
@@ -360,8 +402,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 const uint32_t aH = sbase + OFF_H;
                 // G of this tile was issued after tile k-2's epilogue released the
                 // set, so C h^T's columns are free; h_in^T of this tile is written.
-                mbar_wait(&bars[B_G + s], par, err);
-                mbar_wait(&bars[B_HW + s], par, err);
+                if (!mbar_wait(&bars[B_G + s], par, p, abort_s)) break;
+                if (!mbar_wait(&bars[B_HW + s], par, p, abort_s)) break;
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -371,8 +413,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 mma_commit(&bars[B_YO + s]);     // done with the h_in^T buffer
                 mma_commit(&bars[B_EMPTY + s]);  // with G and S: done with the {C, B} slot
-                mbar_wait(&bars[B_M + s], par, err);
-                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, err);
+                if (!mbar_wait(&bars[B_M + s], par, p, abort_s)) break;
+                if (!mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s)) break;
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -383,6 +425,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 mma_commit(&bars[B_Y + s]);
                 mma_commit(&bars[B_XEMPTY + xs]);  // with the W threads: done with the X slot
             }
+            mma_commit(&bars[B_DRAIN + 1]);
+            mbar_wait_drain(&bars[B_DRAIN + 1], 0, p, abort_s);
         }
     } else if (warp < STATE_W0) {
         // ------------------------------------------------ math warpgroup
@@ -395,9 +439,9 @@ __global__ void __launch_bounds__(NTH, 1)
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
             const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
-            mbar_wait(&bars[B_CS + s], par, err);
+            if (!warp_ok(mbar_wait(&bars[B_CS + s], par, p, abort_s))) break;
             const float v = csk[row], Dh = dh_s[s];
-            mbar_wait(&bars[B_G + s], par, err);
+            if (!warp_ok(mbar_wait(&bars[B_G + s], par, p, abort_s))) break;
             tc_fence_after();
             if (!so) {
 #pragma unroll 1
@@ -416,7 +460,7 @@ __global__ void __launch_bounds__(NTH, 1)
             const Tile t = decode_tile(p, k);
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
-            mbar_wait(&bars[B_CS + s], par, err);
+            if (!warp_ok(mbar_wait(&bars[B_CS + s], par, p, abort_s))) break;
             const float lam = lam_s[s];
             if (t.c == 0) {
                 if (p.init_state) {
@@ -431,7 +475,7 @@ __global__ void __launch_bounds__(NTH, 1)
             if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle)
                 // the one buffer was last read by C h^T of tile k-1; waiting for
                 // that (and not for this tile's G) lets C h^T go as early as it can
-                if (k > 0) mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, err);
+                if (k > 0 && !warp_ok(mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s))) break;
                 uint8_t *sh = sm + OFF_H;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -443,7 +487,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 fence_proxy_async_smem();
             }
             mbar_arrive(&bars[B_HW + s]);  // C h_in^T may go
-            mbar_wait(&bars[B_S + s], par, err);
+            if (!warp_ok(mbar_wait(&bars[B_S + s], par, p, abort_s))) break;
             tc_fence_after();
             {  // h_out = exp(lam) h_in + S, 32 columns at a time
                 const float el = __expf(lam);
@@ -482,7 +526,17 @@ __global__ void __launch_bounds__(NTH, 1)
             Dn = p.D ? p.D[tn.h] : 0.f;
         }
         Tile prev{};  // tile k-1, whose y this step writes
+        // A failed wait skips the rest of the step; the warpgroup stops together
+        // at the next step, deciding from votes cast before its first named
+        // barrier, so that no warp is left waiting at a barrier.
+        bool failed = false;
         for (int k = 0; k <= ntl; ++k) {
+            if (failed) {
+                if (k == ntl) break;  // no barrier left: leave alone
+                if (lane == 0) votes[quad] = 1;
+            } else if (lane == 0 && k < ntl) {
+                votes[quad] = *abort_s;
+            }
             Tile cur{};
             if (k < ntl) {
                 cur = tn;
@@ -503,6 +557,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 if (lane == 31) wtot[quad] = v;
                 named_bar_sync(BAR_MATH, 128);
+                if (votes[0] | votes[1] | votes[2] | votes[3]) break;  // uniform over the warpgroup
                 for (int w = 0; w < quad; ++w) v += wtot[w];
                 csk[row] = v;
                 dtk[row] = d;
@@ -517,8 +572,11 @@ __global__ void __launch_bounds__(NTH, 1)
                 mbar_arrive(&bars[B_CS + s]);
                 // W (one buffer): the previous tile's S must have read it
                 const int xs = k % X_SLOTS;
-                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, err);
-                if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, err);
+                if (!warp_ok(mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s)) ||
+                    (k > 0 && !warp_ok(mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s)))) {
+                    failed = true;
+                    continue;
+                }
                 // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
                 // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
                 // SM sub-partition also builds the most M blocks, skips it and the warp
@@ -538,7 +596,10 @@ __global__ void __launch_bounds__(NTH, 1)
                 const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s + lane_off;
                 const Tile t = prev;
                 const float e = __expf(cs[s * QT + row]);
-                mbar_wait(&bars[B_Y + s], par, err);
+                if (!warp_ok(mbar_wait(&bars[B_Y + s], par, p, abort_s))) {
+                    failed = true;
+                    continue;
+                }
                 tc_fence_after();
                 if (!t.state_only) {
                     __nv_bfloat16 *yrow = p.y + (((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h) * PD;
@@ -604,10 +665,15 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
 
 struct DevInfo {
     bool init = false;
+    void *ctx = nullptr;  // the context the kernel attribute was set in
     int sms = 0;
 };
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
+
+// Test-only fault injection (set through ssd_debug_inject_stall).
+std::atomic<int> g_withhold{0};
+std::atomic<unsigned long long> g_wait_ns{0};
 
 // Split nchunks into `runs` runs so that every run's CTA has about the same
 // work: run r streams its run_start[r] predecessors state-only (cost ALPHA per
@@ -635,6 +701,11 @@ void split_runs(int nchunks, int runs, int *start) {
 
 }  // namespace
 
+void set_tc_fault_injection(int withhold, unsigned long long wait_ns) {
+    g_wait_ns.store(wait_ns);
+    g_withhold.store(withhold ? 1 : 0);
+}
+
 bool tc_supported(int headdim, int dstate, int seqlen) {
     return headdim == PD && dstate == ND && seqlen >= QT;
 }
@@ -652,11 +723,14 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     {
         std::lock_guard<std::mutex> lk(g_dev_mu);
         DevInfo &di = g_dev[dev];
-        if (!di.init) {
+        void *ctx = current_context();
+        if (!di.init || di.ctx != ctx) {
+            di.init = false;
             if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SMEM_ALLOC)) != cudaSuccess)
                 return e;
             if ((e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+            di.ctx = ctx;
             di.init = true;
         }
     }
@@ -686,6 +760,9 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     p.runs = runs;
     split_runs(p.nchunks, runs, p.run_start);
     p.dev_error = a.dev_error;
+    const unsigned long long wns = g_wait_ns.load();
+    p.wait_ns = wns ? wns : WAIT_NS;
+    p.withhold = g_withhold.load();
 
     const int items = p.bH * runs;
     const int grid = std::min(items, di.sms);  // one CTA per SM

@@ -8,6 +8,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 
 #include "../../include/ssd.h"
@@ -38,24 +39,33 @@ ssd_status cuda_fail(cudaError_t e, const char *what) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Device address of the error word in the current context, looked up once per
+// (device, context) with that device current.
 int *device_error_ptr(ssd_status *st) {
-    static int *cache[64] = {nullptr};
+    struct Entry {
+        void *ctx;
+        int *ptr;
+    };
+    static Entry cache[64] = {};
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess || dev < 0 || dev >= 64) {
         *st = cuda_fail(e, "cudaGetDevice");
         return nullptr;
     }
-    if (!cache[dev]) {
+    void *ctx = ssd::current_context();
+    std::lock_guard<std::mutex> lk(mu);
+    if (!cache[dev].ptr || cache[dev].ctx != ctx) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_ssd_device_error);
         if (e != cudaSuccess) {
             *st = cuda_fail(e, "cudaGetSymbolAddress(device error word)");
             return nullptr;
         }
-        cache[dev] = static_cast<int *>(p);
+        cache[dev] = Entry{ctx, static_cast<int *>(p)};
     }
-    return cache[dev];
+    return cache[dev].ptr;
 }
 
 constexpr int kMaxHeaddim = 256;
@@ -199,6 +209,23 @@ bool valid_dtype(ssd_dtype d) { return d == SSD_F32 || d == SSD_BF16; }
 
 namespace ssd {
 void set_last_error(const char *msg) { g_last_error = msg; }
+
+void *current_context() {
+    // cuCtxGetCurrent, fetched through the runtime so that libssd needs no link
+    // against the driver library.
+    typedef int (*GetCurrent)(void **);
+    static GetCurrent fn = [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (GetCurrent) nullptr;
+        return reinterpret_cast<GetCurrent>(f);
+    }();
+    void *ctx = nullptr;
+    if (!fn || fn(&ctx) != 0) return nullptr;
+    return ctx;
+}
 }  // namespace ssd
 
 // The backward scans (real or complex), after validation.
@@ -350,6 +377,11 @@ ssd_status ssd_get_device_status(void *stream) {
         return fail(SSD_ERR_TIMEOUT, "a bounded inter-block wait gave up on the device; the "
                     "outputs of the call that raised it are invalid");
     return fail(SSD_ERR_CUDA, "device error code %d", code);
+}
+
+ssd_status ssd_debug_inject_stall(int withhold_first_load, unsigned long long wait_limit_ns) {
+    ssd::set_tc_fault_injection(withhold_first_load, wait_limit_ns);
+    return SSD_OK;
 }
 
 const char *ssd_last_error(void) { return g_last_error.c_str(); }

@@ -80,6 +80,9 @@ bool tc_supported(int headdim, int dstate, int seqlen);
 size_t tc_workspace_bytes(int batch, int nheads);
 cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st);
 int tc_kernel_launches();
+// Test only: with withhold != 0 the tensor-core kernel's producer issues no load,
+// so every bounded wait runs out; wait_ns (0: the default) bounds each wait.
+void set_tc_fault_injection(int withhold, unsigned long long wait_ns);
 
 cudaError_t launch_state_update(float *state, const void *x, const float *dt, const float *A,
                                 const void *B, const void *C, const float *D, void *y,
@@ -106,6 +109,13 @@ cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_stat
 
 // Sets the message ssd_last_error() returns on this host thread.
 void set_last_error(const char *msg);
+
+// The calling thread's current CUDA context (the driver's CUcontext, as an
+// opaque pointer; NULL when there is none or the query is unavailable).  The
+// per-device caches of device addresses and kernel attributes are keyed on it,
+// so they are looked up again after the context changes (for example after
+// cudaDeviceReset destroyed the primary context and a new one was created).
+void *current_context();
 
 static inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
