@@ -736,6 +736,296 @@ def bench_ours(args, shape):
     return 0
 
 
+# ------------------------------------------------- packed projection input
+def packed_bytes(shape) -> dict:
+    """Per call.  fused: the projection output read once (bf16), y written, the
+    final state written.  unpacked: the block's separate unpacking pass (read the
+    projection, write x float32, B and C complex64, dt float32) and then the scan
+    reading those.  The difference is what reading the slices in place saves."""
+    b, T, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    tok = b * T
+    W = H * (P + 4 * N + 1)
+    proj = tok * W * 2
+    out = tok * H * P * 4 + b * H * P * N * 8
+    unpacked = tok * (H * P * 4 + 2 * H * N * 8 + H * 4)
+    return {"fused": proj + out + 8 * H, "unpack_then_scan": proj + 2 * unpacked + out + 8 * H}
+
+
+def bench_packed(args, shape):
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+    inp = inputs.packed_inputs(shape, "bf16")
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    H, P, N = shape.nheads, shape.headdim, shape.dstate
+    y = torch.empty((shape.batch, shape.seqlen, H, P), dtype=torch.float32, device=dev)
+    fs = torch.empty((shape.batch, H, P, N), dtype=torch.complex64, device=dev)
+    ws = torch.zeros(max(16, ssd.ssd_scan_workspace_size(shape.batch, shape.seqlen, H, P, H, N, shape.chunk, True,
+                                                         ssd.SSD_F32)), dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_scan_fwd_complex_packed(d["proj"], d["A"], d["D"], None, nheads=H, headdim=P, dstate=N,
+                                        dt_bias=d["dt_bias"], chunk_size=shape.chunk, y=y, final_state=fs,
+                                        workspace=ws)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    warm_ms = []
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b_))
+    ssd.ssd_get_device_status()
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    torch.cuda._sleep(20_000_000)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [a.elapsed_time(b_) for a, b_ in zip(starts, ends)]
+    total_s = dist_max(sum(per_step_ms) / 1e3, dev)
+    t_call = statistics.median(per_step_ms) / 1e3
+    peaks = load_peaks()
+    by = packed_bytes(shape)
+    line = {
+        "metric": METRIC, "value": shape.tokens * world * steps / total_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "ours", "config": dict(scan_config(shape, world), io_dtype="bf16 projection"),
+        "roofline": {"bound": "hbm", "achieved": by["fused"] / t_call / 1e9, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": by["fused"] / t_call / 1e9 / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "complex scan from the packed projection (3 launches, timed as one call)",
+                     "algorithmic_bytes_per_launch": by["fused"],
+                     "bytes_unpack_then_scan": by["unpack_then_scan"],
+                     "bytes_saved": by["unpack_then_scan"] - by["fused"], "kernel_time_us": 1e6 * t_call},
+        "cpu_baseline": None, "e2e": None, "clocks": sampler.summary(t0, t1), "gpu_launches": 3 * steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+# ------------------------------------------------------------- variants
+SFU_EXP_PER_CLK_SM = 16  # exponentials per clock per SM (4 per sub-partition)
+
+
+def bench_variant(args, name):
+    """The conv1d prologue or the Mamba-1 selective scan, one call per step."""
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+    peaks = load_peaks()
+    if name == inputs.MAMBA2_CONV.name:
+        sh = inputs.MAMBA2_CONV
+        inp = inputs.conv_inputs(sh)
+        d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+        Ct = sh.x_channels + 2 * sh.bc_channels
+        out = (torch.empty((sh.batch, sh.seqlen, sh.x_channels), dtype=d["xbc"].dtype, device=dev),
+               torch.empty((sh.batch, sh.seqlen, sh.bc_channels), dtype=d["xbc"].dtype, device=dev),
+               torch.empty((sh.batch, sh.seqlen, sh.bc_channels), dtype=d["xbc"].dtype, device=dev))
+        step = lambda: ssd.ssd_conv1d_xbc(d["xbc"], d["weight"], d["bias"], None, x_channels=sh.x_channels,
+                                          bc_channels=sh.bc_channels, silu=sh.silu, out=out)
+        tokens = sh.batch * sh.seqlen
+        esz = 2 if sh.io_dtype == "bf16" else 4
+        abytes = 2 * sh.batch * sh.seqlen * Ct * esz + Ct * (sh.width + 1) * 4
+        kernel, bound, alu_peak = "conv1d_xbc_kernel", "hbm", None
+    else:
+        sh = inputs.MAMBA1_50M
+        inp = inputs.selective_inputs(sh)
+        d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+        y = torch.empty_like(d["x"])
+        fs = torch.empty((sh.batch, sh.channels, sh.dstate), dtype=torch.float32, device=dev)
+        step = lambda: ssd.ssd_selective_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                                              y=y, final_state=fs)
+        tokens = sh.tokens
+        esz = 2 if sh.io_dtype == "bf16" else 4
+        abytes = (sh.tokens * sh.channels * (2 * esz + 4) + 2 * sh.tokens * sh.ngroups * sh.dstate * esz
+                  + sh.batch * sh.channels * sh.dstate * 4 + sh.channels * (sh.dstate + 1) * 4)
+        exps = sh.tokens * sh.channels * sh.dstate
+        kernel = "selective_scan_kernel"
+        alu_peak = 148 * SFU_EXP_PER_CLK_SM * 1.965e9  # exponentials per second at the max SM clock
+        bound = "alu" if exps / alu_peak > abytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    warm_ms = []
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b_))
+    ssd.ssd_get_device_status()
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    torch.cuda._sleep(20_000_000)
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [a.elapsed_time(b_) for a, b_ in zip(starts, ends)]
+    total_s = dist_max(sum(per_step_ms) / 1e3, dev)
+    t_call = statistics.median(per_step_ms) / 1e3
+    if bound == "alu":
+        roof = {"bound": "alu", "achieved": exps / t_call / 1e12, "peak": alu_peak / 1e12, "unit": "Texp/s",
+                "frac": exps / t_call / alu_peak,
+                "peak_source": "derived: 148 SMs x 16 exponentials per clock x 1965 MHz",
+                "hbm_frac": abytes / t_call / 1e9 / peaks["hbm_gbs"]}
+    else:
+        roof = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"]}
+    roof.update({"traffic": None, "kernel": kernel, "algorithmic_bytes_per_launch": abytes,
+                 "kernel_time_us": 1e6 * t_call})
+    line = {
+        "metric": METRIC, "value": tokens * world * steps / total_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "impl": "ours", "config": dict(dataclasses_asdict(sh), parallelism="1 GPU" if world == 1 else f"replicas x{world}"),
+        "roofline": roof, "cpu_baseline": None, "e2e": None, "clocks": sampler.summary(t0, t1), "gpu_launches": steps,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def dataclasses_asdict(obj):
+    import dataclasses
+
+    dd = dataclasses.asdict(obj)
+    dd["workload"] = dd.pop("name")
+    return dd
+
+
+# ------------------------------------------------------- sequence split
+def bench_seqpar(args, shape):
+    """One sequence of shape.seqlen tokens cut into consecutive slices, one per
+    rank: state-only scan of each slice, all-gather of the slice end states and
+    log-decays over NCCL, fold, full scan of each slice from its entering state
+    (selective_state_space_22_b200.seqpar).  Strong scaling: the whole job is one
+    sequence whatever the number of GPUs; value = its tokens / max over ranks."""
+    import torch
+
+    import selective_state_space_22_b200 as ssd
+    from selective_state_space_22_b200 import inputs
+    from selective_state_space_22_b200.seqpar import scan_fwd_sequence_parallel
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init("nccl")
+    ssd.load_library()
+    inp = inputs.scan_inputs(shape)
+    t0, t1 = shape.seqlen * rank // world, shape.seqlen * (rank + 1) // world
+    sl = lambda t: None if t is None else t[:, t0:t1].contiguous().to(dev)
+    d = {k: sl(inp[k]) for k in ("x", "dt", "B", "C")}
+    d.update(A=inp["A"].to(dev), D=inp["D"].to(dev),
+             init_state=inp["init_state"].to(dev) if (rank == 0 and inp["init_state"] is not None) else None)
+
+    def step():
+        return scan_fwd_sequence_parallel(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"],
+                                          chunk_size=shape.chunk)
+
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    sampler = ClockSampler(local).start()
+    warm_ms = []
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        warm_ms.append(a.elapsed_time(b))
+    ssd.ssd_get_device_status()
+    steps = int(dist_max(float(pick_steps(args, warm_ms)), dev))
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    t_0 = time.perf_counter()
+    for i in range(steps):
+        flush.fill_(i & 0xFF)
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    t_1 = time.perf_counter()
+    dist_barrier()
+    sampler.stop()
+    ssd.ssd_get_device_status()
+    per_step_ms = [a.elapsed_time(b) for a, b in zip(starts, ends)]
+    total_s = dist_max(sum(per_step_ms) / 1e3, dev)
+    value = shape.tokens * steps / total_s
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "impl": "ours",
+        "config": dict(scan_config(shape, world), parallelism=f"sequence split x{world}"),
+        "roofline": None, "cpu_baseline": None, "e2e": None, "clocks": sampler.summary(t_0, t_1),
+        "gpu_launches": None,
+        "note": "per step per rank: state-only scan of its slice, NCCL all-gather of (end state, log-decay), "
+                "fold, full scan of the slice",
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 # --------------------------------------------------------------- backward
 BWD_METRIC = {False: "SSD scan backward tokens/s at Mamba-2 1B layer shape (float32); % of HBM roofline",
               True: "SSD complex scan backward tokens/s at Mamba-3-Lite layer shape (float32); % of HBM roofline"}
@@ -872,7 +1162,8 @@ def bench_bwd(args, shape):
     e2e = None
     if not args.no_e2e:
         hin = {k: v.pin_memory() for k, v in list(inp.items()) + list(up.items()) if v is not None}
-        dsets = [{k: (d[k] if k in d else u[k]) for k in hin}, {k: torch.empty_like(v) for k, v in hin.items()}]
+        dsets = [{k: (d[k] if k in d else u[k]) for k in hin}, {}]
+        dsets[1] = {k: torch.empty_like(v) for k, v in dsets[0].items()}
         step()
         torch.cuda.synchronize()
         douts = [{k: v for k, v in out.items() if v is not None}, {}]
@@ -966,9 +1257,23 @@ def main(argv=None):
     if args.workload == inputs.DECODE.name:
         shape = inputs.DECODE
         return bench_reference_decode(args, shape) if args.impl == "reference" else bench_decode(args, shape)
+    if args.workload in (inputs.MAMBA2_CONV.name, inputs.MAMBA1_50M.name):
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the variant workloads are timed against their "
+                              "roofline only; their oracle is used for parity"}))
+            return 0
+        return bench_variant(args, args.workload)
+    if args.workload == inputs.MAMBA3_PACKED.name:
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the packed-input workload has no separate "
+                              "reference arm: the oracle of the complex workload covers the same scan"}))
+            return 0
+        return bench_packed(args, inputs.MAMBA3_PACKED)
     shape = inputs.WORKLOADS[args.workload]
     if args.impl == "reference":
         return bench_reference(args, shape)
+    if shape is inputs.LONG and dist_env()[1] > 1:
+        return bench_seqpar(args, shape)  # one long sequence split across the GPUs
     return bench_ours(args, shape)
 
 

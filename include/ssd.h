@@ -127,11 +127,17 @@ ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A,
  *  final_state [batch, nheads, headdim, dstate] complex, or NULL
  *  y           [batch, seqlen, nheads, headdim] float32 = Re(h_t C_t) + D x_t
  *
- * Runs in float32 (complex64) throughout, on CUDA cores: three launches and a
- * workspace (ssd_scan_workspace_size with is_complex = 1).  Each token's C and B
- * are rotated by its cumulative phase, which leaves a real decay magnitude, so
- * every contraction is a real float32 product over the 2 dstate interleaved
- * values.  Other arguments as ssd_scan_fwd.
+ * Three launches and a workspace (ssd_scan_workspace_size with is_complex = 1):
+ * chunk states, the state pass over chunks, the chunk scan.  Every contraction
+ * is a real product over the 2 dstate interleaved (re, im) values, with the
+ * complex decay folded into C and B.  headdim 64 and dstate 64 (the Mamba-3-Lite
+ * head) run the chunk states and chunk scan on tcgen05 tensor cores in
+ * 128-token chunks, with each float32 operand split into bf16 hi and lo parts
+ * and three products per contraction (float32 accumulation; about 1e-5 of the
+ * float32 result), and chunks whose real log-decay spans more than 140 on
+ * CUDA cores; other sizes run float32 CUDA-core kernels that honour chunk_size.
+ * State and accumulation are float32 (complex64).  Other arguments as
+ * ssd_scan_fwd.
  */
 ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A,
                                 const float *B, const float *C, const float *D,
@@ -139,6 +145,133 @@ ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A,
                                 int batch, int seqlen, int nheads, int headdim,
                                 int ngroups, int dstate, int chunk_size,
                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * The complex scan reading the packed input-projection output directly.
+ *
+ * "Block Anatomy, Numerical Stability & Scaling", Block Anatomy section 4.1-4.3:
+ * a Mamba-3-Lite block's projection emits per token W = H (D + 4N + 1) values in
+ * head-major slices, in this order: x (H*D), Re B (H*N), Im B (H*N), Re C
+ * (H*N), Im C (H*N), dt (H); Numerical Stability section 4 (_discretise) applies
+ * softplus to dt.  This call reads those slices in place (float32 or bf16,
+ * widened exactly), pairs the real and imaginary parts, and computes
+ * dt = softplus(dt_raw + dt_bias[h]) inside the scan's own loads, so the
+ * separate unpacking pass of the block (the float32 copies and the complex64
+ * B and C) never touches HBM.  The result equals ssd_scan_fwd_complex given the
+ * unpacked tensors.
+ *
+ *  proj        [batch, seqlen, W] in proj_dtype, W = nheads (headdim + 4 dstate + 1)
+ *  dt_bias     [nheads] float32 added before the softplus, or NULL for none
+ *  A, D, init_state, final_state, y, chunk_size, workspace: as ssd_scan_fwd_complex,
+ *  with one group per head (ngroups = nheads; workspace from
+ *  ssd_scan_workspace_size(batch, seqlen, nheads, headdim, nheads, dstate,
+ *  chunk_size, 1, SSD_F32)).
+ */
+ssd_status ssd_scan_fwd_complex_packed(const void *proj, ssd_dtype proj_dtype,
+                                       const float *dt_bias, const float *A, const float *D,
+                                       const float *init_state, float *final_state, float *y,
+                                       int batch, int seqlen, int nheads, int headdim,
+                                       int dstate, int chunk_size, void *workspace,
+                                       size_t workspace_bytes, void *stream);
+
+/*
+ * Sequence split across devices, step 1: the final state of a slice of the
+ * sequence, and its total log-decay, without its outputs.
+ *
+ * "Block Anatomy, Numerical Stability & Scaling" (Numerical Stability, section
+ * 4) carries each chunk's end state into later chunks through the decay between
+ * them; the same holds for consecutive slices of a sequence held by different
+ * devices.  A device scans its slice from a zero state (the first slice from
+ * the caller's initial state) with this call, which runs the state part of the
+ * scan only (cumulative decay, chunk states, state passing; no C, no y).
+ *
+ *  x, dt, A, B, init_state, io_dtype, sizes, chunk_size, workspace: as
+ *    ssd_scan_fwd (same workspace size).
+ *  final_state      [batch, nheads, headdim, dstate] float32, required.
+ *  total_log_decay  [batch, nheads] float32 = A[h] * sum over the slice of
+ *    dt[b, t, h] (summed in double), or NULL.
+ * For seqlen 0 the final state is init_state (or zeros) and the log-decay 0.
+ */
+ssd_status ssd_scan_final_state(const void *x, const float *dt, const float *A,
+                                const void *B, const float *init_state,
+                                float *final_state, float *total_log_decay,
+                                ssd_dtype io_dtype, int batch, int seqlen, int nheads,
+                                int headdim, int ngroups, int dstate, int chunk_size,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Sequence split across devices, step 2: the state entering a slice.
+ *
+ * Given the final states S_0 .. S_{n-1} of the n slices before it (S_0 from the
+ * caller's initial state, the others from zero) and their total log-decays,
+ * out = h_{n-1} with h_0 = S_0 and h_j = exp(log_decay_j) h_{j-1} + S_j, the
+ * inter-chunk recurrence of the pages applied per slice.  Elementwise, float32.
+ *
+ *  states     [nstates, batch, nheads, headdim, dstate] float32
+ *  log_decay  [nstates, batch, nheads] float32 (entry 0 unused; may be NULL
+ *             when nstates == 1)
+ *  out        [batch, nheads, headdim, dstate] float32 (may not alias states)
+ */
+ssd_status ssd_fold_states(const float *states, const float *log_decay, int nstates,
+                           float *out, int batch, int nheads, int headdim, int dstate,
+                           void *stream);
+
+/*
+ * The causal depthwise convolution Mamba-1 and Mamba-2 run before the scan
+ * ("Block Anatomy, Numerical Stability & Scaling", Block Anatomy section 5.1:
+ * each channel at position t becomes a learned combination of positions
+ * t-K+1 .. t, K = 4), over the packed x | B | C channels of a Mamba-2 input
+ * projection, written straight into the scan's separate inputs:
+ *
+ *   out[b,t,c] = act(bias[c] + sum_{k<K} weight[c,k] * xbc[b, t-K+1+k, c])
+ *
+ * with act the identity, or SiLU v / (1 + exp(-v)) when silu != 0 (the pages
+ * name the convolution only; Mamba-2 follows it with SiLU).  Positions before
+ * t = 0 read conv_init (the last K-1 inputs of a preceding part of the same
+ * sequence) or zero.
+ *
+ *  xbc        [batch, seqlen, x_channels + 2 bc_channels]  io_dtype
+ *  weight     [x_channels + 2 bc_channels, width] float32; bias the same
+ *             channels, float32, or NULL
+ *  conv_init  [batch, x_channels + 2 bc_channels, width - 1] io_dtype, or NULL
+ *  x_out      [batch, seqlen, x_channels] io_dtype (channels 0 .. x_channels-1;
+ *             for the scan: [batch, seqlen, nheads, headdim])
+ *  B_out, C_out [batch, seqlen, bc_channels] io_dtype (the next two channel
+ *             ranges; for the scan: [batch, seqlen, ngroups, dstate])
+ *  conv_final [batch, x_channels + 2 bc_channels, width - 1] io_dtype, or NULL:
+ *             the last width-1 inputs, the conv_init of a continuation
+ *  width      1 .. 8.
+ * Float32 arithmetic; one read of every input, one write of every output.
+ */
+ssd_status ssd_conv1d_xbc(const void *xbc, const float *weight, const float *bias,
+                          const void *conv_init, void *x_out, void *B_out, void *C_out,
+                          void *conv_final, ssd_dtype io_dtype, int batch, int seqlen,
+                          int x_channels, int bc_channels, int width, int silu, void *stream);
+
+/*
+ * The Mamba-1 selective scan: one decay rate per state component ("Block
+ * Anatomy, Numerical Stability & Scaling", Block Anatomy section 4.4: A of shape
+ * (H, N); the "Mamba-50M" card: a Mamba selective-SSM language model).  Each
+ * channel d has its own step and dstate states:
+ *
+ *   h_t[n] = exp(dt_t[d] A[d,n]) h_{t-1}[n] + dt_t[d] B_t[n] x_t[d]
+ *   y_t[d] = sum_n C_t[n] h_t[n] + D[d] x_t[d]
+ *
+ *  x, y        [batch, seqlen, channels]  io_dtype
+ *  dt          [batch, seqlen, channels]  float32 (after softplus and bias)
+ *  A           [channels, dstate]         float32
+ *  B, C        [batch, seqlen, ngroups, dstate]  io_dtype; channel d reads group
+ *              d / (channels / ngroups)
+ *  D           [channels] float32 or NULL
+ *  init_state, final_state [batch, channels, dstate] float32 or NULL
+ *  dstate      4, 8, 16 or 32 (SSD_ERR_UNSUPPORTED otherwise).
+ * Sequential in time (the per-state decay has no chunked matrix form),
+ * parallel over (batch, channel): one launch, no workspace, float32 state.
+ */
+ssd_status ssd_selective_scan(const void *x, const float *dt, const float *A, const void *B,
+                              const void *C, const float *D, const float *init_state,
+                              float *final_state, void *y, ssd_dtype io_dtype, int batch,
+                              int seqlen, int channels, int ngroups, int dstate, void *stream);
 
 /*
  * One recurrent decoding step, in place on the state (real variant):

@@ -62,6 +62,10 @@ def _declare(lib):
     for name in ("oracle_state_update_real", "oracle_state_update_complex"):
         getattr(lib, name).argtypes = upd_args
         getattr(lib, name).restype = ctypes.c_int
+    lib.oracle_causal_conv1d.argtypes = [_D, _D, _D, _D, ctypes.c_int, _D, _L, _L, _L, _L]
+    lib.oracle_causal_conv1d.restype = ctypes.c_int
+    lib.oracle_selective_scan.argtypes = [_D] * 9 + [_L] * 5
+    lib.oracle_selective_scan.restype = ctypes.c_int
     bwd_args = [_D] * 16 + [_L] * 6
     for name in ("oracle_scan_bwd_real", "oracle_scan_bwd_complex"):
         getattr(lib, name).argtypes = bwd_args
@@ -146,3 +150,35 @@ def scan_bwd(x, dt, A, B, C, D, init_state, dy, dfinal=None, lib=None):
     if rc != 0:
         raise ValueError("oracle rejected the arguments")
     return out
+
+
+def causal_conv1d(x, w, bias=None, init=None, silu=False, lib=None):
+    """Causal depthwise convolution, x [b,T,C] float64, w [C,K], bias [C],
+    init [b,C,K-1] (the inputs before t = 0) or None.  Returns out [b,T,C]."""
+    lib = lib or load()
+    b, T, Cn = x.shape
+    K = w.shape[1]
+    out = np.zeros((b, T, Cn), np.float64)
+    rc = lib.oracle_causal_conv1d(_ptr(x, np.float64), _ptr(w, np.float64), _ptr(bias, np.float64),
+                                  _ptr(init, np.float64), int(bool(silu)), _ptr(out, np.float64), b, T, Cn, K)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return out
+
+
+def selective_scan(x, dt, A, B, C, D=None, init_state=None, lib=None):
+    """Mamba-1 selective scan with a per-state A: x, dt [b,T,Dc], A [Dc,N],
+    B, C [b,T,G,N], D [Dc], init_state [b,Dc,N].  Returns (y [b,T,Dc],
+    final_state [b,Dc,N])."""
+    lib = lib or load()
+    b, T, Dc = x.shape
+    G, N = B.shape[2], B.shape[3]
+    y = np.zeros((b, T, Dc), np.float64)
+    fs = np.zeros((b, Dc, N), np.float64)
+    rc = lib.oracle_selective_scan(_ptr(x, np.float64), _ptr(dt, np.float64), _ptr(A, np.float64),
+                                   _ptr(B, np.float64), _ptr(C, np.float64), _ptr(D, np.float64),
+                                   _ptr(init_state, np.float64), _ptr(y, np.float64), _ptr(fs, np.float64),
+                                   b, T, Dc, G, N)
+    if rc != 0:
+        raise ValueError("oracle rejected the arguments")
+    return y, fs

@@ -424,3 +424,86 @@ int oracle_scan_bwd_complex(const double *x, const double *dt, const double *A,
     free(hist); free(Gs);
     return 0;
 }
+
+/* ------------------------------------------------------------------------
+ * Variants named on the pages beside the Mamba-2 / Mamba-3-Lite scan.
+ *
+ * Causal depthwise convolution ("Block Anatomy, Numerical Stability &
+ * Scaling", Block Anatomy section 5.1): Mamba-1 and Mamba-2 convolve each
+ * channel of the projected input over the current and the K-1 previous
+ * positions (K = 4) before the scan.  out[t][c] = bias[c] + sum_k w[c][k] *
+ * in[t - (K-1) + k][c]; inputs before t = 0 come from init (the previous K-1
+ * inputs of a continued sequence, [b][c][K-1]) or are zero.  With silu != 0 the
+ * result goes through v / (1 + exp(-v)) (the Mamba-2 activation; the pages
+ * name the convolution only, so the activation is the caller's choice).
+ *
+ * Layouts: in, out [b][t][c]; w [c][K]; bias [c]; init [b][c][K-1].
+ */
+int oracle_causal_conv1d(const double *in, const double *w, const double *bias,
+                         const double *init, int silu, double *out, long batch,
+                         long seqlen, long channels, long width) {
+    if (batch < 0 || seqlen < 0 || channels <= 0 || width <= 0) return -1;
+    for (long b = 0; b < batch; ++b)
+        for (long t = 0; t < seqlen; ++t)
+            for (long c = 0; c < channels; ++c) {
+                double v = bias ? bias[c] : 0.0;
+                for (long k = 0; k < width; ++k) {
+                    const long s = t - (width - 1) + k;
+                    double u = 0.0;
+                    if (s >= 0)
+                        u = in[(b * seqlen + s) * channels + c];
+                    else if (init)  /* s = -1 is init[..][K-2], s = -(K-1) is init[..][0] */
+                        u = init[(b * channels + c) * (width - 1) + (width - 1) + s];
+                    v += w[c * width + k] * u;
+                }
+                if (silu) v = v / (1.0 + exp(-v));
+                out[(b * seqlen + t) * channels + c] = v;
+            }
+    return 0;
+}
+
+/*
+ * Mamba-1 selective scan: a per-state decay ("Block Anatomy, Numerical
+ * Stability & Scaling", Block Anatomy section 4.4: A of shape (H, N), one decay
+ * rate per state component; the "Mamba-50M" card: a Mamba (selective SSM)
+ * model).  Each channel d has its own step dt and N states:
+ *
+ *   h_t[n] = exp(dt_t[d] A[d][n]) h_{t-1}[n] + dt_t[d] B_t[n] x_t[d]
+ *   y_t[d] = sum_n C_t[n] h_t[n] + D[d] x_t[d]
+ *
+ * Channel d reads group d / (channels / ngroups) of B and C.
+ * Layouts: x, dt, y [b][t][d]; A [d][n]; B, C [b][t][g][n]; D [d];
+ * state [b][d][n].
+ */
+int oracle_selective_scan(const double *x, const double *dt, const double *A,
+                          const double *B, const double *C, const double *D,
+                          const double *init_state, double *y, double *final_state,
+                          long batch, long seqlen, long channels, long ngroups,
+                          long dstate) {
+    if (batch < 0 || seqlen < 0 || channels <= 0 || ngroups <= 0 || dstate <= 0 ||
+        channels % ngroups != 0)
+        return -1;
+    double *h = (double *)malloc((size_t)dstate * sizeof(double));
+    if (!h) return -1;
+    for (long b = 0; b < batch; ++b)
+        for (long d = 0; d < channels; ++d) {
+            const long g = d / (channels / ngroups);
+            for (long n = 0; n < dstate; ++n)
+                h[n] = init_state ? init_state[(b * channels + d) * dstate + n] : 0.0;
+            for (long t = 0; t < seqlen; ++t) {
+                const size_t bt = (size_t)(b * seqlen + t);
+                const double u = x[bt * channels + d], step = dt[bt * channels + d];
+                double acc = 0.0;
+                for (long n = 0; n < dstate; ++n) {
+                    const size_t bc = (bt * ngroups + g) * dstate + n;
+                    h[n] = exp(step * A[d * dstate + n]) * h[n] + step * B[bc] * u;
+                    acc += C[bc] * h[n];
+                }
+                y[bt * channels + d] = acc + (D ? D[d] * u : 0.0);
+            }
+            if (final_state)
+                for (long n = 0; n < dstate; ++n) final_state[(b * channels + d) * dstate + n] = h[n];
+        }
+    free(h);
+    return 0;
+}

@@ -23,7 +23,8 @@ __all__ = ["SSDError", "ssd_scan_fwd", "ssd_scan_fwd_complex", "ssd_state_update
            "ssd_state_update_complex", "ssd_scan_workspace_size", "ssd_scan_kernel_launches", "ssd_get_device_status",
            "ssd_scan_fwd_noalloc", "ssd_last_error", "ssd_version", "load_library", "LIB_PATH",
            "SSD_WORKSPACE_INVALID", "ssd_scan_bwd", "ssd_scan_bwd_workspace_size",
-           "ssd_scan_bwd_complex", "ssd_scan_bwd_complex_workspace_size"]
+           "ssd_scan_bwd_complex", "ssd_scan_bwd_complex_workspace_size", "ssd_scan_final_state",
+           "ssd_fold_states", "ssd_scan_fwd_complex_packed", "ssd_conv1d_xbc", "ssd_selective_scan"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libssd.so")
 
@@ -77,6 +78,16 @@ def load_library(path: str | None = None):
         lib.ssd_scan_bwd_complex_workspace_size.restype = _SZ
         lib.ssd_scan_bwd_complex.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, _SZ, _VP]
         lib.ssd_scan_bwd_complex.restype = _I
+        lib.ssd_conv1d_xbc.argtypes = [_VP] * 8 + [_I] * 7 + [_VP]
+        lib.ssd_conv1d_xbc.restype = _I
+        lib.ssd_selective_scan.argtypes = [_VP] * 9 + [_I] * 6 + [_VP]
+        lib.ssd_selective_scan.restype = _I
+        lib.ssd_scan_fwd_complex_packed.argtypes = [_VP, _I] + [_VP] * 6 + [_I] * 6 + [_VP, _SZ, _VP]
+        lib.ssd_scan_fwd_complex_packed.restype = _I
+        lib.ssd_scan_final_state.argtypes = [_VP] * 7 + [_I] * 8 + [_VP, _SZ, _VP]
+        lib.ssd_scan_final_state.restype = _I
+        lib.ssd_fold_states.argtypes = [_VP, _VP, _I, _VP, _I, _I, _I, _I, _VP]
+        lib.ssd_fold_states.restype = _I
         lib.ssd_debug_inject_stall.argtypes = [_I, ctypes.c_ulonglong]
         lib.ssd_debug_inject_stall.restype = _I
         lib.ssd_get_device_status.argtypes = [_VP]
@@ -198,6 +209,159 @@ def ssd_scan_fwd(x, dt, A, B, C, D=None, init_state=None, *, chunk_size=256, y=N
                               _ptr(ws), 0 if ws is None else ws.numel(), _stream_handle(stream))
     _check(st)
     return y, final_state
+
+
+def ssd_conv1d_xbc(xbc, weight, bias=None, conv_init=None, *, x_channels, bc_channels, silu=True,
+                   out=None, conv_final=None, stream=None):
+    """Causal depthwise conv over packed x|B|C channels, split into the scan's
+    inputs.  xbc [b,T,Cx+2Cb] bf16/float32, weight [Cx+2Cb, K] float32, bias
+    [Cx+2Cb] float32, conv_init [b, Cx+2Cb, K-1].  Returns (x [b,T,Cx],
+    B [b,T,Cb], C [b,T,Cb]) (``out`` may pass them preallocated)."""
+    lib = load_library()
+    dev = xbc.device
+    b, T, Ct = xbc.shape
+    if Ct != x_channels + 2 * bc_channels:
+        raise ValueError("xbc width must be x_channels + 2 bc_channels")
+    io = {torch.bfloat16: SSD_BF16, torch.float32: SSD_F32}.get(xbc.dtype)
+    if io is None:
+        raise ValueError("xbc must be bfloat16 or float32")
+    K = weight.shape[1]
+    _need(xbc, "xbc", xbc.dtype, dev)
+    _need(weight, "weight", torch.float32, dev, (Ct, K))
+    _need(bias, "bias", torch.float32, dev, (Ct,), allow_none=True)
+    _need(conv_init, "conv_init", xbc.dtype, dev, (b, Ct, K - 1), allow_none=True)
+    _need(conv_final, "conv_final", xbc.dtype, dev, (b, Ct, K - 1), allow_none=True)
+    if out is None:
+        out = (torch.empty((b, T, x_channels), dtype=xbc.dtype, device=dev),
+               torch.empty((b, T, bc_channels), dtype=xbc.dtype, device=dev),
+               torch.empty((b, T, bc_channels), dtype=xbc.dtype, device=dev))
+    xo, bo, co = out
+    with torch.cuda.device(dev):
+        st = lib.ssd_conv1d_xbc(_ptr(xbc), _ptr(weight), _ptr(bias), _ptr(conv_init), _ptr(xo), _ptr(bo), _ptr(co),
+                                _ptr(conv_final), io, b, T, x_channels, bc_channels, K, int(bool(silu)),
+                                _stream_handle(stream))
+    _check(st)
+    return xo, bo, co
+
+
+def ssd_selective_scan(x, dt, A, B, C, D=None, init_state=None, *, y=None, final_state=None,
+                       return_final_state=True, stream=None):
+    """Mamba-1 selective scan (per-state A).  x [b,T,Dc] bf16/float32, dt [b,T,Dc]
+    float32, A [Dc,N] float32, B, C [b,T,G,N] (dtype of x), D [Dc], init_state
+    [b,Dc,N] float32.  Returns (y [b,T,Dc], final_state or None)."""
+    lib = load_library()
+    dev = x.device
+    b, T, Dc = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = {torch.bfloat16: SSD_BF16, torch.float32: SSD_F32}.get(x.dtype)
+    if io is None:
+        raise ValueError("x must be bfloat16 or float32")
+    _need(x, "x", x.dtype, dev)
+    _need(dt, "dt", torch.float32, dev, (b, T, Dc))
+    _need(A, "A", torch.float32, dev, (Dc, N))
+    _need(B, "B", x.dtype, dev, (b, T, G, N))
+    _need(C, "C", x.dtype, dev, (b, T, G, N))
+    _need(D, "D", torch.float32, dev, (Dc,), allow_none=True)
+    _need(init_state, "init_state", torch.float32, dev, (b, Dc, N), allow_none=True)
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, Dc, N), dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        st = lib.ssd_selective_scan(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(init_state),
+                                    _ptr(final_state), _ptr(y), io, b, T, Dc, G, N, _stream_handle(stream))
+    _check(st)
+    return y, final_state
+
+
+def ssd_scan_fwd_complex_packed(proj, A, D=None, init_state=None, *, nheads, headdim, dstate, dt_bias=None,
+                                chunk_size=256, y=None, final_state=None, return_final_state=True, workspace=None,
+                                stream=None):
+    """The complex scan reading the packed projection output in place.
+
+    proj [b, T, H (headdim + 4 dstate + 1)] float32 or bf16, head-major slices
+    x | Re B | Im B | Re C | Im C | dt; dt = softplus(dt + dt_bias) inside the scan.
+    A [H] complex64, D [H] float32, dt_bias [H] float32, init_state [b,H,P,N]
+    complex64.  Returns (y [b,T,H,P] float32, final_state or None)."""
+    lib = load_library()
+    dev = proj.device
+    b, T, W = proj.shape
+    H, P, N = nheads, headdim, dstate
+    if W != H * (P + 4 * N + 1):
+        raise ValueError(f"proj width {W} != nheads (headdim + 4 dstate + 1) = {H * (P + 4 * N + 1)}")
+    io = {torch.bfloat16: SSD_BF16, torch.float32: SSD_F32}.get(proj.dtype)
+    if io is None:
+        raise ValueError("proj must be bfloat16 or float32")
+    _need(proj, "proj", proj.dtype, dev)
+    _need(A, "A", torch.complex64, dev, (H,))
+    _need(D, "D", torch.float32, dev, (H,), allow_none=True)
+    _need(dt_bias, "dt_bias", torch.float32, dev, (H,), allow_none=True)
+    _need(init_state, "init_state", torch.complex64, dev, (b, H, P, N), allow_none=True)
+    if y is None:
+        y = torch.empty((b, T, H, P), dtype=torch.float32, device=dev)
+    _need(y, "y", torch.float32, dev, (b, T, H, P))
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, H, P, N), dtype=torch.complex64, device=dev)
+    _need(final_state, "final_state", torch.complex64, dev, (b, H, P, N), allow_none=True)
+    nbytes = ssd_scan_workspace_size(b, T, H, P, H, N, chunk_size, True, SSD_F32)
+    ws = workspace if workspace is not None else _workspace(dev, nbytes)
+    with torch.cuda.device(dev):
+        st = lib.ssd_scan_fwd_complex_packed(_ptr(proj), io, _ptr(dt_bias), _ptr(A), _ptr(D), _ptr(init_state),
+                                             _ptr(final_state), _ptr(y), b, T, H, P, N, chunk_size, _ptr(ws),
+                                             0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st)
+    return y, final_state
+
+
+def ssd_scan_final_state(x, dt, A, B, init_state=None, *, chunk_size=256, final_state=None,
+                         total_log_decay=None, workspace=None, stream=None):
+    """Final state and total log-decay of a (slice of a) sequence, without its
+    outputs: the state-only scan.  Returns (final_state [b,H,P,N] float32,
+    total_log_decay [b,H] float32 = A * sum of dt)."""
+    lib = load_library()
+    dev = x.device
+    b, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    io = {torch.bfloat16: SSD_BF16, torch.float32: SSD_F32}.get(x.dtype)
+    if io is None:
+        raise ValueError("x must be bfloat16 or float32")
+    _need(x, "x", x.dtype, dev)
+    _need(dt, "dt", torch.float32, dev, (b, T, H))
+    _need(A, "A", torch.float32, dev, (H,))
+    _need(B, "B", x.dtype, dev, (b, T, G, N))
+    _need(init_state, "init_state", torch.float32, dev, (b, H, P, N), allow_none=True)
+    if final_state is None:
+        final_state = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _need(final_state, "final_state", torch.float32, dev, (b, H, P, N))
+    if total_log_decay is None:
+        total_log_decay = torch.empty((b, H), dtype=torch.float32, device=dev)
+    _need(total_log_decay, "total_log_decay", torch.float32, dev, (b, H))
+    nbytes = ssd_scan_workspace_size(b, T, H, P, G, N, chunk_size, False, io)
+    ws = workspace if workspace is not None else _workspace(dev, nbytes)
+    with torch.cuda.device(dev):
+        st = lib.ssd_scan_final_state(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(init_state), _ptr(final_state),
+                                      _ptr(total_log_decay), io, b, T, H, P, G, N, chunk_size, _ptr(ws),
+                                      0 if ws is None else ws.numel(), _stream_handle(stream))
+    _check(st)
+    return final_state, total_log_decay
+
+
+def ssd_fold_states(states, log_decay, *, out=None, stream=None):
+    """The state entering the slice after the given ones: h_0 = states[0],
+    h_j = exp(log_decay[j]) h_{j-1} + states[j]; returns h_{n-1}.
+    states [n, b, H, P, N] float32, log_decay [n, b, H] float32."""
+    lib = load_library()
+    dev = states.device
+    n, b, H, P, N = states.shape
+    _need(states, "states", torch.float32, dev)
+    _need(log_decay, "log_decay", torch.float32, dev, (n, b, H))
+    if out is None:
+        out = torch.empty((b, H, P, N), dtype=torch.float32, device=dev)
+    _need(out, "out", torch.float32, dev, (b, H, P, N))
+    with torch.cuda.device(dev):
+        st = lib.ssd_fold_states(_ptr(states), _ptr(log_decay), n, _ptr(out), b, H, P, N, _stream_handle(stream))
+    _check(st)
+    return out
 
 
 def ssd_scan_fwd_noalloc(x, dt, A, B, C, D=None, init_state=None, *, chunk_size=256, y=None,

@@ -22,7 +22,9 @@
 // [u_re, -u_im] . [v_re, v_im], so all four contractions are real GEMMs with
 // K = 2N, register-tiled below.  Three kernels, as in the real CUDA-core path:
 // chunk state, the sequential state pass over chunks, and the chunk scan.
+#include "cplx_view.cuh"
 #include "ssd_internal.cuh"
+#include "tc_ptx.cuh"
 
 namespace ssd {
 namespace {
@@ -71,11 +73,13 @@ __device__ void warp_scan_d(double *v, int Q) {
 
 // dt of the chunk and its cumulative log-decay (real and imaginary parts, double)
 // into shared memory; tokens past the sequence end get dt = 0.
-__device__ void chunk_log_decay(const ScanArgs &a, int b, int h, int c, float *dts, double *cre, double *cim) {
+template <typename T>
+__device__ void chunk_log_decay(const ScanArgs &a, const CplxView<T> &v, int b, int h, int c, float *dts, double *cre,
+                                double *cim) {
     const int Q = a.chunk, t0 = c * Q, valid = min(Q, a.seqlen - t0);
     const float Ar = a.A[2 * h], Ai = a.A[2 * h + 1];
     for (int s = threadIdx.x; s < Q; s += NT) {
-        const float d = s < valid ? a.dt[((size_t)b * a.seqlen + t0 + s) * a.nheads + h] : 0.f;
+        const float d = s < valid ? view_dt(v, (size_t)b * a.seqlen + t0 + s, h) : 0.f;
         dts[s] = d;
         cre[s] = (double)d * Ar;
         cim[s] = (double)d * Ai;
@@ -94,7 +98,8 @@ __device__ void chunk_log_decay(const ScanArgs &a, int b, int h, int c, float *d
 // thread: 4 p x 8 interleaved values, columns 4 tj .. 4 tj + 3 and 64 + 4 tj ..
 // 64 + 4 tj + 3 (each 8-thread phase of a 128-bit shared load then reads 128
 // contiguous bytes: no bank conflict).
-__global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w, int npt, int njt) {
+template <typename T>
+__global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w, CplxView<T> v, int npt, int njt) {
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int c = blockIdx.x, h = blockIdx.y;
     const int b = blockIdx.z / (npt * njt), pt = (blockIdx.z / njt) % npt, jt = blockIdx.z % njt;
@@ -111,7 +116,7 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
     float *Xw = reinterpret_cast<float *>(rot + Q);     // [KS][TP]
     float *Bt = Xw + KS * TP;                           // [KS][TJ]
 
-    chunk_log_decay(a, b, h, c, dts, cre, cim);
+    chunk_log_decay(a, v, b, h, c, dts, cre, cim);
     const double R = cre[Q - 1], Th = cim[Q - 1];
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c;
     if (blockIdx.z % (npt * njt) == 0) {
@@ -138,8 +143,6 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-    const float *xg = reinterpret_cast<const float *>(a.x);
-    const cf *Bg = reinterpret_cast<const cf *>(a.B);
     for (int s0 = 0; s0 < valid; s0 += KS) {
         {  // all of a thread's loads are issued before its first shared-memory store
             constexpr int IX = KS * TP / NT, IB = KS * (TJ / 2) / NT;
@@ -148,13 +151,12 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
 #pragma unroll
             for (int it = 0; it < IX; ++it) {
                 const int i = threadIdx.x + it * NT, k = i / TP, p = i % TP, s = s0 + k;
-                xv[it] = (s < valid && p0 + p < P) ? xg[(((size_t)b * a.seqlen + t0 + s) * H + h) * P + p0 + p] : 0.f;
+                xv[it] = (s < valid && p0 + p < P) ? view_x(v, (size_t)b * a.seqlen + t0 + s, h, P, p0 + p) : 0.f;
             }
 #pragma unroll
             for (int it = 0; it < IB; ++it) {
                 const int i = threadIdx.x + it * NT, k = i / (TJ / 2), m = i % (TJ / 2), s = s0 + k;
-                bv[it] = (s < valid && n0 + m < N) ? Bg[(((size_t)b * a.seqlen + t0 + s) * a.ngroups + g) * N + n0 + m]
-                                                   : cf{0.f, 0.f};
+                bv[it] = (s < valid && n0 + m < N) ? view_b(v, (size_t)b * a.seqlen + t0 + s, g, n0 + m) : cf{0.f, 0.f};
             }
 #pragma unroll
             for (int it = 0; it < IX; ++it) {
@@ -238,11 +240,14 @@ __global__ void __launch_bounds__(NT) cplx_state_pass_kernel(ScanArgs a, CWs w) 
 // Block: one (batch, head, chunk), 64 rows l and 64 head-dim columns p;
 // thread: 4 x 4 outputs.
 //   y[l, p] = exp(r_l) Re(C'_l . h_in[p]) + sum_{s <= l} exp(r_l - r_s) dt_s Re(C'_l . B'_s) x_s[p] + D x_l[p]
-__global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, int nrt, int npt) {
+// One (batch, head, chunk, 64-row tile, 64-column tile) of the chunk scan; the
+// kernel below runs one per block, and the tensor-core chunk scan calls it for
+// chunks whose decay is too steep for its factored form.  smem_raw: at least
+// cplx_scan_tile_smem(Q) bytes.
+template <typename T>
+__device__ void cplx_scan_tile(const ScanArgs &a, const CWs &w, const CplxView<T> &v, int b, int h, int c, int rt,
+                               int pt, unsigned char *smem_raw) {
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate, K2 = 2 * N;
-    const int rt = blockIdx.x % nrt, c = blockIdx.x / nrt;
-    const int h = blockIdx.y;
-    const int pt = blockIdx.z % npt, b = blockIdx.z / npt;
     const int g = h / (H / a.ngroups);
     const int t0 = c * Q, valid = min(Q, a.seqlen - t0);
     const int l0 = rt * TL;
@@ -251,7 +256,6 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
     const int p0 = pt * TP;
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c;
 
-    extern __shared__ __align__(16) unsigned char smem_raw[];
     float *rr = reinterpret_cast<float *>(smem_raw);   // r_s (real cumulative log-decay)
     float *dts = rr + Q;
     float2 *ph = reinterpret_cast<float2 *>(dts + Q);  // e^{i theta_s}
@@ -265,21 +269,18 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
         double sn, cn;
         sincos(w.cs[(bhc * 2 + 1) * Q + s], &sn, &cn);
         ph[s] = make_float2((float)cn, (float)sn);
-        dts[s] = s < valid ? a.dt[((size_t)b * a.seqlen + t0 + s) * H + h] : 0.f;
+        dts[s] = s < valid ? view_dt(v, (size_t)b * a.seqlen + t0 + s, h) : 0.f;
     }
     __syncthreads();
 
     const int li = threadIdx.x / 16, pi = threadIdx.x % 16;
-    const cf *Cg = reinterpret_cast<const cf *>(a.C);
-    const cf *Bg = reinterpret_cast<const cf *>(a.B);
-    const float *xg = reinterpret_cast<const float *>(a.x);
     // [C'_re, -C'_im] of row l, complex index n, into At[kk][l] (kk = 2 (n - n0))
     auto stage_c = [&](int kc) {
         for (int i = threadIdx.x; i < (KC / 2) * TL; i += NT) {
             const int l = i / (KC / 2), m = i % (KC / 2), n = kc / 2 + m;
             float vr = 0.f, vi = 0.f;
             if (l < rows && n < N) {
-                const cf cv = Cg[(((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + n];
+                const cf cv = view_c(v, (size_t)b * a.seqlen + t0 + l0 + l, g, n);
                 const float2 e = ph[l0 + l];
                 vr = cv.re * e.x - cv.im * e.y;
                 vi = -(cv.re * e.y + cv.im * e.x);
@@ -342,7 +343,7 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
                 const int s = i / (KC / 2), m = i % (KC / 2), n = kc / 2 + m;
                 float vr = 0.f, vi = 0.f;
                 if (s0 + s < valid && n < N) {
-                    const cf bv = Bg[(((size_t)b * a.seqlen + t0 + s0 + s) * a.ngroups + g) * N + n];
+                    const cf bv = view_b(v, (size_t)b * a.seqlen + t0 + s0 + s, g, n);
                     const float2 e = ph[s0 + s];  // rotate by e^{-i theta_s}
                     vr = bv.re * e.x + bv.im * e.y;
                     vi = bv.im * e.x - bv.re * e.y;
@@ -376,8 +377,7 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
         }
         for (int i = threadIdx.x; i < 64 * TP; i += NT) {
             const int s = i / TP, p = i % TP;
-            Xs[i] = (s0 + s < valid && p0 + p < P) ? xg[(((size_t)b * a.seqlen + t0 + s0 + s) * H + h) * P + p0 + p]
-                                                   : 0.f;
+            Xs[i] = (s0 + s < valid && p0 + p < P) ? view_x(v, (size_t)b * a.seqlen + t0 + s0 + s, h, P, p0 + p) : 0.f;
         }
         __syncthreads();
 #pragma unroll 4
@@ -404,9 +404,17 @@ __global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, 
             const int p = p0 + 4 * pi + j;
             if (p >= P) continue;
             const size_t idx = (((size_t)b * a.seqlen + t0 + l0 + l) * H + h) * P + p;
-            yg[idx] = a.D ? fmaf(Dh, xg[idx], acc[i][j]) : acc[i][j];
+            yg[idx] = a.D ? fmaf(Dh, view_x(v, (size_t)b * a.seqlen + t0 + l0 + l, h, P, p), acc[i][j]) : acc[i][j];
         }
     }
+    __syncthreads();  // the shared memory may be reused by the caller
+}
+
+template <typename T>
+__global__ void __launch_bounds__(NT) cplx_chunk_scan_kernel(ScanArgs a, CWs w, CplxView<T> v, int nrt, int npt) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    cplx_scan_tile<T>(a, w, v, blockIdx.z / npt, blockIdx.y, blockIdx.x / nrt, blockIdx.x % nrt, blockIdx.z % npt,
+                      smem_raw);
 }
 
 // The chunk scan for 2N <= 128: the rotated C of the block's 64 rows is staged
@@ -421,7 +429,8 @@ __device__ __forceinline__ void stage_index(int i, int &m, int &c) {  // i in [0
     m = (blk & 7) * 8 + (lane & 7);
     c = (blk >> 3) * 4 + (lane >> 3);
 }
-__global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, CWs w, int nrt, int npt) {
+template <typename T>
+__global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, CWs w, CplxView<T> v, int nrt, int npt) {
     const int Q = a.chunk, H = a.nheads, P = a.headdim, N = a.dstate;
     const int rt = blockIdx.x % nrt, c = blockIdx.x / nrt;
     const int h = blockIdx.y;
@@ -448,12 +457,9 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
         double sn, cn;
         sincos(w.cs[(bhc * 2 + 1) * Q + s], &sn, &cn);
         ph[s] = make_float2((float)cn, (float)sn);
-        dts[s] = s < valid ? a.dt[((size_t)b * a.seqlen + t0 + s) * H + h] : 0.f;
+        dts[s] = s < valid ? view_dt(v, (size_t)b * a.seqlen + t0 + s, h) : 0.f;
     }
     __syncthreads();
-    const cf *Cg = reinterpret_cast<const cf *>(a.C);
-    const cf *Bg = reinterpret_cast<const cf *>(a.B);
-    const float *xg = reinterpret_cast<const float *>(a.x);
     constexpr int IT = 64 * 64 / NT;  // staged elements per thread
     {
         cf cv[IT];
@@ -461,8 +467,7 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
         for (int it = 0; it < IT; ++it) {
             int m, l;
             stage_index(threadIdx.x + it * NT, m, l);
-            cv[it] = (l < rows && m < N) ? Cg[(((size_t)b * a.seqlen + t0 + l0 + l) * a.ngroups + g) * N + m]
-                                         : cf{0.f, 0.f};
+            cv[it] = (l < rows && m < N) ? view_c(v, (size_t)b * a.seqlen + t0 + l0 + l, g, m) : cf{0.f, 0.f};
         }
 #pragma unroll
         for (int it = 0; it < IT; ++it) {
@@ -480,12 +485,12 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
     for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-    // acc(l, j) += sum_k Ch[k][l] T[k][j] over the 2N interleaved values
-    auto gemm_k = [&](const float *T, float (&o)[4][4]) {
+    // acc(l, j) += sum_k Ch[k][l] Tk[k][j] over the 2N interleaved values
+    auto gemm_k = [&](const float *Tk, float (&o)[4][4]) {
 #pragma unroll 8
         for (int k = 0; k < 128; ++k) {
             const float4 av = *reinterpret_cast<const float4 *>(Ch + k * LD + 4 * li);
-            const float4 bv = *reinterpret_cast<const float4 *>(T + k * LD + 4 * pi);
+            const float4 bv = *reinterpret_cast<const float4 *>(Tk + k * LD + 4 * pi);
             const float aa[4] = {av.x, av.y, av.z, av.w}, bb[4] = {bv.x, bv.y, bv.z, bv.w};
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -532,11 +537,9 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
             for (int it = 0; it < IT; ++it) {
                 int m, sb;
                 stage_index(threadIdx.x + it * NT, m, sb);
-                bv[it] = (s0 + sb < valid && m < N) ? Bg[(((size_t)b * a.seqlen + t0 + s0 + sb) * a.ngroups + g) * N + m]
-                                                    : cf{0.f, 0.f};
+                bv[it] = (s0 + sb < valid && m < N) ? view_b(v, (size_t)b * a.seqlen + t0 + s0 + sb, g, m) : cf{0.f, 0.f};
                 const int i = threadIdx.x + it * NT, s = i / TP, p = i % TP;  // x: p fastest
-                xv[it] = (s0 + s < valid && p0 + p < P) ? xg[(((size_t)b * a.seqlen + t0 + s0 + s) * H + h) * P + p0 + p]
-                                                        : 0.f;
+                xv[it] = (s0 + s < valid && p0 + p < P) ? view_x(v, (size_t)b * a.seqlen + t0 + s0 + s, h, P, p0 + p) : 0.f;
             }
 #pragma unroll
             for (int it = 0; it < IT; ++it) {
@@ -594,14 +597,28 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
             const int p = p0 + 4 * pi + j;
             if (p >= P) continue;
             const size_t idx = (((size_t)b * a.seqlen + t0 + l0 + l) * H + h) * P + p;
-            yg[idx] = a.D ? fmaf(Dh, xg[idx], acc[i][j]) : acc[i][j];
+            yg[idx] = a.D ? fmaf(Dh, view_x(v, (size_t)b * a.seqlen + t0 + l0 + l, h, P, p), acc[i][j]) : acc[i][j];
         }
     }
 }
 
+#include "scan_complex_tc.cuh"
+
 }  // namespace
 
-cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
+size_t cplx_scan_tile_smem(int Q) {
+    return 2 * Q * sizeof(float) + Q * sizeof(float2) + (KC * TL + KC * 64 + 64 * TL + 64 * TP) * sizeof(float);
+}
+
+cudaError_t launch_cplx_state_pass(const ScanArgs &a, void *ws, cudaStream_t st) {
+    const CWs w = carve_c(ws, a);
+    const int PN = a.headdim * a.dstate;
+    cplx_state_pass_kernel<<<dim3((PN + NT - 1) / NT, a.nheads, a.batch), NT, 0, st>>>(a, w);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_complex_cuda_cores(const ScanArgs &a, const CplxView<T> &v, void *ws, cudaStream_t st) {
     const CWs w = carve_c(ws, a);
     const int Q = a.chunk, P = a.headdim, N = a.dstate;
     cudaError_t e;
@@ -609,32 +626,71 @@ cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
     const int npt = (P + TP - 1) / TP, njt = (2 * N + TJ - 1) / TJ;
     const size_t sm1 = 2 * Q * sizeof(double) + 2 * Q * sizeof(float) + Q * sizeof(float2) +
                        (KS * TP + KS * TJ) * sizeof(float);
-    if ((e = cudaFuncSetAttribute(cplx_chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1)) !=
-        cudaSuccess)
+    if ((e = cudaFuncSetAttribute(cplx_chunk_state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm1)) != cudaSuccess)
         return e;
-    cplx_chunk_state_kernel<<<dim3(a.nchunks, a.nheads, a.batch * npt * njt), NT, sm1, st>>>(a, w, npt, njt);
+    cplx_chunk_state_kernel<T><<<dim3(a.nchunks, a.nheads, a.batch * npt * njt), NT, sm1, st>>>(a, w, v, npt, njt);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-    const int PN = P * N;
-    cplx_state_pass_kernel<<<dim3((PN + NT - 1) / NT, a.nheads, a.batch), NT, 0, st>>>(a, w);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_cplx_state_pass(a, ws, st)) != cudaSuccess) return e;
 
     const int nrt = (Q + TL - 1) / TL;
     if (N <= 64) {
         const size_t smf = 2 * Q * sizeof(float) + Q * sizeof(float2) + (2 * 128 + 2 * 64) * LD * sizeof(float);
-        if ((e = cudaFuncSetAttribute(cplx_chunk_scan_n64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if ((e = cudaFuncSetAttribute(cplx_chunk_scan_n64_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)smf)) != cudaSuccess)
             return e;
-        cplx_chunk_scan_n64_kernel<<<dim3(a.nchunks * nrt, a.nheads, a.batch * npt), NT, smf, st>>>(a, w, nrt, npt);
+        cplx_chunk_scan_n64_kernel<T><<<dim3(a.nchunks * nrt, a.nheads, a.batch * npt), NT, smf, st>>>(a, w, v, nrt,
+                                                                                                       npt);
         return cudaGetLastError();
     }
-    const size_t sm3 = 2 * Q * sizeof(float) + Q * sizeof(float2) +
-                       (KC * TL + KC * 64 + 64 * TL + 64 * TP) * sizeof(float);
-    if ((e = cudaFuncSetAttribute(cplx_chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm3)) !=
-        cudaSuccess)
+    const size_t sm3 = cplx_scan_tile_smem(Q);
+    if ((e = cudaFuncSetAttribute(cplx_chunk_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)sm3)) != cudaSuccess)
         return e;
-    cplx_chunk_scan_kernel<<<dim3(a.nchunks * nrt, a.nheads, a.batch * npt), NT, sm3, st>>>(a, w, nrt, npt);
+    cplx_chunk_scan_kernel<T><<<dim3(a.nchunks * nrt, a.nheads, a.batch * npt), NT, sm3, st>>>(a, w, v, nrt, npt);
     return cudaGetLastError();
+}
+bool cplx_tc_supported(int headdim, int dstate) { return headdim == 64 && dstate == 64; }
+
+// The tensor-core path: chunk states (tcgen05), the state pass over chunks, the
+// chunk scan (tcgen05; steep chunks on CUDA cores), in 128-token chunks.
+template <typename T>
+cudaError_t launch_complex_tc(const ScanArgs &a0, const CplxView<T> &v, void *ws, cudaStream_t st) {
+    ScanArgs a = a0;
+    a.chunk = ctc::QT;
+    a.nchunks = (a.seqlen + ctc::QT - 1) / ctc::QT;
+    const CWs w = carve_c(ws, a);
+    cudaError_t e;
+    if ((e = cudaFuncSetAttribute(ctc::state_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ctc::SMEM_STATE)) != cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(ctc::scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ctc::SMEM_SCAN)) != cudaSuccess)
+        return e;
+    const dim3 grid(a.nchunks, a.nheads, a.batch);
+    ctc::state_kernel<T><<<grid, ctc::NTH, ctc::SMEM_STATE, st>>>(a, w, v);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_cplx_state_pass(a, ws, st)) != cudaSuccess) return e;
+    ctc::scan_kernel<T><<<grid, ctc::NTH, ctc::SMEM_SCAN, st>>>(a, w, v);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_complex_view(const ScanArgs &a, const CplxView<T> &v, void *ws, cudaStream_t st) {
+    if (cplx_tc_supported(a.headdim, a.dstate)) return launch_complex_tc<T>(a, v, ws, st);
+    return launch_complex_cuda_cores<T>(a, v, ws, st);
+}
+
+cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
+    return launch_complex_view<float>(a, plain_view(a), ws, st);
+}
+
+cudaError_t launch_complex_packed(const ScanArgs &a, const void *proj, bool proj_bf16, const float *dt_bias, void *ws,
+                                  cudaStream_t st) {
+    if (proj_bf16)
+        return launch_complex_view<__nv_bfloat16>(
+            a, packed_view<__nv_bfloat16>(proj, dt_bias, a.nheads, a.headdim, a.dstate), ws, st);
+    return launch_complex_view<float>(a, packed_view<float>(proj, dt_bias, a.nheads, a.headdim, a.dstate), ws, st);
 }
 
 }  // namespace ssd

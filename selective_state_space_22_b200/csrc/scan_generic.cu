@@ -385,6 +385,7 @@ cudaError_t launch_typed(const ScanArgs &a, void *wsp, cudaStream_t st) {
     dim3 g2((PN + NT - 1) / NT, a.nheads, a.batch);
     state_pass_kernel<<<g2, NT, 0, st>>>(a, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (!a.y) return cudaSuccess;  // final state only
 
     size_t sm3 = Q * sizeof(double) + Q * sizeof(float) + (KT * RT + KT * 64) * sizeof(float) +
                  (ST * RT + ST * PT) * sizeof(float);

@@ -88,7 +88,8 @@ enum {
     // count 1 (TMA bytes or an MMA commit); B_EMPTY ({C, B} slot free): 2, a
     // commit from each MMA issuer
     B_FULL = 0, B_EMPTY = 2, B_G = 4, B_S = 6, B_Y = 8, B_YO = 10,
-    // the X ring; B_XEMPTY counts the 128 W threads and M X's commit
+    // the X ring; B_XEMPTY counts S's commit (S is issued once W has read X)
+    // and M X's commit
     B_XFULL = 12, B_XEMPTY = 15,
     // count 128 (one warpgroup).  B_HW: h_in^T written; B_H: chunk state read
     B_CS = 18, B_W = 20, B_M = 22, B_H = 24, B_FREE = 26, B_HW = 28,
@@ -97,7 +98,7 @@ enum {
     B_DRAIN = 30, NBARS = 32
 };
 // misc: cs[2][128], dtv[2][128], bfac[2][128] floats, lam[2], dh[2], wtot[4],
-// abort word + 4 votes (8 ints), bars, tmem base
+// the abort word (+ 7 spare ints), bars, tmem base
 constexpr int MISC_BYTES = 3 * 2 * QT * 4 + 8 + 8 + 16 + 32 + NBARS * 8 + 8;
 constexpr int SMEM_ALLOC = OFF_MISC + MISC_BYTES + 1024;
 
@@ -165,25 +166,40 @@ __device__ __forceinline__ unsigned long long now_ns() {
 }
 
 // Bounded wait on an mbarrier phase.  Returns false, without waiting further,
-// once the CTA's abort word is set; sets the device error word and the abort
-// word when the bound runs out.  A role that gets false stops issuing work and
-// leaves its tile loop (warps decide together: warp_ok).
-__device__ bool mbar_wait(uint64_t *bar, uint32_t parity, const TcParams &p, volatile int *abort_s) {
-    if (mbar_try_wait(bar, parity)) return true;
+// once the CTA's abort word is set; a wait that runs out sets the device error
+// word and the abort word.  After an abort, the single-thread roles (the TMA
+// producer and the MMA issuers) leave their tile loops and wait for the loads
+// and MMAs they issued; the warpgroup roles run their remaining tiles with every
+// wait falling through (their TMEM and shared-memory accesses stay in bounds and
+// their named barriers stay matched; the outputs are invalid and reported so).
+// They arrive only on barriers of their own warpgroup, so no phase count is
+// overrun.  Only the first probe is inlined; the polling loop, which looks at
+// the abort word once a wait has lasted 20 us, is one out-of-line copy, so that
+// the many wait sites of the hot loops stay small.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_s, int *err,
+                                            unsigned long long limit) {
     const unsigned long long t0 = now_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (*abort_s) return false;
-        if (now_ns() - t0 > p.wait_ns) {
-            atomicCAS(p.dev_error, 0, DEV_TIMEOUT);
-            *abort_s = 1;
-            return false;
+        const unsigned long long waited = now_ns() - t0;
+        if (waited > 20000) {  // the abort word is only looked at once a wait is long
+            if (*abort_s) return false;
+            if (waited > limit) {
+                atomicCAS(err, 0, DEV_TIMEOUT);
+                *abort_s = 1;
+                return false;
+            }
         }
     }
     return true;
 }
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const TcParams &p, volatile int *abort_s) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_slow(bar, parity, abort_s, p.dev_error, p.wait_ns);
+}
 // The same without the abort shortcut: how a role waits for its own TMA loads
 // or MMAs to finish before the CTA exits (still bounded).
-__device__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, const TcParams &p, volatile int *abort_s) {
+__device__ __noinline__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, const TcParams &p,
+                                             volatile int *abort_s) {
     const unsigned long long t0 = now_ns();
     while (!mbar_try_wait(bar, parity)) {
         if (now_ns() - t0 > p.wait_ns) {
@@ -193,8 +209,6 @@ __device__ void mbar_wait_drain(uint64_t *bar, uint32_t parity, const TcParams &
         }
     }
 }
-// A warp goes on only if every lane's wait succeeded.
-__device__ __forceinline__ bool warp_ok(bool ok) { return __all_sync(0xffffffffu, ok); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);  // .x (low half) = lo
@@ -298,15 +312,14 @@ __global__ void __launch_bounds__(NTH, 1)
     float *lam_s = bfac + 2 * QT;                          // [2]
     float *dh_s = lam_s + 2;                               // [2]
     float *wtot = dh_s + 2;                                // [4]
-    volatile int *abort_s = reinterpret_cast<volatile int *>(wtot + 4);  // [1], then votes [4]
-    volatile int *votes = abort_s + 4;
+    volatile int *abort_s = reinterpret_cast<volatile int *>(wtot + 4);  // [1]
     uint64_t *bars = reinterpret_cast<uint64_t *>(wtot + 12);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBARS);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int i = 0; i < B_CS; ++i)
-            mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1) ? 2 : (i >= B_XEMPTY && i < B_XEMPTY + 3) ? 129 : 1);
+            mbar_init(&bars[i], (i == B_EMPTY || i == B_EMPTY + 1 || (i >= B_XEMPTY && i < B_XEMPTY + 3)) ? 2 : 1);
         for (int i = B_CS; i < B_DRAIN; ++i) mbar_init(&bars[i], 128);
         mbar_init(&bars[B_DRAIN], 1);
         mbar_init(&bars[B_DRAIN + 1], 1);
@@ -386,6 +399,7 @@ __global__ void __launch_bounds__(NTH, 1)
                            smem_desc_sw128(aW + kk * 2048, 8192, 1024), IDESC_S, kk > 0);
                 mma_commit(&bars[B_S + s]);
                 mma_commit(&bars[B_EMPTY + s]);  // G and S are done with the slot's B and C
+                mma_commit(&bars[B_XEMPTY + k % X_SLOTS]);  // W (issued after W was built) is done with X
             }
             mma_commit(&bars[B_DRAIN]);  // this thread's MMAs are done before the CTA exits
             mbar_wait_drain(&bars[B_DRAIN], 0, p, abort_s);
@@ -439,9 +453,9 @@ __global__ void __launch_bounds__(NTH, 1)
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
             const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
-            if (!warp_ok(mbar_wait(&bars[B_CS + s], par, p, abort_s))) break;
+            mbar_wait(&bars[B_CS + s], par, p, abort_s);
             const float v = csk[row], Dh = dh_s[s];
-            if (!warp_ok(mbar_wait(&bars[B_G + s], par, p, abort_s))) break;
+            mbar_wait(&bars[B_G + s], par, p, abort_s);
             tc_fence_after();
             if (!so) {
 #pragma unroll 1
@@ -460,7 +474,7 @@ __global__ void __launch_bounds__(NTH, 1)
             const Tile t = decode_tile(p, k);
             const int s = k & 1;
             const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s + lane_off;
-            if (!warp_ok(mbar_wait(&bars[B_CS + s], par, p, abort_s))) break;
+            mbar_wait(&bars[B_CS + s], par, p, abort_s);
             const float lam = lam_s[s];
             if (t.c == 0) {
                 if (p.init_state) {
@@ -475,7 +489,7 @@ __global__ void __launch_bounds__(NTH, 1)
             if (!t.state_only) {  // h_in^T (rows n, bf16, 128-byte swizzle)
                 // the one buffer was last read by C h^T of tile k-1; waiting for
                 // that (and not for this tile's G) lets C h^T go as early as it can
-                if (k > 0 && !warp_ok(mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s))) break;
+                if (k > 0) mbar_wait(&bars[B_YO + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s);
                 uint8_t *sh = sm + OFF_H;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
@@ -487,7 +501,7 @@ __global__ void __launch_bounds__(NTH, 1)
                 fence_proxy_async_smem();
             }
             mbar_arrive(&bars[B_HW + s]);  // C h_in^T may go
-            if (!warp_ok(mbar_wait(&bars[B_S + s], par, p, abort_s))) break;
+            mbar_wait(&bars[B_S + s], par, p, abort_s);
             tc_fence_after();
             {  // h_out = exp(lam) h_in + S, 32 columns at a time
                 const float el = __expf(lam);
@@ -526,17 +540,7 @@ __global__ void __launch_bounds__(NTH, 1)
             Dn = p.D ? p.D[tn.h] : 0.f;
         }
         Tile prev{};  // tile k-1, whose y this step writes
-        // A failed wait skips the rest of the step; the warpgroup stops together
-        // at the next step, deciding from votes cast before its first named
-        // barrier, so that no warp is left waiting at a barrier.
-        bool failed = false;
         for (int k = 0; k <= ntl; ++k) {
-            if (failed) {
-                if (k == ntl) break;  // no barrier left: leave alone
-                if (lane == 0) votes[quad] = 1;
-            } else if (lane == 0 && k < ntl) {
-                votes[quad] = *abort_s;
-            }
             Tile cur{};
             if (k < ntl) {
                 cur = tn;
@@ -557,7 +561,6 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 if (lane == 31) wtot[quad] = v;
                 named_bar_sync(BAR_MATH, 128);
-                if (votes[0] | votes[1] | votes[2] | votes[3]) break;  // uniform over the warpgroup
                 for (int w = 0; w < quad; ++w) v += wtot[w];
                 csk[row] = v;
                 dtk[row] = d;
@@ -572,11 +575,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 mbar_arrive(&bars[B_CS + s]);
                 // W (one buffer): the previous tile's S must have read it
                 const int xs = k % X_SLOTS;
-                if (!warp_ok(mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s)) ||
-                    (k > 0 && !warp_ok(mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s)))) {
-                    failed = true;
-                    continue;
-                }
+                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s);
+                if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s);
                 // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
                 // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
                 // SM sub-partition also builds the most M blocks, skips it and the warp
@@ -589,17 +589,13 @@ __global__ void __launch_bounds__(NTH, 1)
                 if (quad == 0) w_row(96 + lane);
                 fence_proxy_async_smem();
                 mbar_arrive(&bars[B_W + s]);
-                mbar_arrive(&bars[B_XEMPTY + xs]);  // this thread is done reading the X slot
             }
             if (k > 0) {  // y of tile k-1
                 const int j = k - 1, s = j & 1;
                 const uint32_t par = (j >> 1) & 1, tm = tmem + 256 * s + lane_off;
                 const Tile t = prev;
                 const float e = __expf(cs[s * QT + row]);
-                if (!warp_ok(mbar_wait(&bars[B_Y + s], par, p, abort_s))) {
-                    failed = true;
-                    continue;
-                }
+                mbar_wait(&bars[B_Y + s], par, p, abort_s);
                 tc_fence_after();
                 if (!t.state_only) {
                     __nv_bfloat16 *yrow = p.y + (((size_t)t.b * p.seqlen + t.t0 + row) * p.nheads + t.h) * PD;

@@ -109,6 +109,12 @@ Plan plan_scan(int batch, int seqlen, int nheads, int headdim, int ngroups, int 
         p.launches = ssd::tc_kernel_launches();
         return p;
     }
+    if (cplx && ssd::cplx_tc_supported(headdim, dstate)) {  // tensor-core path: 128-token chunks
+        p.ws = ssd::generic_workspace_bytes(batch, nheads, headdim, dstate, 128, seqlen > 0 ? (seqlen + 127) / 128 : 0,
+                                            true);
+        p.launches = 3;
+        return p;
+    }
     p.ws = ssd::generic_workspace_bytes(batch, nheads, headdim, dstate, chunk, nchunks, cplx);
     p.launches = 3;
     return p;
@@ -123,7 +129,7 @@ ssd_status run_scan(const void *x, const float *dt, const float *A, const void *
     const size_t state_floats = (size_t)batch * nheads * headdim * dstate * (cplx ? 2 : 1);
     const bool any_tokens = (size_t)batch * seqlen > 0;
     if (any_tokens) {
-        if (!x || !dt || !A || !B || !C || !y)
+        if (!x || !dt || !A || !B || !C || (!y && !final_state))
             return fail(SSD_ERR_INVALID_ARG, "x, dt, A, B, C and y must be non-null");
         const void *ptrs[] = {x, dt, A, B, C, y, D, init_state, final_state};
         for (const void *p : ptrs)
@@ -174,6 +180,77 @@ ssd_status run_scan(const void *x, const float *dt, const float *A, const void *
     a.dev_error = dev_err;
     cudaError_t e = pl.tc ? ssd::launch_tc_scan(a, workspace, st)
                           : ssd::launch_generic_scan(a, cplx, bf16, workspace, st);
+    if (e != cudaSuccess) return cuda_fail(e, "scan launch");
+    return SSD_OK;
+}
+
+// The state-only scan of one slice of a sequence: final state and total log-decay.
+ssd_status run_final_state(const void *x, const float *dt, const float *A, const void *B, const float *init_state,
+                           float *final_state, float *total_log_decay, bool bf16, int batch, int seqlen, int nheads,
+                           int headdim, int ngroups, int dstate, int chunk, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+    ssd_status s = check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, chunk);
+    if (s != SSD_OK) return s;
+    if (!final_state || !A) return fail(SSD_ERR_INVALID_ARG, "final_state and A are required");
+    const bool any_tokens = (size_t)batch * seqlen > 0;
+    if (any_tokens && (!x || !dt || !B)) return fail(SSD_ERR_INVALID_ARG, "x, dt and B must be non-null");
+    const void *ptrs[] = {x, dt, A, B, init_state, final_state, total_log_decay};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (total_log_decay) {
+        cudaError_t e = any_tokens ? ssd::launch_log_decay_sum(dt, A, total_log_decay, batch, seqlen, nheads, st)
+                                   : cudaMemsetAsync(total_log_decay, 0, (size_t)batch * nheads * sizeof(float), st);
+        if (e != cudaSuccess) return cuda_fail(e, "log-decay sum launch");
+    }
+    // y = NULL selects the state-only form of the scan; C is never read then.
+    return run_scan(x, dt, A, B, B, nullptr, init_state, final_state, nullptr, false, bf16, batch, seqlen, nheads,
+                    headdim, ngroups, dstate, chunk, workspace, workspace_bytes, stream);
+}
+
+// The complex scan reading the packed projection output.
+ssd_status run_scan_packed(const void *proj, bool proj_bf16, const float *dt_bias, const float *A, const float *D,
+                           const float *init_state, float *final_state, float *y, int batch, int seqlen, int nheads,
+                           int headdim, int dstate, int chunk, void *workspace, size_t workspace_bytes, void *stream) {
+    ssd_status s = check_scan_dims(batch, seqlen, nheads, headdim, nheads, dstate, chunk);
+    if (s != SSD_OK) return s;
+    const bool any_tokens = (size_t)batch * seqlen > 0;
+    if (any_tokens && (!proj || !A || !y)) return fail(SSD_ERR_INVALID_ARG, "proj, A and y must be non-null");
+    const void *ptrs[] = {proj, dt_bias, A, D, init_state, final_state, y};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (!any_tokens) {
+        if (final_state && final_state != init_state) {
+            cudaError_t e = ssd::launch_copy_or_zero_state(init_state, final_state,
+                                                           (size_t)batch * nheads * headdim * dstate * 2, st);
+            if (e != cudaSuccess) return cuda_fail(e, "state copy launch");
+        }
+        return SSD_OK;
+    }
+    Plan pl = plan_scan(batch, seqlen, nheads, headdim, nheads, dstate, chunk, true, false);
+    if (!workspace) return fail(SSD_ERR_WORKSPACE, "workspace is NULL; %zu bytes are needed", pl.ws);
+    if (workspace_bytes < pl.ws)
+        return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes is too small; %zu are needed", workspace_bytes, pl.ws);
+    if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    int *dev_err = device_error_ptr(&s);
+    if (!dev_err) return s;
+    ssd::ScanArgs a{};
+    a.A = A;
+    a.D = D;
+    a.init_state = init_state;
+    a.final_state = final_state;
+    a.y = y;
+    a.batch = batch;
+    a.seqlen = seqlen;
+    a.nheads = nheads;
+    a.headdim = headdim;
+    a.ngroups = nheads;
+    a.dstate = dstate;
+    a.chunk = chunk;
+    a.nchunks = (seqlen + chunk - 1) / chunk;
+    a.dev_error = dev_err;
+    cudaError_t e = ssd::launch_complex_packed(a, proj, proj_bf16, dt_bias, workspace, st);
     if (e != cudaSuccess) return cuda_fail(e, "scan launch");
     return SSD_OK;
 }
@@ -296,9 +373,36 @@ ssd_status ssd_scan_fwd(const void *x, const float *dt, const float *A, const vo
                         int ngroups, int dstate, int chunk_size, void *workspace,
                         size_t workspace_bytes, void *stream) {
     if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    if (!y && (long long)batch * seqlen > 0) return fail(SSD_ERR_INVALID_ARG, "y must be non-null");
     return run_scan(x, dt, A, B, C, D, init_state, final_state, y, false, io_dtype == SSD_BF16, batch,
                     seqlen, nheads, headdim, ngroups, dstate, chunk_size, workspace, workspace_bytes,
                     stream);
+}
+
+ssd_status ssd_scan_final_state(const void *x, const float *dt, const float *A, const void *B,
+                                const float *init_state, float *final_state, float *total_log_decay,
+                                ssd_dtype io_dtype, int batch, int seqlen, int nheads, int headdim, int ngroups,
+                                int dstate, int chunk_size, void *workspace, size_t workspace_bytes, void *stream) {
+    if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    return run_final_state(x, dt, A, B, init_state, final_state, total_log_decay, io_dtype == SSD_BF16, batch,
+                           seqlen, nheads, headdim, ngroups, dstate, chunk_size, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_fold_states(const float *states, const float *log_decay, int nstates, float *out, int batch,
+                           int nheads, int headdim, int dstate, void *stream) {
+    if (nstates <= 0 || batch < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "nstates, nheads, headdim and dstate must be > 0 and batch >= 0");
+    if ((long long)batch * nheads * headdim * dstate * nstates > (1LL << 40))
+        return fail(SSD_ERR_UNSUPPORTED, "states too large");
+    if (batch == 0) return SSD_OK;
+    if (!states || !out || (nstates > 1 && !log_decay))
+        return fail(SSD_ERR_INVALID_ARG, "states, out (and log_decay when nstates > 1) must be non-null");
+    for (const void *p : {(const void *)states, (const void *)log_decay, (const void *)out})
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = ssd::launch_fold_states(states, log_decay, nstates, out, batch, nheads, headdim, dstate,
+                                            static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "fold launch");
+    return SSD_OK;
 }
 
 ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A, const float *B,
@@ -306,8 +410,73 @@ ssd_status ssd_scan_fwd_complex(const float *x, const float *dt, const float *A,
                                 float *final_state, float *y, int batch, int seqlen, int nheads,
                                 int headdim, int ngroups, int dstate, int chunk_size, void *workspace,
                                 size_t workspace_bytes, void *stream) {
+    if (!y && (long long)batch * seqlen > 0) return fail(SSD_ERR_INVALID_ARG, "y must be non-null");
     return run_scan(x, dt, A, B, C, D, init_state, final_state, y, true, false, batch, seqlen, nheads,
                     headdim, ngroups, dstate, chunk_size, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_scan_fwd_complex_packed(const void *proj, ssd_dtype proj_dtype, const float *dt_bias, const float *A,
+                                       const float *D, const float *init_state, float *final_state, float *y,
+                                       int batch, int seqlen, int nheads, int headdim, int dstate, int chunk_size,
+                                       void *workspace, size_t workspace_bytes, void *stream) {
+    if (!valid_dtype(proj_dtype)) return fail(SSD_ERR_INVALID_ARG, "proj_dtype must be SSD_F32 or SSD_BF16");
+    return run_scan_packed(proj, proj_dtype == SSD_BF16, dt_bias, A, D, init_state, final_state, y, batch, seqlen,
+                           nheads, headdim, dstate, chunk_size, workspace, workspace_bytes, stream);
+}
+
+ssd_status ssd_conv1d_xbc(const void *xbc, const float *weight, const float *bias, const void *conv_init,
+                          void *x_out, void *B_out, void *C_out, void *conv_final, ssd_dtype io_dtype, int batch,
+                          int seqlen, int x_channels, int bc_channels, int width, int silu, void *stream) {
+    if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    if (batch < 0 || seqlen < 0 || x_channels <= 0 || bc_channels < 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch and seqlen must be >= 0, x_channels > 0, bc_channels >= 0");
+    if (width < 1 || width > 8) return fail(SSD_ERR_UNSUPPORTED, "width must be in 1..8 (got %d)", width);
+    if ((long long)batch * seqlen > (1LL << 31) || batch > 65535 || (long long)x_channels + 2LL * bc_channels > (1 << 24))
+        return fail(SSD_ERR_UNSUPPORTED, "sizes beyond the supported grid");
+    if ((long long)batch * seqlen == 0) return SSD_OK;
+    if (!xbc || !weight || !x_out || (bc_channels > 0 && (!B_out || !C_out)))
+        return fail(SSD_ERR_INVALID_ARG, "xbc, weight, x_out, B_out and C_out must be non-null");
+    for (const void *p : {(const void *)xbc, (const void *)weight, (const void *)bias, (const void *)conv_init,
+                          (const void *)x_out, (const void *)B_out, (const void *)C_out, (const void *)conv_final})
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaError_t e = ssd::launch_conv1d_xbc(xbc, weight, bias, conv_init, x_out, B_out, C_out, conv_final,
+                                           io_dtype == SSD_BF16, batch, seqlen, x_channels, bc_channels, width,
+                                           silu != 0, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "conv1d launch");
+    return SSD_OK;
+}
+
+ssd_status ssd_selective_scan(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                              const float *D, const float *init_state, float *final_state, void *y,
+                              ssd_dtype io_dtype, int batch, int seqlen, int channels, int ngroups, int dstate,
+                              void *stream) {
+    if (!valid_dtype(io_dtype)) return fail(SSD_ERR_INVALID_ARG, "io_dtype must be SSD_F32 or SSD_BF16");
+    if (batch < 0 || seqlen < 0 || channels <= 0 || ngroups <= 0 || dstate <= 0)
+        return fail(SSD_ERR_INVALID_ARG, "batch, seqlen >= 0 and channels, ngroups, dstate > 0 required");
+    if (channels % ngroups != 0)
+        return fail(SSD_ERR_INVALID_ARG, "ngroups (%d) must divide channels (%d)", ngroups, channels);
+    if (!ssd::selective_dstate_supported(dstate))
+        return fail(SSD_ERR_UNSUPPORTED, "dstate must be 4, 8, 16 or 32 (got %d)", dstate);
+    if (batch > 65535 || (long long)batch * seqlen > (1LL << 31))
+        return fail(SSD_ERR_UNSUPPORTED, "sizes beyond the supported grid");
+    if (batch == 0) return SSD_OK;
+    if (!A || (seqlen > 0 && (!x || !dt || !B || !C || !y)))
+        return fail(SSD_ERR_INVALID_ARG, "x, dt, A, B, C and y must be non-null");
+    for (const void *p : {(const void *)x, (const void *)dt, (const void *)A, (const void *)B, (const void *)C,
+                          (const void *)D, (const void *)init_state, (const void *)final_state, (const void *)y})
+        if (p && !aligned16(p)) return fail(SSD_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (seqlen == 0) {
+        e = final_state && final_state != init_state
+                ? ssd::launch_copy_or_zero_state(init_state, final_state, (size_t)batch * channels * dstate, st)
+                : cudaSuccess;
+    } else {
+        e = ssd::launch_selective_scan(x, dt, A, B, C, D, init_state, final_state, y, io_dtype == SSD_BF16, batch,
+                                       seqlen, channels, ngroups, dstate, st);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "selective scan launch");
+    return SSD_OK;
 }
 
 ssd_status ssd_state_update(float *state, const void *x, const float *dt, const float *A,

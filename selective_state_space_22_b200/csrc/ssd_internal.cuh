@@ -69,9 +69,15 @@ enum : int { DEV_OK = 0, DEV_TIMEOUT = 1 };
 // Each returns cudaSuccess or the launch error; none synchronises.
 size_t generic_workspace_bytes(int batch, int nheads, int headdim, int dstate, int chunk,
                                int nchunks, bool cplx);
-// Complex scan on CUDA cores (scan_complex.cu); same workspace layout and size as
-// generic_workspace_bytes(..., cplx = true).
+// Complex scan (scan_complex.cu); same workspace layout and size as
+// generic_workspace_bytes(..., cplx = true), with the chunk 128 when
+// cplx_tc_supported (the tensor-core path evaluates 128-token chunks).
+bool cplx_tc_supported(int headdim, int dstate);
 cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st);
+// The same reading x, B, C and dt from the packed projection output
+// [batch, seqlen, H (P + 4N + 1)] (float32 or bf16), dt = softplus(dt + dt_bias).
+cudaError_t launch_complex_packed(const ScanArgs &a, const void *proj, bool proj_bf16, const float *dt_bias, void *ws,
+                                  cudaStream_t st);
 cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *ws,
                                 cudaStream_t st);
 
@@ -106,6 +112,23 @@ cudaError_t launch_scan_bwd_complex(const BwdCall &call, void *ws, cudaStream_t 
 
 cudaError_t launch_copy_or_zero_state(const float *init_state, float *final_state,
                                       size_t nfloats, cudaStream_t st);
+
+// Sequence split across devices (seqpar.cu): total log-decay of each (batch,
+// head) over a slice, and the ordered fold of the slices' end states.
+cudaError_t launch_log_decay_sum(const float *dt, const float *A, float *out, int batch, int seqlen, int nheads,
+                                 cudaStream_t st);
+cudaError_t launch_fold_states(const float *states, const float *lam, int nstates, float *out, int batch,
+                               int nheads, int headdim, int dstate, cudaStream_t st);
+
+// The variants (variants.cu): the causal conv1d prologue over packed x|B|C
+// channels, and the Mamba-1 selective scan (dstate 4, 8, 16 or 32).
+cudaError_t launch_conv1d_xbc(const void *in, const float *w, const float *bias, const void *cinit, void *xo,
+                              void *bo, void *co, void *cfinal, bool bf16, int batch, int seqlen, int cx, int cb,
+                              int width, int silu, cudaStream_t st);
+bool selective_dstate_supported(int dstate);
+cudaError_t launch_selective_scan(const void *x, const float *dt, const float *A, const void *B, const void *C,
+                                  const float *D, const float *init_state, float *final_state, void *y, bool bf16,
+                                  int batch, int seqlen, int channels, int ngroups, int dstate, cudaStream_t st);
 
 // Sets the message ssd_last_error() returns on this host thread.
 void set_last_error(const char *msg);

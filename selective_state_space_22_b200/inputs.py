@@ -164,6 +164,124 @@ def scan_inputs(shape: ScanShape, seqlen: int | None = None, batch: int | None =
     return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D, "init_state": init}
 
 
+def packed_inputs(shape: ScanShape, proj_dtype: str = "f32") -> dict:
+    """Inputs of the packed complex scan: the projection output proj
+    [b, T, H (P + 4N + 1)] in head-major slices x | Re B | Im B | Re C | Im C | dt
+    ("Block Anatomy, Numerical Stability & Scaling", Block Anatomy 4.1-4.2), and
+    dt_bias, A, D and the initial state.  x ~ N(0, 1); the B and C slices
+    N(0, 1/2) (so E|B|^2 = 1); the dt slice N(0, 1) before the bias;
+    dt_bias_h = log(expm1(dt0_h)) with dt0_h log-uniform in [1e-3, 0.1] (the
+    scan applies softplus(dt + dt_bias) itself).  One group per head."""
+    b, T, H, P, N = shape.batch, shape.seqlen, shape.nheads, shape.headdim, shape.dstate
+    gen = torch.Generator().manual_seed(shape.seed)
+    s = 1.0 / math.sqrt(2.0)
+    x = torch.randn((b, T, H * P), generator=gen)
+    bc = torch.randn((b, T, 4 * H * N), generator=gen) * s
+    z = torch.randn((b, T, H), generator=gen)
+    lo, hi = math.log(1e-3), math.log(0.1)
+    dt0 = torch.exp(torch.rand(H, generator=gen) * (hi - lo) + lo)
+    dt_bias = torch.log(torch.expm1(dt0))
+    A = _complex_A(gen, H)
+    D = torch.randn(H, generator=gen)
+    init = _cnormal(gen, (b, H, P, N)) if shape.init_state else None
+    proj = torch.cat([x, bc, z], dim=-1).to(_tdtype(proj_dtype)).contiguous()
+    return {"proj": proj, "dt_bias": dt_bias.contiguous(), "A": A, "D": D, "init_state": init}
+
+
+def unpack_projection(proj: torch.Tensor, nheads: int, headdim: int, dstate: int) -> dict:
+    """The slices of a packed projection output as separate CPU tensors (x
+    [b,T,H,P], B and C complex [b,T,H,N], raw dt [b,T,H]), widened exactly to
+    float64 / complex128: how the block unpacks them before a scan that takes
+    separate tensors.  Slicing only, no scan arithmetic."""
+    b, T, _ = proj.shape
+    H, P, N = nheads, headdim, dstate
+    p = proj.to(torch.float64)
+    o = [0, H * P, H * P + H * N, H * P + 2 * H * N, H * P + 3 * H * N, H * P + 4 * H * N]
+    x = p[..., o[0]:o[1]].reshape(b, T, H, P)
+    B = torch.complex(p[..., o[1]:o[2]], p[..., o[2]:o[3]]).reshape(b, T, H, N)
+    C = torch.complex(p[..., o[3]:o[4]], p[..., o[4]:o[5]]).reshape(b, T, H, N)
+    dt_raw = p[..., o[5]:]
+    return {"x": x.contiguous(), "B": B.contiguous(), "C": C.contiguous(), "dt_raw": dt_raw.contiguous()}
+
+
+# The Mamba-3-Lite layer fed from its packed projection output, bf16 (the
+# projection's dtype under the block's bf16 autocast).
+MAMBA3_PACKED = ScanShape("mamba3lite-complex-packed-bf16", 4, 2048, 16, 64, 16, 64, 256, "bf16", complex=True,
+                          seed=SEED_BASE + 7)
+
+
+@dataclass(frozen=True)
+class ConvShape:
+    """The causal conv1d prologue over packed x | B | C channels."""
+    name: str
+    batch: int
+    seqlen: int
+    x_channels: int
+    bc_channels: int
+    width: int
+    io_dtype: str
+    silu: bool = True
+    init: bool = False
+    seed: int = SEED_BASE + 8
+
+
+@dataclass(frozen=True)
+class SelectiveShape:
+    """The Mamba-1 selective scan (per-state A)."""
+    name: str
+    batch: int
+    seqlen: int
+    channels: int
+    ngroups: int
+    dstate: int
+    io_dtype: str
+    init_state: bool = False
+    seed: int = SEED_BASE + 9
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+# The BitMamba-1B layer's prologue: x (64 heads x 64) and B, C (one group x 128)
+# channels, kernel 4, SiLU.
+MAMBA2_CONV = ConvShape("mamba2-conv1d-bitmamba1b-bf16", 2, 2048, 4096, 128, 4, "bf16")
+# A Mamba-1 layer at the "Mamba-50M" card's batch (64) and context (512); the
+# card gives no widths, so d_inner 1024 and d_state 16 (the Mamba-1 default).
+MAMBA1_50M = SelectiveShape("mamba1-50m-layer-bf16", 64, 512, 1024, 1, 16, "bf16")
+
+
+def conv_inputs(shape: ConvShape) -> dict:
+    """xbc [b,T,Cx+2Cb] ~ N(0,1), weight [C,K] ~ N(0, 1/K), bias [C] ~ N(0, 0.1^2),
+    conv_init [b,C,K-1] ~ N(0,1) when asked for."""
+    gen = torch.Generator().manual_seed(shape.seed)
+    Ct = shape.x_channels + 2 * shape.bc_channels
+    io = _tdtype(shape.io_dtype)
+    xbc = torch.randn((shape.batch, shape.seqlen, Ct), generator=gen).to(io).contiguous()
+    w = (torch.randn((Ct, shape.width), generator=gen) / math.sqrt(shape.width)).contiguous()
+    bias = (torch.randn(Ct, generator=gen) * 0.1).contiguous()
+    init = None
+    if shape.init:
+        init = torch.randn((shape.batch, Ct, shape.width - 1), generator=gen).to(io).contiguous()
+    return {"xbc": xbc, "weight": w, "bias": bias, "conv_init": init}
+
+
+def selective_inputs(shape: SelectiveShape) -> dict:
+    """x, B, C ~ N(0,1) (io dtype); dt as for the scans (c12 recipe, per channel);
+    A[d,n] = -U[1,16] per state; D ~ N(0,1); init N(0,1) when asked for."""
+    gen = torch.Generator().manual_seed(shape.seed)
+    b, T, Dc, G, N = shape.batch, shape.seqlen, shape.channels, shape.ngroups, shape.dstate
+    io = _tdtype(shape.io_dtype)
+    x = torch.randn((b, T, Dc), generator=gen).to(io).contiguous()
+    dt = _dt_draw(gen, (b, T, Dc), Dc)
+    A = (-(torch.rand((Dc, N), generator=gen) * 15.0 + 1.0)).contiguous()
+    B = torch.randn((b, T, G, N), generator=gen).to(io).contiguous()
+    C = torch.randn((b, T, G, N), generator=gen).to(io).contiguous()
+    D = torch.randn(Dc, generator=gen)
+    init = torch.randn((b, Dc, N), generator=gen) if shape.init_state else None
+    return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D, "init_state": init}
+
+
 def decode_step_inputs(gen: torch.Generator, shape: DecodeShape) -> dict:
     """Per-step decode inputs x [b,H,P], dt [b,H], B, C [b,G,N] (io dtype)."""
     b, H, P, G, N = shape.batch, shape.nheads, shape.headdim, shape.ngroups, shape.dstate

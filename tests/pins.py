@@ -460,6 +460,106 @@ def pin_gradient_chunkwise(lib, cplx=False, seed=13):
     return err
 
 
+# ----------------------------------------------------------- the variants
+def pin_conv1d_library(lib, seed=20):
+    """The causal depthwise convolution equals numpy's full convolution of each
+    channel with its reversed kernel, cut to the first T outputs (a library
+    routine), plus the bias; SiLU equals torch's; the identity kernel returns
+    the input and the one-step shift kernel the input delayed by one token."""
+    import torch
+
+    rng = np.random.default_rng(seed)
+    err = 0.0
+    b, T, Cn, K = 2, 11, 5, 4
+    x = rng.standard_normal((b, T, Cn))
+    w = rng.standard_normal((Cn, K))
+    bias = rng.standard_normal(Cn)
+    ref = np.zeros_like(x)
+    for bi in range(b):
+        for c in range(Cn):
+            ref[bi, :, c] = np.convolve(x[bi, :, c], w[c, ::-1])[:T] + bias[c]
+    err = max(err, rel_err(oracle.causal_conv1d(x, w, bias, lib=lib), ref))
+    silu = torch.nn.functional.silu(torch.from_numpy(ref)).numpy()
+    err = max(err, rel_err(oracle.causal_conv1d(x, w, bias, silu=True, lib=lib), silu))
+    eye = np.zeros((Cn, K))
+    eye[:, K - 1] = 1.0
+    err = max(err, rel_err(oracle.causal_conv1d(x, eye, lib=lib), x))
+    shift = np.zeros((Cn, K))
+    shift[:, K - 2] = 1.0
+    delayed = np.concatenate([np.zeros((b, 1, Cn)), x[:, :-1]], axis=1)
+    err = max(err, rel_err(oracle.causal_conv1d(x, shift, lib=lib), delayed))
+    return err
+
+
+def pin_conv1d_continuation(lib, seed=21):
+    """A sequence convolved in two parts, the second given the last K-1 inputs of
+    the first as its initial window, equals the whole sequence convolved."""
+    rng = np.random.default_rng(seed)
+    b, T1, T2, Cn, K = 2, 7, 6, 3, 4
+    x = rng.standard_normal((b, T1 + T2, Cn))
+    w = rng.standard_normal((Cn, K))
+    whole = oracle.causal_conv1d(x, w, lib=lib)
+    init = np.ascontiguousarray(np.transpose(x[:, T1 - (K - 1):T1], (0, 2, 1)))
+    part = oracle.causal_conv1d(np.ascontiguousarray(x[:, T1:]), w, init=init, lib=lib)
+    return rel_err(part, whole[:, T1:])
+
+
+def _selective_problem(rng, b, T, Dc, G, N, init=True):
+    return dict(x=rng.standard_normal((b, T, Dc)), dt=rng.uniform(1e-3, 0.1, (b, T, Dc)),
+                A=-rng.uniform(1.0, 16.0, (Dc, N)), B=rng.standard_normal((b, T, G, N)),
+                C=rng.standard_normal((b, T, G, N)), D=rng.standard_normal(Dc),
+                init_state=rng.standard_normal((b, Dc, N)) if init else None)
+
+
+def pin_selective_scalar_A_is_ssd(lib, seed=22):
+    """With the same A for every state of a channel, the Mamba-1 scan is the
+    scalar-A scan with one head per channel and head dim 1 (the pinned SSD
+    oracle)."""
+    rng = np.random.default_rng(seed)
+    b, T, Dc, G, N = 2, 13, 6, 2, 5
+    p = _selective_problem(rng, b, T, Dc, G, N)
+    a = -rng.uniform(1.0, 16.0, Dc)
+    A = np.ascontiguousarray(np.repeat(a[:, None], N, axis=1))
+    y, fs = oracle.selective_scan(p["x"], p["dt"], A, p["B"], p["C"], p["D"], p["init_state"], lib=lib)
+    c = np.ascontiguousarray
+    y_ref, fs_ref = oracle.scan(c(p["x"][..., None]), p["dt"], a, p["B"], p["C"], p["D"],
+                                c(p["init_state"][:, :, None, :]), lib=lib)
+    return max(rel_err(y, y_ref[..., 0]), rel_err(fs, fs_ref[:, :, 0, :]))
+
+
+def pin_selective_brute_force(lib, seed=23):
+    """Short sequences against the explicit sum over source tokens, each state
+    with its own decay: y_t = sum_n C_t[n] (sum_{s<=t} exp(A[n] sum_{s<u<=t} dt_u)
+    dt_s B_s[n] x_s + exp(A[n] sum_{u<=t} dt_u) h0[n]) + D x_t; and with x = 0
+    the pure decay of h0."""
+    rng = np.random.default_rng(seed)
+    b, T, Dc, G, N = 1, 6, 4, 2, 3
+    p = _selective_problem(rng, b, T, Dc, G, N)
+    y, fs = oracle.selective_scan(p["x"], p["dt"], p["A"], p["B"], p["C"], p["D"], p["init_state"], lib=lib)
+    ref = np.zeros_like(y)
+    for d in range(Dc):
+        g = d // (Dc // G)
+        for t in range(T):
+            tot = 0.0
+            for n in range(N):
+                s_sum = 0.0
+                for s in range(t + 1):
+                    decay = np.exp(p["A"][d, n] * p["dt"][0, s + 1:t + 1, d].sum())
+                    s_sum += decay * p["dt"][0, s, d] * p["B"][0, s, g, n] * p["x"][0, s, d]
+                s_sum += np.exp(p["A"][d, n] * p["dt"][0, :t + 1, d].sum()) * p["init_state"][0, d, n]
+                tot += p["C"][0, t, g, n] * s_sum
+            ref[0, t, d] = tot + p["D"][d] * p["x"][0, t, d]
+    err = rel_err(y, ref)
+    z = dict(p, x=np.zeros_like(p["x"]))
+    _, fs0 = oracle.selective_scan(z["x"], z["dt"], z["A"], z["B"], z["C"], z["D"], z["init_state"], lib=lib)
+    closed = np.exp(p["A"][None] * p["dt"].sum(axis=1)[:, :, None]) * p["init_state"]
+    return max(err, rel_err(fs0, closed))
+
+
+VARIANT_PINS = [pin_conv1d_library, pin_conv1d_continuation, pin_selective_scalar_A_is_ssd,
+                pin_selective_brute_force]
+
+
 REAL_PINS = [pin_brute_force, pin_chunkwise, pin_zero_input, pin_prefix_sum, pin_linearity,
              pin_continuation, pin_decode_equals_scan, pin_contraction,
              pin_gradient_finite_difference, pin_gradient_empty_and_dfinal, pin_gradient_chunkwise]
@@ -472,7 +572,7 @@ def all_pins():
     for f in REAL_PINS:
         out.append((f.__name__ + "[real]", lambda lib, f=f: f(lib, cplx=False)))
         out.append((f.__name__ + "[complex]", lambda lib, f=f: f(lib, cplx=True)))
-    for f in COMPLEX_ONLY_PINS:
+    for f in COMPLEX_ONLY_PINS + VARIANT_PINS:
         out.append((f.__name__, f))
     return out
 

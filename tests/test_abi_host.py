@@ -166,3 +166,25 @@ def test_header_compiles_as_c_and_cpp(tmp_path, lang, std):
     cc = "gcc" if lang == "c" else "g++"
     subprocess.check_call([cc, f"-std={std}", "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
                            "-x", lang, "-I", os.path.join(ROOT, "include"), str(src)])
+
+
+def test_final_state_and_fold_validation(lib):
+    def fs_call(**over):
+        a = dict(x=FAKE, dt=FAKE, A=FAKE, B=FAKE, init=None, final=FAKE, lam=None, io=ssd.SSD_BF16, b=1, T=256,
+                 H=2, P=64, G=1, N=128, Q=256, ws=FAKE, wsb=1 << 30, stream=None)
+        a.update(over)
+        return lib.ssd_scan_final_state(a["x"], a["dt"], a["A"], a["B"], a["init"], a["final"], a["lam"],
+                                        a["io"], a["b"], a["T"], a["H"], a["P"], a["G"], a["N"], a["Q"],
+                                        a["ws"], a["wsb"], a["stream"])
+
+    assert fs_call(final=None) == ssd.SSD_ERR_INVALID_ARG and "final_state" in ssd.ssd_last_error()
+    assert fs_call(B=None) == ssd.SSD_ERR_INVALID_ARG and "non-null" in ssd.ssd_last_error()
+    assert fs_call(lam=ctypes.c_void_p((1 << 20) + 4)) == ssd.SSD_ERR_INVALID_ARG
+    assert fs_call(G=3) == ssd.SSD_ERR_INVALID_ARG
+    assert fs_call(io=5) == ssd.SSD_ERR_INVALID_ARG
+    # y NULL stays an error for the full scan (only the final-state entry point omits it)
+    assert scan_call(lib, y=None, final=FAKE) == ssd.SSD_ERR_INVALID_ARG
+    fold = lambda n, lam, out: lib.ssd_fold_states(FAKE, lam, n, out, 1, 2, 64, 128, None)
+    assert fold(0, FAKE, FAKE) == ssd.SSD_ERR_INVALID_ARG
+    assert fold(2, None, FAKE) == ssd.SSD_ERR_INVALID_ARG and "log_decay" in ssd.ssd_last_error()
+    assert fold(2, FAKE, None) == ssd.SSD_ERR_INVALID_ARG

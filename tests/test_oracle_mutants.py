@@ -48,6 +48,18 @@ MUTANTS = {
                                            "Gs[IDX2(p, n, dstate)] += Ct[n] * dyt[p];"),
     "bwd_complex_ddt_imag_part": ("creal(ga * conj(Ac[h] * a))", "cimag(ga * conj(Ac[h] * a))"),
     "bwd_complex_input_grad_imag_part": ("rp += creal(conj(Bt[n]) * Gs", "rp += cimag(conj(Bt[n]) * Gs"),
+    # the variants
+    "conv_kernel_reversed": ("v += w[c * width + k] * u;", "v += w[c * width + (width - 1 - k)] * u;"),
+    "conv_not_causal": ("const long s = t - (width - 1) + k;", "const long s = t + k;"),
+    "conv_init_reversed": ("init[(b * channels + c) * (width - 1) + (width - 1) + s]",
+                           "init[(b * channels + c) * (width - 1) - 1 - s]"),
+    "conv_silu_sign": ("if (silu) v = v / (1.0 + exp(-v));", "if (silu) v = v / (1.0 + exp(v));"),
+    "selective_A_first_state": ("h[n] = exp(step * A[d * dstate + n]) * h[n] + step * B[bc] * u;",
+                                "h[n] = exp(step * A[d * dstate]) * h[n] + step * B[bc] * u;"),
+    "selective_readout_before_update": ("                    acc += C[bc] * h[n];",
+                                        "                    acc += C[bc] * (h[n] - step * B[bc] * u);"),
+    "selective_group_modulo": ("const long g = d / (channels / ngroups);\n            for (long n = 0; n < dstate; ++n)\n                h[n] = init_state",
+                               "const long g = d % ngroups;\n            for (long n = 0; n < dstate; ++n)\n                h[n] = init_state"),
 }
 
 
