@@ -32,6 +32,7 @@ template <typename T> struct CplxView {
     int bc_gs, bc_es;
     const float *dt_bias;        // dt + dt_bias[h] before softplus (nullable)
     int softplus;                // dt <- softplus(dt + dt_bias)
+    int vec;                     // 16-byte loads of 4 states / 8 x values are aligned (set on the host)
 };
 
 template <typename T>
@@ -46,12 +47,83 @@ template <typename T> __device__ __forceinline__ cf view_c(const CplxView<T> &v,
     const size_t o = bt * v.bc_ts + (size_t)g * v.bc_gs + (size_t)n * v.bc_es;
     return {to_f32<T>(v.cre[o]), to_f32<T>(v.cim[o])};
 }
+// Four consecutive states n0 .. n0+3 (n0 a multiple of 4) of B or C at one
+// token: two 16-byte loads (interleaved float32) or one per part (split real
+// and imaginary slices) when the view allows, else element by element.
+template <typename T>
+__device__ __forceinline__ void view_cplx4(const CplxView<T> &v, const T *re, const T *im, size_t bt, int g, int n0,
+                                           cf (&out)[4]) {
+    const size_t o = bt * v.bc_ts + (size_t)g * v.bc_gs + (size_t)n0 * v.bc_es;
+    if (v.vec) {
+        if constexpr (sizeof(T) == 4) {
+            if (v.bc_es == 2) {  // (re, im) pairs
+                const float4 a = *reinterpret_cast<const float4 *>(re + o);
+                const float4 b = *reinterpret_cast<const float4 *>(re + o + 4);
+                out[0] = {a.x, a.y}, out[1] = {a.z, a.w}, out[2] = {b.x, b.y}, out[3] = {b.z, b.w};
+            } else {
+                const float4 a = *reinterpret_cast<const float4 *>(re + o);
+                const float4 b = *reinterpret_cast<const float4 *>(im + o);
+                out[0] = {a.x, b.x}, out[1] = {a.y, b.y}, out[2] = {a.z, b.z}, out[3] = {a.w, b.w};
+            }
+        } else {  // bf16, split slices: 8 bytes per part
+            const uint2 a = *reinterpret_cast<const uint2 *>(re + o);
+            const uint2 b = *reinterpret_cast<const uint2 *>(im + o);
+            out[0] = {__uint_as_float(a.x << 16), __uint_as_float(b.x << 16)};
+            out[1] = {__uint_as_float(a.x & 0xffff0000u), __uint_as_float(b.x & 0xffff0000u)};
+            out[2] = {__uint_as_float(a.y << 16), __uint_as_float(b.y << 16)};
+            out[3] = {__uint_as_float(a.y & 0xffff0000u), __uint_as_float(b.y & 0xffff0000u)};
+        }
+        return;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+        out[q] = {to_f32<T>(re[o + (size_t)q * v.bc_es]), to_f32<T>(im[o + (size_t)q * v.bc_es])};
+}
+// Eight consecutive x values p0 .. p0+7 (p0 a multiple of 8) at one token and head.
+template <typename T>
+__device__ __forceinline__ void view_x8(const CplxView<T> &v, size_t bt, int h, int P, int p0, float (&out)[8]) {
+    const T *px = v.x + bt * v.x_ts + (size_t)h * P + p0;
+    if (v.vec) {
+        if constexpr (sizeof(T) == 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(px), b = *reinterpret_cast<const float4 *>(px + 4);
+            out[0] = a.x, out[1] = a.y, out[2] = a.z, out[3] = a.w, out[4] = b.x, out[5] = b.y, out[6] = b.z,
+            out[7] = b.w;
+        } else {
+            const uint4 a = *reinterpret_cast<const uint4 *>(px);
+            const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                out[2 * e] = __uint_as_float(w[e] << 16);
+                out[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+            }
+        }
+        return;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) out[e] = to_f32<T>(px[e]);
+}
+
 // softplus(u) = log(1 + e^u), computed as u + log1p(e^-u) for large u
 __device__ __forceinline__ float softplus_f(float u) { return u > 15.f ? u + log1pf(__expf(-u)) : log1pf(__expf(u)); }
 template <typename T> __device__ __forceinline__ float view_dt(const CplxView<T> &v, size_t bt, int h) {
     float d = to_f32<T>(v.dt[bt * v.dt_ts + h]);
     if (v.softplus) d = softplus_f(d + (v.dt_bias ? v.dt_bias[h] : 0.f));
     return d;
+}
+
+// Whether the vector loads above are aligned for every token, group and head:
+// base pointers aligned to the load and every stride a multiple of it.  With
+// interleaved pairs (bc_es == 2) the imaginary pointer is the real one plus a
+// float and is never dereferenced by the vector path.
+template <typename T> inline bool view_vec_ok(const CplxView<T> &v, int headdim, int dstate) {
+    auto al = [](const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; };
+    const long long xv = 16 / (long long)sizeof(T);  // x elements per 16-byte load
+    const uintptr_t ba = 4 * sizeof(T);               // bytes per B/C load of one part (4 elements)
+    const bool pairs = sizeof(T) == 4 && v.bc_es == 2;
+    const bool bc_ok = pairs ? (al(v.bre, 16) && al(v.cre, 16))
+                             : (v.bc_es == 1 && al(v.bre, ba) && al(v.bim, ba) && al(v.cre, ba) && al(v.cim, ba));
+    return bc_ok && al(v.x, 16) && v.x_ts % xv == 0 && headdim % 8 == 0 && v.bc_ts % 4 == 0 &&
+           v.bc_gs % 4 == 0 && dstate % 4 == 0;
 }
 
 // The separate tensors of ssd_scan_fwd_complex: x, dt float32; B, C complex64
@@ -71,6 +143,7 @@ inline CplxView<float> plain_view(const ScanArgs &a) {
     v.bc_es = 2;
     v.dt_bias = nullptr;
     v.softplus = 0;
+    v.vec = view_vec_ok(v, a.headdim, a.dstate);
     return v;
 }
 
@@ -91,6 +164,7 @@ inline CplxView<T> packed_view(const void *proj, const float *dt_bias, int nhead
     v.bc_es = 1;
     v.dt_bias = dt_bias;
     v.softplus = 1;
+    v.vec = view_vec_ok(v, headdim, dstate);
     return v;
 }
 

@@ -96,8 +96,12 @@ __device__ void stage_x(uint8_t *sm, int off_hi, int off_lo, const ScanArgs &a, 
     for (int u = threadIdx.x; u < QT * 8; u += NTH) {
         const int s = u >> 3, ch = u & 7;
         float val[8];
+        if (s < valid) {
+            view_x8(v, bt0 + s, h, a.headdim, 8 * ch, val);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) val[e] = s < valid ? view_x(v, bt0 + s, h, a.headdim, 8 * ch + e) : 0.f;
+            for (int e = 0; e < 8; ++e) val[e] = 0.f;
+        }
         put8(sm, off_hi, off_lo, sw_off(s, ch, QT * 128), val);
     }
 }
@@ -142,13 +146,12 @@ template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanAr
     for (int u = tid; u < QT * 16; u += NTH) {
         const int s = u >> 4, ch = u & 15;
         float val[8];
+        cf bq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        if (s < valid) view_cplx4(v, v.bre, v.bim, bt0 + s, g, 4 * ch, bq);
+        const float2 ws = wf[s];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            cf z = {0.f, 0.f};
-            if (s < valid) {
-                const float2 ws = wf[s];
-                z = cmul(view_b(v, bt0 + s, g, 4 * ch + q), cf{ws.x, ws.y});
-            }
+            const cf z = cmul(bq[q], cf{ws.x, ws.y});
             val[2 * q] = z.re;
             val[2 * q + 1] = z.im;
         }
@@ -228,13 +231,14 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
         const int r = u >> 4, ch = u & 15;
         float vc[8], vb[8];
         const float2 fc = fC[r], fb = fB[r];
+        cf cq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}}, bq[4] = {cq[0], cq[1], cq[2], cq[3]};
+        if (r < valid) {
+            view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq);
+            view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq);
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            cf zc = {0.f, 0.f}, zb = {0.f, 0.f};
-            if (r < valid) {
-                zc = cmul(view_c(v, bt0 + r, g, 4 * ch + q), cf{fc.x, fc.y});
-                zb = cmul(view_b(v, bt0 + r, g, 4 * ch + q), cf{fb.x, fb.y});
-            }
+            const cf zc = cmul(cq[q], cf{fc.x, fc.y}), zb = cmul(bq[q], cf{fb.x, fb.y});
             vc[2 * q] = zc.re;
             vc[2 * q + 1] = -zc.im;
             vb[2 * q] = zb.re;

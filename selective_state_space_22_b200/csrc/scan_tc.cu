@@ -752,9 +752,14 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     // Whole sequences per CTA when there are enough of them to fill ~3/4 of the
     // SMs; otherwise runs, as many as the SMs allow.
     int runs = 1;
-    if (4 * p.bH < 3 * di.sms) runs = std::max(1, std::min({di.sms / p.bH, p.nchunks, MAX_RUNS}));
+    if (!a.y) {
+        // State-only form (no C, no y): every tile of every sequence state-only.
+        p.run_start[0] = p.run_start[1] = p.nchunks;
+    } else {
+        if (4 * p.bH < 3 * di.sms) runs = std::max(1, std::min({di.sms / p.bH, p.nchunks, MAX_RUNS}));
+        split_runs(p.nchunks, runs, p.run_start);
+    }
     p.runs = runs;
-    split_runs(p.nchunks, runs, p.run_start);
     p.dev_error = a.dev_error;
     const unsigned long long wns = g_wait_ns.load();
     p.wait_ns = wns ? wns : WAIT_NS;
