@@ -21,6 +21,11 @@ namespace ssd {
 template <typename T> __device__ __forceinline__ float to_f32(T v);
 template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+// The scan's inputs are read-only while it runs (outputs never alias them), so
+// they are read through the read-only global path: besides the cache, that
+// tells the compiler a load cannot alias the shared-memory stores of the
+// staging loops, so loads of later rows can be issued ahead of them.
+template <typename T> __device__ __forceinline__ float ldg_f32(const T *p) { return to_f32<T>(__ldg(p)); }
 
 // Element (b, t, ...) of a view lives at base + (b * seqlen + t) * token_stride + ...
 template <typename T> struct CplxView {
@@ -37,15 +42,15 @@ template <typename T> struct CplxView {
 
 template <typename T>
 __device__ __forceinline__ float view_x(const CplxView<T> &v, size_t bt, int h, int P, int p) {
-    return to_f32<T>(v.x[bt * v.x_ts + (size_t)h * P + p]);
+    return ldg_f32<T>(v.x + bt * v.x_ts + (size_t)h * P + p);
 }
 template <typename T> __device__ __forceinline__ cf view_b(const CplxView<T> &v, size_t bt, int g, int n) {
     const size_t o = bt * v.bc_ts + (size_t)g * v.bc_gs + (size_t)n * v.bc_es;
-    return {to_f32<T>(v.bre[o]), to_f32<T>(v.bim[o])};
+    return {ldg_f32<T>(v.bre + o), ldg_f32<T>(v.bim + o)};
 }
 template <typename T> __device__ __forceinline__ cf view_c(const CplxView<T> &v, size_t bt, int g, int n) {
     const size_t o = bt * v.bc_ts + (size_t)g * v.bc_gs + (size_t)n * v.bc_es;
-    return {to_f32<T>(v.cre[o]), to_f32<T>(v.cim[o])};
+    return {ldg_f32<T>(v.cre + o), ldg_f32<T>(v.cim + o)};
 }
 // Four consecutive states n0 .. n0+3 (n0 a multiple of 4) of B or C at one
 // token: two 16-byte loads (interleaved float32) or one per part (split real
@@ -57,17 +62,17 @@ __device__ __forceinline__ void view_cplx4(const CplxView<T> &v, const T *re, co
     if (v.vec) {
         if constexpr (sizeof(T) == 4) {
             if (v.bc_es == 2) {  // (re, im) pairs
-                const float4 a = *reinterpret_cast<const float4 *>(re + o);
-                const float4 b = *reinterpret_cast<const float4 *>(re + o + 4);
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(re + o));
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(re + o + 4));
                 out[0] = {a.x, a.y}, out[1] = {a.z, a.w}, out[2] = {b.x, b.y}, out[3] = {b.z, b.w};
             } else {
-                const float4 a = *reinterpret_cast<const float4 *>(re + o);
-                const float4 b = *reinterpret_cast<const float4 *>(im + o);
+                const float4 a = __ldg(reinterpret_cast<const float4 *>(re + o));
+                const float4 b = __ldg(reinterpret_cast<const float4 *>(im + o));
                 out[0] = {a.x, b.x}, out[1] = {a.y, b.y}, out[2] = {a.z, b.z}, out[3] = {a.w, b.w};
             }
         } else {  // bf16, split slices: 8 bytes per part
-            const uint2 a = *reinterpret_cast<const uint2 *>(re + o);
-            const uint2 b = *reinterpret_cast<const uint2 *>(im + o);
+            const uint2 a = __ldg(reinterpret_cast<const uint2 *>(re + o));
+            const uint2 b = __ldg(reinterpret_cast<const uint2 *>(im + o));
             out[0] = {__uint_as_float(a.x << 16), __uint_as_float(b.x << 16)};
             out[1] = {__uint_as_float(a.x & 0xffff0000u), __uint_as_float(b.x & 0xffff0000u)};
             out[2] = {__uint_as_float(a.y << 16), __uint_as_float(b.y << 16)};
@@ -77,7 +82,7 @@ __device__ __forceinline__ void view_cplx4(const CplxView<T> &v, const T *re, co
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q)
-        out[q] = {to_f32<T>(re[o + (size_t)q * v.bc_es]), to_f32<T>(im[o + (size_t)q * v.bc_es])};
+        out[q] = {ldg_f32<T>(re + o + (size_t)q * v.bc_es), ldg_f32<T>(im + o + (size_t)q * v.bc_es)};
 }
 // Eight consecutive x values p0 .. p0+7 (p0 a multiple of 8) at one token and head.
 template <typename T>
@@ -85,11 +90,11 @@ __device__ __forceinline__ void view_x8(const CplxView<T> &v, size_t bt, int h, 
     const T *px = v.x + bt * v.x_ts + (size_t)h * P + p0;
     if (v.vec) {
         if constexpr (sizeof(T) == 4) {
-            const float4 a = *reinterpret_cast<const float4 *>(px), b = *reinterpret_cast<const float4 *>(px + 4);
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(px)), b = __ldg(reinterpret_cast<const float4 *>(px + 4));
             out[0] = a.x, out[1] = a.y, out[2] = a.z, out[3] = a.w, out[4] = b.x, out[5] = b.y, out[6] = b.z,
             out[7] = b.w;
         } else {
-            const uint4 a = *reinterpret_cast<const uint4 *>(px);
+            const uint4 a = __ldg(reinterpret_cast<const uint4 *>(px));
             const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -100,14 +105,14 @@ __device__ __forceinline__ void view_x8(const CplxView<T> &v, size_t bt, int h, 
         return;
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) out[e] = to_f32<T>(px[e]);
+    for (int e = 0; e < 8; ++e) out[e] = ldg_f32<T>(px + e);
 }
 
 // softplus(u) = log(1 + e^u), computed as u + log1p(e^-u) for large u
 __device__ __forceinline__ float softplus_f(float u) { return u > 15.f ? u + log1pf(__expf(-u)) : log1pf(__expf(u)); }
 template <typename T> __device__ __forceinline__ float view_dt(const CplxView<T> &v, size_t bt, int h) {
-    float d = to_f32<T>(v.dt[bt * v.dt_ts + h]);
-    if (v.softplus) d = softplus_f(d + (v.dt_bias ? v.dt_bias[h] : 0.f));
+    float d = ldg_f32<T>(v.dt + bt * v.dt_ts + h);
+    if (v.softplus) d = softplus_f(d + (v.dt_bias ? __ldg(v.dt_bias + h) : 0.f));
     return d;
 }
 

@@ -93,8 +93,9 @@ __device__ bool wait_bounded(uint64_t *bar, uint32_t parity, int *err) {
 template <typename T>
 __device__ void stage_x(uint8_t *sm, int off_hi, int off_lo, const ScanArgs &a, const CplxView<T> &v, size_t bt0, int h,
                         int valid) {
-    for (int u = threadIdx.x; u < QT * 8; u += NTH) {
-        const int s = u >> 3, ch = u & 7;
+#pragma unroll 4
+    for (int it = 0; it < QT * 8 / NTH; ++it) {
+        const int u = threadIdx.x + it * NTH, s = u >> 3, ch = u & 7;
         float val[8];
         if (s < valid) {
             view_x8(v, bt0 + s, h, a.headdim, 8 * ch, val);
@@ -143,8 +144,9 @@ template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanAr
     }
     __syncthreads();
     // B''_s = w_s B_s as interleaved (re, im), rows s
-    for (int u = tid; u < QT * 16; u += NTH) {
-        const int s = u >> 4, ch = u & 15;
+#pragma unroll 4
+    for (int it = 0; it < QT * 16 / NTH; ++it) {
+        const int u = tid + it * NTH, s = u >> 4, ch = u & 15;
         float val[8];
         cf bq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
         if (s < valid) view_cplx4(v, v.bre, v.bim, bt0 + s, g, 4 * ch, bq);
@@ -227,8 +229,9 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
     }
     __syncthreads();
     // C' as (re, -im) and B' as (re, im), rows = tokens, 4 complex states per chunk of 8
-    for (int u = tid; u < QT * 16; u += NTH) {
-        const int r = u >> 4, ch = u & 15;
+#pragma unroll 4
+    for (int it = 0; it < QT * 16 / NTH; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
         float vc[8], vb[8];
         const float2 fc = fC[r], fb = fB[r];
         cf cq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}}, bq[4] = {cq[0], cq[1], cq[2], cq[3]};
@@ -252,11 +255,12 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
     {  // h' = exp(rho) h_in as (re, im), rows p
         const float er = (float)exp(rho);
         const float *hin = reinterpret_cast<const float *>(w.S + bhc * (size_t)P * N);
-        for (int u = tid; u < 64 * 16; u += NTH) {
-            const int p = u >> 4, ch = u & 15;
+#pragma unroll 4
+        for (int it = 0; it < 64 * 16 / NTH; ++it) {  // h_in was written by earlier launches: read-only here
+            const int u = tid + it * NTH, p = u >> 4, ch = u & 15;
             float val[8];
-            const float4 h0 = *reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2);
-            const float4 h1 = *reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2 + 4);
+            const float4 h0 = __ldg(reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2));
+            const float4 h1 = __ldg(reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2 + 4));
             val[0] = er * h0.x, val[1] = er * h0.y, val[2] = er * h0.z, val[3] = er * h0.w;
             val[4] = er * h1.x, val[5] = er * h1.y, val[6] = er * h1.z, val[7] = er * h1.w;
             put8(sm, S_HH, S_HL, sw_off(p, ch, 64 * 128), val);

@@ -9,26 +9,32 @@
 //    into the scan's separate x, B and C tensors.  A thread slides a K-token
 //    window along a run of tokens, so each input is read once (plus a K-1 token
 //    halo per run, an L2 hit) and each output written once: HBM-bound.  Where
-//    the channel ranges and pointers allow (K <= 4), a thread owns 16 bytes of
-//    channels (8 bf16 or 4 float32) and moves them with one load and one store
-//    per token; otherwise one channel per thread.
+//    the channel ranges allow (K <= 4), a block copies a 256-channel x 32-token
+//    tile into shared memory with asynchronous copies and each thread convolves
+//    a channel pair from there; otherwise one channel per thread.
 //
 // 2. The Mamba-1 selective scan, one decay rate per state component:
 //      h_t[n] = exp(dt_t[d] A[d][n]) h_{t-1}[n] + dt_t[d] B_t[n] x_t[d],
 //      y_t[d] = sum_n C_t[n] h_t[n] + D[d] x_t[d].
 //    With a decay per state the segsum decay is no longer one scalar per token
 //    pair, so there is no chunked matrix form; the scan is sequential in time
-//    and parallel over (batch, channel).  Four lanes share a channel, each with
-//    N/4 of its states in registers, and add their parts of the readout with
-//    two shuffles; a warp covers 8 consecutive channels, and B and C of a step
-//    are one vector load per lane (the same for all channels of a group).
-//    Bound by the N exponentials per channel and step (SFU), then by HBM.
+//    and parallel over (batch, channel).  Where 64-channel blocks lie inside one
+//    B/C group, two lanes share a channel (N/2 states each) and a block stages
+//    x, dt, B and C of 32-token runs in shared memory; otherwise four lanes
+//    share a channel and read global memory directly.  Either way the lanes of
+//    a channel add their parts of the readout with shuffles.  Bound by the N
+//    exponentials per channel and step (SFU), then by HBM.
 #include "ssd_internal.cuh"
 
 namespace ssd {
 namespace {
 
 template <typename T> __device__ __forceinline__ float ldf(const T *p) { return ld_f32<T>(p); }
+
+// SiLU v / (1 + e^-v).  The exponent is capped at 80 so that the fast divide
+// (exact to 2 ulp for divisors below 2^126) always sees a finite divisor; past
+// the cap the quotient is below 1e-33 |v|.
+__device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.f + __expf(fminf(-v, 80.f))); }
 
 constexpr int CONV_TT = 32;   // tokens per thread run
 constexpr int CONV_MAXK = 8;
@@ -82,87 +88,93 @@ __global__ void __launch_bounds__(128) conv1d_xbc_kernel(const T *__restrict__ i
 #pragma unroll
         for (int k = 0; k < CONV_MAXK; ++k)
             if (k < K) v = fmaf(wk[k], win[k], v);
-        if (silu) v = v / (1.f + __expf(-v));
+        if (silu) v = silu_f(v);
         st_f32(dst + (rowb + t) * cn + cc, v);
     }
     if (cfinal && t1 == seqlen)  // the last K-1 inputs, for a continued sequence
         for (int j = 0; j < K - 1; ++j) st_f32(cfinal + ((size_t)b * ctot + c) * (K - 1) + j, win[j + 1]);
 }
 
-// 16 bytes of T <-> floats.
-template <typename T> struct Vec16;
-template <> struct Vec16<float> {
-    static constexpr int V = 4;
-    static __device__ __forceinline__ void load(const float *p, float (&v)[4]) {
-        const float4 q = *reinterpret_cast<const float4 *>(p);
-        v[0] = q.x, v[1] = q.y, v[2] = q.z, v[3] = q.w;
-    }
-    static __device__ __forceinline__ void store(float *p, const float (&v)[4]) {
-        *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
-    }
+// Two consecutive channels of T <-> floats.
+template <typename T> struct Pair;
+template <> struct Pair<float> {
+    static __device__ __forceinline__ float2 load(const float *p) { return *reinterpret_cast<const float2 *>(p); }
+    static __device__ __forceinline__ void store(float *p, float2 v) { *reinterpret_cast<float2 *>(p) = v; }
 };
-template <> struct Vec16<__nv_bfloat16> {
-    static constexpr int V = 8;
-    static __device__ __forceinline__ void load(const __nv_bfloat16 *p, float (&v)[8]) {
-        const uint4 q = *reinterpret_cast<const uint4 *>(p);
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            v[2 * e] = __uint_as_float(w[e] << 16);
-            v[2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-        }
+template <> struct Pair<__nv_bfloat16> {
+    static __device__ __forceinline__ float2 load(const __nv_bfloat16 *p) {
+        const uint32_t r = *reinterpret_cast<const uint32_t *>(p);
+        return make_float2(__uint_as_float(r << 16), __uint_as_float(r & 0xffff0000u));
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16 *p, const float (&v)[8]) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-            w[e] = *reinterpret_cast<const uint32_t *>(&h);
-        }
-        *reinterpret_cast<uint4 *>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    static __device__ __forceinline__ void store(__nv_bfloat16 *p, float2 v) {
+        *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
     }
 };
 
-constexpr int CONV_TV = 16;  // tokens per thread run (vector kernel)
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
+                 "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-// The convolution with one thread per 16 bytes of channels c0 .. c0+V-1 (all in
-// one of the x, B, C ranges), K <= 4: the kernel is right-aligned into four taps,
-// out[t] = bias + sum_{j<4} w4[j] in[t - 3 + j] with w4[j] = w[j - (4 - K)] (zero
-// for j < 4 - K), so the window always holds the three tokens before t.
+constexpr int CONV_CH = 256;  // channels per block of the tiled kernel (128 threads x 2)
+constexpr int CONV_TV = 32;   // tokens per block of the tiled kernel
+
+// The convolution for a tile of 256 channels x 32 tokens, K <= 4.  The tile's
+// input rows (and the three before it) are copied into shared memory with
+// asynchronous 16-byte copies, which hold no registers while in flight, so a
+// block has its whole tile in flight at once; then each thread convolves its
+// channel pair (c0, c0 + 1), both in one of the x, B, C ranges, from shared
+// memory.  The kernel is right-aligned into four taps,
+// out[t] = bias + sum_{j<4} w4[j] in[t - 3 + j], w4[j] = w[j - (4 - K)] (zero for
+// j < 4 - K), so the window always holds the three tokens before t.
 template <typename T>
-__global__ void __launch_bounds__(128) conv1d_xbc_vec_kernel(const T *__restrict__ in, const float *__restrict__ w,
-                                                            const float *__restrict__ bias,
-                                                            const T *__restrict__ cinit, T *__restrict__ xo,
-                                                            T *__restrict__ bo, T *__restrict__ co,
-                                                            T *__restrict__ cfinal, int seqlen, int cx, int cb, int K,
-                                                            int silu) {
-    using IO = Vec16<T>;
-    constexpr int V = IO::V;
+__global__ void __launch_bounds__(128) conv1d_xbc_tile_kernel(const T *__restrict__ in, const float *__restrict__ w,
+                                                             const float *__restrict__ bias,
+                                                             const T *__restrict__ cinit, T *__restrict__ xo,
+                                                             T *__restrict__ bo, T *__restrict__ co,
+                                                             T *__restrict__ cfinal, int seqlen, int cx, int cb, int K,
+                                                             int silu) {
+    using IO = Pair<T>;
+    constexpr int E16 = 16 / (int)sizeof(T);  // elements per 16-byte copy
+    __shared__ __align__(16) T tile[(CONV_TV + 3) * CONV_CH];
     const int ctot = cx + 2 * cb;
-    const int c0 = (blockIdx.x * 128 + threadIdx.x) * V;
-    const int t0 = blockIdx.y * CONV_TV, b = blockIdx.z;
-    if (c0 >= ctot || t0 >= seqlen) return;
-    float wk[4][V], bc[V], win[3][V];
-#pragma unroll
-    for (int e = 0; e < V; ++e) {
+    const int cbase = blockIdx.x * CONV_CH, t0 = blockIdx.y * CONV_TV, b = blockIdx.z;
+    const int nch = min(CONV_CH, ctot - cbase), n = min(CONV_TV, seqlen - t0);
+    const size_t rowb = (size_t)b * seqlen;
+    // rows r = 0 .. n + 2 hold tokens t0 - 3 + r; rows before the sequence are
+    // filled per thread below
+    const int cpr = nch / E16, r0 = t0 >= 3 ? 0 : 3 - t0;
+    for (int u = threadIdx.x; u < (n + 3 - r0) * cpr; u += 128) {
+        const int r = r0 + u / cpr, k = u % cpr;
+        cp_async16(tile + r * CONV_CH + k * E16, in + (rowb + t0 - 3 + r) * ctot + cbase + k * E16);
+    }
+    const int c0 = cbase + 2 * threadIdx.x;
+    float2 wk[4], bc = make_float2(0.f, 0.f);
+    if (c0 < ctot) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int k = j - (4 - K);
-            wk[j][e] = k >= 0 ? w[(size_t)(c0 + e) * K + k] : 0.f;
+            wk[j] = k >= 0 ? make_float2(w[(size_t)c0 * K + k], w[(size_t)(c0 + 1) * K + k]) : make_float2(0.f, 0.f);
         }
-        bc[e] = bias ? bias[c0 + e] : 0.f;
+        if (bias) bc = make_float2(bias[c0], bias[c0 + 1]);
     }
-    const size_t rowb = (size_t)b * seqlen;
+    cp_async_wait_all();
+    __syncthreads();
+    if (c0 >= ctot) return;
+    const T *col = tile + 2 * threadIdx.x;
+    float2 win[3];
 #pragma unroll
     for (int j = 0; j < 3; ++j) {  // win[j] = in[t0 - 3 + j]: the sequence, conv_init or zero
         const int s = t0 - 3 + j;
         if (s >= 0) {
-            IO::load(in + (rowb + s) * ctot + c0, win[j]);
+            win[j] = IO::load(col + j * CONV_CH);
+        } else if (cinit && K - 1 + s >= 0) {
+            const T *ci = cinit + ((size_t)b * ctot + c0) * (K - 1) + (K - 1) + s;
+            win[j] = make_float2(ldf(ci), ldf(ci + (K - 1)));
         } else {
-#pragma unroll
-            for (int e = 0; e < V; ++e)
-                win[j][e] = (cinit && K - 1 + s >= 0) ? ldf(cinit + ((size_t)b * ctot + c0 + e) * (K - 1) + (K - 1) + s)
-                                                      : 0.f;
+            win[j] = make_float2(0.f, 0.f);
         }
     }
     T *dst;
@@ -174,36 +186,24 @@ __global__ void __launch_bounds__(128) conv1d_xbc_vec_kernel(const T *__restrict
     } else {
         dst = co, cc = c0 - cx - cb, cn = cb;
     }
-    const int t1 = min(t0 + CONV_TV, seqlen);
-#pragma unroll
-    for (int q = 0; q < CONV_TV; q += 4) {  // four tokens' loads in flight at a time
-        float cur[4][V];
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (t0 + q + i < t1) IO::load(in + (rowb + t0 + q + i) * ctot + c0, cur[i]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int t = t0 + q + i;
-            if (t < t1) {
-                float out[V];
-#pragma unroll
-                for (int e = 0; e < V; ++e) {
-                    float v = fmaf(wk[0][e], win[0][e], bc[e]);
-                    v = fmaf(wk[1][e], win[1][e], v);
-                    v = fmaf(wk[2][e], win[2][e], v);
-                    v = fmaf(wk[3][e], cur[i][e], v);
-                    out[e] = silu ? v / (1.f + __expf(-v)) : v;
-                    win[0][e] = win[1][e], win[1][e] = win[2][e], win[2][e] = cur[i][e];
-                }
-                IO::store(dst + (rowb + t) * cn + cc, out);
-            }
-        }
+    T *pd = dst + (rowb + t0) * cn + cc;
+#pragma unroll 4
+    for (int i = 0; i < n; ++i) {
+        const float2 cur = IO::load(col + (i + 3) * CONV_CH);
+        float2 v;
+        v.x = fmaf(wk[3].x, cur.x, fmaf(wk[2].x, win[2].x, fmaf(wk[1].x, win[1].x, fmaf(wk[0].x, win[0].x, bc.x))));
+        v.y = fmaf(wk[3].y, cur.y, fmaf(wk[2].y, win[2].y, fmaf(wk[1].y, win[1].y, fmaf(wk[0].y, win[0].y, bc.y))));
+        if (silu) v = make_float2(silu_f(v.x), silu_f(v.y));
+        IO::store(pd, v);
+        pd += cn;
+        win[0] = win[1], win[1] = win[2], win[2] = cur;
     }
-    if (cfinal && t1 == seqlen)  // the last K-1 inputs, for a continued sequence
-        for (int j = 0; j < K - 1; ++j)
-#pragma unroll
-            for (int e = 0; e < V; ++e)
-                st_f32(cfinal + ((size_t)b * ctot + c0 + e) * (K - 1) + j, win[3 - (K - 1) + j][e]);
+    if (cfinal && t0 + n == seqlen)  // the last K-1 inputs, for a continued sequence
+        for (int j = 0; j < K - 1; ++j) {
+            const float2 v = win[3 - (K - 1) + j];
+            st_f32(cfinal + ((size_t)b * ctot + c0) * (K - 1) + j, v.x);
+            st_f32(cfinal + ((size_t)b * ctot + c0 + 1) * (K - 1) + j, v.y);
+        }
 }
 
 // Four lanes per channel: lane 4i + q of a warp holds states q*N/4 .. of channel
@@ -313,12 +313,99 @@ __global__ void __launch_bounds__(128) selective_scan_q4_kernel(const T *__restr
         for (int n = 0; n < NQ; ++n) hT[((size_t)b * channels + d) * N + n0 + n] = h[n];
 }
 
+constexpr int SEL_TT = 32;  // tokens per staged run
+constexpr int SEL_CH = 64;  // channels per block (two lanes each)
+
+// The selective scan for blocks of 64 channels that lie in one B/C group.  Two
+// lanes share a channel, each with N/2 of its states in registers.  Per run of
+// 32 tokens the block copies x, dt (64 channels) and B, C (the group's N
+// states, as float32) into shared memory with coalesced loads, runs the
+// recurrence from there (two vector shared loads of B and C per lane and step,
+// no address arithmetic in global memory), and writes the run's y back as
+// coalesced rows.
+template <typename T, int N>
+__global__ void __launch_bounds__(128) selective_scan_tile_kernel(const T *__restrict__ x, const float *__restrict__ dt,
+                                                                 const float *__restrict__ A, const T *__restrict__ B,
+                                                                 const T *__restrict__ C, const float *__restrict__ D,
+                                                                 const float *__restrict__ h0, float *__restrict__ hT,
+                                                                 T *__restrict__ y, int seqlen, int channels,
+                                                                 int ngroups) {
+    constexpr int NH = N / 2;
+    static_assert(NH % 4 == 0, "states per lane read as float4");
+    __shared__ float xs[SEL_TT][SEL_CH], ds[SEL_TT][SEL_CH], ys[SEL_TT][SEL_CH];
+    __shared__ __align__(16) float bs[SEL_TT][N], cs[SEL_TT][N];
+    const int tid = threadIdx.x, ch = tid >> 1, half = tid & 1;
+    const int cbase = blockIdx.x * SEL_CH, b = blockIdx.y, d = cbase + ch;
+    const int g = cbase / (channels / ngroups), n0 = half * NH;
+    float a2[NH], h[NH];
+#pragma unroll
+    for (int n = 0; n < NH; ++n) {
+        a2[n] = A[(size_t)d * N + n0 + n] * 1.4426950408889634f;
+        h[n] = h0 ? h0[((size_t)b * channels + d) * N + n0 + n] : 0.f;
+    }
+    const float Dd = D ? D[d] : 0.f;
+    for (int t0 = 0; t0 < seqlen; t0 += SEL_TT) {
+        const int nt = min(SEL_TT, seqlen - t0);
+        const size_t row0 = (size_t)b * seqlen + t0;
+        for (int u = tid; u < nt * SEL_CH; u += 128) {
+            const int i = u / SEL_CH, c = u % SEL_CH;
+            const size_t o = (row0 + i) * channels + cbase + c;
+            xs[i][c] = ldf(x + o);
+            ds[i][c] = dt[o];
+        }
+        for (int u = tid; u < nt * N; u += 128) {
+            const int i = u / N, n = u % N;
+            const size_t o = ((row0 + i) * ngroups + g) * N + n;
+            bs[i][n] = ldf(B + o);
+            cs[i][n] = ldf(C + o);
+        }
+        __syncthreads();
+#pragma unroll 2
+        for (int i = 0; i < nt; ++i) {
+            const float xt = xs[i][ch], st = ds[i][ch], u = st * xt;
+            float bv[NH], cv[NH];
+#pragma unroll
+            for (int n = 0; n < NH; n += 4) {
+                const float4 b4 = *reinterpret_cast<const float4 *>(&bs[i][n0 + n]);
+                const float4 c4 = *reinterpret_cast<const float4 *>(&cs[i][n0 + n]);
+                bv[n] = b4.x, bv[n + 1] = b4.y, bv[n + 2] = b4.z, bv[n + 3] = b4.w;
+                cv[n] = c4.x, cv[n + 1] = c4.y, cv[n + 2] = c4.z, cv[n + 3] = c4.w;
+            }
+            float acc = 0.f;
+#pragma unroll
+            for (int n = 0; n < NH; ++n) {
+                h[n] = fmaf(ex2_approx(st * a2[n]), h[n], u * bv[n]);
+                acc = fmaf(cv[n], h[n], acc);
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            if (half == 0) ys[i][ch] = fmaf(Dd, xt, acc);
+        }
+        __syncthreads();
+        for (int u = tid; u < nt * SEL_CH; u += 128) {
+            const int i = u / SEL_CH, c = u % SEL_CH;
+            st_f32(y + (row0 + i) * channels + cbase + c, ys[i][c]);
+        }
+    }
+    if (hT)
+#pragma unroll
+        for (int n = 0; n < NH; ++n) hT[((size_t)b * channels + d) * N + n0 + n] = h[n];
+}
+
 template <typename T, int N>
 cudaError_t launch_sel(const void *x, const float *dt, const float *A, const void *B, const void *C, const float *D,
                        const float *h0, float *hT, void *y, int batch, int seqlen, int channels, int ngroups,
                        cudaStream_t st) {
     // The four-lane form reads each lane's N/4 states of B and C as one vector:
     // aligned when B and C are (the API asks for 16 bytes) and N/4 elements per lane.
+    if constexpr (N >= 8) {  // two lanes of N/2 >= 4 states (whole float4 reads)
+        if ((channels / ngroups) % SEL_CH == 0) {  // every block inside one group
+            dim3 grid(channels / SEL_CH, batch);
+            selective_scan_tile_kernel<T, N><<<grid, 128, 0, st>>>(
+                static_cast<const T *>(x), dt, A, static_cast<const T *>(B), static_cast<const T *>(C), D, h0, hT,
+                static_cast<T *>(y), seqlen, channels, ngroups);
+            return cudaGetLastError();
+        }
+    }
     dim3 grid((channels + 31) / 32, batch);
     selective_scan_q4_kernel<T, N><<<grid, 128, 0, st>>>(static_cast<const T *>(x), dt, A, static_cast<const T *>(B),
                                                          static_cast<const T *>(C), D, h0, hT, static_cast<T *>(y),
@@ -357,19 +444,19 @@ cudaError_t launch_conv1d_xbc(const void *in, const float *w, const float *bias,
                               void *bo, void *co, void *cfinal, bool bf16, int batch, int seqlen, int cx, int cb,
                               int width, int silu, cudaStream_t st) {
     const int ctot = cx + 2 * cb;
-    // 16-byte channel groups when no group straddles the x / B / C ranges and
-    // every row and output base is 16-byte aligned (K <= 4).
-    const int V = bf16 ? 8 : 4;
-    auto al = [](const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
-    if (width <= 4 && cx % V == 0 && cb % V == 0 && al(in) && al(xo) && al(bo) && al(co)) {
-        dim3 grid((ctot / V + 127) / 128, (seqlen + CONV_TV - 1) / CONV_TV, batch);
+    // The tiled kernel when no channel pair straddles the x / B / C ranges, every
+    // token row is a whole number of 16-byte copies (the API asks for 16-byte
+    // aligned pointers) and K <= 4.
+    const int e16 = bf16 ? 8 : 4;
+    if (width <= 4 && cx % 2 == 0 && cb % 2 == 0 && ctot % e16 == 0) {
+        dim3 grid((ctot + CONV_CH - 1) / CONV_CH, (seqlen + CONV_TV - 1) / CONV_TV, batch);
         if (bf16) {
             using T = __nv_bfloat16;
-            conv1d_xbc_vec_kernel<T><<<grid, 128, 0, st>>>(
+            conv1d_xbc_tile_kernel<T><<<grid, 128, 0, st>>>(
                 static_cast<const T *>(in), w, bias, static_cast<const T *>(cinit), static_cast<T *>(xo),
                 static_cast<T *>(bo), static_cast<T *>(co), static_cast<T *>(cfinal), seqlen, cx, cb, width, silu);
         } else {
-            conv1d_xbc_vec_kernel<float><<<grid, 128, 0, st>>>(
+            conv1d_xbc_tile_kernel<float><<<grid, 128, 0, st>>>(
                 static_cast<const float *>(in), w, bias, static_cast<const float *>(cinit), static_cast<float *>(xo),
                 static_cast<float *>(bo), static_cast<float *>(co), static_cast<float *>(cfinal), seqlen, cx, cb,
                 width, silu);
