@@ -666,6 +666,9 @@ def bench_ours(args, shape):
         achieved, peak, unit = aflops / t_launch / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     if tc_path:
         kernel, src_name = "ssd_scan_tc_kernel", "scan_tc.cu"
+    elif cplx and shape.headdim == 64 and shape.dstate == 64:  # the tcgen05 complex kernels
+        kernel, src_name = ("state_kernel+cplx_state_pass+scan_kernel (3 launches, tcgen05, timed as one call)",
+                            "scan_complex_tc.cuh")
     elif cplx:
         kernel, src_name = "cplx_chunk_state+cplx_state_pass+cplx_chunk_scan (3 kernels)", "scan_complex.cu"
     else:
@@ -862,7 +865,7 @@ def bench_variant(args, name):
         tokens = sh.batch * sh.seqlen
         esz = 2 if sh.io_dtype == "bf16" else 4
         abytes = 2 * sh.batch * sh.seqlen * Ct * esz + Ct * (sh.width + 1) * 4
-        kernel, bound, alu_peak = "conv1d_xbc_kernel", "hbm", None
+        kernel, bound, alu_peak = "conv1d_xbc_tile_kernel", "hbm", None
     else:
         sh = inputs.MAMBA1_50M
         inp = inputs.selective_inputs(sh)
@@ -876,7 +879,7 @@ def bench_variant(args, name):
         abytes = (sh.tokens * sh.channels * (2 * esz + 4) + 2 * sh.tokens * sh.ngroups * sh.dstate * esz
                   + sh.batch * sh.channels * sh.dstate * 4 + sh.channels * (sh.dstate + 1) * 4)
         exps = sh.tokens * sh.channels * sh.dstate
-        kernel = "selective_scan_kernel"
+        kernel = "selective_scan_tile_kernel"
         alu_peak = 148 * SFU_EXP_PER_CLK_SM * 1.965e9  # exponentials per second at the max SM clock
         bound = "alu" if exps / alu_peak > abytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -920,8 +923,9 @@ def bench_variant(args, name):
     else:
         roof = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"]}
-    roof.update({"traffic": None, "kernel": kernel, "algorithmic_bytes_per_launch": abytes,
-                 "kernel_time_us": 1e6 * t_call})
+    roof.update({"traffic": lookup_traffic(kernel, os.path.join(ROOT, "selective_state_space_22_b200", "csrc",
+                                                                "variants.cu"), sh.name),
+                 "kernel": kernel, "algorithmic_bytes_per_launch": abytes, "kernel_time_us": 1e6 * t_call})
     line = {
         "metric": METRIC, "value": tokens * world * steps / total_s, "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": max(args.warmup, 3), "ms_per_step": 1e3 * total_s / steps,

@@ -12,6 +12,8 @@
 //      (two kernels)
 // Sums run in a fixed order, so repeated calls give identical bits.  The complex
 // variant (scan_bwd_complex_body.cuh) runs the same six steps on 32-token chunks.
+#include <mutex>
+
 #include "scan_bwd_body.cuh"
 #include "scan_bwd_complex_body.cuh"
 #include "ssd_internal.cuh"
@@ -34,7 +36,9 @@ __global__ void __launch_bounds__(NT) bwd_chunk_state(BwdArgs a) {
     k1_state(a, c, h, b, tid, m);
 }
 
-__global__ void __launch_bounds__(NT) bwd_state_fwd(BwdArgs a) { k2_pass(a, blockIdx.x, blockIdx.y, threadIdx.x); }
+__global__ void __launch_bounds__(NT) bwd_state_fwd(BwdArgs a) {
+    k2_pass(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
+}
 
 __global__ void __launch_bounds__(NT) bwd_readout(BwdArgs a) {
     extern __shared__ float sm[];
@@ -45,7 +49,9 @@ __global__ void __launch_bounds__(NT) bwd_readout(BwdArgs a) {
     k3_r(a, c, h, b, tid, m);
 }
 
-__global__ void __launch_bounds__(NT) bwd_state_bwd(BwdArgs a) { k4_pass(a, blockIdx.x, blockIdx.y, threadIdx.x); }
+__global__ void __launch_bounds__(NT) bwd_state_bwd(BwdArgs a) {
+    k4_pass(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
+}
 
 __global__ void __launch_bounds__(NT) bwd_chunk_grad(BwdArgs a) {
     extern __shared__ float sm[];
@@ -57,9 +63,18 @@ __global__ void __launch_bounds__(NT) bwd_chunk_grad(BwdArgs a) {
     __syncthreads();
     k5_tokens(a, tid, m);
     __syncthreads();
-    k5_decay(a, c, h, b, tid, m);
+    k5_gb(a, tid, m);
     __syncthreads();
-    k5_out(a, c, h, b, tid, m);
+    k5_db(a, c, h, b, tid, m);
+    __syncthreads();
+    k5_ksr(a, tid, m);
+    __syncthreads();
+    k5_dc(a, c, h, b, tid, m);
+    __syncthreads();
+    k5_f(a, tid, m);
+    __syncthreads();
+    k5_decay(a, c, h, b, tid, m);
+    k5_dx(a, c, h, b, tid, m);
 }
 
 __global__ void __launch_bounds__(NT) bwd_group_sum(BwdArgs a, size_t total) {
@@ -205,31 +220,37 @@ cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
     a.nchunks = (call.seqlen + QB - 1) / QB;
     carve(a, static_cast<float *>(ws));
 
-    // the shared-memory opt-in is per function and per device
-    static bool attr_set[64] = {false};
+    // the shared-memory opt-in is per function, device and context
+    static void *attr_ctx[64] = {nullptr};
+    static std::mutex attr_mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!attr_set[dev]) {
-        for (const void *f : {(const void *)bwd_chunk_state, (const void *)bwd_readout,
-                              (const void *)bwd_chunk_grad}) {
-            e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-            if (e != cudaSuccess) return e;
+    {
+        std::lock_guard<std::mutex> lk(attr_mu);
+        void *ctx = current_context();
+        if (!ctx || attr_ctx[dev] != ctx) {
+            for (const void *f : {(const void *)bwd_chunk_state, (const void *)bwd_readout,
+                                  (const void *)bwd_chunk_grad}) {
+                e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+                if (e != cudaSuccess) return e;
+            }
+            attr_ctx[dev] = ctx;
         }
-        attr_set[dev] = true;
     }
+    const unsigned pn_blocks = (unsigned)(((size_t)a.headdim * a.dstate + NT - 1) / NT);
     if (a.batch > 0 && a.nchunks > 0) {
-        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(a.nheads, a.batch);
-        bwd_chunk_state<<<gc, NT, SMEM_BYTES, st>>>(a);
+        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(pn_blocks, a.nheads, a.batch);
+        bwd_chunk_state<<<gc, NT, SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
         bwd_state_fwd<<<gh, NT, 0, st>>>(a);
-        bwd_readout<<<gc, NT, SMEM_BYTES, st>>>(a);
+        bwd_readout<<<gc, NT, SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwd_state_bwd<<<gh, NT, 0, st>>>(a);
         bwd_chunk_grad<<<gc, NT, SMEM_BYTES, st>>>(a);
         const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;
         bwd_group_sum<<<(unsigned)((total + NT - 1) / NT), NT, 0, st>>>(a, total);
     } else if (a.batch > 0) {  // empty sequences: dinit = dfinal (or zero)
-        bwd_state_bwd<<<dim3(a.nheads, a.batch), NT, 0, st>>>(a);
+        bwd_state_bwd<<<dim3(pn_blocks, a.nheads, a.batch), NT, 0, st>>>(a);
     }
     bwd_head_sum<<<(a.nheads + NT - 1) / NT, NT, 0, st>>>(a);
     return cudaGetLastError();

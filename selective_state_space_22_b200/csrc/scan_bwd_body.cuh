@@ -23,14 +23,34 @@
 // Every phase is a __host__ __device__ function of (block, thread): the CUDA
 // kernels run them separated by __syncthreads(), and a CPU harness in the tests
 // runs the same functions thread by thread between the same barriers.
+//
+// The per-chunk products run as register-tiled matrix products on the CUDA
+// cores: the 256 threads form a 16 x 16 grid, each owns a 4 x 4 or 4 x 8 tile of
+// the result, and operands come from shared memory as 16-byte vectors (row
+// strides of 4 mod 32 words keep every access pattern free of bank conflicts).
+// Sums across threads go through a shared array of partial sums, added in a
+// fixed order, so repeated calls stay bitwise equal.
 #pragma once
 
 #include <math.h>
 #include <stddef.h>
+#include <stdint.h>
 
 #ifndef __CUDACC__
 #define __host__
 #define __device__
+#endif
+
+// The inputs and the workspace written by earlier launches are read-only while
+// a phase runs; on the device they are read through the read-only path, which
+// lets the compiler keep many rows' loads in flight ahead of the shared-memory
+// stores of the loading loops.  BWD_UNROLL unrolls those loops on the device.
+#ifdef __CUDA_ARCH__
+#define BWD_LDG(p) __ldg(p)
+#define BWD_UNROLL _Pragma("unroll 8")
+#else
+#define BWD_LDG(p) (*(p))
+#define BWD_UNROLL
 #endif
 
 namespace ssd {
@@ -40,9 +60,9 @@ constexpr int QB = 64;       // tokens per chunk
 constexpr int NT = 256;      // threads per block
 constexpr int P_MAX = 64;    // head dim
 constexpr int N_MAX = 128;   // state dim
-// Shared-memory row strides, one float longer than a row, so that lanes walking
-// down a column hit 32 different banks.
-constexpr int PS = P_MAX + 1, NS = N_MAX + 1, QS = QB + 1;
+// Shared-memory row strides: four floats longer than a row, so rows stay 16-byte
+// aligned and consecutive rows start 4 banks apart.
+constexpr int PS = P_MAX + 4, NS = N_MAX + 4, QS = QB + 4;
 
 struct BwdArgs {
     const float *x, *dt, *A, *B, *C, *D, *init, *dy, *dfinal;
@@ -101,19 +121,25 @@ __host__ __device__ inline size_t ix_pn(const BwdArgs &a, int b, int h, int c) {
 __host__ __device__ inline int group_of(const BwdArgs &a, int h) { return h / (a.nheads / a.ngroups); }
 
 // ------------------------------------------------ shared-memory layout
-// One layout serves every chunk kernel (fixed row strides PS, NS, QS).
+// One layout serves every chunk kernel (fixed row strides PS, NS, QS).  Arrays
+// are zero beyond headdim / dstate, so the products always run over P_MAX and
+// N_MAX.
 struct Smem {
     float *d, *acs, *e, *w;           // [QB]
     float *X, *dY;                    // [QB][PS]
     float *Bs, *Cs;                   // [QB][NS]
     float *Hin, *Gh;                  // [P_MAX][NS]
-    float *GL, *XY, *K;               // [QB][QS]
+    float *GL, *XY, *K;               // [QB][QS]; XY later holds B Gh^T
     float *rowE, *colG, *F, *Ksr;     // [QB]
     float *red;                       // [2 * QB]
+    float *part;                      // [QB][16]: partial row sums, one per thread column
     float *misc;                      // [4]: lam, ...
 };
 constexpr size_t SMEM_FLOATS = 4 * QB + 2 * QB * PS + 2 * QB * NS + 2 * P_MAX * NS + 3 * QB * QS +
-                               4 * QB + 2 * QB + 4;
+                               4 * QB + 2 * QB + 16 * QB + 4;
+// The chunk-state phase uses the layout up to Bs, the readout phase up to Cs.
+constexpr size_t SMEM_FLOATS_K1 = 4 * QB + 2 * QB * PS + QB * NS;
+constexpr size_t SMEM_FLOATS_K3 = 4 * QB + 2 * QB * PS + 2 * QB * NS;
 __host__ __device__ inline Smem smem_map(float *s) {
     Smem m;
     m.d = s; s += QB;
@@ -134,36 +160,125 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.F = s; s += QB;
     m.Ksr = s; s += QB;
     m.red = s; s += 2 * QB;
+    m.part = s; s += 16 * QB;
     m.misc = s;
     return m;
 }
 
+// ---------------------------------------------- register-tiled products
+struct alignas(16) f4 {
+    float x, y, z, w;
+};
+__host__ __device__ inline f4 ld4(const float *p) { return *reinterpret_cast<const f4 *>(p); }
+__host__ __device__ inline float comp(const f4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+// Thread (tr, tc) = (tid / 16, tid % 16) owns rows r0 = 4 tr .. 4 tr + 3.
+// "nt": acc[i][j] += sum_k A[r0+i][k] B[tc+16j][k]   (both k-contiguous rows; k0, k1 multiples of 4)
+template <int NJ>
+__host__ __device__ inline void mm_nt(float (&acc)[4][NJ], const float *A, int lda, int r0, const float *B, int ldb,
+                                      int tc, int k0, int k1) {
+    for (int k = k0; k < k1; k += 4) {
+        f4 a[4], b[NJ];
+        for (int i = 0; i < 4; ++i) a[i] = ld4(A + (r0 + i) * lda + k);
+        for (int j = 0; j < NJ; ++j) b[j] = ld4(B + (tc + 16 * j) * ldb + k);
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < NJ; ++j)
+                acc[i][j] = fmaf(a[i].w, b[j].w, fmaf(a[i].z, b[j].z, fmaf(a[i].y, b[j].y, fmaf(a[i].x, b[j].x, acc[i][j]))));
+    }
+}
+// "tn": acc[i][j] += sum_k sc[k] A[k][r0+i] B[k][c(j)],  c(j) = 4 tc + j (+ 60 for j >= 4: 64 + 4 tc + j - 4)
+// (sc may be null: no scaling)
+template <int NJ>
+__host__ __device__ inline void mm_tn(float (&acc)[4][NJ], const float *A, int lda, int r0, const float *sc,
+                                      const float *B, int ldb, int tc, int k0, int k1) {
+    for (int k = k0; k < k1; ++k) {
+        f4 a = ld4(A + k * lda + r0);
+        if (sc) {
+            const float f = sc[k];
+            a.x *= f, a.y *= f, a.z *= f, a.w *= f;
+        }
+        f4 b[NJ / 4];
+        for (int q = 0; q < NJ / 4; ++q) b[q] = ld4(B + k * ldb + 64 * q + 4 * tc);
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(comp(a, i), comp(b[j / 4], j % 4), acc[i][j]);
+    }
+}
+// "nn": acc[i][j] += sum_k A[r0+i][k] B[k][c(j)]   (k0, k1 multiples of 4)
+template <int NJ>
+__host__ __device__ inline void mm_nn(float (&acc)[4][NJ], const float *A, int lda, int r0, const float *B, int ldb,
+                                      int tc, int k0, int k1) {
+    for (int k = k0; k < k1; k += 4) {
+        f4 a[4];
+        for (int i = 0; i < 4; ++i) a[i] = ld4(A + (r0 + i) * lda + k);
+        for (int kk = 0; kk < 4; ++kk) {
+            f4 b[NJ / 4];
+            for (int q = 0; q < NJ / 4; ++q) b[q] = ld4(B + (k + kk) * ldb + 64 * q + 4 * tc);
+            for (int i = 0; i < 4; ++i)
+                for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(comp(a[i], kk), comp(b[j / 4], j % 4), acc[i][j]);
+        }
+    }
+}
+template <int NJ> __host__ __device__ inline void zero(float (&acc)[4][NJ]) {
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+}
+// Column of element j of a "tn"/"nn" tile.
+__host__ __device__ inline int tile_col(int tc, int j) { return 64 * (j / 4) + 4 * tc + j % 4; }
+
+// Four consecutive values to dst[0..3] of a row holding `valid` values from
+// column col: one 16-byte store when all four are valid and aligned.
+__host__ __device__ inline void store_row4(float *dst, int col, int valid, const float *v) {
+    if (col + 3 < valid && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        *reinterpret_cast<f4 *>(dst) = f4{v[0], v[1], v[2], v[3]};
+    } else {
+        for (int q = 0; q < 4; ++q)
+            if (col + q < valid) dst[q] = v[q];
+    }
+}
+
 // ------------------------------------------------ shared loading phases
-// dt of the chunk (0 past the end), and x or dy [QB][P], B or C [QB][N].
+// dt of the chunk (0 past the end), and x or dy [QB][P], B or C [QB][N]; zero
+// past the sequence end and beyond headdim / dstate.
 __host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     for (int i = tid; i < QB; i += NT) {
         const int t = c * QB + i;
-        m.d[i] = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
+        m.d[i] = t < a.seqlen ? BWD_LDG(a.dt + ix_dt(a, b, t, h)) : 0.f;
     }
 }
 __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
                                             float *dst) {
-    for (int i = tid; i < QB * a.headdim; i += NT) {
-        const int s = i / a.headdim, p = i % a.headdim, t = c * QB + s;
-        dst[s * PS + p] = t < a.seqlen ? src[ix_x(a, b, t, h, p)] : 0.f;
+    BWD_UNROLL
+    for (int i = tid; i < QB * P_MAX; i += NT) {
+        const int s = i / P_MAX, p = i % P_MAX, t = c * QB + s;
+        dst[s * PS + p] = (t < a.seqlen && p < a.headdim) ? BWD_LDG(src + ix_x(a, b, t, h, p)) : 0.f;
     }
 }
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
-    for (int i = tid; i < QB * a.dstate; i += NT) {
-        const int s = i / a.dstate, n = i % a.dstate, t = c * QB + s;
-        dst[s * NS + n] = t < a.seqlen ? src[ix_bc(a, b, t, g, n)] : 0.f;
+    BWD_UNROLL
+    for (int i = tid; i < QB * N_MAX; i += NT) {
+        const int s = i / N_MAX, n = i % N_MAX, t = c * QB + s;
+        dst[s * NS + n] = (t < a.seqlen && n < a.dstate) ? BWD_LDG(src + ix_bc(a, b, t, g, n)) : 0.f;
     }
 }
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
-    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
-        const int p = i / a.dstate, n = i % a.dstate;
-        dst[p * NS + n] = src[i];
+    BWD_UNROLL
+    for (int i = tid; i < P_MAX * N_MAX; i += NT) {
+        const int p = i / N_MAX, n = i % N_MAX;
+        dst[p * NS + n] = (p < a.headdim && n < a.dstate) ? BWD_LDG(src + (size_t)p * a.dstate + n) : 0.f;
+    }
+}
+// A P x N tile (rows p = 4 tr + i, columns tile_col(tc, j)) to a row-major P x N
+// array in global memory.
+__host__ __device__ inline void store_pn(const BwdArgs &a, float *dst, int tid, const float (&acc)[4][8]) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    for (int i = 0; i < 4; ++i) {
+        const int p = r0 + i;
+        if (p >= a.headdim) continue;
+        for (int q = 0; q < 2; ++q) {
+            const int n0 = tile_col(tc, 4 * q);
+            if (n0 < a.dstate) store_row4(dst + (size_t)p * a.dstate + n0, n0, a.dstate, &acc[i][4 * q]);
+        }
     }
 }
 
@@ -184,63 +299,55 @@ __host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b,
         m.acs[i] = v;
         acs_g[i] = v;
     }
-    m.misc[0] = v;
     a.lam[ix_bh(a, b, h) * a.nchunks + c] = v;
     for (int i = 0; i < QB; ++i) m.w[i] = expf(v - m.acs[i]) * m.d[i];
 }
 // S[p][n] = sum_s w_s x_s[p] B_s[n]
 __host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
-    float *S = a.st + ix_pn(a, b, h, c);
-    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
-        const int p = i / a.dstate, n = i % a.dstate;
-        float acc = 0.f;
-        for (int s = 0; s < QB; ++s) acc += m.w[s] * m.X[s * PS + p] * m.Bs[s * NS + n];
-        S[i] = acc;
-    }
+    float acc[4][8];
+    zero(acc);
+    mm_tn<8>(acc, m.X, PS, 4 * (tid >> 4), m.w, m.Bs, NS, tid & 15, 0, QB);
+    store_pn(a, a.st + ix_pn(a, b, h, c), tid, acc);
 }
 
 // ------------------------------------- 2: state entering each chunk (forward)
-__host__ __device__ inline void k2_pass(const BwdArgs &a, int h, int b, int tid) {
-    const size_t pn = (size_t)a.headdim * a.dstate;
-    for (size_t i = tid; i < pn; i += NT) {
-        float hv = a.init ? a.init[ix_bh(a, b, h) * pn + i] : 0.f;
-        for (int c = 0; c < a.nchunks; ++c) {
-            const size_t o = ix_pn(a, b, h, c) + i;
-            a.hin[o] = hv;
-            hv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * hv + a.st[o];
-        }
+// Element i = blk * NT + tid of the P x N state of (batch b, head h).
+__host__ __device__ inline void k2_pass(const BwdArgs &a, int blk, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
+    if (i >= pn) return;
+    float hv = a.init ? a.init[ix_bh(a, b, h) * pn + i] : 0.f;
+    for (int c = 0; c < a.nchunks; ++c) {
+        const size_t o = ix_pn(a, b, h, c) + i;
+        a.hin[o] = hv;
+        hv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * hv + a.st[o];
     }
 }
 
 // ------------------------------- 3: readout terms R = sum_l e^{acs[l]} dy_l C_l^T
 __host__ __device__ inline void k3_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     const float *acs_g = a.acs + (ix_bh(a, b, h) * a.nchunks + c) * QB;
-    for (int i = tid; i < QB; i += NT) m.e[i] = expf(acs_g[i]);
+    for (int i = tid; i < QB; i += NT) m.e[i] = expf(BWD_LDG(acs_g + i));
     load_rows_p(a, a.dy, c, h, b, tid, m.dY);
     load_rows_n(a, a.C, c, group_of(a, h), b, tid, m.Cs);
 }
 __host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
-    float *R = a.st + ix_pn(a, b, h, c);  // the chunk states were consumed by pass 2
-    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
-        const int p = i / a.dstate, n = i % a.dstate;
-        float acc = 0.f;
-        for (int l = 0; l < QB; ++l) acc += m.e[l] * m.dY[l * PS + p] * m.Cs[l * NS + n];
-        R[i] = acc;
-    }
+    float acc[4][8];
+    zero(acc);
+    mm_tn<8>(acc, m.dY, PS, 4 * (tid >> 4), m.e, m.Cs, NS, tid & 15, 0, QB);
+    store_pn(a, a.st + ix_pn(a, b, h, c), tid, acc);  // the chunk states were consumed by pass 2
 }
 
 // --------------------- 4: gradient of the state leaving each chunk (backward)
-__host__ __device__ inline void k4_pass(const BwdArgs &a, int h, int b, int tid) {
-    const size_t pn = (size_t)a.headdim * a.dstate;
-    for (size_t i = tid; i < pn; i += NT) {
-        float gv = a.dfinal ? a.dfinal[ix_bh(a, b, h) * pn + i] : 0.f;
-        for (int c = a.nchunks - 1; c >= 0; --c) {
-            const size_t o = ix_pn(a, b, h, c) + i;
-            a.gh[o] = gv;
-            gv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * gv + a.st[o];
-        }
-        if (a.dinit) a.dinit[ix_bh(a, b, h) * pn + i] = gv;
+__host__ __device__ inline void k4_pass(const BwdArgs &a, int blk, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
+    if (i >= pn) return;
+    float gv = a.dfinal ? a.dfinal[ix_bh(a, b, h) * pn + i] : 0.f;
+    for (int c = a.nchunks - 1; c >= 0; --c) {
+        const size_t o = ix_pn(a, b, h, c) + i;
+        a.gh[o] = gv;
+        gv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * gv + a.st[o];
     }
+    if (a.dinit) a.dinit[ix_bh(a, b, h) * pn + i] = gv;
 }
 
 // ------------------------------------------------ 5: gradients of one chunk
@@ -251,10 +358,11 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     const float lam = a.lam[ix_bh(a, b, h) * a.nchunks + c];
     for (int i = tid; i < QB; i += NT) {
         const int t = c * QB + i;
-        const float d = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
-        m.acs[i] = acs_g[i];
-        m.e[i] = expf(acs_g[i]);
-        m.w[i] = expf(lam - acs_g[i]) * d;
+        const float d = t < a.seqlen ? BWD_LDG(a.dt + ix_dt(a, b, t, h)) : 0.f;
+        const float ac = BWD_LDG(acs_g + i);
+        m.acs[i] = ac;
+        m.e[i] = expf(ac);
+        m.w[i] = expf(lam - ac) * d;
     }
     if (tid == 0) m.misc[0] = lam;
     load_rows_p(a, a.x, c, h, b, tid, m.X);
@@ -264,65 +372,142 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     load_pn(a, a.hin + ix_pn(a, b, h, c), tid, m.Hin);
     load_pn(a, a.gh + ix_pn(a, b, h, c), tid, m.Gh);
 }
-// GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY.
+// GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY; thread tile rows
+// l = 4 tr + i, columns s = tc + 16 j.
 __host__ __device__ inline void k5_mats(const BwdArgs &a, int tid, const Smem &m) {
-    for (int i = tid; i < QB * QB; i += NT) {
-        const int l = i / QB, s = i % QB;
-        float gm = 0.f, xy = 0.f;
-        for (int n = 0; n < a.dstate; ++n) gm += m.Cs[l * NS + n] * m.Bs[s * NS + n];
-        for (int p = 0; p < a.headdim; ++p) xy += m.dY[l * PS + p] * m.X[s * PS + p];
-        m.XY[l * QS + s] = xy;
-        if (l >= s) {
-            const float L = expf(m.acs[l] - m.acs[s]);
-            m.GL[l * QS + s] = gm * L;
-            m.K[l * QS + s] = L * m.d[s] * xy;
-        } else {
-            m.GL[l * QS + s] = 0.f;
-            m.K[l * QS + s] = 0.f;
+    (void)a;
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    float g[4][4], xy[4][4];
+    zero(g);
+    zero(xy);
+    mm_nt<4>(g, m.Cs, NS, r0, m.Bs, NS, tc, 0, N_MAX);
+    mm_nt<4>(xy, m.dY, PS, r0, m.X, PS, tc, 0, P_MAX);
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 4; ++j) {
+            const int l = r0 + i, s = tc + 16 * j;
+            m.XY[l * QS + s] = xy[i][j];
+            if (l >= s) {
+                const float L = expf(m.acs[l] - m.acs[s]);
+                m.GL[l * QS + s] = g[i][j] * L;
+                m.K[l * QS + s] = L * m.d[s] * xy[i][j];
+            } else {
+                m.GL[l * QS + s] = 0.f;
+                m.K[l * QS + s] = 0.f;
+            }
+        }
+}
+// Per token: the row sums of E = GL o XY o dt_s, the column sums of GL o XY; the
+// last 128 threads reduce <Gh, h_in> and dy . x.  Rows are walked from a
+// per-thread start so that the 32 lanes of a warp read 32 different banks.
+__host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    if (tid < QB) {
+        const int t = tid;
+        float re = 0.f;
+        for (int q = 0; q < QB; ++q) {
+            const int s = (q + t) & (QB - 1);
+            re += m.GL[t * QS + s] * m.XY[t * QS + s] * m.d[s];
+        }
+        m.rowE[t] = re;
+    } else if (tid < 2 * QB) {
+        const int t = tid - QB;
+        float cg = 0.f;
+        for (int l = 0; l < QB; ++l) cg += m.GL[l * QS + t] * m.XY[l * QS + t];
+        m.colG[t] = cg;
+    } else if (tid < 3 * QB) {
+        const int r = tid - 2 * QB;
+        float h0 = 0.f;
+        for (int i = r; i < P_MAX * N_MAX; i += QB) {
+            const int p = i / N_MAX, n = i % N_MAX;
+            h0 += m.Gh[p * NS + n] * m.Hin[p * NS + n];
+        }
+        m.red[r] = h0;
+    } else {
+        const int r = tid - 3 * QB;
+        float dd = 0.f;
+        for (int i = r; i < QB * P_MAX; i += QB) {
+            const int s = i / P_MAX, p = i % P_MAX;
+            dd += m.dY[s * PS + p] * m.X[s * PS + p];
+        }
+        m.red[QB + r] = dd;
+    }
+}
+// GB = B Gh^T into the XY buffer (XY is no longer needed): rows s, columns p.
+__host__ __device__ inline void k5_gb(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    float gb[4][4];
+    zero(gb);
+    mm_nt<4>(gb, m.Bs, NS, r0, m.Gh, NS, tc, 0, N_MAX);
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 4; ++j) m.XY[(r0 + i) * QS + tc + 16 * j] = gb[i][j];
+}
+// This head's dB: dB_s = sum_l K[l][s] C_l + w_s (x_s Gh); with the partial sums
+// of Ksr[s] = B_s . (x_s Gh) per thread column.
+__host__ __device__ inline void k5_db(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    float acc[4][8];
+    zero(acc);
+    mm_nn<8>(acc, m.X, PS, r0, m.Gh, NS, tc, 0, P_MAX);  // x Gh
+    for (int i = 0; i < 4; ++i) {
+        const int s = r0 + i;
+        float ks = 0.f;
+        for (int j = 0; j < 8; ++j) ks = fmaf(m.Bs[s * NS + tile_col(tc, j)], acc[i][j], ks);
+        m.part[s * 16 + tc] = ks;
+        for (int j = 0; j < 8; ++j) acc[i][j] *= m.w[s];
+    }
+    mm_tn<8>(acc, m.K, QS, r0, nullptr, m.Cs, NS, tc, r0, QB);  // K[l][s] = 0 for l < s
+    for (int i = 0; i < 4; ++i) {
+        const int s = r0 + i, t = c * QB + s;
+        if (t >= a.seqlen) continue;
+        float *row = a.dBh + (((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate;
+        for (int q = 0; q < 2; ++q) {
+            const int n0 = tile_col(tc, 4 * q);
+            if (n0 < a.dstate) store_row4(row + n0, n0, a.dstate, &acc[i][4 * q]);
         }
     }
 }
-// Per token: the row sums of E, the column sums of GL o XY, and the two
-// state-coupling dot products; the last 64 threads reduce <Gh, h_in> and dy.x.
-__host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem &m) {
+// Ksr from its partial sums (fixed order).
+__host__ __device__ inline void k5_ksr(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
     if (tid < QB) {
-        const int t = tid;
-        float re = 0.f, cg = 0.f;
-        for (int s = 0; s < QB; ++s) re += m.GL[t * QS + s] * m.XY[t * QS + s] * m.d[s];
-        for (int l = 0; l < QB; ++l) cg += m.GL[l * QS + t] * m.XY[l * QS + t];
-        m.rowE[t] = re;
-        m.colG[t] = cg;
-    } else if (tid < 2 * QB) {  // F[t] = e^{acs[t]} dy_t . (h_in C_t)
-        const int t = tid - QB;
-        float acc = 0.f;
-        for (int p = 0; p < a.headdim; ++p) {
-            float hc = 0.f;
-            for (int n = 0; n < a.dstate; ++n) hc += m.Hin[p * NS + n] * m.Cs[t * NS + n];
-            acc += m.dY[t * PS + p] * hc;
+        float v = 0.f;
+        for (int q = 0; q < 16; ++q) v += m.part[tid * 16 + q];
+        m.Ksr[tid] = v;
+    }
+}
+// This head's dC: dC_l = sum_s K[l][s] B_s + e_l (dy_l h_in); with the partial sums
+// of F[l] / e_l = C_l . (dy_l h_in).
+__host__ __device__ inline void k5_dc(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    float acc[4][8];
+    zero(acc);
+    mm_nn<8>(acc, m.dY, PS, r0, m.Hin, NS, tc, 0, P_MAX);  // dy h_in
+    for (int i = 0; i < 4; ++i) {
+        const int l = r0 + i;
+        float f = 0.f;
+        for (int j = 0; j < 8; ++j) f = fmaf(m.Cs[l * NS + tile_col(tc, j)], acc[i][j], f);
+        m.part[l * 16 + tc] = f;
+        for (int j = 0; j < 8; ++j) acc[i][j] *= m.e[l];
+    }
+    mm_nn<8>(acc, m.K, QS, r0, m.Bs, NS, tc, 0, r0 + 4);  // K[l][s] = 0 for s > l
+    for (int i = 0; i < 4; ++i) {
+        const int l = r0 + i, t = c * QB + l;
+        if (t >= a.seqlen) continue;
+        float *row = a.dCh + (((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate;
+        for (int q = 0; q < 2; ++q) {
+            const int n0 = tile_col(tc, 4 * q);
+            if (n0 < a.dstate) store_row4(row + n0, n0, a.dstate, &acc[i][4 * q]);
         }
-        m.F[t] = m.e[t] * acc;
-    } else if (tid < 3 * QB) {  // Ksr[t] = x_t . (Gh B_t)
-        const int t = tid - 2 * QB;
-        float acc = 0.f;
-        for (int p = 0; p < a.headdim; ++p) {
-            float gb = 0.f;
-            for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * NS + n] * m.Bs[t * NS + n];
-            acc += m.X[t * PS + p] * gb;
-        }
-        m.Ksr[t] = acc;
-    } else if (tid < 4 * QB) {
-        const int r = tid - 3 * QB;
-        float h0 = 0.f, dd = 0.f;
-        for (int i = r; i < a.headdim * a.dstate; i += QB) {
-            const int p = i / a.dstate, n = i % a.dstate;
-            h0 += m.Gh[p * NS + n] * m.Hin[p * NS + n];
-        }
-        for (int i = r; i < QB * a.headdim; i += QB) {
-            const int s = i / a.headdim, p = i % a.headdim;
-            dd += m.dY[s * PS + p] * m.X[s * PS + p];
-        }
-        m.red[r] = h0;
-        m.red[QB + r] = dd;
+    }
+}
+// F from its partial sums.
+__host__ __device__ inline void k5_f(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    if (tid < QB) {
+        float v = 0.f;
+        for (int q = 0; q < 16; ++q) v += m.part[tid * 16 + q];
+        m.F[tid] = m.e[tid] * v;
     }
 }
 // Thread 0: the decay gradient (reverse cumulative sum), ddt, and the dA and dD
@@ -351,30 +536,22 @@ __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, 
     a.dAp[ix_bh(a, b, h) * a.nchunks + c] = dAp;
     a.dDp[ix_bh(a, b, h) * a.nchunks + c] = dd;
 }
-// dx, and this head's share of dB and dC.
-__host__ __device__ inline void k5_out(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+// dx_s = dt_s sum_l GL[l][s] dy_l + D dy_s + w_s GB[s]  (rows s, columns p)
+__host__ __device__ inline void k5_dx(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
     const float Dh = a.D ? a.D[h] : 0.f;
-    for (int i = tid; i < QB * a.headdim; i += NT) {
-        const int s = i / a.headdim, p = i % a.headdim, t = c * QB + s;
+    float acc[4][4];
+    zero(acc);
+    mm_tn<4>(acc, m.GL, QS, r0, nullptr, m.dY, PS, tc, r0, QB);  // GL[l][s] = 0 for l < s
+    const int p0 = 4 * tc;
+    if (p0 >= a.headdim) return;
+    for (int i = 0; i < 4; ++i) {
+        const int s = r0 + i, t = c * QB + s;
         if (t >= a.seqlen) continue;
-        float acc = 0.f, gb = 0.f;
-        for (int l = s; l < QB; ++l) acc += m.GL[l * QS + s] * m.dY[l * PS + p];
-        for (int n = 0; n < a.dstate; ++n) gb += m.Gh[p * NS + n] * m.Bs[s * NS + n];
-        a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * PS + p] + m.w[s] * gb;
-    }
-    for (int i = tid; i < QB * a.dstate; i += NT) {
-        const int s = i / a.dstate, n = i % a.dstate, t = c * QB + s;
-        if (t >= a.seqlen) continue;
-        float db = 0.f, dc = 0.f, xg = 0.f, yh = 0.f;
-        for (int l = s; l < QB; ++l) db += m.K[l * QS + s] * m.Cs[l * NS + n];
-        for (int r = 0; r <= s; ++r) dc += m.K[s * QS + r] * m.Bs[r * NS + n];
-        for (int p = 0; p < a.headdim; ++p) {
-            xg += m.X[s * PS + p] * m.Gh[p * NS + n];
-            yh += m.dY[s * PS + p] * m.Hin[p * NS + n];
-        }
-        const size_t o = (((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n;
-        a.dBh[o] = db + m.w[s] * xg;
-        a.dCh[o] = dc + m.e[s] * yh;
+        float v[4];
+        for (int j = 0; j < 4; ++j)
+            v[j] = m.d[s] * acc[i][j] + Dh * m.dY[s * PS + p0 + j] + m.w[s] * m.XY[s * QS + p0 + j];
+        store_row4(a.dx + ix_x(a, b, t, h, p0), p0, a.headdim, v);
     }
 }
 

@@ -27,6 +27,15 @@
 #define __device__
 #endif
 
+// Read-only loads and unrolled loading loops on the device (see scan_bwd_body.cuh).
+#ifdef __CUDA_ARCH__
+#define BWDC_LDG(p) __ldg(p)
+#define BWDC_UNROLL _Pragma("unroll 8")
+#else
+#define BWDC_LDG(p) (*(p))
+#define BWDC_UNROLL
+#endif
+
 namespace ssd {
 namespace bwdc {
 
@@ -156,29 +165,32 @@ __host__ __device__ inline Smem smem_map(float *s) {
 __host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     for (int i = tid; i < QC; i += NT) {
         const int t = c * QC + i;
-        m.d[i] = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
+        m.d[i] = t < a.seqlen ? BWDC_LDG(a.dt + ix_dt(a, b, t, h)) : 0.f;
     }
 }
 __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
                                             float *dst) {
+    BWDC_UNROLL
     for (int i = tid; i < QC * a.headdim; i += NT) {
         const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
-        dst[s * PS + p] = t < a.seqlen ? src[ix_x(a, b, t, h, p)] : 0.f;
+        dst[s * PS + p] = t < a.seqlen ? BWDC_LDG(src + ix_x(a, b, t, h, p)) : 0.f;
     }
 }
 // complex rows of B or C: [QC][N] pairs
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
+    BWDC_UNROLL
     for (int i = tid; i < QC * 2 * a.dstate; i += NT) {
         const int s = i / (2 * a.dstate), f = i % (2 * a.dstate), t = c * QC + s;
-        dst[s * NS + f] = t < a.seqlen ? src[2 * ix_bc(a, b, t, g, 0) + f] : 0.f;
+        dst[s * NS + f] = t < a.seqlen ? BWDC_LDG(src + 2 * ix_bc(a, b, t, g, 0) + f) : 0.f;
     }
 }
 // a complex [P][N] block
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
+    BWDC_UNROLL
     for (int i = tid; i < a.headdim * 2 * a.dstate; i += NT) {
         const int p = i / (2 * a.dstate), f = i % (2 * a.dstate);
-        dst[p * NS + f] = src[i];
+        dst[p * NS + f] = BWDC_LDG(src + i);
     }
 }
 __host__ __device__ inline c2 sm2(const float *row, int k) { return c2{row[2 * k], row[2 * k + 1]}; }
@@ -269,7 +281,7 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     const c2 lam = ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c));
     for (int i = tid; i < QC; i += NT) {
         const int t = c * QC + i;
-        const float d = t < a.seqlen ? a.dt[ix_dt(a, b, t, h)] : 0.f;
+        const float d = t < a.seqlen ? BWDC_LDG(a.dt + ix_dt(a, b, t, h)) : 0.f;
         const c2 ac = ld2(acs_g + 2 * i);
         st2(m.acs + 2 * i, ac);
         st2(m.e + 2 * i, cexpc(ac));
