@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_state(bwdc::BwdArgs a) {
 }
 
 __global__ void __launch_bounds__(bwdc::NT) bwdc_state_fwd(bwdc::BwdArgs a) {
-    bwdc::k2_pass(a, blockIdx.x, blockIdx.y, threadIdx.x);
+    bwdc::k2_pass(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
 }
 
 __global__ void __launch_bounds__(bwdc::NT) bwdc_readout(bwdc::BwdArgs a) {
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_readout(bwdc::BwdArgs a) {
 }
 
 __global__ void __launch_bounds__(bwdc::NT) bwdc_state_bwd(bwdc::BwdArgs a) {
-    bwdc::k4_pass(a, blockIdx.x, blockIdx.y, threadIdx.x);
+    bwdc::k4_pass(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
 }
 
 __global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_grad(bwdc::BwdArgs a) {
@@ -128,9 +128,12 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_grad(bwdc::BwdArgs a) {
     __syncthreads();
     bwdc::k5_tokens(a, tid, m);
     __syncthreads();
-    bwdc::k5_decay(a, c, h, b, tid, m);
+    bwdc::k5_bc(a, c, h, b, tid, m);
     __syncthreads();
-    bwdc::k5_out(a, c, h, b, tid, m);
+    bwdc::k5_fk(a, tid, m);
+    __syncthreads();
+    bwdc::k5_decay(a, c, h, b, tid, m);
+    bwdc::k5_dx(a, c, h, b, tid, m);
 }
 
 __global__ void __launch_bounds__(bwdc::NT) bwdc_group_sum(bwdc::BwdArgs a, size_t total) {
@@ -143,17 +146,22 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_head_sum(bwdc::BwdArgs a) {
     if (h < a.nheads) bwdc::k6_head(a, h);
 }
 
-cudaError_t set_smem_attr(const void *const *fs, int nf, size_t bytes, bool (&done)[64]) {
+// The shared-memory opt-in is per function, device and CUDA context: done[dev]
+// holds the context it was last made in.
+cudaError_t set_smem_attr(const void *const *fs, int nf, size_t bytes, void *(&done)[64]) {
+    static std::mutex mu;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (done[dev]) return cudaSuccess;
+    std::lock_guard<std::mutex> lk(mu);
+    void *ctx = current_context();
+    if (ctx && done[dev] == ctx) return cudaSuccess;
     for (int i = 0; i < nf; ++i) {
         e = cudaFuncSetAttribute(fs[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
         if (e != cudaSuccess) return e;
     }
-    done[dev] = true;
+    done[dev] = ctx;
     return cudaSuccess;
 }
 
@@ -179,22 +187,23 @@ cudaError_t launch_scan_bwd_complex(const BwdCall &call, void *ws, cudaStream_t 
     a.nchunks = (call.seqlen + bwdc::QC - 1) / bwdc::QC;
     bwdc::carve(a, static_cast<float *>(ws));
 
-    static bool attr_set[64] = {false};  // the shared-memory opt-in is per function and per device
+    static void *attr_set[64] = {nullptr};
     const void *fs[3] = {(const void *)bwdc_chunk_state, (const void *)bwdc_readout, (const void *)bwdc_chunk_grad};
     cudaError_t e = set_smem_attr(fs, 3, SMEM_BYTES_C, attr_set);
     if (e != cudaSuccess) return e;
     const int nt = bwdc::NT;
+    const unsigned pn_blocks = (unsigned)(((size_t)a.headdim * a.dstate + nt - 1) / nt);
     if (a.batch > 0 && a.nchunks > 0) {
-        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(a.nheads, a.batch);
-        bwdc_chunk_state<<<gc, nt, SMEM_BYTES_C, st>>>(a);
+        const dim3 gc(a.nchunks, a.nheads, a.batch), gh(pn_blocks, a.nheads, a.batch);
+        bwdc_chunk_state<<<gc, nt, bwdc::SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
         bwdc_state_fwd<<<gh, nt, 0, st>>>(a);
-        bwdc_readout<<<gc, nt, SMEM_BYTES_C, st>>>(a);
+        bwdc_readout<<<gc, nt, bwdc::SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwdc_state_bwd<<<gh, nt, 0, st>>>(a);
         bwdc_chunk_grad<<<gc, nt, SMEM_BYTES_C, st>>>(a);
         const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;
         bwdc_group_sum<<<(unsigned)((total + nt - 1) / nt), nt, 0, st>>>(a, total);
     } else if (a.batch > 0) {  // empty sequences: dinit = dfinal (or zero)
-        bwdc_state_bwd<<<dim3(a.nheads, a.batch), nt, 0, st>>>(a);
+        bwdc_state_bwd<<<dim3(pn_blocks, a.nheads, a.batch), nt, 0, st>>>(a);
     }
     bwdc_head_sum<<<(a.nheads + nt - 1) / nt, nt, 0, st>>>(a);
     return cudaGetLastError();

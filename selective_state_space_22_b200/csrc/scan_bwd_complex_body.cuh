@@ -133,10 +133,14 @@ struct Smem {
     float *XY;                   // [QC][QS1]
     float *rowE, *colG, *F, *Ksr;  // [QC][2]
     float *red;                  // [3][RED]: <conj(Gh), h_in> re, im; dy.x
+    float *pF, *pK;              // [QC][NS]: per (token, state) terms of F and Ksr
     float *misc;                 // [4]: lam re, im
 };
 constexpr size_t SMEM_FLOATS = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS + 2 * P_MAX * NS + 2 * QC * QS2 +
-                               QC * QS1 + 4 * 2 * QC + 3 * RED + 4;
+                               QC * QS1 + 4 * 2 * QC + 3 * RED + 2 * QC * NS + 4;
+// The chunk-state phase uses the layout up to Bs, the readout phase up to Cs.
+constexpr size_t SMEM_FLOATS_K1 = QC + 3 * 2 * QC + 2 * QC * PS + QC * NS;
+constexpr size_t SMEM_FLOATS_K3 = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS;
 __host__ __device__ inline Smem smem_map(float *s) {
     Smem m;
     m.d = s; s += QC;
@@ -157,6 +161,8 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.F = s; s += 2 * QC;
     m.Ksr = s; s += 2 * QC;
     m.red = s; s += 3 * RED;
+    m.pF = s; s += QC * NS;
+    m.pK = s; s += QC * NS;
     m.misc = s;
     return m;
 }
@@ -211,7 +217,6 @@ __host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b,
         st2(m.acs + 2 * i, v);
         st2(acs_g + 2 * i, v);
     }
-    st2(m.misc, v);
     st2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c), v);
     for (int i = 0; i < QC; ++i) st2(m.w + 2 * i, cscale(cexpc(csub(v, ld2(m.acs + 2 * i))), m.d[i]));
 }
@@ -228,15 +233,15 @@ __host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, 
 }
 
 // ------------------------------------- 2: state entering each chunk (forward)
-__host__ __device__ inline void k2_pass(const BwdArgs &a, int h, int b, int tid) {
-    const size_t pn = (size_t)a.headdim * a.dstate;
-    for (size_t i = tid; i < pn; i += NT) {
-        c2 hv = a.init ? ld2(a.init + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
-        for (int c = 0; c < a.nchunks; ++c) {
-            const size_t o = 2 * (ix_pn(a, b, h, c) + i);
-            st2(a.hin + o, hv);
-            hv = cadd(cmul(cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c))), hv), ld2(a.st + o));
-        }
+// Element i = blk * NT + tid of the P x N state of (batch b, head h).
+__host__ __device__ inline void k2_pass(const BwdArgs &a, int blk, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
+    if (i >= pn) return;
+    c2 hv = a.init ? ld2(a.init + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
+    for (int c = 0; c < a.nchunks; ++c) {
+        const size_t o = 2 * (ix_pn(a, b, h, c) + i);
+        st2(a.hin + o, hv);
+        hv = cadd(cmul(cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c))), hv), ld2(a.st + o));
     }
 }
 
@@ -259,18 +264,17 @@ __host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int 
 }
 
 // --------------------- 4: gradient of the state leaving each chunk (backward)
-__host__ __device__ inline void k4_pass(const BwdArgs &a, int h, int b, int tid) {
-    const size_t pn = (size_t)a.headdim * a.dstate;
-    for (size_t i = tid; i < pn; i += NT) {
-        c2 gv = a.dfinal ? ld2(a.dfinal + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
-        for (int c = a.nchunks - 1; c >= 0; --c) {
-            const size_t o = 2 * (ix_pn(a, b, h, c) + i);
-            st2(a.gh + o, gv);
-            const c2 el = cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c)));
-            gv = cadd(cmul(cconj(el), gv), ld2(a.st + o));
-        }
-        if (a.dinit) st2(a.dinit + 2 * (ix_bh(a, b, h) * pn + i), gv);
+__host__ __device__ inline void k4_pass(const BwdArgs &a, int blk, int h, int b, int tid) {
+    const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
+    if (i >= pn) return;
+    c2 gv = a.dfinal ? ld2(a.dfinal + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
+    for (int c = a.nchunks - 1; c >= 0; --c) {
+        const size_t o = 2 * (ix_pn(a, b, h, c) + i);
+        st2(a.gh + o, gv);
+        const c2 el = cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c)));
+        gv = cadd(cmul(cconj(el), gv), ld2(a.st + o));
     }
+    if (a.dinit) st2(a.dinit + 2 * (ix_bh(a, b, h) * pn + i), gv);
 }
 
 // ------------------------------------------------ 5: gradients of one chunk
@@ -323,26 +327,7 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
         for (int l = 0; l < QC; ++l) cg = cadd(cg, cscale(ld2(m.GL + l * QS2 + 2 * t), m.XY[l * QS1 + t]));
         st2(m.rowE + 2 * t, re);
         st2(m.colG + 2 * t, cg);
-    } else if (tid < 2 * QC) {  // F[t] = e_t dy_t . (h_in C_t)
-        const int t = tid - QC;
-        c2 acc = cmk(0.f, 0.f);
-        for (int p = 0; p < a.headdim; ++p) {
-            c2 hc = cmk(0.f, 0.f);
-            for (int n = 0; n < a.dstate; ++n) hc = cadd(hc, cmul(sm2(m.Hin + p * NS, n), sm2(m.Cs + t * NS, n)));
-            acc = cadd(acc, cscale(hc, m.dY[t * PS + p]));
-        }
-        st2(m.F + 2 * t, cmul(ld2(m.e + 2 * t), acc));
-    } else if (tid < 3 * QC) {  // Ksr[t] = x_t . (conj(Gh) B_t)
-        const int t = tid - 2 * QC;
-        c2 acc = cmk(0.f, 0.f);
-        for (int p = 0; p < a.headdim; ++p) {
-            c2 gb = cmk(0.f, 0.f);
-            for (int n = 0; n < a.dstate; ++n)
-                gb = cadd(gb, cmul(cconj(sm2(m.Gh + p * NS, n)), sm2(m.Bs + t * NS, n)));
-            acc = cadd(acc, cscale(gb, m.X[t * PS + p]));
-        }
-        st2(m.Ksr + 2 * t, acc);
-    } else if (tid < 3 * QC + RED) {  // <conj(Gh), h_in> and dy . x, partial sums
+    } else if (tid >= 3 * QC && tid < 3 * QC + RED) {  // <conj(Gh), h_in> and dy . x, partial sums
         const int r = tid - 3 * QC;
         c2 h0 = cmk(0.f, 0.f);
         float dd = 0.f;
@@ -389,7 +374,42 @@ __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, 
     st2(a.dAp + 2 * (ix_bh(a, b, h) * a.nchunks + c), dAp);
     a.dDp[ix_bh(a, b, h) * a.nchunks + c] = dd;
 }
-__host__ __device__ inline void k5_out(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+// This head's dB and dC, and the per-(token, state) terms of F and Ksr:
+// F[t] = e_t dy_t . (h_in C_t) = e_t sum_n C_t[n] (dy_t h_in)[n] and
+// Ksr[t] = x_t . (conj(Gh) B_t) = sum_n B_t[n] conj((x_t Gh)[n]), from the same
+// dy_t h_in and x_t Gh that dC and dB use.
+__host__ __device__ inline void k5_bc(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    for (int i = tid; i < QC * a.dstate; i += NT) {
+        const int s = i / a.dstate, n = i % a.dstate, t = c * QC + s;
+        c2 db = cmk(0.f, 0.f), dc = cmk(0.f, 0.f), xg = cmk(0.f, 0.f), yh = cmk(0.f, 0.f);
+        for (int l = s; l < QC; ++l) db = cadd(db, cmul(ld2(m.K + l * QS2 + 2 * s), sm2(m.Cs + l * NS, n)));
+        for (int r = 0; r <= s; ++r) dc = cadd(dc, cmul(ld2(m.K + s * QS2 + 2 * r), sm2(m.Bs + r * NS, n)));
+        for (int p = 0; p < a.headdim; ++p) {
+            xg = cadd(xg, cscale(sm2(m.Gh + p * NS, n), m.X[s * PS + p]));
+            yh = cadd(yh, cscale(sm2(m.Hin + p * NS, n), m.dY[s * PS + p]));
+        }
+        st2(m.pF + s * NS + 2 * n, cmul(sm2(m.Cs + s * NS, n), yh));
+        st2(m.pK + s * NS + 2 * n, cmul(sm2(m.Bs + s * NS, n), cconj(xg)));
+        if (t >= a.seqlen) continue;
+        const size_t o = 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n);
+        st2(a.dBh + o, cadd(cconj(db), cmul(cconj(ld2(m.w + 2 * s)), xg)));
+        st2(a.dCh + o, cconj(cadd(dc, cmul(ld2(m.e + 2 * s), yh))));
+    }
+}
+// F and Ksr from their per-state terms (fixed order).
+__host__ __device__ inline void k5_fk(const BwdArgs &a, int tid, const Smem &m) {
+    if (tid < QC) {
+        c2 v = cmk(0.f, 0.f);
+        for (int n = 0; n < a.dstate; ++n) v = cadd(v, sm2(m.pF + tid * NS, n));
+        st2(m.F + 2 * tid, cmul(ld2(m.e + 2 * tid), v));
+    } else if (tid < 2 * QC) {
+        const int t = tid - QC;
+        c2 v = cmk(0.f, 0.f);
+        for (int n = 0; n < a.dstate; ++n) v = cadd(v, sm2(m.pK + t * NS, n));
+        st2(m.Ksr + 2 * t, v);
+    }
+}
+__host__ __device__ inline void k5_dx(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     const float Dh = a.D ? a.D[h] : 0.f;
     for (int i = tid; i < QC * a.headdim; i += NT) {
         const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
@@ -399,20 +419,6 @@ __host__ __device__ inline void k5_out(const BwdArgs &a, int c, int h, int b, in
         for (int l = s; l < QC; ++l) acc += ld2(m.GL + l * QS2 + 2 * s).re * m.dY[l * PS + p];
         for (int n = 0; n < a.dstate; ++n) gb = cadd(gb, cmul(cconj(sm2(m.Bs + s * NS, n)), sm2(m.Gh + p * NS, n)));
         a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * PS + p] + cmul(cconj(ld2(m.w + 2 * s)), gb).re;
-    }
-    for (int i = tid; i < QC * a.dstate; i += NT) {
-        const int s = i / a.dstate, n = i % a.dstate, t = c * QC + s;
-        if (t >= a.seqlen) continue;
-        c2 db = cmk(0.f, 0.f), dc = cmk(0.f, 0.f), xg = cmk(0.f, 0.f), yh = cmk(0.f, 0.f);
-        for (int l = s; l < QC; ++l) db = cadd(db, cmul(ld2(m.K + l * QS2 + 2 * s), sm2(m.Cs + l * NS, n)));
-        for (int r = 0; r <= s; ++r) dc = cadd(dc, cmul(ld2(m.K + s * QS2 + 2 * r), sm2(m.Bs + r * NS, n)));
-        for (int p = 0; p < a.headdim; ++p) {
-            xg = cadd(xg, cscale(sm2(m.Gh + p * NS, n), m.X[s * PS + p]));
-            yh = cadd(yh, cscale(sm2(m.Hin + p * NS, n), m.dY[s * PS + p]));
-        }
-        const size_t o = 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n);
-        st2(a.dBh + o, cadd(cconj(db), cmul(cconj(ld2(m.w + 2 * s)), xg)));
-        st2(a.dCh + o, cconj(cadd(dc, cmul(ld2(m.e + 2 * s), yh))));
     }
 }
 

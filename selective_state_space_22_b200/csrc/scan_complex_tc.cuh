@@ -28,17 +28,22 @@ constexpr int QT = 128;         // tokens per chunk (tcgen05 M)
 constexpr int NTH = 256;
 constexpr double SPAN = 140.0;  // |Re Lam| bound of the factored form
 
-// chunk scan: shared memory (1024-aligned tiles, 128-byte swizzled rows)
-constexpr int S_CH = 0, S_CL = 32768;       // C'  [128 l][128 k], hi and lo (two 64-column halves each)
-constexpr int S_BH = 65536, S_BL = 98304;   // B'  [128 s][128 k]
-constexpr int S_XH = 131072, S_XL = 147456; // X   [128 s][64 p]
-constexpr int S_HH = 163840, S_HL = 180224; // h'  [64 p][128 k] (two 8 KB halves)
-constexpr int S_MISC = 196608;
+// chunk scan: shared memory (1024-aligned tiles, 128-byte swizzled rows).  The
+// contraction over k = 2N runs in two halves of 64, so each operand tile holds
+// one half; X later reuses the C' tiles.  About 83 KB, so two CTAs share an SM.
+constexpr int S_CH = 0, S_CL = 16384;       // C'  [128 l][64 k], hi and lo
+constexpr int S_BH = 32768, S_BL = 49152;   // B'  [128 s][64 k]
+constexpr int S_HH = 65536, S_HL = 73728;   // h'  [64 p][64 k]
+constexpr int S_XH = 0, S_XL = 16384;       // X   [128 s][64 p], after the products have read C'
+constexpr int S_MISC = 81920;
 constexpr int SMEM_SCAN = S_MISC + QT * 16 + 64 + 1024;
-static_assert(SMEM_SCAN <= 232448, "shared memory");
-// chunk state: B'' [128 s][128 k] and X [128 s][64 p], hi and lo
-constexpr int A_BH = 0, A_BL = 32768, A_XH = 65536, A_XL = 81920, A_MISC = 98304;
+static_assert(2 * (SMEM_SCAN + 1024) <= 233472, "two CTAs per SM");
+// chunk state: B'' [64 s][128 k] and X [64 s][64 p], hi and lo: the contraction
+// over the chunk's tokens runs in two halves of 64, so four CTAs share an SM.
+constexpr int HT = 64;  // tokens per half
+constexpr int A_BH = 0, A_BL = 16384, A_XH = 32768, A_XL = 40960, A_MISC = 49152;
 constexpr int SMEM_STATE = A_MISC + QT * (16 + 4 + 8) + 64 + 1024;
+static_assert(4 * (SMEM_STATE + 1024) <= 233472, "four CTAs per SM");
 
 constexpr uint32_t IDESC_G = idesc_bf16_f32(128, 128, 0, 0);   // C' (K-major) x B' (K-major)
 constexpr uint32_t IDESC_H = idesc_bf16_f32(128, 64, 0, 0);    // C' (K-major) x h' (K-major)
@@ -108,7 +113,7 @@ __device__ void stage_x(uint8_t *sm, int off_hi, int off_lo, const ScanArgs &a, 
 }
 
 // ------------------------------------------------------------ chunk state
-template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanArgs a, CWs w, CplxView<T> v) {
+template <typename T> __global__ void __launch_bounds__(NTH, 4) state_kernel(ScanArgs a, CWs w, CplxView<T> v) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, H = a.nheads, P = a.headdim, N = a.dstate;
     const int g = h / (H / a.ngroups), t0 = c * QT, valid = min(QT, a.seqlen - t0);
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c, bt0 = (size_t)b * a.seqlen + t0;
@@ -121,7 +126,8 @@ template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanAr
     uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 2);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -142,41 +148,62 @@ template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanAr
         w.lam[bhc * 2] = R;
         w.lam[bhc * 2 + 1] = Th;
     }
-    __syncthreads();
-    // B''_s = w_s B_s as interleaved (re, im), rows s
-#pragma unroll 4
-    for (int it = 0; it < QT * 16 / NTH; ++it) {
-        const int u = tid + it * NTH, s = u >> 4, ch = u & 15;
-        float val[8];
-        cf bq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-        if (s < valid) view_cplx4(v, v.bre, v.bim, bt0 + s, g, 4 * ch, bq);
-        const float2 ws = wf[s];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const cf z = cmul(bq[q], cf{ws.x, ws.y});
-            val[2 * q] = z.re;
-            val[2 * q + 1] = z.im;
-        }
-        put8(sm, A_BH, A_BL, sw_off(s, ch, QT * 128), val);
-    }
-    stage_x(sm, A_XH, A_XL, a, v, bt0, h, valid);
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tslot, sb = smem_u32(sm);
-    if (tid == 0) {
 #pragma unroll 1
-        for (int pass = 0; pass < 3; ++pass) {  // hi.hi + hi.lo + lo.hi
-            const uint32_t aB = sb + (pass == 2 ? A_BL : A_BH), aX = sb + (pass == 1 ? A_XL : A_XH);
-#pragma unroll 1
-            for (int kk = 0; kk < 8; ++kk)
-                mma_ss(tmem, smem_desc_sw128(aB + kk * 2048, 16384, 1024), smem_desc_sw128(aX + kk * 2048, 8192, 1024),
-                       IDESC_S, pass > 0 || kk > 0);
+    for (int th = 0; th < 2; ++th) {  // tokens 64 th .. 64 th + 63
+        if (th == 1) {  // the first half's products have read the tiles
+            wait_bounded(&bar[0], 0, a.dev_error);
+            tc_fence_after();
         }
-        mma_commit(bar);
+        // B''_s = w_s B_s as interleaved (re, im), rows s
+#pragma unroll 4
+        for (int it = 0; it < HT * 16 / NTH; ++it) {
+            const int u = tid + it * NTH, sl = u >> 4, ch = u & 15, s = HT * th + sl;
+            float val[8];
+            cf bq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+            if (s < valid) view_cplx4(v, v.bre, v.bim, bt0 + s, g, 4 * ch, bq);
+            const float2 ws = wf[s];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const cf z = cmul(bq[q], cf{ws.x, ws.y});
+                val[2 * q] = z.re;
+                val[2 * q + 1] = z.im;
+            }
+            put8(sm, A_BH, A_BL, sw_off(sl, ch, HT * 128), val);
+        }
+        // X rows s as bf16 hi/lo
+#pragma unroll 2
+        for (int it = 0; it < HT * 8 / NTH; ++it) {
+            const int u = tid + it * NTH, sl = u >> 3, ch = u & 7, s = HT * th + sl;
+            float val[8];
+            if (s < valid) {
+                view_x8(v, bt0 + s, h, a.headdim, 8 * ch, val);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) val[e] = 0.f;
+            }
+            put8(sm, A_XH, A_XL, sw_off(sl, ch, HT * 128), val);
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
+#pragma unroll 1
+            for (int pass = 0; pass < 3; ++pass) {  // hi.hi + hi.lo + lo.hi
+                const uint32_t aB = sb + (pass == 2 ? A_BL : A_BH), aX = sb + (pass == 1 ? A_XL : A_XH);
+#pragma unroll 1
+                for (int kk = 0; kk < HT / 16; ++kk)
+                    mma_ss(tmem, smem_desc_sw128(aB + kk * 2048, HT * 128, 1024),
+                           smem_desc_sw128(aX + kk * 2048, HT * 128, 1024), IDESC_S, th > 0 || pass > 0 || kk > 0);
+            }
+            mma_commit(&bar[th]);
+        }
     }
-    wait_bounded(bar, 0, a.dev_error);
+    wait_bounded(&bar[1], 0, a.dev_error);
     tc_fence_after();
     {  // S[p][n] (complex) from TMEM lane k = 2n + (re, im), column p
         const int q = warp & 3, cb = 32 * (warp >> 2), k = 32 * q + lane;
@@ -192,8 +219,10 @@ template <typename T> __global__ void __launch_bounds__(NTH) state_kernel(ScanAr
 }
 
 // -------------------------------------------------------------- chunk scan
+// TMEM (256 columns, so two CTAs share an SM): G in 0..127, overwritten in place
+// by M's hi part (bf16 pairs, 0..63); y in 128..191; M's lo part in 192..255.
 template <typename T>
-__global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxView<T> v) {
+__global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxView<T> v) {
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, H = a.nheads, P = a.headdim, N = a.dstate;
     const int g = h / (H / a.ngroups), t0 = c * QT, valid = min(QT, a.seqlen - t0);
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c, bt0 = (size_t)b * a.seqlen + t0;
@@ -206,15 +235,14 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
     }
     float2 *fC = reinterpret_cast<float2 *>(sm + S_MISC), *fB = fC + QT;
     uint64_t *bars = reinterpret_cast<uint64_t *>(fB + QT);
-    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 2);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + 3);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        mbar_init(&bars[0], 1);
-        mbar_init(&bars[1], 1);
+        for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(tslot, 512);
+        tmem_alloc(tslot, 256);
         tmem_relinquish();
     }
     const double rho = 0.5 * Rr;
@@ -227,76 +255,86 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
         fC[s] = make_float2(ec * (float)cn, ec * (float)sn);
         fB[s] = make_float2(eb * (float)cn, -eb * (float)sn);
     }
+    tc_fence_before();
     __syncthreads();
-    // C' as (re, -im) and B' as (re, im), rows = tokens, 4 complex states per chunk of 8
-#pragma unroll 4
-    for (int it = 0; it < QT * 16 / NTH; ++it) {
-        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
-        float vc[8], vb[8];
-        const float2 fc = fC[r], fb = fB[r];
-        cf cq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}}, bq[4] = {cq[0], cq[1], cq[2], cq[3]};
-        if (r < valid) {
-            view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq);
-            view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq);
+    tc_fence_after();
+    const uint32_t tm = *tslot, sb = smem_u32(sm);
+    constexpr uint32_t COL_Y = 128, COL_MH = 0, COL_ML = 192;
+    const float er = (float)exp(rho);
+    const float *hin = reinterpret_cast<const float *>(w.S + bhc * (size_t)P * N);
+    bool ok = true;
+#pragma unroll 1
+    for (int kh = 0; kh < 2; ++kh) {  // k = 64 kh .. 64 kh + 63: complex states 32 kh .. 32 kh + 31
+        if (kh == 1) {  // the first half's products have read the tiles
+            ok = wait_bounded(&bars[0], 0, a.dev_error) && ok;
+            tc_fence_after();
         }
+        // C' as (re, -im) and B' as (re, im), rows = tokens, 4 complex states per chunk of 8
+#pragma unroll 4
+        for (int it = 0; it < QT * 8 / NTH; ++it) {
+            const int u = tid + it * NTH, r = u >> 3, cl = u & 7, ch = 8 * kh + cl;
+            float vc[8], vb[8];
+            const float2 fc = fC[r], fb = fB[r];
+            cf cq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}}, bq[4] = {cq[0], cq[1], cq[2], cq[3]};
+            if (r < valid) {
+                view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq);
+                view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq);
+            }
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const cf zc = cmul(cq[q], cf{fc.x, fc.y}), zb = cmul(bq[q], cf{fb.x, fb.y});
-            vc[2 * q] = zc.re;
-            vc[2 * q + 1] = -zc.im;
-            vb[2 * q] = zb.re;
-            vb[2 * q + 1] = zb.im;
+            for (int q = 0; q < 4; ++q) {
+                const cf zc = cmul(cq[q], cf{fc.x, fc.y}), zb = cmul(bq[q], cf{fb.x, fb.y});
+                vc[2 * q] = zc.re;
+                vc[2 * q + 1] = -zc.im;
+                vb[2 * q] = zb.re;
+                vb[2 * q + 1] = zb.im;
+            }
+            const uint32_t o = sw_off(r, cl, QT * 128);
+            put8(sm, S_CH, S_CL, o, vc);
+            put8(sm, S_BH, S_BL, o, vb);
         }
-        const uint32_t o = sw_off(r, ch, QT * 128);
-        put8(sm, S_CH, S_CL, o, vc);
-        put8(sm, S_BH, S_BL, o, vb);
-    }
-    stage_x(sm, S_XH, S_XL, a, v, bt0, h, valid);
-    {  // h' = exp(rho) h_in as (re, im), rows p
-        const float er = (float)exp(rho);
-        const float *hin = reinterpret_cast<const float *>(w.S + bhc * (size_t)P * N);
-#pragma unroll 4
-        for (int it = 0; it < 64 * 16 / NTH; ++it) {  // h_in was written by earlier launches: read-only here
-            const int u = tid + it * NTH, p = u >> 4, ch = u & 15;
+        // h' = exp(rho) h_in as (re, im), rows p (h_in was written by earlier launches: read-only here)
+#pragma unroll 2
+        for (int it = 0; it < 64 * 8 / NTH; ++it) {
+            const int u = tid + it * NTH, p = u >> 3, cl = u & 7, ch = 8 * kh + cl;
             float val[8];
             const float4 h0 = __ldg(reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2));
             const float4 h1 = __ldg(reinterpret_cast<const float4 *>(hin + ((size_t)p * N + 4 * ch) * 2 + 4));
             val[0] = er * h0.x, val[1] = er * h0.y, val[2] = er * h0.z, val[3] = er * h0.w;
             val[4] = er * h1.x, val[5] = er * h1.y, val[6] = er * h1.z, val[7] = er * h1.w;
-            put8(sm, S_HH, S_HL, sw_off(p, ch, 64 * 128), val);
+            put8(sm, S_HH, S_HL, sw_off(p, cl, 64 * 128), val);
         }
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tm = *tslot, sb = smem_u32(sm);
-    constexpr uint32_t COL_Y = 128, COL_MH = 256, COL_ML = 320;
-    if (tid == 0) {
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0) {
 #pragma unroll 1
-        for (int pass = 0; pass < 3; ++pass) {  // G = C' B'^T and y = C' h'^T, hi.hi + hi.lo + lo.hi
-            const uint32_t aC = sb + (pass == 2 ? S_CL : S_CH), aB = sb + (pass == 1 ? S_BL : S_BH);
-            const uint32_t aH = sb + (pass == 1 ? S_HL : S_HH);
+            for (int pass = 0; pass < 3; ++pass) {  // G = C' B'^T and y = C' h'^T, hi.hi + hi.lo + lo.hi
+                const uint32_t aC = sb + (pass == 2 ? S_CL : S_CH), aB = sb + (pass == 1 ? S_BL : S_BH);
+                const uint32_t aH = sb + (pass == 1 ? S_HL : S_HH);
 #pragma unroll 1
-            for (int kk = 0; kk < 8; ++kk) {
-                const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-                mma_ss(tm, smem_desc_sw128(aC + off, 16, 1024), smem_desc_sw128(aB + off, 16, 1024), IDESC_G,
-                       pass > 0 || kk > 0);
-                mma_ss(tm + COL_Y, smem_desc_sw128(aC + off, 16, 1024),
-                       smem_desc_sw128(aH + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), IDESC_H, pass > 0 || kk > 0);
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint32_t acc = kh > 0 || pass > 0 || kk > 0;
+                    mma_ss(tm, smem_desc_sw128(aC + 32 * kk, 16, 1024), smem_desc_sw128(aB + 32 * kk, 16, 1024),
+                           IDESC_G, acc);
+                    mma_ss(tm + COL_Y, smem_desc_sw128(aC + 32 * kk, 16, 1024),
+                           smem_desc_sw128(aH + 32 * kk, 16, 1024), IDESC_H, acc);
+                }
             }
+            mma_commit(&bars[kh]);
         }
-        mma_commit(&bars[0]);
     }
-    bool ok = wait_bounded(&bars[0], 0, a.dev_error);
+    ok = wait_bounded(&bars[1], 0, a.dev_error) && ok;  // every product of both halves is done
     tc_fence_after();
-    {  // M = the masked product + D on the diagonal, split into hi and lo, in TMEM
-        const int q = warp & 3, hf = warp >> 2;
+    if (warp < 4) {
+        // M = the masked product + D on the diagonal, split into hi and lo, by the warp
+        // of the rows' lane quadrant, blocks in order: M's hi block j lands on G
+        // columns this thread has already read.
+        const int q = warp;
         const uint32_t lo_ = (uint32_t)(32 * q) << 16;
         const float Dh = a.D ? a.D[h] : 0.f;
 #pragma unroll 1
-        for (int jj = 0; jj < 2; ++jj) {
-            const int j = 2 * hf + jj;
+        for (int j = 0; j < 4; ++j) {
             uint32_t ph[16], pl[16];
             if (j > q) {
 #pragma unroll
@@ -321,6 +359,21 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
             tmem_st16(tm + lo_ + COL_ML + 16 * j, pl);
         }
         tmem_wait_st();
+    } else {
+        // X of the chunk as bf16 hi/lo rows [s][p], into the C' tiles
+#pragma unroll 4
+        for (int it = 0; it < QT * 8 / (NTH - 128); ++it) {
+            const int u = (tid - 128) + it * (NTH - 128), s = u >> 3, ch = u & 7;
+            float val[8];
+            if (s < valid) {
+                view_x8(v, bt0 + s, h, a.headdim, 8 * ch, val);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) val[e] = 0.f;
+            }
+            put8(sm, S_XH, S_XL, sw_off(s, ch, QT * 128), val);
+        }
+        fence_proxy_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -335,9 +388,9 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
                     mma_ts(tm + COL_Y, aM + 8 * kk, smem_desc_sw128(aX + kk * 2048, 8192, 1024), IDESC_MX, 1);
             }
         }
-        mma_commit(&bars[1]);
+        mma_commit(&bars[2]);
     }
-    wait_bounded(&bars[1], 0, a.dev_error);
+    wait_bounded(&bars[2], 0, a.dev_error);
     tc_fence_after();
     {  // y rows: lane quadrant (warp & 3), columns 32 (warp >> 2) ..
         const int q = warp & 3, cb = 32 * (warp >> 2), l = 32 * q + lane;
@@ -353,7 +406,7 @@ __global__ void __launch_bounds__(NTH, 1) scan_kernel(ScanArgs a, CWs w, CplxVie
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tm, 512);
+    if (warp == 0) tmem_dealloc(tm, 256);
 }
 
 }  // namespace ctc

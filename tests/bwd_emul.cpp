@@ -105,31 +105,36 @@ extern "C" int emulate_scan_bwd_complex(const float *x, const float *dt, const f
     std::vector<float> ws(ws_floats(batch, seqlen, nheads, headdim, dstate, a.nchunks) + 4,
                           std::numeric_limits<float>::quiet_NaN());
     carve(a, ws.data());
-    std::vector<float> sm(SMEM_FLOATS);
-    const Smem m = smem_map(sm.data());
-    auto fresh = [&] { std::fill(sm.begin(), sm.end(), std::numeric_limits<float>::quiet_NaN()); };
+    std::vector<float> sm(SMEM_FLOATS), sm1(SMEM_FLOATS_K1), sm3(SMEM_FLOATS_K3);
+    const Smem m = smem_map(sm.data()), m1 = smem_map(sm1.data()), m3 = smem_map(sm3.data());
+    auto fresh = [&] {
+        for (auto *v : {&sm, &sm1, &sm3}) std::fill(v->begin(), v->end(), std::numeric_limits<float>::quiet_NaN());
+    };
     auto each = [&](auto &&f) { for (int tid = 0; tid < NT; ++tid) f(tid); };
+    const int pn_blocks = (headdim * dstate + NT - 1) / NT;
 
     if (batch > 0 && a.nchunks > 0) {
         for (int b = 0; b < batch; ++b)
             for (int h = 0; h < nheads; ++h)
                 for (int c = 0; c < a.nchunks; ++c) {
                     fresh();
-                    each([&](int t) { k1_load(a, c, h, b, t, m); });
-                    each([&](int t) { k1_cumsum(a, c, h, b, t, m); });
-                    each([&](int t) { k1_state(a, c, h, b, t, m); });
+                    each([&](int t) { k1_load(a, c, h, b, t, m1); });
+                    each([&](int t) { k1_cumsum(a, c, h, b, t, m1); });
+                    each([&](int t) { k1_state(a, c, h, b, t, m1); });
                 }
         for (int b = 0; b < batch; ++b)
-            for (int h = 0; h < nheads; ++h) each([&](int t) { k2_pass(a, h, b, t); });
+            for (int h = 0; h < nheads; ++h)
+                for (int blk = 0; blk < pn_blocks; ++blk) each([&](int t) { k2_pass(a, blk, h, b, t); });
         for (int b = 0; b < batch; ++b)
             for (int h = 0; h < nheads; ++h)
                 for (int c = 0; c < a.nchunks; ++c) {
                     fresh();
-                    each([&](int t) { k3_load(a, c, h, b, t, m); });
-                    each([&](int t) { k3_r(a, c, h, b, t, m); });
+                    each([&](int t) { k3_load(a, c, h, b, t, m3); });
+                    each([&](int t) { k3_r(a, c, h, b, t, m3); });
                 }
         for (int b = 0; b < batch; ++b)
-            for (int h = 0; h < nheads; ++h) each([&](int t) { k4_pass(a, h, b, t); });
+            for (int h = 0; h < nheads; ++h)
+                for (int blk = 0; blk < pn_blocks; ++blk) each([&](int t) { k4_pass(a, blk, h, b, t); });
         for (int b = 0; b < batch; ++b)
             for (int h = 0; h < nheads; ++h)
                 for (int c = 0; c < a.nchunks; ++c) {
@@ -137,14 +142,19 @@ extern "C" int emulate_scan_bwd_complex(const float *x, const float *dt, const f
                     each([&](int t) { k5_load(a, c, h, b, t, m); });
                     each([&](int t) { k5_mats(a, t, m); });
                     each([&](int t) { k5_tokens(a, t, m); });
-                    each([&](int t) { k5_decay(a, c, h, b, t, m); });
-                    each([&](int t) { k5_out(a, c, h, b, t, m); });
+                    each([&](int t) { k5_bc(a, c, h, b, t, m); });
+                    each([&](int t) { k5_fk(a, t, m); });
+                    each([&](int t) {
+                        k5_decay(a, c, h, b, t, m);
+                        k5_dx(a, c, h, b, t, m);
+                    });
                 }
         const size_t total = (size_t)batch * seqlen * ngroups * dstate;
         for (size_t i = 0; i < total; ++i) k6_group(a, i);
     } else if (batch > 0) {
         for (int b = 0; b < batch; ++b)
-            for (int h = 0; h < nheads; ++h) each([&](int t) { k4_pass(a, h, b, t); });
+            for (int h = 0; h < nheads; ++h)
+                for (int blk = 0; blk < pn_blocks; ++blk) each([&](int t) { k4_pass(a, blk, h, b, t); });
     }
     for (int h = 0; h < nheads; ++h) k6_head(a, h);
     return 0;
