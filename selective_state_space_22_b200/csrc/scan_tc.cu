@@ -167,15 +167,18 @@ __device__ __forceinline__ unsigned long long now_ns() {
 
 // Bounded wait on an mbarrier phase.  Returns false, without waiting further,
 // once the CTA's abort word is set; a wait that runs out sets the device error
-// word and the abort word.  After an abort, the single-thread roles (the TMA
-// producer and the MMA issuers) leave their tile loops and wait for the loads
-// and MMAs they issued; the warpgroup roles run their remaining tiles with every
-// wait falling through (their TMEM and shared-memory accesses stay in bounds and
-// their named barriers stay matched; the outputs are invalid and reported so).
-// They arrive only on barriers of their own warpgroup, so no phase count is
-// overrun.  Only the first probe is inlined; the polling loop, which looks at
-// the abort word once a wait has lasted 20 us, is one out-of-line copy, so that
-// the many wait sites of the hot loops stay small.
+// word and the abort word.  After an abort the TMA producer stops at its first
+// failed wait; every other role runs its remaining tiles with each wait giving
+// up after 20 us (so the kernel ends within milliseconds),
+// its shared-memory and TMEM accesses in bounds and its named barriers matched;
+// the outputs are invalid and reported so.  Arrivals that then come early (MMA
+// commits, warpgroup arrivals: plain counts, no transaction bytes) only complete
+// barrier phases early.  At the end the TMA
+// producer waits (bounded) for the last load of every slot and each MMA issuer
+// for a commit of everything it issued, so nothing is in flight when the CTA
+// frees TMEM and exits.  Only the first probe is inlined; the polling loop,
+// which looks at the abort word once a wait has lasted 20 us, is one
+// out-of-line copy, so that the many wait sites of the hot loops stay small.
 __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_s, int *err,
                                             unsigned long long limit) {
     const unsigned long long t0 = now_ns();
@@ -340,7 +343,10 @@ __global__ void __launch_bounds__(NTH, 1)
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0 && !p.withhold) {
-            int last_cb[2] = {-1, -1}, last_x[X_SLOTS] = {-1, -1, -1};  // last tile loaded per slot
+            // After an abort the producer stops issuing at its first failed wait, so
+            // that a slot is never reloaded while its last load is in flight; ncb
+            // and nx count the {C, B} and X loads issued (tiles 0 .. n - 1).
+            int ncb = 0, nx = 0;
             for (int k = 0; k < ntl; ++k) {
                 const Tile t = decode_tile(p, k);
                 const int s = k & 1;
@@ -354,19 +360,25 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 tma_load_4d(st + OFF_B, &tm_b, full, 0, t.g, t.t0, t.b);
                 tma_load_4d(st + OFF_B + 16384, &tm_b, full, 64, t.g, t.t0, t.b);
-                last_cb[s] = k;
+                ncb = k + 1;
                 const int xs = k % X_SLOTS;
                 if (!mbar_wait(&bars[B_XEMPTY + xs], ((k / X_SLOTS) & 1) ^ 1, p, abort_s)) break;
                 mbar_arrive_expect_tx(&bars[B_XFULL + xs], LOAD_X);
                 tma_load_4d(sm + OFF_XR + xs * 16384, &tm_x, &bars[B_XFULL + xs], 0, t.h, t.t0, t.b);
-                last_x[xs] = k;
+                nx = k + 1;
             }
             // Every load issued must have landed before the CTA's shared memory
             // is released (after an abort its consumer may never have waited).
-            for (int s = 0; s < 2; ++s)
-                if (last_cb[s] >= 0) mbar_wait_drain(&bars[B_FULL + s], (last_cb[s] >> 1) & 1, p, abort_s);
+            for (int s = 0; s < 2; ++s)  // the last tile loaded into each slot
+                if (ncb - 1 >= s) {
+                    const int kl = ncb - 1 - ((ncb - 1 - s) & 1);
+                    mbar_wait_drain(&bars[B_FULL + s], (kl >> 1) & 1, p, abort_s);
+                }
             for (int xs = 0; xs < X_SLOTS; ++xs)
-                if (last_x[xs] >= 0) mbar_wait_drain(&bars[B_XFULL + xs], (last_x[xs] / X_SLOTS) & 1, p, abort_s);
+                if (nx - 1 >= xs) {
+                    const int kl = nx - 1 - (nx - 1 - xs) % X_SLOTS;
+                    mbar_wait_drain(&bars[B_XFULL + xs], (kl / X_SLOTS) & 1, p, abort_s);
+                }
         }
     } else if (warp == 1) {
         // ------------------------------------------- MMA issuer: G and S
@@ -377,8 +389,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * CB_BYTES + OFF_C, aB = sbase + s * CB_BYTES + OFF_B;
-                if (!mbar_wait(&bars[B_FULL + s], par, p, abort_s)) break;
-                if (!mbar_wait(&bars[B_FREE + s], par ^ 1, p, abort_s)) break;
+                mbar_wait(&bars[B_FULL + s], par, p, abort_s);
+                mbar_wait(&bars[B_FREE + s], par ^ 1, p, abort_s);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -389,9 +401,9 @@ __global__ void __launch_bounds__(NTH, 1)
                     }
                 }
                 mma_commit(&bars[B_G + s]);
-                if (!mbar_wait(&bars[B_W + s], par, p, abort_s)) break;
+                mbar_wait(&bars[B_W + s], par, p, abort_s);
                 // S's columns held the chunk state of tile k-2 until its state update
-                if (k >= 2 && !mbar_wait(&bars[B_H + s], par ^ 1, p, abort_s)) break;
+                if (k >= 2) mbar_wait(&bars[B_H + s], par ^ 1, p, abort_s);
                 tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)  // S = B^T W
@@ -416,8 +428,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 const uint32_t aH = sbase + OFF_H;
                 // G of this tile was issued after tile k-2's epilogue released the
                 // set, so C h^T's columns are free; h_in^T of this tile is written.
-                if (!mbar_wait(&bars[B_G + s], par, p, abort_s)) break;
-                if (!mbar_wait(&bars[B_HW + s], par, p, abort_s)) break;
+                mbar_wait(&bars[B_G + s], par, p, abort_s);
+                mbar_wait(&bars[B_HW + s], par, p, abort_s);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
@@ -427,8 +439,8 @@ __global__ void __launch_bounds__(NTH, 1)
                 }
                 mma_commit(&bars[B_YO + s]);     // done with the h_in^T buffer
                 mma_commit(&bars[B_EMPTY + s]);  // with G and S: done with the {C, B} slot
-                if (!mbar_wait(&bars[B_M + s], par, p, abort_s)) break;
-                if (!mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s)) break;
+                mbar_wait(&bars[B_M + s], par, p, abort_s);
+                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s);
                 tc_fence_after();
                 if (!so) {
 #pragma unroll 1
