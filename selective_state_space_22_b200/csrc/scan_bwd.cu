@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_chunk_state(bwdc::BwdArgs a) {
     __syncthreads();
     bwdc::k1_cumsum(a, c, h, b, tid, m);
     __syncthreads();
+    bwdc::k1_scale(a, tid, m);
+    __syncthreads();
     bwdc::k1_state(a, c, h, b, tid, m);
 }
 
@@ -110,6 +112,8 @@ __global__ void __launch_bounds__(bwdc::NT) bwdc_readout(bwdc::BwdArgs a) {
     const bwdc::Smem m = bwdc::smem_map(sm);
     const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
     bwdc::k3_load(a, c, h, b, tid, m);
+    __syncthreads();
+    bwdc::k3_scale(a, tid, m);
     __syncthreads();
     bwdc::k3_r(a, c, h, b, tid, m);
 }

@@ -16,11 +16,15 @@
 //   dalpha = reverse cumulative sum of dacs;  ddt += Re(conj(dalpha) A);  dA += sum dt dalpha.
 // (C_l.B_s = sum_n C_l[n] B_s[n], no conjugate, as in the forward readout.)  The
 // chunk is 32 tokens so that the complex tiles fit in shared memory.  As in the
-// real variant, every phase is a __host__ __device__ function of (block, thread).
+// real variant, every phase is a __host__ __device__ function of (block, thread),
+// and the products are register-tiled: 256 threads as a 16 x 16 grid, each with
+// a tile of 2 x 2 to 4 x 4 complex results, operands read from shared memory as
+// 16-byte vectors (two complex values), rows strided 4 mod 32 words.
 #pragma once
 
 #include <math.h>
 #include <stddef.h>
+#include <stdint.h>
 
 #ifndef __CUDACC__
 #define __host__
@@ -44,8 +48,9 @@ constexpr int NT = 256;       // threads per block
 constexpr int P_MAX = 64;     // head dim
 constexpr int N_MAX = 64;     // complex state dim
 constexpr int RED = 64;       // threads of the block reductions
-// Row strides in floats, odd so that lanes walking down a column spread over banks.
-constexpr int PS = P_MAX + 1, NS = 2 * N_MAX + 1, QS2 = 2 * QC + 1, QS1 = QC + 1;
+// Row strides in floats: 4 more than a row, so rows stay 16-byte aligned and
+// consecutive rows start 4 banks apart.
+constexpr int PS = P_MAX + 4, NS = 2 * N_MAX + 4, QS2 = 2 * QC + 4, QS1 = QC + 4;
 
 struct c2 {
     float re, im;
@@ -123,6 +128,7 @@ __host__ __device__ inline size_t ix_pn(const BwdArgs &a, int b, int h, int c) {
 __host__ __device__ inline int group_of(const BwdArgs &a, int h) { return h / (a.nheads / a.ngroups); }
 
 // ------------------------------------------------ shared-memory layout
+// Arrays are zero beyond headdim / dstate, so the products run over P_MAX, N_MAX.
 struct Smem {
     float *d;                    // [QC]
     float *acs, *e, *w;          // [QC][2]
@@ -133,11 +139,11 @@ struct Smem {
     float *XY;                   // [QC][QS1]
     float *rowE, *colG, *F, *Ksr;  // [QC][2]
     float *red;                  // [3][RED]: <conj(Gh), h_in> re, im; dy.x
-    float *pF, *pK;              // [QC][NS]: per (token, state) terms of F and Ksr
+    float *part;                 // [2][QC][16][2]: per-thread-column terms of Ksr and F
     float *misc;                 // [4]: lam re, im
 };
 constexpr size_t SMEM_FLOATS = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS + 2 * P_MAX * NS + 2 * QC * QS2 +
-                               QC * QS1 + 4 * 2 * QC + 3 * RED + 2 * QC * NS + 4;
+                               QC * QS1 + 4 * 2 * QC + 3 * RED + 2 * QC * 16 * 2 + 4;
 // The chunk-state phase uses the layout up to Bs, the readout phase up to Cs.
 constexpr size_t SMEM_FLOATS_K1 = QC + 3 * 2 * QC + 2 * QC * PS + QC * NS;
 constexpr size_t SMEM_FLOATS_K3 = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS;
@@ -161,8 +167,7 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.F = s; s += 2 * QC;
     m.Ksr = s; s += 2 * QC;
     m.red = s; s += 3 * RED;
-    m.pF = s; s += QC * NS;
-    m.pK = s; s += QC * NS;
+    m.part = s; s += 2 * QC * 16 * 2;
     m.misc = s;
     return m;
 }
@@ -177,29 +182,83 @@ __host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, i
 __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
                                             float *dst) {
     BWDC_UNROLL
-    for (int i = tid; i < QC * a.headdim; i += NT) {
-        const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
-        dst[s * PS + p] = t < a.seqlen ? BWDC_LDG(src + ix_x(a, b, t, h, p)) : 0.f;
+    for (int i = tid; i < QC * P_MAX; i += NT) {
+        const int s = i / P_MAX, p = i % P_MAX, t = c * QC + s;
+        dst[s * PS + p] = (t < a.seqlen && p < a.headdim) ? BWDC_LDG(src + ix_x(a, b, t, h, p)) : 0.f;
     }
 }
 // complex rows of B or C: [QC][N] pairs
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
     BWDC_UNROLL
-    for (int i = tid; i < QC * 2 * a.dstate; i += NT) {
-        const int s = i / (2 * a.dstate), f = i % (2 * a.dstate), t = c * QC + s;
-        dst[s * NS + f] = t < a.seqlen ? BWDC_LDG(src + 2 * ix_bc(a, b, t, g, 0) + f) : 0.f;
+    for (int i = tid; i < QC * 2 * N_MAX; i += NT) {
+        const int s = i / (2 * N_MAX), f = i % (2 * N_MAX), t = c * QC + s;
+        dst[s * NS + f] = (t < a.seqlen && f < 2 * a.dstate) ? BWDC_LDG(src + 2 * ix_bc(a, b, t, g, 0) + f) : 0.f;
     }
 }
 // a complex [P][N] block
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
     BWDC_UNROLL
-    for (int i = tid; i < a.headdim * 2 * a.dstate; i += NT) {
-        const int p = i / (2 * a.dstate), f = i % (2 * a.dstate);
-        dst[p * NS + f] = BWDC_LDG(src + i);
+    for (int i = tid; i < P_MAX * 2 * N_MAX; i += NT) {
+        const int p = i / (2 * N_MAX), f = i % (2 * N_MAX);
+        dst[p * NS + f] = (p < a.headdim && f < 2 * a.dstate) ? BWDC_LDG(src + (size_t)p * 2 * a.dstate + f) : 0.f;
     }
 }
 __host__ __device__ inline c2 sm2(const float *row, int k) { return c2{row[2 * k], row[2 * k + 1]}; }
+
+// --------------------------------------------------- register tiles
+struct alignas(16) f4 {
+    float x, y, z, w;
+};
+__host__ __device__ inline f4 ld4(const float *p) { return *reinterpret_cast<const f4 *>(p); }
+__host__ __device__ inline float comp(const f4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+// The complex columns of a thread's "n" tile: n(j) = 2 tc + (j & 1) + 32 (j >> 1),
+// at float offset 4 tc + 2 (j & 1) + 64 (j >> 1) of a row.
+__host__ __device__ inline int ncol(int tc, int j) { return 2 * tc + (j & 1) + 32 * (j >> 1); }
+// acc[i][j] += a * v[j] for one real a and the four complex values of a row at
+// float offsets 4 tc and 64 + 4 tc.
+__host__ __device__ inline void axpy4(c2 (&acc)[4], float a, const float *row, int tc) {
+    const f4 u = ld4(row + 4 * tc), v = ld4(row + 64 + 4 * tc);
+    acc[0].re = fmaf(a, u.x, acc[0].re), acc[0].im = fmaf(a, u.y, acc[0].im);
+    acc[1].re = fmaf(a, u.z, acc[1].re), acc[1].im = fmaf(a, u.w, acc[1].im);
+    acc[2].re = fmaf(a, v.x, acc[2].re), acc[2].im = fmaf(a, v.y, acc[2].im);
+    acc[3].re = fmaf(a, v.z, acc[3].re), acc[3].im = fmaf(a, v.w, acc[3].im);
+}
+// acc[j] += z * row[n(j)] for a complex z (no conjugate).
+__host__ __device__ inline void czpy4(c2 (&acc)[4], c2 z, const float *row, int tc) {
+    const f4 u = ld4(row + 4 * tc), v = ld4(row + 64 + 4 * tc);
+    const c2 r[4] = {c2{u.x, u.y}, c2{u.z, u.w}, c2{v.x, v.y}, c2{v.z, v.w}};
+    for (int j = 0; j < 4; ++j) acc[j] = cadd(acc[j], cmul(z, r[j]));
+}
+// Complex values n = 2 tc .. 2 tc + 1 and 2 tc + 32 .. 33 of a row (acc[0..3]) to a
+// global row of `valid` complex values, 16 bytes at a time where aligned.
+__host__ __device__ inline void store_n4(float *row, int tc, int valid, const c2 (&v)[4]) {
+    for (int q = 0; q < 2; ++q) {
+        const int n = 2 * tc + 32 * q;
+        float *dst = row + 2 * n;
+        if (n + 1 < valid && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+            *reinterpret_cast<f4 *>(dst) = f4{v[2 * q].re, v[2 * q].im, v[2 * q + 1].re, v[2 * q + 1].im};
+        } else {
+            if (n < valid) st2(dst, v[2 * q]);
+            if (n + 1 < valid) st2(dst + 2, v[2 * q + 1]);
+        }
+    }
+}
+// out[p][n] = sum_k A[k][p] M[k][n] over k < QC for rows p = 4 tr .. 4 tr + 3 (A real,
+// [QC][PS]) and the thread's four complex columns (M [QC][NS]), stored to a
+// complex P x N array.
+__host__ __device__ inline void tn_pn(const BwdArgs &a, const float *A, const float *M, float *dst, int tid) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    c2 acc[4][4];
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 4; ++j) acc[i][j] = cmk(0.f, 0.f);
+    for (int k = 0; k < QC; ++k) {
+        const f4 av = ld4(A + k * PS + r0);
+        for (int i = 0; i < 4; ++i) axpy4(acc[i], comp(av, i), M + k * NS, tc);
+    }
+    for (int i = 0; i < 4; ++i)
+        if (r0 + i < a.headdim) store_n4(dst + 2 * (size_t)(r0 + i) * a.dstate, tc, a.dstate, acc[i]);
+}
 
 // ---------------------------------------------- 1: chunk states (forward)
 __host__ __device__ inline void k1_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
@@ -220,16 +279,17 @@ __host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b,
     st2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c), v);
     for (int i = 0; i < QC; ++i) st2(m.w + 2 * i, cscale(cexpc(csub(v, ld2(m.acs + 2 * i))), m.d[i]));
 }
-// S[p][n] = sum_s w_s x_s[p] B_s[n]
-__host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
-    float *S = a.st + 2 * ix_pn(a, b, h, c);
-    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
-        const int p = i / a.dstate, n = i % a.dstate;
-        c2 acc = cmk(0.f, 0.f);
-        for (int s = 0; s < QC; ++s)
-            acc = cadd(acc, cscale(cmul(ld2(m.w + 2 * s), sm2(m.Bs + s * NS, n)), m.X[s * PS + p]));
-        st2(S + 2 * i, acc);
+// B_s <- w_s B_s in place
+__host__ __device__ inline void k1_scale(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    for (int i = tid; i < QC * N_MAX; i += NT) {
+        const int s = i / N_MAX, n = i % N_MAX;
+        st2(m.Bs + s * NS + 2 * n, cmul(ld2(m.w + 2 * s), sm2(m.Bs + s * NS, n)));
     }
+}
+// S[p][n] = sum_s x_s[p] (w_s B_s[n])
+__host__ __device__ inline void k1_state(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    tn_pn(a, m.X, m.Bs, a.st + 2 * ix_pn(a, b, h, c), tid);
 }
 
 // ------------------------------------- 2: state entering each chunk (forward)
@@ -252,15 +312,16 @@ __host__ __device__ inline void k3_load(const BwdArgs &a, int c, int h, int b, i
     load_rows_p(a, a.dy, c, h, b, tid, m.dY);
     load_rows_n(a, a.C, c, group_of(a, h), b, tid, m.Cs);
 }
-__host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
-    float *R = a.st + 2 * ix_pn(a, b, h, c);  // the chunk states were consumed by pass 2
-    for (int i = tid; i < a.headdim * a.dstate; i += NT) {
-        const int p = i / a.dstate, n = i % a.dstate;
-        c2 acc = cmk(0.f, 0.f);
-        for (int l = 0; l < QC; ++l)
-            acc = cadd(acc, cscale(cconj(cmul(ld2(m.e + 2 * l), sm2(m.Cs + l * NS, n))), m.dY[l * PS + p]));
-        st2(R + 2 * i, acc);
+// C_l <- conj(e_l C_l) in place
+__host__ __device__ inline void k3_scale(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    for (int i = tid; i < QC * N_MAX; i += NT) {
+        const int l = i / N_MAX, n = i % N_MAX;
+        st2(m.Cs + l * NS + 2 * n, cconj(cmul(ld2(m.e + 2 * l), sm2(m.Cs + l * NS, n))));
     }
+}
+__host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    tn_pn(a, m.dY, m.Cs, a.st + 2 * ix_pn(a, b, h, c), tid);  // the chunk states were consumed by pass 2
 }
 
 // --------------------- 4: gradient of the state leaving each chunk (backward)
@@ -299,24 +360,47 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     load_pn(a, a.hin + 2 * ix_pn(a, b, h, c), tid, m.Hin);
     load_pn(a, a.gh + 2 * ix_pn(a, b, h, c), tid, m.Gh);
 }
-// GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY.
+// GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY; thread tile rows
+// l = 2 tr + i, columns s = tc + 16 j.
 __host__ __device__ inline void k5_mats(const BwdArgs &a, int tid, const Smem &m) {
-    for (int i = tid; i < QC * QC; i += NT) {
-        const int l = i / QC, s = i % QC;
-        c2 gm = cmk(0.f, 0.f);
-        float xy = 0.f;
-        for (int n = 0; n < a.dstate; ++n) gm = cadd(gm, cmul(sm2(m.Cs + l * NS, n), sm2(m.Bs + s * NS, n)));
-        for (int p = 0; p < a.headdim; ++p) xy += m.dY[l * PS + p] * m.X[s * PS + p];
-        m.XY[l * QS1 + s] = xy;
-        if (l >= s) {
-            const c2 L = cexpc(csub(ld2(m.acs + 2 * l), ld2(m.acs + 2 * s)));
-            st2(m.GL + l * QS2 + 2 * s, cmul(gm, L));
-            st2(m.K + l * QS2 + 2 * s, cscale(L, m.d[s] * xy));
-        } else {
-            st2(m.GL + l * QS2 + 2 * s, cmk(0.f, 0.f));
-            st2(m.K + l * QS2 + 2 * s, cmk(0.f, 0.f));
-        }
+    (void)a;
+    const int r0 = 2 * (tid >> 4), tc = tid & 15;
+    c2 g[2][2];
+    float xy[2][2];
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 2; ++j) g[i][j] = cmk(0.f, 0.f), xy[i][j] = 0.f;
+    for (int k = 0; k < 2 * N_MAX; k += 4) {  // two complex states per step
+        f4 ca[2], bb[2];
+        for (int i = 0; i < 2; ++i) ca[i] = ld4(m.Cs + (r0 + i) * NS + k);
+        for (int j = 0; j < 2; ++j) bb[j] = ld4(m.Bs + (tc + 16 * j) * NS + k);
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 2; ++j) {
+                const f4 &u = ca[i], &v = bb[j];
+                g[i][j].re = fmaf(u.x, v.x, fmaf(-u.y, v.y, fmaf(u.z, v.z, fmaf(-u.w, v.w, g[i][j].re))));
+                g[i][j].im = fmaf(u.x, v.y, fmaf(u.y, v.x, fmaf(u.z, v.w, fmaf(u.w, v.z, g[i][j].im))));
+            }
     }
+    for (int p = 0; p < P_MAX; p += 4) {
+        f4 ya[2], xb[2];
+        for (int i = 0; i < 2; ++i) ya[i] = ld4(m.dY + (r0 + i) * PS + p);
+        for (int j = 0; j < 2; ++j) xb[j] = ld4(m.X + (tc + 16 * j) * PS + p);
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 2; ++j)
+                xy[i][j] = fmaf(ya[i].x, xb[j].x, fmaf(ya[i].y, xb[j].y, fmaf(ya[i].z, xb[j].z, fmaf(ya[i].w, xb[j].w, xy[i][j]))));
+    }
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 2; ++j) {
+            const int l = r0 + i, s = tc + 16 * j;
+            m.XY[l * QS1 + s] = xy[i][j];
+            if (l >= s) {
+                const c2 L = cexpc(csub(ld2(m.acs + 2 * l), ld2(m.acs + 2 * s)));
+                st2(m.GL + l * QS2 + 2 * s, cmul(g[i][j], L));
+                st2(m.K + l * QS2 + 2 * s, cscale(L, m.d[s] * xy[i][j]));
+            } else {
+                st2(m.GL + l * QS2 + 2 * s, cmk(0.f, 0.f));
+                st2(m.K + l * QS2 + 2 * s, cmk(0.f, 0.f));
+            }
+        }
 }
 __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem &m) {
     if (tid < QC) {  // rows of E and columns of GL o XY
@@ -342,6 +426,98 @@ __host__ __device__ inline void k5_tokens(const BwdArgs &a, int tid, const Smem 
         m.red[r] = h0.re;
         m.red[RED + r] = h0.im;
         m.red[2 * RED + r] = dd;
+    }
+}
+// This head's dB and dC, with each thread's column share of Ksr and F:
+//   xg = x Gh, yh = dy h_in (tiles rows 2 tr + i, complex columns n(j)),
+//   dB_s = conj(sum_l K[l][s] C_l) + conj(w_s) xg_s,   Ksr[s] = sum_n B_s[n] conj(xg_s[n]),
+//   dC_l = conj(sum_s K[l][s] B_s + e_l yh_l),          F[l] / e_l = sum_n C_l[n] yh_l[n].
+__host__ __device__ inline void k5_bc(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int r0 = 2 * (tid >> 4), tc = tid & 15;
+    float *part_k = m.part, *part_f = m.part + QC * 16 * 2;
+    {
+        c2 acc[2][4];
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 4; ++j) acc[i][j] = cmk(0.f, 0.f);
+        for (int p = 0; p < P_MAX; p += 4) {  // x Gh
+            f4 xa[2];
+            for (int i = 0; i < 2; ++i) xa[i] = ld4(m.X + (r0 + i) * PS + p);
+            for (int pp = 0; pp < 4; ++pp)
+                for (int i = 0; i < 2; ++i) axpy4(acc[i], comp(xa[i], pp), m.Gh + (p + pp) * NS, tc);
+        }
+        c2 kc[2][4];
+        for (int i = 0; i < 2; ++i) {
+            const int s = r0 + i;
+            c2 ks = cmk(0.f, 0.f);
+            for (int j = 0; j < 4; ++j) {
+                ks = cadd(ks, cmul(sm2(m.Bs + s * NS, ncol(tc, j)), cconj(acc[i][j])));
+                kc[i][j] = cmk(0.f, 0.f);
+            }
+            st2(part_k + (s * 16 + tc) * 2, ks);
+        }
+        for (int l = r0; l < QC; ++l) {  // sum_l K[l][s] C_l, K[l][s] = 0 for l < s
+            const f4 kv = ld4(m.K + l * QS2 + 2 * r0);
+            czpy4(kc[0], c2{kv.x, kv.y}, m.Cs + l * NS, tc);
+            czpy4(kc[1], c2{kv.z, kv.w}, m.Cs + l * NS, tc);
+        }
+        for (int i = 0; i < 2; ++i) {
+            const int s = r0 + i, t = c * QC + s;
+            if (t >= a.seqlen) continue;
+            const c2 wc = cconj(ld2(m.w + 2 * s));
+            c2 v[4];
+            for (int j = 0; j < 4; ++j) v[j] = cadd(cconj(kc[i][j]), cmul(wc, acc[i][j]));
+            store_n4(a.dBh + 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate), tc, a.dstate, v);
+        }
+    }
+    {
+        c2 acc[2][4];
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 4; ++j) acc[i][j] = cmk(0.f, 0.f);
+        for (int p = 0; p < P_MAX; p += 4) {  // dy h_in
+            f4 ya[2];
+            for (int i = 0; i < 2; ++i) ya[i] = ld4(m.dY + (r0 + i) * PS + p);
+            for (int pp = 0; pp < 4; ++pp)
+                for (int i = 0; i < 2; ++i) axpy4(acc[i], comp(ya[i], pp), m.Hin + (p + pp) * NS, tc);
+        }
+        for (int i = 0; i < 2; ++i) {
+            const int l = r0 + i;
+            c2 f = cmk(0.f, 0.f);
+            const c2 el = ld2(m.e + 2 * l);
+            for (int j = 0; j < 4; ++j) {
+                f = cadd(f, cmul(sm2(m.Cs + l * NS, ncol(tc, j)), acc[i][j]));
+                acc[i][j] = cmul(el, acc[i][j]);
+            }
+            st2(part_f + (l * 16 + tc) * 2, f);
+        }
+        for (int k = 0; k < r0 + 2; k += 2) {  // sum_s K[l][s] B_s, K[l][s] = 0 for s > l
+            for (int i = 0; i < 2; ++i) {
+                const f4 kv = ld4(m.K + (r0 + i) * QS2 + 2 * k);
+                czpy4(acc[i], c2{kv.x, kv.y}, m.Bs + k * NS, tc);
+                czpy4(acc[i], c2{kv.z, kv.w}, m.Bs + (k + 1) * NS, tc);
+            }
+        }
+        for (int i = 0; i < 2; ++i) {
+            const int l = r0 + i, t = c * QC + l;
+            if (t >= a.seqlen) continue;
+            c2 v[4];
+            for (int j = 0; j < 4; ++j) v[j] = cconj(acc[i][j]);
+            store_n4(a.dCh + 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate), tc, a.dstate, v);
+        }
+    }
+}
+// F and Ksr from their column shares (fixed order).
+__host__ __device__ inline void k5_fk(const BwdArgs &a, int tid, const Smem &m) {
+    (void)a;
+    const float *part_k = m.part, *part_f = m.part + QC * 16 * 2;
+    if (tid < QC) {
+        c2 v = cmk(0.f, 0.f);
+        for (int q = 0; q < 16; ++q) v = cadd(v, ld2(part_f + (tid * 16 + q) * 2));
+        st2(m.F + 2 * tid, cmul(ld2(m.e + 2 * tid), v));
+    } else if (tid < 2 * QC) {
+        const int t = tid - QC;
+        c2 v = cmk(0.f, 0.f);
+        for (int q = 0; q < 16; ++q) v = cadd(v, ld2(part_k + (t * 16 + q) * 2));
+        st2(m.Ksr + 2 * t, v);
     }
 }
 __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
@@ -374,51 +550,44 @@ __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, 
     st2(a.dAp + 2 * (ix_bh(a, b, h) * a.nchunks + c), dAp);
     a.dDp[ix_bh(a, b, h) * a.nchunks + c] = dd;
 }
-// This head's dB and dC, and the per-(token, state) terms of F and Ksr:
-// F[t] = e_t dy_t . (h_in C_t) = e_t sum_n C_t[n] (dy_t h_in)[n] and
-// Ksr[t] = x_t . (conj(Gh) B_t) = sum_n B_t[n] conj((x_t Gh)[n]), from the same
-// dy_t h_in and x_t Gh that dC and dB use.
-__host__ __device__ inline void k5_bc(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
-    for (int i = tid; i < QC * a.dstate; i += NT) {
-        const int s = i / a.dstate, n = i % a.dstate, t = c * QC + s;
-        c2 db = cmk(0.f, 0.f), dc = cmk(0.f, 0.f), xg = cmk(0.f, 0.f), yh = cmk(0.f, 0.f);
-        for (int l = s; l < QC; ++l) db = cadd(db, cmul(ld2(m.K + l * QS2 + 2 * s), sm2(m.Cs + l * NS, n)));
-        for (int r = 0; r <= s; ++r) dc = cadd(dc, cmul(ld2(m.K + s * QS2 + 2 * r), sm2(m.Bs + r * NS, n)));
-        for (int p = 0; p < a.headdim; ++p) {
-            xg = cadd(xg, cscale(sm2(m.Gh + p * NS, n), m.X[s * PS + p]));
-            yh = cadd(yh, cscale(sm2(m.Hin + p * NS, n), m.dY[s * PS + p]));
-        }
-        st2(m.pF + s * NS + 2 * n, cmul(sm2(m.Cs + s * NS, n), yh));
-        st2(m.pK + s * NS + 2 * n, cmul(sm2(m.Bs + s * NS, n), cconj(xg)));
-        if (t >= a.seqlen) continue;
-        const size_t o = 2 * ((((size_t)b * a.seqlen + t) * a.nheads + h) * a.dstate + n);
-        st2(a.dBh + o, cadd(cconj(db), cmul(cconj(ld2(m.w + 2 * s)), xg)));
-        st2(a.dCh + o, cconj(cadd(dc, cmul(ld2(m.e + 2 * s), yh))));
-    }
-}
-// F and Ksr from their per-state terms (fixed order).
-__host__ __device__ inline void k5_fk(const BwdArgs &a, int tid, const Smem &m) {
-    if (tid < QC) {
-        c2 v = cmk(0.f, 0.f);
-        for (int n = 0; n < a.dstate; ++n) v = cadd(v, sm2(m.pF + tid * NS, n));
-        st2(m.F + 2 * tid, cmul(ld2(m.e + 2 * tid), v));
-    } else if (tid < 2 * QC) {
-        const int t = tid - QC;
-        c2 v = cmk(0.f, 0.f);
-        for (int n = 0; n < a.dstate; ++n) v = cadd(v, sm2(m.pK + t * NS, n));
-        st2(m.Ksr + 2 * t, v);
-    }
-}
+// dx_s = dt_s sum_l Re(GL[l][s]) dy_l + D dy_s + Re(conj(w_s) sum_n conj(B_s[n]) Gh[.][n]),
+// thread tile rows s = 2 tr + i, columns p = tc + 16 j.
 __host__ __device__ inline void k5_dx(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
+    const int r0 = 2 * (tid >> 4), tc = tid & 15;
     const float Dh = a.D ? a.D[h] : 0.f;
-    for (int i = tid; i < QC * a.headdim; i += NT) {
-        const int s = i / a.headdim, p = i % a.headdim, t = c * QC + s;
+    float acc[2][4];
+    c2 gb[2][4];
+    for (int i = 0; i < 2; ++i)
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f, gb[i][j] = cmk(0.f, 0.f);
+    for (int l = r0; l < QC; ++l) {  // GL[l][s] = 0 for l < s
+        const f4 gl = ld4(m.GL + l * QS2 + 2 * r0);
+        for (int j = 0; j < 4; ++j) {
+            const float yv = m.dY[l * PS + tc + 16 * j];
+            acc[0][j] = fmaf(gl.x, yv, acc[0][j]);
+            acc[1][j] = fmaf(gl.z, yv, acc[1][j]);
+        }
+    }
+    for (int k = 0; k < 2 * N_MAX; k += 4) {  // conj(B_s) . Gh[p], two complex states per step
+        f4 ba[2], gv[4];
+        for (int i = 0; i < 2; ++i) ba[i] = ld4(m.Bs + (r0 + i) * NS + k);
+        for (int j = 0; j < 4; ++j) gv[j] = ld4(m.Gh + (tc + 16 * j) * NS + k);
+        for (int i = 0; i < 2; ++i)
+            for (int j = 0; j < 4; ++j) {
+                const f4 &u = ba[i], &v = gv[j];
+                gb[i][j].re = fmaf(u.x, v.x, fmaf(u.y, v.y, fmaf(u.z, v.z, fmaf(u.w, v.w, gb[i][j].re))));
+                gb[i][j].im = fmaf(u.x, v.y, fmaf(-u.y, v.x, fmaf(u.z, v.w, fmaf(-u.w, v.z, gb[i][j].im))));
+            }
+    }
+    for (int i = 0; i < 2; ++i) {
+        const int s = r0 + i, t = c * QC + s;
         if (t >= a.seqlen) continue;
-        float acc = 0.f;
-        c2 gb = cmk(0.f, 0.f);
-        for (int l = s; l < QC; ++l) acc += ld2(m.GL + l * QS2 + 2 * s).re * m.dY[l * PS + p];
-        for (int n = 0; n < a.dstate; ++n) gb = cadd(gb, cmul(cconj(sm2(m.Bs + s * NS, n)), sm2(m.Gh + p * NS, n)));
-        a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc + Dh * m.dY[s * PS + p] + cmul(cconj(ld2(m.w + 2 * s)), gb).re;
+        const c2 ws = ld2(m.w + 2 * s);
+        for (int j = 0; j < 4; ++j) {
+            const int p = tc + 16 * j;
+            if (p >= a.headdim) continue;
+            a.dx[ix_x(a, b, t, h, p)] = m.d[s] * acc[i][j] + Dh * m.dY[s * PS + p] + ws.re * gb[i][j].re +
+                                        ws.im * gb[i][j].im;
+        }
     }
 }
 

@@ -120,6 +120,7 @@ extern "C" int emulate_scan_bwd_complex(const float *x, const float *dt, const f
                     fresh();
                     each([&](int t) { k1_load(a, c, h, b, t, m1); });
                     each([&](int t) { k1_cumsum(a, c, h, b, t, m1); });
+                    each([&](int t) { k1_scale(a, t, m1); });
                     each([&](int t) { k1_state(a, c, h, b, t, m1); });
                 }
         for (int b = 0; b < batch; ++b)
@@ -130,6 +131,7 @@ extern "C" int emulate_scan_bwd_complex(const float *x, const float *dt, const f
                 for (int c = 0; c < a.nchunks; ++c) {
                     fresh();
                     each([&](int t) { k3_load(a, c, h, b, t, m3); });
+                    each([&](int t) { k3_scale(a, t, m3); });
                     each([&](int t) { k3_r(a, c, h, b, t, m3); });
                 }
         for (int b = 0; b < batch; ++b)
