@@ -206,34 +206,48 @@ __global__ void __launch_bounds__(NT) cplx_chunk_state_kernel(ScanArgs a, CWs w,
 
 // ------------------------------------------------------------ 2. state pass
 // h_c = exp(A_cs total of chunk c) h_{c-1} + S_c per state element, in place:
-// S_c becomes the state entering chunk c; the last h is the final state.
-__global__ void __launch_bounds__(NT) cplx_state_pass_kernel(ScanArgs a, CWs w) {
+// S_c becomes the state entering chunk c; the last h is the final state.  The
+// chunks' complex decay factors are computed once per block (NT chunks at a
+// time) into shared memory; every thread stays to the end for the barriers.
+__global__ void __launch_bounds__(NT, 4) cplx_state_pass_kernel(ScanArgs a, CWs w) {
+    __shared__ cf fac[NT];
+    ptx::grid_dep_wait();    // the chunk states are complete
+    ptx::grid_dep_launch();  // the chunk scan may start its prologue
     const int PN = a.headdim * a.dstate;
     const int e = blockIdx.x * NT + threadIdx.x;
     const int h = blockIdx.y, b = blockIdx.z;
-    if (e >= PN) return;
+    const bool live = e < PN;
     const size_t bh = (size_t)b * a.nheads + h;
     cf run = {0.f, 0.f};
-    if (a.init_state) run = reinterpret_cast<const cf *>(a.init_state)[bh * PN + e];
-    constexpr int GRP = 8;  // chunk states loaded together, then folded in order
-    for (int c0 = 0; c0 < a.nchunks; c0 += GRP) {
-        const int n = min(GRP, a.nchunks - c0);
-        cf sv[GRP];
-#pragma unroll
-        for (int i = 0; i < GRP; ++i)
-            if (i < n) sv[i] = w.S[(bh * a.nchunks + c0 + i) * PN + e];
-#pragma unroll
-        for (int i = 0; i < GRP; ++i) {
-            if (i >= n) break;
-            const size_t bhc = bh * a.nchunks + c0 + i;
-            w.S[bhc * PN + e] = run;
+    if (live && a.init_state) run = reinterpret_cast<const cf *>(a.init_state)[bh * PN + e];
+    constexpr int GRP = 16;  // chunk states loaded together, then folded in order
+    for (int f0 = 0; f0 < a.nchunks; f0 += NT) {
+        const int nf = min(NT, a.nchunks - f0);
+        __syncthreads();  // the previous factors are no longer read
+        if ((int)threadIdx.x < nf) {
+            const size_t bhc = bh * a.nchunks + f0 + threadIdx.x;
             const float mag = expf((float)w.lam[bhc * 2]);
             float sn, cn;
             sincosf((float)w.lam[bhc * 2 + 1], &sn, &cn);
-            run = cfma({mag * cn, mag * sn}, run, sv[i]);
+            fac[threadIdx.x] = {mag * cn, mag * sn};
+        }
+        __syncthreads();
+        if (!live) continue;
+        for (int c0 = 0; c0 < nf; c0 += GRP) {
+            const int n = min(GRP, nf - c0);
+            cf sv[GRP];
+#pragma unroll
+            for (int i = 0; i < GRP; ++i)
+                if (i < n) sv[i] = w.S[(bh * a.nchunks + f0 + c0 + i) * PN + e];
+#pragma unroll
+            for (int i = 0; i < GRP; ++i) {
+                if (i >= n) break;
+                w.S[(bh * a.nchunks + f0 + c0 + i) * PN + e] = run;
+                run = cfma(fac[c0 + i], run, sv[i]);
+            }
         }
     }
-    if (a.final_state) reinterpret_cast<cf *>(a.final_state)[bh * PN + e] = run;
+    if (live && a.final_state) reinterpret_cast<cf *>(a.final_state)[bh * PN + e] = run;
 }
 
 // ------------------------------------------------------------- 3. chunk scan
@@ -606,6 +620,24 @@ __global__ void __launch_bounds__(NT, 2) cplx_chunk_scan_n64_kernel(ScanArgs a, 
 
 }  // namespace
 
+// Launch with programmatic stream serialization: the kernel may begin while its
+// predecessor in the stream is ending, and waits for it (grid_dep_wait) before
+// it reads what the predecessor wrote.
+template <typename... P, typename... Args>
+cudaError_t launch_after(void (*kern)(P...), dim3 grid, int threads, size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 size_t cplx_scan_tile_smem(int Q) {
     return 2 * Q * sizeof(float) + Q * sizeof(float2) + (KC * TL + KC * 64 + 64 * TL + 64 * TP) * sizeof(float);
 }
@@ -613,8 +645,7 @@ size_t cplx_scan_tile_smem(int Q) {
 cudaError_t launch_cplx_state_pass(const ScanArgs &a, void *ws, cudaStream_t st) {
     const CWs w = carve_c(ws, a);
     const int PN = a.headdim * a.dstate;
-    cplx_state_pass_kernel<<<dim3((PN + NT - 1) / NT, a.nheads, a.batch), NT, 0, st>>>(a, w);
-    return cudaGetLastError();
+    return launch_after(cplx_state_pass_kernel, dim3((PN + NT - 1) / NT, a.nheads, a.batch), NT, 0, st, a, w);
 }
 
 template <typename T>
@@ -671,8 +702,7 @@ cudaError_t launch_complex_tc(const ScanArgs &a0, const CplxView<T> &v, void *ws
     ctc::state_kernel<T><<<grid, ctc::NTH, ctc::SMEM_STATE, st>>>(a, w, v);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_cplx_state_pass(a, ws, st)) != cudaSuccess) return e;
-    ctc::scan_kernel<T><<<grid, ctc::NTH, ctc::SMEM_SCAN, st>>>(a, w, v);
-    return cudaGetLastError();
+    return launch_after(ctc::scan_kernel<T>, grid, ctc::NTH, ctc::SMEM_SCAN, st, a, w, v);
 }
 
 template <typename T>

@@ -136,13 +136,30 @@ template <typename T> __global__ void __launch_bounds__(NTH, 4) state_kernel(Sca
     }
     chunk_log_decay(a, v, b, h, c, dts, cre, cim);  // ends with a block barrier
     const double R = cre[QT - 1], Th = cim[QT - 1];
-    for (int s = tid; s < QT; s += NTH) {
-        w.cs[(bhc * 2) * QT + s] = cre[s];
-        w.cs[(bhc * 2 + 1) * QT + s] = cim[s];
+    // The chunk scan's per-token factors go to the chunk's log-decay slot (2 x 128
+    // float2 in the place of 2 x 128 doubles): C' = exp(A_cs - rho) and
+    // B' = exp(rho - A_cs) dt, rho = R / 2.  A chunk too steep for that form keeps
+    // its cumulative log-decays there for the CUDA-core tile code.  Threads below
+    // QT take C' and B', the others the chunk-state weights.
+    const bool steep = fabs(R) > SPAN;
+    float2 *fac = reinterpret_cast<float2 *>(w.cs + (bhc * 2) * QT);
+    for (int u = tid; u < 2 * QT; u += NTH) {
+        const int s = u & (QT - 1);
         double sn, cn;
-        sincos(Th - cim[s], &sn, &cn);
-        const float m = (float)exp(R - cre[s]) * dts[s];
-        wf[s] = make_float2(m * (float)cn, m * (float)sn);
+        if (u >= QT) {
+            sincos(Th - cim[s], &sn, &cn);
+            const float m = (float)exp(R - cre[s]) * dts[s];
+            wf[s] = make_float2(m * (float)cn, m * (float)sn);
+        } else if (steep) {
+            w.cs[(bhc * 2) * QT + s] = cre[s];
+            w.cs[(bhc * 2 + 1) * QT + s] = cim[s];
+        } else {
+            const double rho = 0.5 * R;
+            sincos(cim[s], &sn, &cn);
+            const float ec = (float)exp(cre[s] - rho), eb = (float)exp(rho - cre[s]) * dts[s];
+            fac[s] = make_float2(ec * (float)cn, ec * (float)sn);
+            fac[QT + s] = make_float2(eb * (float)cn, -eb * (float)sn);
+        }
     }
     if (tid == 0) {
         w.lam[bhc * 2] = R;
@@ -230,6 +247,7 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const double Rr = w.lam[bhc * 2];
     if (fabs(Rr) > SPAN) {  // too steep for the factored form: the CUDA-core tile code
+        grid_dep_wait();    // h_in is written by the state pass
         for (int rt = 0; rt * 64 < valid; ++rt) cplx_scan_tile<T>(a, w, v, b, h, c, rt, 0, sm);
         return;
     }
@@ -246,14 +264,9 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
         tmem_relinquish();
     }
     const double rho = 0.5 * Rr;
-    for (int s = tid; s < QT; s += NTH) {
-        const double cr = w.cs[(bhc * 2) * QT + s], ci = w.cs[(bhc * 2 + 1) * QT + s];
-        double sn, cn;
-        sincos(ci, &sn, &cn);
-        const float d = s < valid ? view_dt(v, bt0 + s, h) : 0.f;
-        const float ec = (float)exp(cr - rho), eb = (float)exp(rho - cr) * d;
-        fC[s] = make_float2(ec * (float)cn, ec * (float)sn);
-        fB[s] = make_float2(eb * (float)cn, -eb * (float)sn);
+    {  // C' and B' factors of the chunk, written by the chunk-state kernel
+        const float2 *fac = reinterpret_cast<const float2 *>(w.cs + (bhc * 2) * QT);
+        for (int u = tid; u < 2 * QT; u += NTH) fC[u] = __ldg(fac + u);  // fB = fC + QT
     }
     tc_fence_before();
     __syncthreads();
@@ -263,6 +276,7 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
     const float er = (float)exp(rho);
     const float *hin = reinterpret_cast<const float *>(w.S + bhc * (size_t)P * N);
     bool ok = true;
+#pragma unroll 1
 #pragma unroll 1
     for (int kh = 0; kh < 2; ++kh) {  // k = 64 kh .. 64 kh + 63: complex states 32 kh .. 32 kh + 31
         if (kh == 1) {  // the first half's products have read the tiles
@@ -292,7 +306,9 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
             put8(sm, S_CH, S_CL, o, vc);
             put8(sm, S_BH, S_BL, o, vb);
         }
-        // h' = exp(rho) h_in as (re, im), rows p (h_in was written by earlier launches: read-only here)
+        // h' = exp(rho) h_in as (re, im), rows p (h_in was written by earlier launches: read-only here;
+        // the state pass that writes it may still be running until grid_dep_wait returns)
+        if (kh == 0) grid_dep_wait();
 #pragma unroll 2
         for (int it = 0; it < 64 * 8 / NTH; ++it) {
             const int u = tid + it * NTH, p = u >> 3, cl = u & 7, ch = 8 * kh + cl;
@@ -322,6 +338,22 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
                 }
             }
             mma_commit(&bars[kh]);
+        }
+    }
+    // Warps 4-7 load X of the chunk while the products run; it is written over
+    // the C' tiles once they are done.
+    constexpr int XIT = QT * 8 / (NTH - 128);
+    float xr[XIT][8];
+    if (warp >= 4) {
+#pragma unroll
+        for (int it = 0; it < XIT; ++it) {
+            const int u = (tid - 128) + it * (NTH - 128), s = u >> 3, ch = u & 7;
+            if (s < valid) {
+                view_x8(v, bt0 + s, h, a.headdim, 8 * ch, xr[it]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) xr[it][e] = 0.f;
+            }
         }
     }
     ok = wait_bounded(&bars[1], 0, a.dev_error) && ok;  // every product of both halves is done
@@ -361,17 +393,10 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
         tmem_wait_st();
     } else {
         // X of the chunk as bf16 hi/lo rows [s][p], into the C' tiles
-#pragma unroll 4
-        for (int it = 0; it < QT * 8 / (NTH - 128); ++it) {
-            const int u = (tid - 128) + it * (NTH - 128), s = u >> 3, ch = u & 7;
-            float val[8];
-            if (s < valid) {
-                view_x8(v, bt0 + s, h, a.headdim, 8 * ch, val);
-            } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) val[e] = 0.f;
-            }
-            put8(sm, S_XH, S_XL, sw_off(s, ch, QT * 128), val);
+        for (int it = 0; it < XIT; ++it) {
+            const int u = (tid - 128) + it * (NTH - 128), s = u >> 3, ch = u & 7;
+            put8(sm, S_XH, S_XL, sw_off(s, ch, QT * 128), xr[it]);
         }
         fence_proxy_async_smem();
     }
