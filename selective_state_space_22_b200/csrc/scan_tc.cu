@@ -685,9 +685,12 @@ std::atomic<unsigned long long> g_wait_ns{0};
 
 // Split nchunks into `runs` runs so that every run's CTA has about the same
 // work: run r streams its run_start[r] predecessors state-only (cost ALPHA per
-// chunk relative to a full chunk) and then its own chunks in full.
+// chunk relative to a full chunk) and then its own chunks in full.  A state-only
+// chunk costs about 0.65 of a full one: it is bound by the latency of its B and X
+// loads through the two {C, B} slots, not by its work (measured: 1.7 against
+// 2.6 us per chunk at T = 65536, 64 heads).
 void split_runs(int nchunks, int runs, int *start) {
-    const double ALPHA = 0.35;
+    const double ALPHA = 0.65;
     auto last = [&](double K) {
         double x = 0;
         for (int r = 0; r < runs; ++r) x += K - ALPHA * x;
