@@ -245,6 +245,20 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
     const size_t bhc = ((size_t)b * H + h) * a.nchunks + c, bt0 = (size_t)b * a.seqlen + t0;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // The first k half's C and B values go in flight before anything else: they
+    // depend on nothing this kernel computes.
+    constexpr int CBIT = QT * 8 / NTH;
+    cf cq0[CBIT][4], bq0[CBIT][4];
+#pragma unroll
+    for (int it = 0; it < CBIT; ++it) {
+        const int u = threadIdx.x + it * NTH, r = u >> 3, ch = u & 7;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cq0[it][q] = bq0[it][q] = cf{0.f, 0.f};
+        if (r < valid) {
+            view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq0[it]);
+            view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq0[it]);
+        }
+    }
     const double Rr = w.lam[bhc * 2];
     if (fabs(Rr) > SPAN) {  // too steep for the factored form: the CUDA-core tile code
         grid_dep_wait();    // h_in is written by the state pass
@@ -276,8 +290,7 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
     const float er = (float)exp(rho);
     const float *hin = reinterpret_cast<const float *>(w.S + bhc * (size_t)P * N);
     bool ok = true;
-#pragma unroll 1
-#pragma unroll 1
+#pragma unroll
     for (int kh = 0; kh < 2; ++kh) {  // k = 64 kh .. 64 kh + 63: complex states 32 kh .. 32 kh + 31
         if (kh == 1) {  // the first half's products have read the tiles
             ok = wait_bounded(&bars[0], 0, a.dev_error) && ok;
@@ -285,14 +298,15 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
         }
         // C' as (re, -im) and B' as (re, im), rows = tokens, 4 complex states per chunk of 8
 #pragma unroll 4
-        for (int it = 0; it < QT * 8 / NTH; ++it) {
+        for (int it = 0; it < CBIT; ++it) {
             const int u = tid + it * NTH, r = u >> 3, cl = u & 7, ch = 8 * kh + cl;
             float vc[8], vb[8];
             const float2 fc = fC[r], fb = fB[r];
             cf cq[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}}, bq[4] = {cq[0], cq[1], cq[2], cq[3]};
-            if (r < valid) {
-                view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq);
-                view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                cq[q] = cq0[it][q];
+                bq[q] = bq0[it][q];
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -338,6 +352,18 @@ __global__ void __launch_bounds__(NTH, 2) scan_kernel(ScanArgs a, CWs w, CplxVie
                 }
             }
             mma_commit(&bars[kh]);
+        }
+        if (kh == 0) {  // the second half's C and B, in flight while the first half's products run
+#pragma unroll
+            for (int it = 0; it < CBIT; ++it) {
+                const int u = tid + it * NTH, r = u >> 3, ch = 8 + (u & 7);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) cq0[it][q] = bq0[it][q] = cf{0.f, 0.f};
+                if (r < valid) {
+                    view_cplx4(v, v.cre, v.cim, bt0 + r, g, 4 * ch, cq0[it]);
+                    view_cplx4(v, v.bre, v.bim, bt0 + r, g, 4 * ch, bq0[it]);
+                }
+            }
         }
     }
     // Warps 4-7 load X of the chunk while the products run; it is written over
