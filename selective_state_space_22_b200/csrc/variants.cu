@@ -35,18 +35,6 @@ template <typename T> __device__ __forceinline__ float ldf(const T *p) { return 
 // (exact to 2 ulp for divisors below 2^126) always sees a finite divisor; past
 // the cap the quotient is below 1e-33 |v|.
 __device__ __forceinline__ float silu_f(float v) { return __fdividef(v, 1.f + __expf(fminf(-v, 80.f))); }
-// For bf16 outputs: v sigmoid(v) = v/2 (1 + tanh(v/2)) with the hardware tanh
-// (relative error about 2^-11, below the 2^-9 rounding of the bf16 result); one
-// exponential-unit operation instead of two.
-__device__ __forceinline__ float silu_bf16out(float v) {
-    const float hv = 0.5f * v;
-    float t;
-    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(hv));
-    return fmaf(hv, t, hv);
-}
-template <typename T> __device__ __forceinline__ float silu_out(float v);
-template <> __device__ __forceinline__ float silu_out<float>(float v) { return silu_f(v); }
-template <> __device__ __forceinline__ float silu_out<__nv_bfloat16>(float v) { return silu_bf16out(v); }
 
 constexpr int CONV_TT = 32;   // tokens per thread run
 constexpr int CONV_MAXK = 8;
@@ -122,6 +110,40 @@ template <> struct Pair<__nv_bfloat16> {
         *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(v.x, v.y);
     }
 };
+
+// Packed float32 pairs (sm_100): one instruction does both lanes, each lane
+// rounded as the scalar fmaf / multiply would.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
+          "l"(*reinterpret_cast<unsigned long long *>(&c)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+__device__ __forceinline__ float2 fmul2v(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
+    return *reinterpret_cast<float2 *>(&r);
+}
+// SiLU of a pair for bf16 outputs: v sigmoid(v) = v/2 (1 + tanh(v/2)) with the
+// hardware tanh (relative error about 2^-11, below the 2^-9 rounding of the bf16
+// result): one exponential-unit operation instead of two; the multiply and the
+// fma packed.
+__device__ __forceinline__ float2 silu2_bf16out(float2 v) {
+    const float2 hv = fmul2v(make_float2(0.5f, 0.5f), v);
+    float2 t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.x) : "f"(hv.x));
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t.y) : "f"(hv.y));
+    return ffma2(hv, t, hv);
+}
+template <typename T> __device__ __forceinline__ float2 silu2_out(float2 v);
+template <> __device__ __forceinline__ float2 silu2_out<float>(float2 v) {
+    return make_float2(silu_f(v.x), silu_f(v.y));
+}
+template <> __device__ __forceinline__ float2 silu2_out<__nv_bfloat16>(float2 v) { return silu2_bf16out(v); }
 
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(smem)),
@@ -202,10 +224,8 @@ __global__ void __launch_bounds__(128) conv1d_xbc_tile_kernel(const T *__restric
 #pragma unroll 4
     for (int i = 0; i < n; ++i) {
         const float2 cur = IO::load(col + (i + 3) * CONV_CH);
-        float2 v;
-        v.x = fmaf(wk[3].x, cur.x, fmaf(wk[2].x, win[2].x, fmaf(wk[1].x, win[1].x, fmaf(wk[0].x, win[0].x, bc.x))));
-        v.y = fmaf(wk[3].y, cur.y, fmaf(wk[2].y, win[2].y, fmaf(wk[1].y, win[1].y, fmaf(wk[0].y, win[0].y, bc.y))));
-        if (silu) v = make_float2(silu_out<T>(v.x), silu_out<T>(v.y));
+        float2 v = ffma2(wk[3], cur, ffma2(wk[2], win[2], ffma2(wk[1], win[1], ffma2(wk[0], win[0], bc))));
+        if (silu) v = silu2_out<T>(v);
         IO::store(pd, v);
         pd += cn;
         win[0] = win[1], win[1] = win[2], win[2] = cur;
@@ -329,12 +349,30 @@ constexpr int SEL_TT = 32;  // tokens per staged run
 constexpr int SEL_CH = 64;  // channels per block (two lanes each)
 
 // The selective scan for blocks of 64 channels that lie in one B/C group.  Two
-// lanes share a channel, each with N/2 of its states in registers.  Per run of
-// 32 tokens the block copies x, dt (64 channels) and B, C (the group's N
-// states, as float32) into shared memory with coalesced loads, runs the
-// recurrence from there (two vector shared loads of B and C per lane and step,
-// no address arithmetic in global memory), and writes the run's y back as
-// coalesced rows.
+// lanes share a channel, each with N/2 of its states in registers.  Runs of 32
+// tokens (16 for float32 inputs with 32 states) of x, dt (64 channels) and B, C (the group's N states) are copied into
+// shared memory as they are stored, with asynchronous 16-byte copies, double
+// buffered: run r+1's copies are in flight while run r is computed, so no load
+// latency sits between runs.  The recurrence reads B and C with vector shared
+// loads (no address arithmetic in global memory), works on pairs of states with
+// packed float32 instructions, and each run's y goes back as coalesced rows.
+// Needs 16-byte aligned x, dt, B, C rows (checked by the launcher).
+template <typename T> __device__ __forceinline__ void unpack8(const T *p, float (&v)[8]);
+template <> __device__ __forceinline__ void unpack8<float>(const float *p, float (&v)[8]) {
+    const float4 a = *reinterpret_cast<const float4 *>(p), b = *reinterpret_cast<const float4 *>(p + 4);
+    v[0] = a.x, v[1] = a.y, v[2] = a.z, v[3] = a.w, v[4] = b.x, v[5] = b.y, v[6] = b.z, v[7] = b.w;
+}
+template <> __device__ __forceinline__ void unpack8<__nv_bfloat16>(const __nv_bfloat16 *p, float (&v)[8]) {
+    const uint4 q = *reinterpret_cast<const uint4 *>(p);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+template <typename T> __device__ __forceinline__ float smem_f(const T *p) { return ld_f32<T>(p); }
+
 template <typename T, int N>
 __global__ void __launch_bounds__(128) selective_scan_tile_kernel(const T *__restrict__ x, const float *__restrict__ dt,
                                                                  const float *__restrict__ A, const T *__restrict__ B,
@@ -343,56 +381,90 @@ __global__ void __launch_bounds__(128) selective_scan_tile_kernel(const T *__res
                                                                  T *__restrict__ y, int seqlen, int channels,
                                                                  int ngroups) {
     constexpr int NH = N / 2;
-    static_assert(NH % 4 == 0, "states per lane read as float4");
-    __shared__ float xs[SEL_TT][SEL_CH], ds[SEL_TT][SEL_CH], ys[SEL_TT][SEL_CH];
-    __shared__ __align__(16) float bs[SEL_TT][N], cs[SEL_TT][N];
+    static_assert(NH % 8 == 0 || NH == 4, "states per lane read as 16-byte vectors");
+    constexpr int XE = 16 / (int)sizeof(T);  // elements of x, B, C per 16-byte copy
+    // tokens per run: 32, or 16 where two runs of float32 x, B and C with 32 states
+    // would not fit in 48 KB of static shared memory
+    constexpr int TT = (sizeof(T) == 4 && N >= 32) ? SEL_TT / 2 : SEL_TT;
+    __shared__ __align__(16) T xs[2][TT][SEL_CH];
+    __shared__ __align__(16) float ds[2][TT][SEL_CH];
+    __shared__ __align__(16) T bs[2][TT][N], cs[2][TT][N];
+    __shared__ float ys[TT][SEL_CH];
     const int tid = threadIdx.x, ch = tid >> 1, half = tid & 1;
     const int cbase = blockIdx.x * SEL_CH, b = blockIdx.y, d = cbase + ch;
     const int g = cbase / (channels / ngroups), n0 = half * NH;
-    float a2[NH], h[NH];
+    // Run r's copies into buffer r % 2 (rows past the sequence are not copied).
+    auto copy_run = [&](int r) {
+        const int t0 = r * TT, nt = min(TT, seqlen - t0), buf = r & 1;
+        const size_t row0 = (size_t)b * seqlen + t0;
+        for (int u = tid; u < nt * (SEL_CH / XE); u += 128) {
+            const int i = u / (SEL_CH / XE), k = u % (SEL_CH / XE);
+            cp_async16(&xs[buf][i][k * XE], x + (row0 + i) * channels + cbase + k * XE);
+        }
+        for (int u = tid; u < nt * (SEL_CH / 4); u += 128) {
+            const int i = u / (SEL_CH / 4), k = u % (SEL_CH / 4);
+            cp_async16(&ds[buf][i][k * 4], dt + (row0 + i) * channels + cbase + k * 4);
+        }
+        for (int u = tid; u < nt * (N / XE); u += 128) {
+            const int i = u / (N / XE), k = u % (N / XE);
+            const size_t o = ((row0 + i) * ngroups + g) * N + k * XE;
+            cp_async16(&bs[buf][i][k * XE], B + o);
+            cp_async16(&cs[buf][i][k * XE], C + o);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const int nruns = (seqlen + TT - 1) / TT;
+    if (nruns > 0) copy_run(0);
+    float2 a2[NH / 2], h[NH / 2];
 #pragma unroll
-    for (int n = 0; n < NH; ++n) {
-        a2[n] = A[(size_t)d * N + n0 + n] * 1.4426950408889634f;
-        h[n] = h0 ? h0[((size_t)b * channels + d) * N + n0 + n] : 0.f;
+    for (int n = 0; n < NH / 2; ++n) {
+        const size_t o = (size_t)d * N + n0 + 2 * n;
+        a2[n] = make_float2(A[o] * 1.4426950408889634f, A[o + 1] * 1.4426950408889634f);
+        const size_t oh = ((size_t)b * channels + d) * N + n0 + 2 * n;
+        h[n] = h0 ? make_float2(h0[oh], h0[oh + 1]) : make_float2(0.f, 0.f);
     }
     const float Dd = D ? D[d] : 0.f;
-    for (int t0 = 0; t0 < seqlen; t0 += SEL_TT) {
-        const int nt = min(SEL_TT, seqlen - t0);
-        const size_t row0 = (size_t)b * seqlen + t0;
-        for (int u = tid; u < nt * SEL_CH; u += 128) {
-            const int i = u / SEL_CH, c = u % SEL_CH;
-            const size_t o = (row0 + i) * channels + cbase + c;
-            xs[i][c] = ldf(x + o);
-            ds[i][c] = dt[o];
+    for (int r = 0; r < nruns; ++r) {
+        const int t0 = r * TT, nt = min(TT, seqlen - t0), buf = r & 1;
+        if (r + 1 < nruns) {
+            copy_run(r + 1);  // into the buffer run r-1 used: its reads ended at the last barrier
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
-        for (int u = tid; u < nt * N; u += 128) {
-            const int i = u / N, n = u % N;
-            const size_t o = ((row0 + i) * ngroups + g) * N + n;
-            bs[i][n] = ldf(B + o);
-            cs[i][n] = ldf(C + o);
-        }
-        __syncthreads();
+        __syncthreads();  // run r's copies from every thread have landed
 #pragma unroll 2
         for (int i = 0; i < nt; ++i) {
-            const float xt = xs[i][ch], st = ds[i][ch], u = st * xt;
+            const float xt = smem_f(&xs[buf][i][ch]), st = ds[buf][i][ch], u = st * xt;
             float bv[NH], cv[NH];
 #pragma unroll
-            for (int n = 0; n < NH; n += 4) {
-                const float4 b4 = *reinterpret_cast<const float4 *>(&bs[i][n0 + n]);
-                const float4 c4 = *reinterpret_cast<const float4 *>(&cs[i][n0 + n]);
-                bv[n] = b4.x, bv[n + 1] = b4.y, bv[n + 2] = b4.z, bv[n + 3] = b4.w;
-                cv[n] = c4.x, cv[n + 1] = c4.y, cv[n + 2] = c4.z, cv[n + 3] = c4.w;
-            }
-            float acc = 0.f;
+            for (int n = 0; n < NH; n += 8 < NH ? 8 : NH) {
+                if constexpr (NH >= 8) {
+                    float tb[8], tc[8];
+                    unpack8<T>(&bs[buf][i][n0 + n], tb);
+                    unpack8<T>(&cs[buf][i][n0 + n], tc);
 #pragma unroll
-            for (int n = 0; n < NH; ++n) {
-                h[n] = fmaf(ex2_approx(st * a2[n]), h[n], u * bv[n]);
-                acc = fmaf(cv[n], h[n], acc);
+                    for (int e = 0; e < 8; ++e) bv[n + e] = tb[e], cv[n + e] = tc[e];
+                } else {
+#pragma unroll
+                    for (int e = 0; e < NH; ++e) bv[e] = smem_f(&bs[buf][i][n0 + e]), cv[e] = smem_f(&cs[buf][i][n0 + e]);
+                }
             }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            if (half == 0) ys[i][ch] = fmaf(Dd, xt, acc);
+            const float2 st2 = make_float2(st, st), u2 = make_float2(u, u);
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int n = 0; n < NH / 2; ++n) {
+                const float2 arg = fmul2v(st2, a2[n]);
+                const float2 e = make_float2(ex2_approx(arg.x), ex2_approx(arg.y));
+                h[n] = ffma2(e, h[n], fmul2v(u2, make_float2(bv[2 * n], bv[2 * n + 1])));
+                acc = ffma2(make_float2(cv[2 * n], cv[2 * n + 1]), h[n], acc);
+            }
+            float accs = acc.x + acc.y;
+            accs += __shfl_xor_sync(0xffffffffu, accs, 1);
+            if (half == 0) ys[i][ch] = fmaf(Dd, xt, accs);
         }
-        __syncthreads();
+        __syncthreads();  // ys complete; buffer buf is free for run r+2
+        const size_t row0 = (size_t)b * seqlen + t0;
         for (int u = tid; u < nt * SEL_CH; u += 128) {
             const int i = u / SEL_CH, c = u % SEL_CH;
             st_f32(y + (row0 + i) * channels + cbase + c, ys[i][c]);
@@ -400,7 +472,11 @@ __global__ void __launch_bounds__(128) selective_scan_tile_kernel(const T *__res
     }
     if (hT)
 #pragma unroll
-        for (int n = 0; n < NH; ++n) hT[((size_t)b * channels + d) * N + n0 + n] = h[n];
+        for (int n = 0; n < NH / 2; ++n) {
+            const size_t oh = ((size_t)b * channels + d) * N + n0 + 2 * n;
+            hT[oh] = h[n].x;
+            hT[oh + 1] = h[n].y;
+        }
 }
 
 template <typename T, int N>
@@ -409,8 +485,12 @@ cudaError_t launch_sel(const void *x, const float *dt, const float *A, const voi
                        cudaStream_t st) {
     // The four-lane form reads each lane's N/4 states of B and C as one vector:
     // aligned when B and C are (the API asks for 16 bytes) and N/4 elements per lane.
-    if constexpr (N >= 8) {  // two lanes of N/2 >= 4 states (whole float4 reads)
-        if ((channels / ngroups) % SEL_CH == 0) {  // every block inside one group
+    if constexpr (N >= 8) {  // two lanes of N/2 >= 4 states (whole 16-byte reads)
+        const bool aligned = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(dt) |
+                               reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(C)) & 15) == 0 &&
+                             ((size_t)channels * sizeof(T)) % 16 == 0 && channels % 4 == 0 &&
+                             ((size_t)N * sizeof(T)) % 16 == 0;
+        if ((channels / ngroups) % SEL_CH == 0 && aligned) {  // every block inside one group
             dim3 grid(channels / SEL_CH, batch);
             selective_scan_tile_kernel<T, N><<<grid, 128, 0, st>>>(
                 static_cast<const T *>(x), dt, A, static_cast<const T *>(B), static_cast<const T *>(C), D, h0, hT,
