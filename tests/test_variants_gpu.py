@@ -82,8 +82,12 @@ def sel_case(shape, sample=None):
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 @pytest.mark.parametrize("T,Dc,G,N,init", [(1, 64, 1, 16, True), (17, 100, 2, 8, False), (300, 256, 1, 16, True),
-                                           (130, 96, 3, 32, True), (64, 33, 1, 4, False)])
+                                           (130, 96, 3, 32, True), (64, 33, 1, 4, False),
+                                           (150, 128, 2, 32, True), (45, 128, 1, 8, False)])
 def test_selective_scan(io, T, Dc, G, N, init):
+    """Both kernels: 64-channel groups take the double-buffered tile kernel (runs
+    of 32 tokens, 16 for float32 with 32 states; N = 8 reads B and C per element),
+    the others the per-lane kernel; ragged last runs, one token."""
     sel_case(inputs.SelectiveShape("sel", 2, T, Dc, G, N, io, init_state=init, seed=T + N))
 
 
