@@ -776,8 +776,21 @@ cudaError_t launch_complex_tma(const ScanArgs &a0, void *ws, cudaStream_t st) {
         const cuuint32_t box[2] = {32, (cuuint32_t)P};
         if ((e = make_map_f32(&mh, w.S, 2, dims, str, box)) != cudaSuccess) return e;
     }
-    if ((e = cudaFuncSetAttribute(ctc::state_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  ctc::SMEM_STATE)) != cudaSuccess)
+    CUtensorMap msb, msx;  // the chunk-state kernel's token quarters of B [32 t][2N] and x [32 t][P]
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)N2, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)Bt};
+        const cuuint64_t str[3] = {(cuuint64_t)N2 * 4, (cuuint64_t)G * N2 * 4, (cuuint64_t)T * G * N2 * 4};
+        const cuuint32_t box[4] = {(cuuint32_t)N2, 1, (cuuint32_t)ctc::S_QT, 1};
+        if ((e = make_map_f32(&msb, a.B, 4, dims, str, box)) != cudaSuccess) return e;
+    }
+    {
+        const cuuint64_t dims[4] = {(cuuint64_t)P, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
+        const cuuint64_t str[3] = {(cuuint64_t)P * 4, (cuuint64_t)H * P * 4, (cuuint64_t)T * H * P * 4};
+        const cuuint32_t box[4] = {(cuuint32_t)P, 1, (cuuint32_t)ctc::S_QT, 1};
+        if ((e = make_map_f32(&msx, a.x, 4, dims, str, box)) != cudaSuccess) return e;
+    }
+    if ((e = cudaFuncSetAttribute(ctc::state_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  ctc::SMEM_STMA)) != cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(ctc::scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   ctc::SMEM_TMA)) != cudaSuccess)
@@ -790,13 +803,13 @@ cudaError_t launch_complex_tma(const ScanArgs &a0, void *ws, cudaStream_t st) {
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int nitems = (int)nbhc, grid1 = std::min(nitems, sms);
-    ctc::state_kernel<float><<<dim3(a.nchunks, H, Bt), ctc::NTH, ctc::SMEM_STATE, st>>>(a, w, v);
+    ctc::state_tma_kernel<<<grid1, ctc::SNTH, ctc::SMEM_STMA, st>>>(msb, msx, a, w);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_cplx_state_pass(a, ws, st)) != cudaSuccess) return e;
-    if ((e = launch_after(ctc::scan_tma_kernel, dim3(grid1), ctc::TNTH, (size_t)ctc::SMEM_TMA, st, mc, mb, mx, mh, a,
-                          w)) != cudaSuccess)
-        return e;
-    return launch_after(ctc::steep_chunks_kernel<float>, dim3(grid1), ctc::NTH, (size_t)steep_smem, st, a, w, v);
+    ctc::scan_tma_kernel<<<grid1, ctc::TNTH, ctc::SMEM_TMA, st>>>(mc, mb, mx, mh, a, w);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    ctc::steep_chunks_kernel<float><<<grid1, ctc::NTH, steep_smem, st>>>(a, w, v);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st) {

@@ -635,10 +635,6 @@ __global__ void __launch_bounds__(TNTH, 1)
                 }
                 if (!ok) break;
             }
-            // The kernel ends only after the state pass (steep_chunks_kernel, launched
-            // after it, relies on that even when this CTA had no chunk to load).
-            if (!h_ready) grid_dep_wait();
-            grid_dep_launch();
             // every load issued has landed before the CTA's shared memory is released
             for (int slot = 0; slot < 2; ++slot)
                 if (r - 1 >= slot) {
@@ -866,11 +862,272 @@ __global__ void __launch_bounds__(TNTH, 1)
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+
+// ----------------------------------------------- TMA-fed persistent chunk states
+// state_kernel for float32 inputs in the plain layout, one CTA per SM looping
+// over chunks (steep ones included):
+//   warp 13     TMA producer: per chunk, four token quarters of B [32 t][128 floats]
+//               and X [32 t][64], each into one of three 24 KB raw stages
+//   warps 0-3   chunk j's decays (thread = token: the cumulative log-decay in
+//               double, the weights w_s of B'', the chunk scan's factors and Lambda
+//               into the workspace), then the state S of chunk j-1 out of TMEM
+//   warps 4-11  converters: each quarter -> B'' = w B and X as bf16 hi/lo
+//               (128-byte swizzled rows) in one of two operand stages
+//   warp 12     MMA issuer: S = B''^T X over the four quarters, three passes
+// Two TMEM column sets of 64 hold two chunks' states.
+constexpr int SNTH = 448;
+constexpr int SW_CONV = 4, SW_MMA = 12, SW_TMA = 13;
+constexpr int S_QT = 32;                  // tokens per quarter
+constexpr int S_RAWSZ = 24576, S_NRAW = 3;  // B [32][128] 16 KB, X [32][64] 8 KB
+constexpr int SO_BH = 0, SO_BL = 8192, SO_XH = 16384, SO_XL = 20480, S_OPSZ = 24576;
+constexpr int S_OP = S_NRAW * S_RAWSZ;     // two operand stages
+constexpr int S_WF = S_OP + 2 * S_OPSZ;    // weights [2][128] float2, then [4] double2 warp totals
+constexpr int S_MISCB = S_WF + 2 * QT * 8 + 4 * 16 + 16;
+enum { SB_RAWF = 0, SB_RAWE = 3, SB_OPF = 6, SB_OPE = 8, SB_WRDY = 10, SB_WFREE = 12, SB_SDONE = 14, SB_TFREE = 16,
+       SB_DRAIN = 18, SB_N = 19 };
+constexpr int SMEM_STMA = S_MISCB + SB_N * 8 + 16 + 1024;
+static_assert(S_OP % 1024 == 0 && S_OPSZ % 1024 == 0, "swizzled tiles are 1024-byte aligned");
+static_assert(SMEM_STMA <= 232448, "one CTA per SM");
+
+__global__ void __launch_bounds__(SNTH, 1)
+    state_tma_kernel(const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x, ScanArgs a,
+                     CWs w) {
+    const int P = a.headdim, N = a.dstate, H = a.nheads;
+    const int nitems = a.batch * H * a.nchunks;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float2 *wfs = reinterpret_cast<float2 *>(sm + S_WF);                 // [2][QT]
+    double2 *wtot = reinterpret_cast<double2 *>(sm + S_WF + 2 * QT * 8);  // [4]
+    double2 *last = wtot + 4;                                             // (R, Theta) of the chunk
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S_MISCB);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bars + SB_N);
+    volatile int *abort_s = reinterpret_cast<volatile int *>(tslot + 1);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (tid == 0) {
+        for (int i = 0; i < S_NRAW; ++i) {
+            mbar_init(&bars[SB_RAWF + i], 1);
+            mbar_init(&bars[SB_RAWE + i], 256);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[SB_OPF + i], 256);
+            mbar_init(&bars[SB_OPE + i], 1);
+            mbar_init(&bars[SB_WRDY + i], 128);
+            mbar_init(&bars[SB_WFREE + i], 256);
+            mbar_init(&bars[SB_SDONE + i], 1);
+            mbar_init(&bars[SB_TFREE + i], 128);
+        }
+        mbar_init(&bars[SB_DRAIN], 1);
+        *abort_s = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot, sb = smem_u32(sm);
+
+    if (warp == SW_TMA) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            int r = 0;
+            bool ok = true;
+            for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+                const PItem t = p_item(a, it);
+                for (int tq = 0; tq < 4; ++tq) {
+                    const int slot = r % S_NRAW;
+                    ok = pwait(&bars[SB_RAWE + slot], ((r / S_NRAW) & 1) ^ 1, abort_s, a.dev_error);
+                    if (!ok) break;  // nothing more is issued after an abort
+                    uint8_t *dst = sm + slot * S_RAWSZ;
+                    uint64_t *full = &bars[SB_RAWF + slot];
+                    mbar_arrive_expect_tx(full, S_RAWSZ);
+                    tma_load_4d(dst, &tm_b, full, 0, t.g, t.c * QT + S_QT * tq, t.b);
+                    tma_load_4d(dst + 16384, &tm_x, full, 0, t.h, t.c * QT + S_QT * tq, t.b);
+                    ++r;
+                }
+            }
+            for (int slot = 0; slot < S_NRAW; ++slot)  // the last load of every slot has landed
+                if (r - 1 >= slot) {
+                    const int kl = r - 1 - (r - 1 - slot) % S_NRAW;
+                    const unsigned long long t0 = now_ns();
+                    while (!mbar_try_wait(&bars[SB_RAWF + slot], (kl / S_NRAW) & 1))
+                        if (now_ns() - t0 > WAIT_NS) {
+                            atomicCAS(a.dev_error, 0, DEV_TIMEOUT);
+                            break;
+                        }
+                }
+        }
+    } else if (warp >= SW_CONV && warp < SW_MMA) {
+        // -------------------------------------------------------- converters
+        const int ct = tid - SW_CONV * 32;  // 0..255
+        int r = 0, j = 0;
+        for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+            const int wb = j & 1;
+            pwait(&bars[SB_WRDY + wb], (j >> 1) & 1, abort_s, a.dev_error);  // chunk j's weights
+            const float2 *wf = wfs + wb * QT;
+#pragma unroll 1
+            for (int tq = 0; tq < 4; ++tq) {
+                const int o = 4 * j + tq, os = o & 1, slot = r % S_NRAW;
+                uint8_t *op = sm + S_OP + os * S_OPSZ;
+                pwait(&bars[SB_RAWF + slot], (r / S_NRAW) & 1, abort_s, a.dev_error);
+                pwait(&bars[SB_OPE + os], ((o >> 1) & 1) ^ 1, abort_s, a.dev_error);  // quarter o-2 is done
+                const float *raw = reinterpret_cast<const float *>(sm + slot * S_RAWSZ);
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {  // B''_s = w_s B_s as interleaved (re, im), rows s
+                    const int u = ct + 256 * i, sl = u >> 4, ch = u & 15;
+                    const float4 b0 = *reinterpret_cast<const float4 *>(raw + sl * 128 + 8 * ch);
+                    const float4 b1 = *reinterpret_cast<const float4 *>(raw + sl * 128 + 8 * ch + 4);
+                    const cf bq[4] = {{b0.x, b0.y}, {b0.z, b0.w}, {b1.x, b1.y}, {b1.z, b1.w}};
+                    const float2 ws = wf[S_QT * tq + sl];
+                    float val[8];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const cf z = cmul(bq[e], cf{ws.x, ws.y});
+                        val[2 * e] = z.re;
+                        val[2 * e + 1] = z.im;
+                    }
+                    put8(op, SO_BH, SO_BL, sw_off(sl, ch, S_QT * 128), val);
+                }
+                {  // X rows s as bf16 hi/lo
+                    const int sl = ct >> 3, ch = ct & 7;
+                    const float4 x0 = *reinterpret_cast<const float4 *>(raw + 4096 + sl * 64 + 8 * ch);
+                    const float4 x1 = *reinterpret_cast<const float4 *>(raw + 4096 + sl * 64 + 8 * ch + 4);
+                    float val[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                    put8(op, SO_XH, SO_XL, sw_off(sl, ch, S_QT * 128), val);
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&bars[SB_OPF + os]);
+                mbar_arrive(&bars[SB_RAWE + slot]);
+                ++r;
+            }
+            mbar_arrive(&bars[SB_WFREE + wb]);  // done with chunk j's weights
+            ++j;
+        }
+    } else if (warp == SW_MMA) {
+        // -------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int j = 0;
+            for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+                const int s = j & 1;
+                const uint32_t tm = tmem + 64 * s;
+                pwait(&bars[SB_TFREE + s], ((j >> 1) & 1) ^ 1, abort_s, a.dev_error);  // S of chunk j-2 is out
+#pragma unroll 1
+                for (int tq = 0; tq < 4; ++tq) {
+                    const int o = 4 * j + tq, os = o & 1;
+                    const uint32_t st = sb + S_OP + os * S_OPSZ;
+                    pwait(&bars[SB_OPF + os], (o >> 1) & 1, abort_s, a.dev_error);
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int pass = 0; pass < 3; ++pass) {  // hi.hi + hi.lo + lo.hi
+                        const uint32_t aB = st + (pass == 2 ? SO_BL : SO_BH), aX = st + (pass == 1 ? SO_XL : SO_XH);
+#pragma unroll 1
+                        for (int kk = 0; kk < S_QT / 16; ++kk)
+                            mma_ss(tm, smem_desc_sw128(aB + kk * 2048, S_QT * 128, 1024),
+                                   smem_desc_sw128(aX + kk * 2048, S_QT * 128, 1024), IDESC_S,
+                                   tq > 0 || pass > 0 || kk > 0);
+                    }
+                    mma_commit(&bars[SB_OPE + os]);
+                }
+                mma_commit(&bars[SB_SDONE + s]);
+                ++j;
+            }
+            mma_commit(&bars[SB_DRAIN]);
+            const unsigned long long t0 = now_ns();
+            while (!mbar_try_wait(&bars[SB_DRAIN], 0))
+                if (now_ns() - t0 > WAIT_NS) {
+                    atomicCAS(a.dev_error, 0, DEV_TIMEOUT);
+                    break;
+                }
+        }
+    } else if (warp < SW_CONV) {
+        // ------------------------------------- decays, then S of the chunk before
+        const int sq = tid;  // token 0..127
+        const int qd = warp;
+        auto state_out = [&](int jj, size_t bhc) {  // S[p][n] (complex) from TMEM lane k = 2n + (re, im), column p
+            const int s = jj & 1;
+            pwait(&bars[SB_SDONE + s], (jj >> 1) & 1, abort_s, a.dev_error);
+            tc_fence_after();
+            const int k = 32 * qd + lane;
+            float *S = reinterpret_cast<float *>(w.S + bhc * (size_t)P * N);
+#pragma unroll 1
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t rr[32];
+                tmem_ld32(tmem + 64 * s + ((uint32_t)(32 * qd) << 16) + cb, rr);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) S[((size_t)(cb + i) * N + (k >> 1)) * 2 + (k & 1)] = __uint_as_float(rr[i]);
+            }
+            tc_fence_before();
+            mbar_arrive(&bars[SB_TFREE + s]);
+        };
+        int j = 0;
+        size_t prev_bhc = 0;
+        for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
+            const PItem t = p_item(a, it);
+            const int wb = j & 1;
+            // the cumulative log-decay of the chunk in double (same sums, same order,
+            // as chunk_log_decay: a warp scan per 32 tokens, then the totals before)
+            const float Ar = a.A[2 * t.h], Ai = a.A[2 * t.h + 1];
+            const float d = sq < t.valid ? a.dt[(t.bt0 + sq) * H + t.h] : 0.f;
+            double vr = (double)d * Ar, vi = (double)d * Ai;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double yr = __shfl_up_sync(0xffffffffu, vr, o), yi = __shfl_up_sync(0xffffffffu, vi, o);
+                if (lane >= o) vr += yr, vi += yi;
+            }
+            if (lane == 31) wtot[qd] = make_double2(vr, vi);
+            named_bar_sync(1, 128);
+            if (qd > 0) {
+                double pr = wtot[0].x, pi = wtot[0].y;
+                for (int q = 1; q < qd; ++q) pr += wtot[q].x, pi += wtot[q].y;
+                vr += pr, vi += pi;
+            }
+            if (sq == QT - 1) *last = make_double2(vr, vi);
+            named_bar_sync(1, 128);
+            const double R = last->x, Th = last->y;
+            // weights of B'' (slot wb: the converters are done with chunk j-2's)
+            pwait(&bars[SB_WFREE + wb], ((j >> 1) & 1) ^ 1, abort_s, a.dev_error);
+            {
+                double sn, cn;
+                sincos(Th - vi, &sn, &cn);
+                const float m = (float)exp(R - vr) * d;
+                wfs[wb * QT + sq] = make_float2(m * (float)cn, m * (float)sn);
+            }
+            mbar_arrive(&bars[SB_WRDY + wb]);
+            // the chunk scan's factors, or the log-decays of a steep chunk; Lambda
+            float2 *fac = reinterpret_cast<float2 *>(w.cs + (t.bhc * 2) * QT);
+            if (fabs(R) > SPAN) {
+                w.cs[(t.bhc * 2) * QT + sq] = vr;
+                w.cs[(t.bhc * 2 + 1) * QT + sq] = vi;
+            } else {
+                const double rho = 0.5 * R;
+                double sn, cn;
+                sincos(vi, &sn, &cn);
+                const float ec = (float)exp(vr - rho), eb = (float)exp(rho - vr) * d;
+                fac[sq] = make_float2(ec * (float)cn, ec * (float)sn);
+                fac[QT + sq] = make_float2(eb * (float)cn, -eb * (float)sn);
+            }
+            if (sq == 0) {
+                w.lam[t.bhc * 2] = R;
+                w.lam[t.bhc * 2 + 1] = Th;
+            }
+            if (j > 0) state_out(j - 1, prev_bhc);
+            prev_bhc = t.bhc;
+            ++j;
+        }
+        if (j > 0) state_out(j - 1, prev_bhc);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 // The chunks the factored form cannot take (|Re Lambda| > SPAN): the CUDA-core tile
 // code, one CTA per chunk in a loop over all chunks.  smem: cplx_scan_tile_smem(QT).
 template <typename T> __global__ void __launch_bounds__(NTH) steep_chunks_kernel(ScanArgs a, CWs w, CplxView<T> v) {
     extern __shared__ uint8_t smem_raw[];
-    grid_dep_wait();  // the chunk scan before it (and so the state pass) is complete
     const int nitems = a.batch * a.nheads * a.nchunks;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x) {
         const PItem t = p_item(a, it);
