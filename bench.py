@@ -667,7 +667,7 @@ def bench_ours(args, shape):
     if tc_path:
         kernel, src_name = "ssd_scan_tc_kernel", "scan_tc.cu"
     elif cplx and shape.headdim == 64 and shape.dstate == 64:  # the tcgen05 complex kernels
-        kernel, src_name = ("state_tma_kernel+cplx_state_pass+scan_tma_kernel+steep_chunks_kernel (4 launches, tcgen05, timed as one call)",
+        kernel, src_name = ("state_kernel+cplx_state_pass+scan_kernel (3 launches, tcgen05, timed as one call)",
                             "scan_complex_tc.cuh")
     elif cplx:
         kernel, src_name = "cplx_chunk_state+cplx_state_pass+cplx_chunk_scan (3 kernels)", "scan_complex.cu"

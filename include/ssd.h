@@ -79,10 +79,8 @@ size_t ssd_scan_workspace_size(int batch, int seqlen, int nheads, int headdim,
 
 /*
  * Number of kernels that one ssd_scan_fwd / ssd_scan_fwd_complex call with these
- * sizes enqueues when seqlen > 0 (0 for invalid sizes); for the complex scan with
- * head dim 64 and 64 states it assumes 16-byte aligned x, B and C (one launch
- * fewer otherwise).  For capture planning and launch accounting; it launches
- * nothing.
+ * sizes enqueues when seqlen > 0 (0 for invalid sizes).  For capture planning
+ * and launch accounting; it launches nothing.
  */
 int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int ngroups,
                              int dstate, int chunk_size, int is_complex, ssd_dtype io_dtype);

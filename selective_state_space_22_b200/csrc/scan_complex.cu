@@ -22,11 +22,6 @@
 // [u_re, -u_im] . [v_re, v_im], so all four contractions are real GEMMs with
 // K = 2N, register-tiled below.  Three kernels, as in the real CUDA-core path:
 // chunk state, the sequential state pass over chunks, and the chunk scan.
-#include <cudaTypedefs.h>
-
-#include <algorithm>
-#include <mutex>
-
 #include "cplx_view.cuh"
 #include "ssd_internal.cuh"
 #include "tc_ptx.cuh"
@@ -716,104 +711,7 @@ cudaError_t launch_complex_view(const ScanArgs &a, const CplxView<T> &v, void *w
     return launch_complex_cuda_cores<T>(a, v, ws, st);
 }
 
-// ---------------------------------------------------- TMA-fed tensor-core path
-PFN_cuTensorMapEncodeTiled_v12000 g_cplx_encode = nullptr;
-std::once_flag g_cplx_encode_once;
-
-// A float32 tensor map without swizzle (rank 2 or 4; strides in bytes for
-// dimensions 1..rank-1), zero fill outside the tensor.
-cudaError_t make_map_f32(CUtensorMap *m, const void *base, int rank, const cuuint64_t *dims, const cuuint64_t *strides,
-                         const cuuint32_t *box) {
-    std::call_once(g_cplx_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_cplx_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    if (!g_cplx_encode) return cudaErrorNotSupported;
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    const CUresult r = g_cplx_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, rank, const_cast<void *>(base), dims, strides,
-                                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
-// float32 x, B, C in the plain layout, 16-byte aligned: chunk states, state pass,
-// the TMA-fed persistent chunk scan and the steep chunks (4 launches).
-bool cplx_tma_ok(const ScanArgs &a) {
-    return cplx_tc_supported(a.headdim, a.dstate) && a.seqlen > 0 && a.batch > 0 &&
-           ((reinterpret_cast<uintptr_t>(a.x) | reinterpret_cast<uintptr_t>(a.B) | reinterpret_cast<uintptr_t>(a.C)) &
-            15) == 0;
-}
-
-cudaError_t launch_complex_tma(const ScanArgs &a0, void *ws, cudaStream_t st) {
-    ScanArgs a = a0;
-    a.chunk = ctc::QT;
-    a.nchunks = (a.seqlen + ctc::QT - 1) / ctc::QT;
-    const CWs w = carve_c(ws, a);
-    const CplxView<float> v = plain_view(a);
-    const int N2 = 2 * a.dstate, P = a.headdim, G = a.ngroups, H = a.nheads, T = a.seqlen, Bt = a.batch;
-    const long long nbhc = (long long)Bt * H * a.nchunks;
-    CUtensorMap mc, mb, mx, mh;
-    cudaError_t e;
-    {  // B and C: floats [b][t][g][2N] (re, im interleaved); box 32 floats x 128 tokens
-        const cuuint64_t dims[4] = {(cuuint64_t)N2, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)Bt};
-        const cuuint64_t str[3] = {(cuuint64_t)N2 * 4, (cuuint64_t)G * N2 * 4, (cuuint64_t)T * G * N2 * 4};
-        const cuuint32_t box[4] = {32, 1, (cuuint32_t)ctc::QT, 1};
-        if ((e = make_map_f32(&mc, a.C, 4, dims, str, box)) != cudaSuccess) return e;
-        if ((e = make_map_f32(&mb, a.B, 4, dims, str, box)) != cudaSuccess) return e;
-    }
-    {  // x: [b][t][h][P]; box P x 128 tokens
-        const cuuint64_t dims[4] = {(cuuint64_t)P, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
-        const cuuint64_t str[3] = {(cuuint64_t)P * 4, (cuuint64_t)H * P * 4, (cuuint64_t)T * H * P * 4};
-        const cuuint32_t box[4] = {(cuuint32_t)P, 1, (cuuint32_t)ctc::QT, 1};
-        if ((e = make_map_f32(&mx, a.x, 4, dims, str, box)) != cudaSuccess) return e;
-    }
-    {  // h_in in the workspace: floats [b h chunk][P][2N]; box 32 floats x P rows
-        const cuuint64_t dims[2] = {(cuuint64_t)N2, (cuuint64_t)(nbhc * P)};
-        const cuuint64_t str[1] = {(cuuint64_t)N2 * 4};
-        const cuuint32_t box[2] = {32, (cuuint32_t)P};
-        if ((e = make_map_f32(&mh, w.S, 2, dims, str, box)) != cudaSuccess) return e;
-    }
-    CUtensorMap msb, msx;  // the chunk-state kernel's token quarters of B [32 t][2N] and x [32 t][P]
-    {
-        const cuuint64_t dims[4] = {(cuuint64_t)N2, (cuuint64_t)G, (cuuint64_t)T, (cuuint64_t)Bt};
-        const cuuint64_t str[3] = {(cuuint64_t)N2 * 4, (cuuint64_t)G * N2 * 4, (cuuint64_t)T * G * N2 * 4};
-        const cuuint32_t box[4] = {(cuuint32_t)N2, 1, (cuuint32_t)ctc::S_QT, 1};
-        if ((e = make_map_f32(&msb, a.B, 4, dims, str, box)) != cudaSuccess) return e;
-    }
-    {
-        const cuuint64_t dims[4] = {(cuuint64_t)P, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)Bt};
-        const cuuint64_t str[3] = {(cuuint64_t)P * 4, (cuuint64_t)H * P * 4, (cuuint64_t)T * H * P * 4};
-        const cuuint32_t box[4] = {(cuuint32_t)P, 1, (cuuint32_t)ctc::S_QT, 1};
-        if ((e = make_map_f32(&msx, a.x, 4, dims, str, box)) != cudaSuccess) return e;
-    }
-    if ((e = cudaFuncSetAttribute(ctc::state_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  ctc::SMEM_STMA)) != cudaSuccess)
-        return e;
-    if ((e = cudaFuncSetAttribute(ctc::scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  ctc::SMEM_TMA)) != cudaSuccess)
-        return e;
-    const int steep_smem = (int)cplx_scan_tile_smem(ctc::QT);
-    if ((e = cudaFuncSetAttribute(ctc::steep_chunks_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  steep_smem)) != cudaSuccess)
-        return e;
-    int dev = 0, sms = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int nitems = (int)nbhc, grid1 = std::min(nitems, sms);
-    ctc::state_tma_kernel<<<grid1, ctc::SNTH, ctc::SMEM_STMA, st>>>(msb, msx, a, w);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_cplx_state_pass(a, ws, st)) != cudaSuccess) return e;
-    ctc::scan_tma_kernel<<<grid1, ctc::TNTH, ctc::SMEM_TMA, st>>>(mc, mb, mx, mh, a, w);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    ctc::steep_chunks_kernel<float><<<grid1, ctc::NTH, steep_smem, st>>>(a, w, v);
-    return cudaGetLastError();
-}
-
 cudaError_t launch_complex_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
-    if (cplx_tma_ok(a)) return launch_complex_tma(a, ws, st);
     return launch_complex_view<float>(a, plain_view(a), ws, st);
 }
 

@@ -112,9 +112,7 @@ Plan plan_scan(int batch, int seqlen, int nheads, int headdim, int ngroups, int 
     if (cplx && ssd::cplx_tc_supported(headdim, dstate)) {  // tensor-core path: 128-token chunks
         p.ws = ssd::generic_workspace_bytes(batch, nheads, headdim, dstate, 128, seqlen > 0 ? (seqlen + 127) / 128 : 0,
                                             true);
-        // chunk states, state pass, the TMA-fed chunk scan and its steep chunks (three
-        // launches when x, B or C is not 16-byte aligned: the per-chunk scan kernel)
-        p.launches = 4;
+        p.launches = 3;
         return p;
     }
     p.ws = ssd::generic_workspace_bytes(batch, nheads, headdim, dstate, chunk, nchunks, cplx);
