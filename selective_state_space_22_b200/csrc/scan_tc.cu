@@ -304,6 +304,22 @@ __device__ __forceinline__ void scale_row(const uint8_t *src, uint8_t *dst, int 
     for (int j = 0; j < 8; ++j) reinterpret_cast<uint4 *>(dst)[j ^ key] = q[j];
 }
 
+// A state-only tile's W: the math warpgroup, which has no M to build for it,
+// scales this thread's row of X into the C half of the tile's {C, B} slot.  Out of
+// line, so that the M build's loop keeps its size.
+__device__ __noinline__ void state_only_w_row(const uint8_t *x_row, uint8_t *w_row, int key, float f) {
+    scale_row(x_row, w_row, key, __float2bfloat162_rn(f));
+}
+
+// SPLIT: the state-only form (no y: every tile state-only).  Then the math
+// warpgroup, which has no M to build, builds each tile's W into the C half of the
+// tile's {C, B} slot (TMA loads only B there), free once the tile two before has
+// released the slot; W of one tile then does not wait for S of the one before, and
+// the epilogue warpgroup only computes the decays (1.24 against 1.49 us per tile
+// at T = 65536, 64 heads).  Otherwise the epilogue warpgroup builds every W, a
+// run's state-only prefix included, into the one W buffer: the same change slowed
+// the full tiles of a launch by 4-15%, more than the prefix gains.
+template <bool SPLIT>
 __global__ void __launch_bounds__(NTH, 1)
     ssd_scan_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                        const __grid_constant__ CUtensorMap tm_c, const TcParams p) {
@@ -383,12 +399,12 @@ __global__ void __launch_bounds__(NTH, 1)
     } else if (warp == 1) {
         // ------------------------------------------- MMA issuer: G and S
         if (lane == 0) {
-            const uint32_t aW = sbase + OFF_W;
             for (int k = 0; k < ntl; ++k) {
                 const bool so = decode_tile(p, k).state_only;
                 const int s = k & 1;
                 const uint32_t par = (k >> 1) & 1, tm = tmem + 256 * s;
                 const uint32_t aC = sbase + s * CB_BYTES + OFF_C, aB = sbase + s * CB_BYTES + OFF_B;
+                const uint32_t aW = (SPLIT && so) ? aC : sbase + OFF_W;
                 mbar_wait(&bars[B_FULL + s], par, p, abort_s);
                 mbar_wait(&bars[B_FREE + s], par ^ 1, p, abort_s);
                 tc_fence_after();
@@ -467,6 +483,17 @@ __global__ void __launch_bounds__(NTH, 1)
             const float *csk = cs + s * QT, *dtk = dtv + s * QT, *bfk = bfac + s * QT;
             mbar_wait(&bars[B_CS + s], par, p, abort_s);
             const float v = csk[row], Dh = dh_s[s];
+            if constexpr (SPLIT) {
+                if (so) {  // W of a state-only tile, into its slot's C half
+                    const int xs = k % X_SLOTS;
+                    mbar_wait(&bars[B_EMPTY + s], par ^ 1, p, abort_s);
+                    mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s);
+                    state_only_w_row(sm + OFF_XR + xs * 16384 + row * 128, sm + s * CB_BYTES + OFF_C + row * 128,
+                                     row & 7, __expf(csk[QT - 1] - v) * dtk[row]);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bars[B_W + s]);
+                }
+            }
             mbar_wait(&bars[B_G + s], par, p, abort_s);
             tc_fence_after();
             if (!so) {
@@ -585,22 +612,25 @@ __global__ void __launch_bounds__(NTH, 1)
                 bfk[row] = __expf(csk[row & ~31] - v) * d;  // exp(A_cs[r] - A_cs[s]) dt_s, r = s's 32-block start
                 named_bar_sync(BAR_MATH, 128);  // every row's decays written
                 mbar_arrive(&bars[B_CS + s]);
-                // W (one buffer): the previous tile's S must have read it
-                const int xs = k % X_SLOTS;
-                mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s);
-                if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s);
-                // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
-                // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
-                // SM sub-partition also builds the most M blocks, skips it and the warp
-                // of quadrant 0 (the fewest) takes those rows too.
-                auto w_row = [&](int r) {
-                    scale_row(sm + OFF_XR + xs * 16384 + r * 128, sm + OFF_W + r * 128, r & 7,
-                              __float2bfloat162_rn(__expf(lam - csk[r]) * dtk[r]));
-                };
-                if (quad != 3) w_row(row);
-                if (quad == 0) w_row(96 + lane);
-                fence_proxy_async_smem();
-                mbar_arrive(&bars[B_W + s]);
+                // W (one buffer): the previous tile's S must have read it.  With SPLIT,
+                // the math warpgroup builds a state-only tile's W.
+                if (!(SPLIT && cur.state_only)) {
+                    const int xs = k % X_SLOTS;
+                    mbar_wait(&bars[B_XFULL + xs], (k / X_SLOTS) & 1, p, abort_s);
+                    if (k > 0) mbar_wait(&bars[B_S + (s ^ 1)], ((k - 1) >> 1) & 1, p, abort_s);
+                    // W row = exp(lam - A_cs[row]) dt x_row (a row keeps its swizzled chunk
+                    // places).  W needs no TMEM lane, so the warp of lane quadrant 3, whose
+                    // SM sub-partition also builds the most M blocks, skips it and the warp
+                    // of quadrant 0 (the fewest) takes those rows too.
+                    auto w_row = [&](int r) {
+                        scale_row(sm + OFF_XR + xs * 16384 + r * 128, sm + OFF_W + r * 128, r & 7,
+                                  __float2bfloat162_rn(__expf(lam - csk[r]) * dtk[r]));
+                    };
+                    if (quad != 3) w_row(row);
+                    if (quad == 0) w_row(96 + lane);
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bars[B_W + s]);
+                }
             }
             if (k > 0) {  // y of tile k-1
                 const int j = k - 1, s = j & 1;
@@ -737,7 +767,10 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
         void *ctx = current_context();
         if (!di.init || di.ctx != ctx) {
             di.init = false;
-            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          SMEM_ALLOC)) != cudaSuccess)
+                return e;
+            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                           SMEM_ALLOC)) != cudaSuccess)
                 return e;
             if ((e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
@@ -787,7 +820,8 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     cfg.blockDim = dim3(NTH);
     cfg.dynamicSmemBytes = SMEM_ALLOC;
     cfg.stream = st;
-    return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel, mx, mb, mc, p);
+    if (!a.y) return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel<true>, mx, mb, mc, p);
+    return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel<false>, mx, mb, mc, p);
 }
 
 }  // namespace ssd
