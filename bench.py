@@ -607,7 +607,8 @@ def bench_ours(args, shape):
     launches = ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
                                             shape.ngroups, shape.dstate, shape.chunk, cplx, io)
     tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
-    kernel_chunk = 128 if tc_path else shape.chunk  # the tensor-core kernel tiles 128 tokens
+    cplx_tc = cplx and shape.headdim == 64 and shape.dstate == 64  # the tcgen05 complex kernels
+    kernel_chunk = 128 if (tc_path or cplx_tc) else shape.chunk  # the tensor-core kernels tile 128 tokens
 
     def step(dd=d, yy=y, ff=fs, w=ws):
         fn(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["init_state"], chunk_size=shape.chunk,
@@ -666,7 +667,7 @@ def bench_ours(args, shape):
         achieved, peak, unit = aflops / t_launch / 1e12, peaks["bf16_tflops"], "TFLOP/s"
     if tc_path:
         kernel, src_name = "ssd_scan_tc_kernel", "scan_tc.cu"
-    elif cplx and shape.headdim == 64 and shape.dstate == 64:  # the tcgen05 complex kernels
+    elif cplx_tc:
         kernel, src_name = ("state_kernel+cplx_state_pass+scan_kernel (3 launches, tcgen05, timed as one call)",
                             "scan_complex_tc.cuh")
     elif cplx:
