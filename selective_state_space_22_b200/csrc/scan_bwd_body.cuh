@@ -53,6 +53,29 @@
 #define BWD_UNROLL
 #endif
 
+// On the device the operand rows come in as 16-byte asynchronous copies
+// (cp.async, zero-filled past the sequence end or the row's width) when the rows
+// are whole 16-byte units, so a thread has all its copies of a phase in flight
+// at once instead of a few registers' worth; bwd_async_wait() at the end of the
+// loading phase waits for them.  The host harness takes the scalar loops.
+#ifndef SSD_BWD_ASYNC_DEFINED
+#define SSD_BWD_ASYNC_DEFINED
+#ifdef __CUDA_ARCH__
+__device__ inline void bwd_cp16(float *dst, const float *src, bool valid) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ inline void bwd_async_wait() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+#else
+inline void bwd_async_wait() {}
+#endif
+// rows of `width` floats starting at src can be copied in 16-byte units
+__host__ __device__ inline bool bwd_vec_rows(const float *src, int width) {
+    return width % 4 == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+}
+#endif
+
 namespace ssd {
 namespace bwd {
 
@@ -63,6 +86,7 @@ constexpr int N_MAX = 128;   // state dim
 // Shared-memory row strides: four floats longer than a row, so rows stay 16-byte
 // aligned and consecutive rows start 4 banks apart.
 constexpr int PS = P_MAX + 4, NS = N_MAX + 4, QS = QB + 4;
+constexpr int PASS_GRP = 8;  // chunks whose loads a state pass issues together
 
 struct BwdArgs {
     const float *x, *dt, *A, *B, *C, *D, *init, *dy, *dfinal;
@@ -133,10 +157,11 @@ struct Smem {
     float *rowE, *colG, *F, *Ksr;     // [QB]
     float *red;                       // [2 * QB]
     float *part;                      // [QB][16]: partial row sums, one per thread column
-    float *misc;                      // [4]: lam, ...
+    float *el;                        // [QB]: exp(lam - acs)
+    float *misc;                      // [4]: lam, exp(lam) <Gh, h_in>, dy . x, sum_s w_s Ksr[s]
 };
 constexpr size_t SMEM_FLOATS = 4 * QB + 2 * QB * PS + 2 * QB * NS + 2 * P_MAX * NS + 3 * QB * QS +
-                               4 * QB + 2 * QB + 16 * QB + 4;
+                               4 * QB + 2 * QB + 16 * QB + QB + 4;
 // The chunk-state phase uses the layout up to Bs, the readout phase up to Cs.
 constexpr size_t SMEM_FLOATS_K1 = 4 * QB + 2 * QB * PS + QB * NS;
 constexpr size_t SMEM_FLOATS_K3 = 4 * QB + 2 * QB * PS + 2 * QB * NS;
@@ -161,6 +186,7 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.Ksr = s; s += QB;
     m.red = s; s += 2 * QB;
     m.part = s; s += 16 * QB;
+    m.el = s; s += QB;
     m.misc = s;
     return m;
 }
@@ -247,6 +273,16 @@ __host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, i
 }
 __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
                                             float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, a.headdim)) {
+        for (int i = tid; i < QB * (P_MAX / 4); i += NT) {
+            const int s = i / (P_MAX / 4), p = 4 * (i % (P_MAX / 4)), t = c * QB + s;
+            const bool v = t < a.seqlen && p < a.headdim;
+            bwd_cp16(dst + s * PS + p, v ? src + ix_x(a, b, t, h, p) : src, v);
+        }
+        return;
+    }
+#endif
     BWD_UNROLL
     for (int i = tid; i < QB * P_MAX; i += NT) {
         const int s = i / P_MAX, p = i % P_MAX, t = c * QB + s;
@@ -255,6 +291,16 @@ __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, 
 }
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, a.dstate)) {
+        for (int i = tid; i < QB * (N_MAX / 4); i += NT) {
+            const int s = i / (N_MAX / 4), n = 4 * (i % (N_MAX / 4)), t = c * QB + s;
+            const bool v = t < a.seqlen && n < a.dstate;
+            bwd_cp16(dst + s * NS + n, v ? src + ix_bc(a, b, t, g, n) : src, v);
+        }
+        return;
+    }
+#endif
     BWD_UNROLL
     for (int i = tid; i < QB * N_MAX; i += NT) {
         const int s = i / N_MAX, n = i % N_MAX, t = c * QB + s;
@@ -262,6 +308,16 @@ __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, 
     }
 }
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, a.dstate)) {
+        for (int i = tid; i < P_MAX * (N_MAX / 4); i += NT) {
+            const int p = i / (N_MAX / 4), n = 4 * (i % (N_MAX / 4));
+            const bool v = p < a.headdim && n < a.dstate;
+            bwd_cp16(dst + p * NS + n, v ? src + (size_t)p * a.dstate + n : src, v);
+        }
+        return;
+    }
+#endif
     BWD_UNROLL
     for (int i = tid; i < P_MAX * N_MAX; i += NT) {
         const int p = i / N_MAX, n = i % N_MAX;
@@ -287,6 +343,7 @@ __host__ __device__ inline void k1_load(const BwdArgs &a, int c, int h, int b, i
     load_dt(a, c, h, b, tid, m);
     load_rows_p(a, a.x, c, h, b, tid, m.X);
     load_rows_n(a, a.B, c, group_of(a, h), b, tid, m.Bs);
+    bwd_async_wait();
 }
 // Thread 0: the inclusive cumulative decay, lam and w.
 __host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
@@ -316,10 +373,17 @@ __host__ __device__ inline void k2_pass(const BwdArgs &a, int blk, int h, int b,
     const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
     if (i >= pn) return;
     float hv = a.init ? a.init[ix_bh(a, b, h) * pn + i] : 0.f;
-    for (int c = 0; c < a.nchunks; ++c) {
-        const size_t o = ix_pn(a, b, h, c) + i;
-        a.hin[o] = hv;
-        hv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * hv + a.st[o];
+    for (int c0 = 0; c0 < a.nchunks; c0 += PASS_GRP) {  // a group's loads in flight together
+        float sv[PASS_GRP], lv[PASS_GRP];
+        for (int j = 0; j < PASS_GRP; ++j)
+            if (c0 + j < a.nchunks) {
+                sv[j] = BWD_LDG(a.st + ix_pn(a, b, h, c0 + j) + i);
+                lv[j] = BWD_LDG(a.lam + ix_bh(a, b, h) * a.nchunks + c0 + j);
+            }
+        for (int j = 0; j < PASS_GRP && c0 + j < a.nchunks; ++j) {
+            a.hin[ix_pn(a, b, h, c0 + j) + i] = hv;
+            hv = expf(lv[j]) * hv + sv[j];
+        }
     }
 }
 
@@ -329,6 +393,7 @@ __host__ __device__ inline void k3_load(const BwdArgs &a, int c, int h, int b, i
     for (int i = tid; i < QB; i += NT) m.e[i] = expf(BWD_LDG(acs_g + i));
     load_rows_p(a, a.dy, c, h, b, tid, m.dY);
     load_rows_n(a, a.C, c, group_of(a, h), b, tid, m.Cs);
+    bwd_async_wait();
 }
 __host__ __device__ inline void k3_r(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     float acc[4][8];
@@ -342,10 +407,17 @@ __host__ __device__ inline void k4_pass(const BwdArgs &a, int blk, int h, int b,
     const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
     if (i >= pn) return;
     float gv = a.dfinal ? a.dfinal[ix_bh(a, b, h) * pn + i] : 0.f;
-    for (int c = a.nchunks - 1; c >= 0; --c) {
-        const size_t o = ix_pn(a, b, h, c) + i;
-        a.gh[o] = gv;
-        gv = expf(a.lam[ix_bh(a, b, h) * a.nchunks + c]) * gv + a.st[o];
+    for (int c0 = a.nchunks - 1; c0 >= 0; c0 -= PASS_GRP) {  // chunks c0, c0 - 1, ...
+        float sv[PASS_GRP], lv[PASS_GRP];
+        for (int j = 0; j < PASS_GRP; ++j)
+            if (c0 - j >= 0) {
+                sv[j] = BWD_LDG(a.st + ix_pn(a, b, h, c0 - j) + i);
+                lv[j] = BWD_LDG(a.lam + ix_bh(a, b, h) * a.nchunks + c0 - j);
+            }
+        for (int j = 0; j < PASS_GRP && c0 - j >= 0; ++j) {
+            a.gh[ix_pn(a, b, h, c0 - j) + i] = gv;
+            gv = expf(lv[j]) * gv + sv[j];
+        }
     }
     if (a.dinit) a.dinit[ix_bh(a, b, h) * pn + i] = gv;
 }
@@ -362,7 +434,8 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
         const float ac = BWD_LDG(acs_g + i);
         m.acs[i] = ac;
         m.e[i] = expf(ac);
-        m.w[i] = expf(lam - ac) * d;
+        m.el[i] = expf(lam - ac);
+        m.w[i] = m.el[i] * d;
     }
     if (tid == 0) m.misc[0] = lam;
     load_rows_p(a, a.x, c, h, b, tid, m.X);
@@ -371,6 +444,7 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     load_rows_n(a, a.C, c, g, b, tid, m.Cs);
     load_pn(a, a.hin + ix_pn(a, b, h, c), tid, m.Hin);
     load_pn(a, a.gh + ix_pn(a, b, h, c), tid, m.Gh);
+    bwd_async_wait();
 }
 // GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY; thread tile rows
 // l = 4 tr + i, columns s = tc + 16 j.
@@ -501,27 +575,34 @@ __host__ __device__ inline void k5_dc(const BwdArgs &a, int c, int h, int b, int
         }
     }
 }
-// F from its partial sums.
+// F from its partial sums; three other threads form the sums the decay gradient
+// needs (each in token order), so that the one thread of k5_decay only runs the
+// reverse cumulative sum.
 __host__ __device__ inline void k5_f(const BwdArgs &a, int tid, const Smem &m) {
     (void)a;
     if (tid < QB) {
         float v = 0.f;
         for (int q = 0; q < 16; ++q) v += m.part[tid * 16 + q];
         m.F[tid] = m.e[tid] * v;
+    } else if (tid == QB) {
+        float h0 = 0.f;
+        for (int r = 0; r < QB; ++r) h0 += m.red[r];
+        m.misc[1] = h0 * expf(m.misc[0]);
+    } else if (tid == QB + 32) {
+        float dd = 0.f;
+        for (int r = 0; r < QB; ++r) dd += m.red[QB + r];
+        m.misc[2] = dd;
+    } else if (tid == QB + 64) {
+        float ksum = 0.f;
+        for (int r = 0; r < QB; ++r) ksum += m.w[r] * m.Ksr[r];
+        m.misc[3] = ksum;
     }
 }
 // Thread 0: the decay gradient (reverse cumulative sum), ddt, and the dA and dD
 // partials of this chunk.
 __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     if (tid != 0) return;
-    const float lam = m.misc[0], Ah = a.A[h];
-    float h0 = 0.f, dd = 0.f, ksum = 0.f;
-    for (int r = 0; r < QB; ++r) {
-        h0 += m.red[r];
-        dd += m.red[QB + r];
-        ksum += m.w[r] * m.Ksr[r];
-    }
-    h0 *= expf(lam);
+    const float Ah = a.A[h], h0 = m.misc[1], dd = m.misc[2], ksum = m.misc[3];
     // colsum of E = dt_t * colsum of GL o XY
     float run = 0.f, dAp = 0.f;
     for (int t = QB - 1; t >= 0; --t) {
@@ -530,7 +611,7 @@ __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, 
         run += dacs;  // dalpha[t] = sum_{t' >= t} dacs[t']
         const int tg = c * QB + t;
         if (tg < a.seqlen)
-            a.ddt[ix_dt(a, b, tg, h)] = m.colG[t] + expf(lam - m.acs[t]) * m.Ksr[t] + Ah * run;
+            a.ddt[ix_dt(a, b, tg, h)] = m.colG[t] + m.el[t] * m.Ksr[t] + Ah * run;
         dAp += m.d[t] * run;
     }
     a.dAp[ix_bh(a, b, h) * a.nchunks + c] = dAp;

@@ -40,6 +40,29 @@
 #define BWDC_UNROLL
 #endif
 
+// On the device the operand rows come in as 16-byte asynchronous copies
+// (cp.async, zero-filled past the sequence end or the row's width) when the rows
+// are whole 16-byte units, so a thread has all its copies of a phase in flight
+// at once instead of a few registers' worth; bwd_async_wait() at the end of the
+// loading phase waits for them.  The host harness takes the scalar loops.
+#ifndef SSD_BWD_ASYNC_DEFINED
+#define SSD_BWD_ASYNC_DEFINED
+#ifdef __CUDA_ARCH__
+__device__ inline void bwd_cp16(float *dst, const float *src, bool valid) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ inline void bwd_async_wait() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+#else
+inline void bwd_async_wait() {}
+#endif
+// rows of `width` floats starting at src can be copied in 16-byte units
+__host__ __device__ inline bool bwd_vec_rows(const float *src, int width) {
+    return width % 4 == 0 && (reinterpret_cast<uintptr_t>(src) & 15) == 0;
+}
+#endif
+
 namespace ssd {
 namespace bwdc {
 
@@ -51,6 +74,7 @@ constexpr int RED = 64;       // threads of the block reductions
 // Row strides in floats: 4 more than a row, so rows stay 16-byte aligned and
 // consecutive rows start 4 banks apart.
 constexpr int PS = P_MAX + 4, NS = 2 * N_MAX + 4, QS2 = 2 * QC + 4, QS1 = QC + 4;
+constexpr int PASS_GRP = 8;  // chunks whose loads a state pass issues together
 
 struct c2 {
     float re, im;
@@ -140,10 +164,11 @@ struct Smem {
     float *rowE, *colG, *F, *Ksr;  // [QC][2]
     float *red;                  // [3][RED]: <conj(Gh), h_in> re, im; dy.x
     float *part;                 // [2][QC][16][2]: per-thread-column terms of Ksr and F
-    float *misc;                 // [4]: lam re, im
+    float *el;                   // [QC][2]: exp(lam - acs)
+    float *misc;                 // [8]: lam; exp(lam) <conj(Gh), h_in>; dy.x
 };
 constexpr size_t SMEM_FLOATS = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS + 2 * P_MAX * NS + 2 * QC * QS2 +
-                               QC * QS1 + 4 * 2 * QC + 3 * RED + 2 * QC * 16 * 2 + 4;
+                               QC * QS1 + 4 * 2 * QC + 3 * RED + 2 * QC * 16 * 2 + 2 * QC + 8;
 // The chunk-state phase uses the layout up to Bs, the readout phase up to Cs.
 constexpr size_t SMEM_FLOATS_K1 = QC + 3 * 2 * QC + 2 * QC * PS + QC * NS;
 constexpr size_t SMEM_FLOATS_K3 = QC + 3 * 2 * QC + 2 * QC * PS + 2 * QC * NS;
@@ -168,6 +193,7 @@ __host__ __device__ inline Smem smem_map(float *s) {
     m.Ksr = s; s += 2 * QC;
     m.red = s; s += 3 * RED;
     m.part = s; s += 2 * QC * 16 * 2;
+    m.el = s; s += 2 * QC;
     m.misc = s;
     return m;
 }
@@ -181,6 +207,16 @@ __host__ __device__ inline void load_dt(const BwdArgs &a, int c, int h, int b, i
 }
 __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, int c, int h, int b, int tid,
                                             float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, a.headdim)) {
+        for (int i = tid; i < QC * (P_MAX / 4); i += NT) {
+            const int s = i / (P_MAX / 4), p = 4 * (i % (P_MAX / 4)), t = c * QC + s;
+            const bool v = t < a.seqlen && p < a.headdim;
+            bwd_cp16(dst + s * PS + p, v ? src + ix_x(a, b, t, h, p) : src, v);
+        }
+        return;
+    }
+#endif
     BWDC_UNROLL
     for (int i = tid; i < QC * P_MAX; i += NT) {
         const int s = i / P_MAX, p = i % P_MAX, t = c * QC + s;
@@ -190,6 +226,16 @@ __host__ __device__ inline void load_rows_p(const BwdArgs &a, const float *src, 
 // complex rows of B or C: [QC][N] pairs
 __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, int c, int g, int b, int tid,
                                             float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, 2 * a.dstate)) {
+        for (int i = tid; i < QC * (2 * N_MAX / 4); i += NT) {
+            const int s = i / (2 * N_MAX / 4), f = 4 * (i % (2 * N_MAX / 4)), t = c * QC + s;
+            const bool v = t < a.seqlen && f < 2 * a.dstate;
+            bwd_cp16(dst + s * NS + f, v ? src + 2 * ix_bc(a, b, t, g, 0) + f : src, v);
+        }
+        return;
+    }
+#endif
     BWDC_UNROLL
     for (int i = tid; i < QC * 2 * N_MAX; i += NT) {
         const int s = i / (2 * N_MAX), f = i % (2 * N_MAX), t = c * QC + s;
@@ -198,6 +244,16 @@ __host__ __device__ inline void load_rows_n(const BwdArgs &a, const float *src, 
 }
 // a complex [P][N] block
 __host__ __device__ inline void load_pn(const BwdArgs &a, const float *src, int tid, float *dst) {
+#ifdef __CUDA_ARCH__
+    if (bwd_vec_rows(src, 2 * a.dstate)) {
+        for (int i = tid; i < P_MAX * (2 * N_MAX / 4); i += NT) {
+            const int p = i / (2 * N_MAX / 4), f = 4 * (i % (2 * N_MAX / 4));
+            const bool v = p < a.headdim && f < 2 * a.dstate;
+            bwd_cp16(dst + p * NS + f, v ? src + (size_t)p * 2 * a.dstate + f : src, v);
+        }
+        return;
+    }
+#endif
     BWDC_UNROLL
     for (int i = tid; i < P_MAX * 2 * N_MAX; i += NT) {
         const int p = i / (2 * N_MAX), f = i % (2 * N_MAX);
@@ -265,6 +321,7 @@ __host__ __device__ inline void k1_load(const BwdArgs &a, int c, int h, int b, i
     load_dt(a, c, h, b, tid, m);
     load_rows_p(a, a.x, c, h, b, tid, m.X);
     load_rows_n(a, a.B, c, group_of(a, h), b, tid, m.Bs);
+    bwd_async_wait();
 }
 __host__ __device__ inline void k1_cumsum(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     if (tid != 0) return;
@@ -298,10 +355,17 @@ __host__ __device__ inline void k2_pass(const BwdArgs &a, int blk, int h, int b,
     const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
     if (i >= pn) return;
     c2 hv = a.init ? ld2(a.init + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
-    for (int c = 0; c < a.nchunks; ++c) {
-        const size_t o = 2 * (ix_pn(a, b, h, c) + i);
-        st2(a.hin + o, hv);
-        hv = cadd(cmul(cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c))), hv), ld2(a.st + o));
+    for (int c0 = 0; c0 < a.nchunks; c0 += PASS_GRP) {  // a group's loads in flight together
+        c2 sv[PASS_GRP], lv[PASS_GRP];
+        for (int j = 0; j < PASS_GRP; ++j)
+            if (c0 + j < a.nchunks) {
+                sv[j] = ld2(a.st + 2 * (ix_pn(a, b, h, c0 + j) + i));
+                lv[j] = ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c0 + j));
+            }
+        for (int j = 0; j < PASS_GRP && c0 + j < a.nchunks; ++j) {
+            st2(a.hin + 2 * (ix_pn(a, b, h, c0 + j) + i), hv);
+            hv = cadd(cmul(cexpc(lv[j]), hv), sv[j]);
+        }
     }
 }
 
@@ -311,6 +375,7 @@ __host__ __device__ inline void k3_load(const BwdArgs &a, int c, int h, int b, i
     for (int i = tid; i < QC; i += NT) st2(m.e + 2 * i, cexpc(ld2(acs_g + 2 * i)));
     load_rows_p(a, a.dy, c, h, b, tid, m.dY);
     load_rows_n(a, a.C, c, group_of(a, h), b, tid, m.Cs);
+    bwd_async_wait();
 }
 // C_l <- conj(e_l C_l) in place
 __host__ __device__ inline void k3_scale(const BwdArgs &a, int tid, const Smem &m) {
@@ -329,11 +394,18 @@ __host__ __device__ inline void k4_pass(const BwdArgs &a, int blk, int h, int b,
     const size_t pn = (size_t)a.headdim * a.dstate, i = (size_t)blk * NT + tid;
     if (i >= pn) return;
     c2 gv = a.dfinal ? ld2(a.dfinal + 2 * (ix_bh(a, b, h) * pn + i)) : cmk(0.f, 0.f);
-    for (int c = a.nchunks - 1; c >= 0; --c) {
-        const size_t o = 2 * (ix_pn(a, b, h, c) + i);
-        st2(a.gh + o, gv);
-        const c2 el = cexpc(ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c)));
-        gv = cadd(cmul(cconj(el), gv), ld2(a.st + o));
+    for (int c0 = a.nchunks - 1; c0 >= 0; c0 -= PASS_GRP) {  // chunks c0, c0 - 1, ...
+        c2 sv[PASS_GRP], lv[PASS_GRP];
+        for (int j = 0; j < PASS_GRP; ++j)
+            if (c0 - j >= 0) {
+                sv[j] = ld2(a.st + 2 * (ix_pn(a, b, h, c0 - j) + i));
+                lv[j] = ld2(a.lam + 2 * (ix_bh(a, b, h) * a.nchunks + c0 - j));
+            }
+        for (int j = 0; j < PASS_GRP && c0 - j >= 0; ++j) {
+            st2(a.gh + 2 * (ix_pn(a, b, h, c0 - j) + i), gv);
+            const c2 el = cexpc(lv[j]);
+            gv = cadd(cmul(cconj(el), gv), sv[j]);
+        }
     }
     if (a.dinit) st2(a.dinit + 2 * (ix_bh(a, b, h) * pn + i), gv);
 }
@@ -350,7 +422,9 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
         const c2 ac = ld2(acs_g + 2 * i);
         st2(m.acs + 2 * i, ac);
         st2(m.e + 2 * i, cexpc(ac));
-        st2(m.w + 2 * i, cscale(cexpc(csub(lam, ac)), d));
+        const c2 wl = cexpc(csub(lam, ac));
+        st2(m.el + 2 * i, wl);
+        st2(m.w + 2 * i, cscale(wl, d));
     }
     if (tid == 0) st2(m.misc, lam);
     load_rows_p(a, a.x, c, h, b, tid, m.X);
@@ -359,6 +433,7 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     load_rows_n(a, a.C, c, g, b, tid, m.Cs);
     load_pn(a, a.hin + 2 * ix_pn(a, b, h, c), tid, m.Hin);
     load_pn(a, a.gh + 2 * ix_pn(a, b, h, c), tid, m.Gh);
+    bwd_async_wait();
 }
 // GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY; thread tile rows
 // l = 2 tr + i, columns s = tc + 16 j.
@@ -518,19 +593,22 @@ __host__ __device__ inline void k5_fk(const BwdArgs &a, int tid, const Smem &m) 
         c2 v = cmk(0.f, 0.f);
         for (int q = 0; q < 16; ++q) v = cadd(v, ld2(part_k + (t * 16 + q) * 2));
         st2(m.Ksr + 2 * t, v);
+    } else if (tid == 2 * QC) {  // the decay gradient's sums, off its one thread
+        c2 h0 = cmk(0.f, 0.f);
+        for (int r = 0; r < RED; ++r) h0 = cadd(h0, cmk(m.red[r], m.red[RED + r]));
+        st2(m.misc + 2, cmul(cexpc(ld2(m.misc)), h0));
+    } else if (tid == 3 * QC) {
+        float dd = 0.f;
+        for (int r = 0; r < RED; ++r) dd += m.red[2 * RED + r];
+        m.misc[4] = dd;
     }
 }
 __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     if (tid != 0) return;
-    const c2 lam = ld2(m.misc), Ah = ld2(a.A + 2 * h);
-    c2 h0 = cmk(0.f, 0.f), ksum = cmk(0.f, 0.f);
-    float dd = 0.f;
-    for (int r = 0; r < RED; ++r) {
-        h0 = cadd(h0, cmk(m.red[r], m.red[RED + r]));
-        dd += m.red[2 * RED + r];
-    }
+    const c2 Ah = ld2(a.A + 2 * h), h0 = ld2(m.misc + 2);
+    const float dd = m.misc[4];
+    c2 ksum = cmk(0.f, 0.f);
     for (int t = 0; t < QC; ++t) ksum = cadd(ksum, cmul(ld2(m.w + 2 * t), ld2(m.Ksr + 2 * t)));
-    h0 = cmul(cexpc(lam), h0);
     c2 run = cmk(0.f, 0.f), dAp = cmk(0.f, 0.f);
     for (int t = QC - 1; t >= 0; --t) {
         // colsum of E = dt_t * colsum of GL o XY
@@ -541,7 +619,7 @@ __host__ __device__ inline void k5_decay(const BwdArgs &a, int c, int h, int b, 
         run = cadd(run, cconj(inner));  // dalpha[t] = sum_{t' >= t} dacs[t']
         const int tg = c * QC + t;
         if (tg < a.seqlen) {
-            const c2 wlam = cexpc(csub(lam, ld2(m.acs + 2 * t)));
+            const c2 wlam = ld2(m.el + 2 * t);
             a.ddt[ix_dt(a, b, tg, h)] =
                 m.colG[2 * t] + cmul(wlam, ld2(m.Ksr + 2 * t)).re + cmul(cconj(run), Ah).re;
         }
