@@ -212,6 +212,25 @@ __host__ __device__ inline void mm_nt(float (&acc)[4][NJ], const float *A, int l
                 acc[i][j] = fmaf(a[i].w, b[j].w, fmaf(a[i].z, b[j].z, fmaf(a[i].y, b[j].y, fmaf(a[i].x, b[j].x, acc[i][j]))));
     }
 }
+// Two fused multiply-adds on a pair of floats: one packed instruction on the
+// device (fma.rn.f32x2, each lane rounded as fmaf), two fmaf on the host.
+__host__ __device__ inline void fma_pair(float a, float b0, float b1, float &c0, float &c1) {
+#ifdef __CUDA_ARCH__
+    unsigned long long r;
+    const float2 av = make_float2(a, a), bv = make_float2(b0, b1), cv = make_float2(c0, c1);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<const unsigned long long *>(&av)),
+          "l"(*reinterpret_cast<const unsigned long long *>(&bv)),
+          "l"(*reinterpret_cast<const unsigned long long *>(&cv)));
+    const float2 rv = *reinterpret_cast<float2 *>(&r);
+    c0 = rv.x;
+    c1 = rv.y;
+#else
+    c0 = fmaf(a, b0, c0);
+    c1 = fmaf(a, b1, c1);
+#endif
+}
 // "tn": acc[i][j] += sum_k sc[k] A[k][r0+i] B[k][c(j)],  c(j) = 4 tc + j (+ 60 for j >= 4: 64 + 4 tc + j - 4)
 // (sc may be null: no scaling)
 template <int NJ>
@@ -226,7 +245,10 @@ __host__ __device__ inline void mm_tn(float (&acc)[4][NJ], const float *A, int l
         f4 b[NJ / 4];
         for (int q = 0; q < NJ / 4; ++q) b[q] = ld4(B + k * ldb + 64 * q + 4 * tc);
         for (int i = 0; i < 4; ++i)
-            for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(comp(a, i), comp(b[j / 4], j % 4), acc[i][j]);
+            for (int q = 0; q < NJ / 4; ++q) {
+                fma_pair(comp(a, i), b[q].x, b[q].y, acc[i][4 * q], acc[i][4 * q + 1]);
+                fma_pair(comp(a, i), b[q].z, b[q].w, acc[i][4 * q + 2], acc[i][4 * q + 3]);
+            }
     }
 }
 // "nn": acc[i][j] += sum_k A[r0+i][k] B[k][c(j)]   (k0, k1 multiples of 4)
@@ -240,7 +262,10 @@ __host__ __device__ inline void mm_nn(float (&acc)[4][NJ], const float *A, int l
             f4 b[NJ / 4];
             for (int q = 0; q < NJ / 4; ++q) b[q] = ld4(B + (k + kk) * ldb + 64 * q + 4 * tc);
             for (int i = 0; i < 4; ++i)
-                for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(comp(a[i], kk), comp(b[j / 4], j % 4), acc[i][j]);
+                for (int q = 0; q < NJ / 4; ++q) {
+                    fma_pair(comp(a[i], kk), b[q].x, b[q].y, acc[i][4 * q], acc[i][4 * q + 1]);
+                    fma_pair(comp(a[i], kk), b[q].z, b[q].w, acc[i][4 * q + 2], acc[i][4 * q + 3]);
+                }
         }
     }
 }
