@@ -68,6 +68,33 @@ def test_timeout_is_reported_quickly_and_the_next_call_is_correct(lib):
     assert rel_err(got_fs, fs_ref) <= TOL_BF16
 
 
+def test_timeout_in_the_state_only_form(lib):
+    """The state-only form (no y) runs its own kernel instance, in which the math
+    warpgroup waits for each tile's slot and X before building W.  With the
+    producer withheld, those waits run out too: SSD_ERR_TIMEOUT within a
+    second, and the next state-only call matches the oracle's final state."""
+    shape = inputs.ScanShape("stall-so", 1, 2048, 8, 64, 1, 128, 128, "bf16", init_state=True, seed=32)
+    inp = inputs.scan_inputs(shape)
+    d = to_dev(inp)
+    ssd.ssd_scan_final_state(d["x"], d["dt"], d["A"], d["B"], d["init_state"], chunk_size=128)
+    assert lib.ssd_get_device_status(_stream()) == ssd.SSD_OK
+    try:
+        assert lib.ssd_debug_inject_stall(1, 10_000_000) == ssd.SSD_OK
+        t0 = time.perf_counter()
+        ssd.ssd_scan_final_state(d["x"], d["dt"], d["A"], d["B"], d["init_state"], chunk_size=128)
+        st = lib.ssd_get_device_status(_stream())
+        elapsed = time.perf_counter() - t0
+    finally:
+        lib.ssd_debug_inject_stall(0, 0)
+    assert st == ssd.SSD_ERR_TIMEOUT, (st, ssd.ssd_last_error())
+    assert elapsed < 1.0, elapsed
+    assert lib.ssd_get_device_status(_stream()) == ssd.SSD_OK
+    fs, _ = ssd.ssd_scan_final_state(d["x"], d["dt"], d["A"], d["B"], d["init_state"], chunk_size=128)
+    assert lib.ssd_get_device_status(_stream()) == ssd.SSD_OK
+    _, fs_ref = oracle_scan(inp, heads=[0, 7], batches=[0])
+    assert rel_err(fs.cpu().numpy()[[0]][:, [0, 7]], fs_ref) <= TOL_BF16
+
+
 SENTINEL = 0x5A
 
 
