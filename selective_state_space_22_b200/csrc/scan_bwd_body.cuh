@@ -198,20 +198,6 @@ struct alignas(16) f4 {
 __host__ __device__ inline f4 ld4(const float *p) { return *reinterpret_cast<const f4 *>(p); }
 __host__ __device__ inline float comp(const f4 &v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
-// Thread (tr, tc) = (tid / 16, tid % 16) owns rows r0 = 4 tr .. 4 tr + 3.
-// "nt": acc[i][j] += sum_k A[r0+i][k] B[tc+16j][k]   (both k-contiguous rows; k0, k1 multiples of 4)
-template <int NJ>
-__host__ __device__ inline void mm_nt(float (&acc)[4][NJ], const float *A, int lda, int r0, const float *B, int ldb,
-                                      int tc, int k0, int k1) {
-    for (int k = k0; k < k1; k += 4) {
-        f4 a[4], b[NJ];
-        for (int i = 0; i < 4; ++i) a[i] = ld4(A + (r0 + i) * lda + k);
-        for (int j = 0; j < NJ; ++j) b[j] = ld4(B + (tc + 16 * j) * ldb + k);
-        for (int i = 0; i < 4; ++i)
-            for (int j = 0; j < NJ; ++j)
-                acc[i][j] = fmaf(a[i].w, b[j].w, fmaf(a[i].z, b[j].z, fmaf(a[i].y, b[j].y, fmaf(a[i].x, b[j].x, acc[i][j]))));
-    }
-}
 // Two fused multiply-adds on a pair of floats: one packed instruction on the
 // device (fma.rn.f32x2, each lane rounded as fmaf), two fmaf on the host.
 __host__ __device__ inline void fma_pair(float a, float b0, float b1, float &c0, float &c1) {
@@ -230,6 +216,47 @@ __host__ __device__ inline void fma_pair(float a, float b0, float b1, float &c0,
     c0 = fmaf(a, b0, c0);
     c1 = fmaf(a, b1, c1);
 #endif
+}
+// Two independent fused multiply-adds (a0 b0 + c0, a1 b1 + c1) as one packed
+// instruction on the device, two fmaf on the host.
+__host__ __device__ inline void fma_pairs(float a0, float a1, float b0, float b1, float &c0, float &c1) {
+#ifdef __CUDA_ARCH__
+    unsigned long long r;
+    const float2 av = make_float2(a0, a1), bv = make_float2(b0, b1), cv = make_float2(c0, c1);
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(r)
+        : "l"(*reinterpret_cast<const unsigned long long *>(&av)),
+          "l"(*reinterpret_cast<const unsigned long long *>(&bv)),
+          "l"(*reinterpret_cast<const unsigned long long *>(&cv)));
+    const float2 rv = *reinterpret_cast<float2 *>(&r);
+    c0 = rv.x;
+    c1 = rv.y;
+#else
+    c0 = fmaf(a0, b0, c0);
+    c1 = fmaf(a1, b1, c1);
+#endif
+}
+// Thread (tr, tc) = (tid / 16, tid % 16) owns rows r0 = 4 tr .. 4 tr + 3.
+// "nt": acc[i][j] += sum_k A[r0+i][k] B[tc+16j][k]   (both k-contiguous rows; k0, k1 multiples of 4)
+// (The even and odd k run as the two lanes of packed float pairs, added at the end.)
+template <int NJ>
+__host__ __device__ inline void mm_nt(float (&acc)[4][NJ], const float *A, int lda, int r0, const float *B, int ldb,
+                                      int tc, int k0, int k1) {
+    float ev[4][NJ], od[4][NJ];
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NJ; ++j) ev[i][j] = od[i][j] = 0.f;
+    for (int k = k0; k < k1; k += 4) {
+        f4 a[4], b[NJ];
+        for (int i = 0; i < 4; ++i) a[i] = ld4(A + (r0 + i) * lda + k);
+        for (int j = 0; j < NJ; ++j) b[j] = ld4(B + (tc + 16 * j) * ldb + k);
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < NJ; ++j) {
+                fma_pairs(a[i].x, a[i].y, b[j].x, b[j].y, ev[i][j], od[i][j]);
+                fma_pairs(a[i].z, a[i].w, b[j].z, b[j].w, ev[i][j], od[i][j]);
+            }
+    }
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < NJ; ++j) acc[i][j] += ev[i][j] + od[i][j];
 }
 // "tn": acc[i][j] += sum_k sc[k] A[k][r0+i] B[k][c(j)],  c(j) = 4 tc + j (+ 60 for j >= 4: 64 + 4 tc + j - 4)
 // (sc may be null: no scaling)
