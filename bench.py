@@ -691,8 +691,7 @@ def bench_ours(args, shape):
     e2e = None
     if not args.no_e2e:
         hin = {k: v.pin_memory() for k, v in inp.items() if v is not None}
-        # two buffer sets (three measured slower: 0.94 against 0.87 ms per step; the
-        # two copy directions together are bound at 0.755 ms per step on this bus)
+        # two buffer sets (three measured slower: 0.94 against 0.87 ms per step)
         dsets = [{k: d[k] for k in hin}, {k: torch.empty_like(d[k]) for k in hin}]
         douts = [{"y": y, "final_state": fs}, {"y": torch.empty_like(y), "final_state": torch.empty_like(fs)}]
         hout = [{k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in o.items()} for o in douts]
