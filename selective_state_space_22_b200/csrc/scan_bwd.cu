@@ -16,6 +16,7 @@
 
 #include "scan_bwd_body.cuh"
 #include "scan_bwd_complex_body.cuh"
+#include "scan_bwd_tc.cuh"
 #include "ssd_internal.cuh"
 
 namespace ssd {
@@ -231,7 +232,10 @@ cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
     a.batch = call.batch; a.seqlen = call.seqlen; a.nheads = call.nheads; a.headdim = call.headdim;
     a.ngroups = call.ngroups; a.dstate = call.dstate;
     a.nchunks = (call.seqlen + QB - 1) / QB;
+    a.dev_error = call.dev_error;
     carve(a, static_cast<float *>(ws));
+    // head dim 64, d_state 128: the chunk states and readout terms on tcgen05
+    const bool tc = a.headdim == bwdtc::PD && a.dstate == bwdtc::ND && a.dev_error;
 
     // the shared-memory opt-in is per function, device and context
     static void *attr_ctx[64] = {nullptr};
@@ -249,15 +253,26 @@ cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
                 e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
                 if (e != cudaSuccess) return e;
             }
+            for (const void *f : {(const void *)bwdtc::chunk_product_kernel<false>,
+                                  (const void *)bwdtc::chunk_product_kernel<true>}) {
+                e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bwdtc::SMEM);
+                if (e != cudaSuccess) return e;
+            }
             attr_ctx[dev] = ctx;
         }
     }
     const unsigned pn_blocks = (unsigned)(((size_t)a.headdim * a.dstate + NT - 1) / NT);
     if (a.batch > 0 && a.nchunks > 0) {
         const dim3 gc(a.nchunks, a.nheads, a.batch), gh(pn_blocks, a.nheads, a.batch);
-        bwd_chunk_state<<<gc, NT, SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
+        if (tc)
+            bwdtc::chunk_product_kernel<false><<<gc, bwdtc::NTH, bwdtc::SMEM, st>>>(a);
+        else
+            bwd_chunk_state<<<gc, NT, SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
         bwd_state_fwd<<<gh, NT, 0, st>>>(a);
-        bwd_readout<<<gc, NT, SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
+        if (tc)
+            bwdtc::chunk_product_kernel<true><<<gc, bwdtc::NTH, bwdtc::SMEM, st>>>(a);
+        else
+            bwd_readout<<<gc, NT, SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwd_state_bwd<<<gh, NT, 0, st>>>(a);
         bwd_chunk_grad<<<gc, NT, SMEM_BYTES, st>>>(a);
         const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;

@@ -102,6 +102,7 @@ struct BwdArgs {
     float *dCh;   // [b][T][h][N]
     float *dAp;   // [b][h][nchunks]
     float *dDp;   // [b][h][nchunks]
+    int *dev_error;  // device error word (tensor-core phases' bounded waits)
 };
 
 // Workspace floats for one call (each region padded to 4 floats).

@@ -1,0 +1,194 @@
+// scan_bwd_tc.cuh -- the two per-chunk contractions of the real backward that
+// have the shape of a chunk state, on tcgen05 (sm_100a), for head dim 64 and
+// d_state 128:
+//   chunk state   S[p][n] = sum_s w_s x_s[p] B_s[n],  w_s = exp(lam - acs[s]) dt_s
+//   readout       R[p][n] = sum_l e_l dy_l[p] C_l[n], e_l = exp(acs[l])
+// ("Block Anatomy, Numerical Stability & Scaling", Numerical Stability section 4:
+// the chunk states; section 5.3: the backward runs through the same exp products.)
+// One CTA of 128 threads per (64-token chunk, head, batch).  The rows [tokens][n]
+// (B or C) are the MMA's A operand, MN-major, and the scaled rows [tokens][p]
+// (w x or e dy) its B operand, MN-major; M = n (128, the TMEM lanes), N = p (64
+// columns), K = the chunk's 64 tokens.  Float32 accuracy from bf16 operands: each
+// value is split into hi + lo (16 significant bits) and the product is
+// hi.hi + hi.lo + lo.hi, accumulated in float32 in TMEM.  The chunk-state kernel
+// also forms the chunk's cumulative decay (a warp scan) and writes acs and lam
+// for the later phases.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "scan_bwd_body.cuh"
+#include "ssd_internal.cuh"
+#include "tc_ptx.cuh"
+
+namespace ssd {
+namespace bwdtc {
+
+using namespace ptx;
+
+constexpr int Q = bwd::QB;   // 64 tokens per chunk
+constexpr int PD = 64;       // head dim of this path
+constexpr int ND = 128;      // d_state of this path
+constexpr int NTH = 128;
+// Shared memory: the [tokens][n] rows as two 64-column halves of [64][128 B]
+// (hi, then lo), the scaled [tokens][p] rows [64][128 B] (hi, then lo).
+constexpr int O_AH = 0, O_AL = 16384, O_BH = 32768, O_BL = 40960, O_MISC = 49152;
+constexpr int SMEM = O_MISC + 3 * Q * 4 + 64 + 1024;
+constexpr uint32_t IDESC = idesc_bf16_f32(128, 64, 1, 1);
+constexpr unsigned long long WAIT_NS = 1000000000ull;
+
+// Byte offset of 16-byte chunk ch (8 bf16) of row r in a tile of 128-byte
+// swizzled rows, the 64-column halves half_bytes apart.
+__device__ __forceinline__ uint32_t swz(int r, int ch, int half_bytes) {
+    return (uint32_t)((ch >> 3) * half_bytes + r * 128 + (((ch & 7) ^ (r & 7)) << 4));
+}
+// Eight floats -> bf16 hi and lo parts at sm + hi_off + o and sm + lo_off + o.
+__device__ __forceinline__ void put_split8(uint8_t *sm, int hi_off, int lo_off, uint32_t o, const float (&v)[8]) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        const float2 hf = __bfloat1622float2(hh);
+        const __nv_bfloat162 ll = __floats2bfloat162_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+        h[e] = *reinterpret_cast<const uint32_t *>(&hh);
+        l[e] = *reinterpret_cast<const uint32_t *>(&ll);
+    }
+    *reinterpret_cast<uint4 *>(sm + hi_off + o) = make_uint4(h[0], h[1], h[2], h[3]);
+    *reinterpret_cast<uint4 *>(sm + lo_off + o) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// READOUT = false: the chunk state (and acs, lam); true: the readout terms.
+template <bool READOUT>
+__global__ void __launch_bounds__(NTH) chunk_product_kernel(bwd::BwdArgs a) {
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = bwd::group_of(a, h), t0 = c * Q, valid = min(Q, a.seqlen - t0);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *scale = reinterpret_cast<float *>(sm + O_MISC);  // [Q]: w_s or e_l
+    float *acs = scale + Q;                                  // [Q]
+    float *wtot = acs + Q;                                   // [2]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(wtot + Q);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 64);
+        tmem_relinquish();
+    }
+    const size_t bh = bwd::ix_bh(a, b, h);
+    float *acs_g = a.acs + (bh * a.nchunks + c) * Q;
+    if constexpr (!READOUT) {
+        // cumulative decay of the chunk: warps 0 and 1 scan 32 tokens each
+        float d = 0.f, v = 0.f;
+        if (tid < Q) {
+            d = tid < valid ? __ldg(a.dt + bwd::ix_dt(a, b, t0 + tid, h)) : 0.f;
+            v = d * __ldg(a.A + h);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += y;
+            }
+            if (lane == 31) wtot[warp] = v;
+        }
+        __syncthreads();
+        if (tid < Q) {
+            if (warp == 1) v += wtot[0];
+            acs[tid] = v;
+            acs_g[tid] = v;
+        }
+        __syncthreads();
+        const float lam = acs[Q - 1];
+        if (tid < Q) scale[tid] = expf(lam - v) * d;
+        if (tid == 0) a.lam[bh * a.nchunks + c] = lam;
+    } else {
+        if (tid < Q) scale[tid] = expf(__ldg(acs_g + tid));
+    }
+    __syncthreads();
+    // operands: the [tokens][n] rows (B or C) and the scaled [tokens][p] rows (x or dy)
+    const float *rows_n = READOUT ? a.C : a.B;
+    const float *rows_p = READOUT ? a.dy : a.x;
+#pragma unroll 4
+    for (int it = 0; it < Q * 16 / NTH; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
+        float v8[8];
+        if (r < valid) {
+            const float *src = rows_n + bwd::ix_bc(a, b, t0 + r, g, 8 * ch);
+            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src));
+            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + 4));
+            v8[0] = x0.x, v8[1] = x0.y, v8[2] = x0.z, v8[3] = x0.w, v8[4] = x1.x, v8[5] = x1.y, v8[6] = x1.z,
+            v8[7] = x1.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] = 0.f;
+        }
+        put_split8(sm, O_AH, O_AL, swz(r, ch, Q * 128), v8);
+    }
+#pragma unroll 4
+    for (int it = 0; it < Q * 8 / NTH; ++it) {
+        const int u = tid + it * NTH, r = u >> 3, ch = u & 7;
+        float v8[8];
+        if (r < valid) {
+            const float f = scale[r];
+            const float *src = rows_p + bwd::ix_x(a, b, t0 + r, h, 8 * ch);
+            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src));
+            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + 4));
+            v8[0] = f * x0.x, v8[1] = f * x0.y, v8[2] = f * x0.z, v8[3] = f * x0.w;
+            v8[4] = f * x1.x, v8[5] = f * x1.y, v8[6] = f * x1.z, v8[7] = f * x1.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] = 0.f;
+        }
+        put_split8(sm, O_BH, O_BL, swz(r, ch, Q * 128), v8);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot, sb = smem_u32(sm);
+    if (tid == 0) {
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {  // hi.hi + hi.lo + lo.hi
+            const uint32_t aA = sb + (pass == 2 ? O_AL : O_AH), aB = sb + (pass == 1 ? O_BL : O_BH);
+#pragma unroll 1
+            for (int kk = 0; kk < Q / 16; ++kk)
+                mma_ss(tmem, smem_desc_sw128(aA + kk * 2048, Q * 128, 1024), smem_desc_sw128(aB + kk * 2048, Q * 128, 1024),
+                       IDESC, pass > 0 || kk > 0);
+        }
+        mma_commit(bar);
+    }
+    // bounded wait for the products (the device error word records a timeout)
+    if (!mbar_try_wait(bar, 0)) {
+        const unsigned long long w0 = globaltimer_ns();
+        while (!mbar_try_wait(bar, 0))
+            if (globaltimer_ns() - w0 > WAIT_NS) {
+                atomicCAS(a.dev_error, 0, DEV_TIMEOUT);
+                break;
+            }
+    }
+    tc_fence_after();
+    {  // TMEM lane n = 32 warp + lane, columns p -> S[p][n] (or R)
+        const int n = 32 * warp + lane;
+        float *out = a.st + bwd::ix_pn(a, b, h, c) + n;
+#pragma unroll 1
+        for (int cb = 0; cb < PD; cb += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + cb, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) out[(size_t)(cb + i) * ND] = __uint_as_float(r[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+}  // namespace bwdtc
+}  // namespace ssd

@@ -337,8 +337,10 @@ static ssd_status run_bwd(bool cplx, const float *x, const float *dt, const floa
                         workspace ? workspace_bytes : (size_t)0);
         if (!aligned16(workspace)) return fail(SSD_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
     }
+    int *dev_err = device_error_ptr(&s);
+    if (!dev_err) return s;
     ssd::BwdCall call{x, dt, A, B, C, D, init_state, dy, dfinal, dx, ddt, dA, dB, dC, dD, dinit,
-                      batch, seqlen, nheads, headdim, ngroups, dstate};
+                      batch, seqlen, nheads, headdim, ngroups, dstate, dev_err};
     cudaError_t e = cplx ? ssd::launch_scan_bwd_complex(call, workspace, static_cast<cudaStream_t>(stream))
                          : ssd::launch_scan_bwd(call, workspace, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "launching the backward scan");

@@ -100,6 +100,7 @@ struct BwdCall {
     const float *x, *dt, *A, *B, *C, *D, *init_state, *dy, *dfinal;
     float *dx, *ddt, *dA, *dB, *dC, *dD, *dinit;
     int batch, seqlen, nheads, headdim, ngroups, dstate;
+    int *dev_error;  // device error word
 };
 bool bwd_supported(int headdim, int dstate);
 size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate);
