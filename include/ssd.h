@@ -320,8 +320,10 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
  *  gradient for D whether or not D was given.
  *
  * Limits: headdim <= 64 and dstate <= 128 (SSD_ERR_UNSUPPORTED otherwise).  Runs
- * on CUDA cores in seven launches.  Sums are taken in a fixed order, so repeated
- * calls give identical bits.  The workspace (ssd_scan_bwd_workspace_size bytes,
+ * in seven launches; with headdim 64 and dstate 128 the chunk states and the
+ * readout terms are tcgen05 products (bf16 hi/lo, three products, float32
+ * accumulation), the rest CUDA cores.  Sums are taken in a fixed order, so
+ * repeated calls give identical bits.  The workspace (ssd_scan_bwd_workspace_size bytes,
  * caller-owned, 16-byte aligned, no initialisation needed) holds the chunk
  * states, the state gradients and per-head partial sums; it grows with
  * batch * nheads * ceil(seqlen / 64) * headdim * dstate * 12 bytes plus
