@@ -83,6 +83,32 @@ __global__ void __launch_bounds__(NTH) chunk_product_kernel(bwd::BwdArgs a) {
         tmem_alloc(tslot, 64);
         tmem_relinquish();
     }
+    // Every row load of the chunk goes in flight first (into registers; nothing
+    // below waits on them until the conversion), then the decays are formed.
+    const float *rows_n = READOUT ? a.C : a.B;   // [tokens][n]: B or C
+    const float *rows_p = READOUT ? a.dy : a.x;  // [tokens][p]: x or dy
+    constexpr int IA = Q * 16 / NTH, IB = Q * 8 / NTH;
+    float4 ra[IA][2], rb[IB][2];
+#pragma unroll
+    for (int it = 0; it < IA; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
+        ra[it][0] = ra[it][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < valid) {
+            const float *src = rows_n + bwd::ix_bc(a, b, t0 + r, g, 8 * ch);
+            ra[it][0] = __ldg(reinterpret_cast<const float4 *>(src));
+            ra[it][1] = __ldg(reinterpret_cast<const float4 *>(src + 4));
+        }
+    }
+#pragma unroll
+    for (int it = 0; it < IB; ++it) {
+        const int u = tid + it * NTH, r = u >> 3, ch = u & 7;
+        rb[it][0] = rb[it][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < valid) {
+            const float *src = rows_p + bwd::ix_x(a, b, t0 + r, h, 8 * ch);
+            rb[it][0] = __ldg(reinterpret_cast<const float4 *>(src));
+            rb[it][1] = __ldg(reinterpret_cast<const float4 *>(src + 4));
+        }
+    }
     const size_t bh = bwd::ix_bh(a, b, h);
     float *acs_g = a.acs + (bh * a.nchunks + c) * Q;
     if constexpr (!READOUT) {
@@ -112,40 +138,21 @@ __global__ void __launch_bounds__(NTH) chunk_product_kernel(bwd::BwdArgs a) {
         if (tid < Q) scale[tid] = expf(__ldg(acs_g + tid));
     }
     __syncthreads();
-    // operands: the [tokens][n] rows (B or C) and the scaled [tokens][p] rows (x or dy)
-    const float *rows_n = READOUT ? a.C : a.B;
-    const float *rows_p = READOUT ? a.dy : a.x;
-#pragma unroll 4
-    for (int it = 0; it < Q * 16 / NTH; ++it) {
-        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
-        float v8[8];
-        if (r < valid) {
-            const float *src = rows_n + bwd::ix_bc(a, b, t0 + r, g, 8 * ch);
-            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src));
-            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + 4));
-            v8[0] = x0.x, v8[1] = x0.y, v8[2] = x0.z, v8[3] = x0.w, v8[4] = x1.x, v8[5] = x1.y, v8[6] = x1.z,
-            v8[7] = x1.w;
-        } else {
+    // operands as bf16 hi/lo: the [tokens][n] rows, and the [tokens][p] rows scaled
+    // by w (chunk state) or e (readout); rows past the sequence are zeros
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v8[e] = 0.f;
-        }
+    for (int it = 0; it < IA; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, ch = u & 15;
+        const float4 x0 = ra[it][0], x1 = ra[it][1];
+        const float v8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         put_split8(sm, O_AH, O_AL, swz(r, ch, Q * 128), v8);
     }
-#pragma unroll 4
-    for (int it = 0; it < Q * 8 / NTH; ++it) {
-        const int u = tid + it * NTH, r = u >> 3, ch = u & 7;
-        float v8[8];
-        if (r < valid) {
-            const float f = scale[r];
-            const float *src = rows_p + bwd::ix_x(a, b, t0 + r, h, 8 * ch);
-            const float4 x0 = __ldg(reinterpret_cast<const float4 *>(src));
-            const float4 x1 = __ldg(reinterpret_cast<const float4 *>(src + 4));
-            v8[0] = f * x0.x, v8[1] = f * x0.y, v8[2] = f * x0.z, v8[3] = f * x0.w;
-            v8[4] = f * x1.x, v8[5] = f * x1.y, v8[6] = f * x1.z, v8[7] = f * x1.w;
-        } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v8[e] = 0.f;
-        }
+    for (int it = 0; it < IB; ++it) {
+        const int u = tid + it * NTH, r = u >> 3, ch = u & 7;
+        const float f = scale[r];
+        const float4 x0 = rb[it][0], x1 = rb[it][1];
+        const float v8[8] = {f * x0.x, f * x0.y, f * x0.z, f * x0.w, f * x1.x, f * x1.y, f * x1.z, f * x1.w};
         put_split8(sm, O_BH, O_BL, swz(r, ch, Q * 128), v8);
     }
     fence_proxy_async_smem();
