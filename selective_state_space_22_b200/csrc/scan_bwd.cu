@@ -190,19 +190,30 @@ cudaError_t launch_scan_bwd_complex(const BwdCall &call, void *ws, cudaStream_t 
     a.batch = call.batch; a.seqlen = call.seqlen; a.nheads = call.nheads; a.headdim = call.headdim;
     a.ngroups = call.ngroups; a.dstate = call.dstate;
     a.nchunks = (call.seqlen + bwdc::QC - 1) / bwdc::QC;
+    a.dev_error = call.dev_error;
     bwdc::carve(a, static_cast<float *>(ws));
+    // head dim 64, 64 complex states: the chunk states and readout terms on tcgen05
+    const bool tc = a.headdim == bwdtc::PD && a.dstate == bwdtc::NCX && a.dev_error;
 
-    static void *attr_set[64] = {nullptr};
+    static void *attr_set[64] = {nullptr}, *attr_set_tc[64] = {nullptr};
     const void *fs[3] = {(const void *)bwdc_chunk_state, (const void *)bwdc_readout, (const void *)bwdc_chunk_grad};
     cudaError_t e = set_smem_attr(fs, 3, SMEM_BYTES_C, attr_set);
     if (e != cudaSuccess) return e;
+    const void *ftc[2] = {(const void *)bwdtc::cplx_product_kernel<false>, (const void *)bwdtc::cplx_product_kernel<true>};
+    if ((e = set_smem_attr(ftc, 2, bwdtc::CSMEM, attr_set_tc)) != cudaSuccess) return e;
     const int nt = bwdc::NT;
     const unsigned pn_blocks = (unsigned)(((size_t)a.headdim * a.dstate + nt - 1) / nt);
     if (a.batch > 0 && a.nchunks > 0) {
         const dim3 gc(a.nchunks, a.nheads, a.batch), gh(pn_blocks, a.nheads, a.batch);
-        bwdc_chunk_state<<<gc, nt, bwdc::SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
+        if (tc)
+            bwdtc::cplx_product_kernel<false><<<gc, bwdtc::NTH, bwdtc::CSMEM, st>>>(a);
+        else
+            bwdc_chunk_state<<<gc, nt, bwdc::SMEM_FLOATS_K1 * sizeof(float), st>>>(a);
         bwdc_state_fwd<<<gh, nt, 0, st>>>(a);
-        bwdc_readout<<<gc, nt, bwdc::SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
+        if (tc)
+            bwdtc::cplx_product_kernel<true><<<gc, bwdtc::NTH, bwdtc::CSMEM, st>>>(a);
+        else
+            bwdc_readout<<<gc, nt, bwdc::SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwdc_state_bwd<<<gh, nt, 0, st>>>(a);
         bwdc_chunk_grad<<<gc, nt, SMEM_BYTES_C, st>>>(a);
         const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;

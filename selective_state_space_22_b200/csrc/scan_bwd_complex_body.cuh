@@ -109,6 +109,7 @@ struct BwdArgs {
     float *dCh;   // [b][T][h][N][2]
     float *dAp;   // [b][h][nchunks][2]
     float *dDp;   // [b][h][nchunks]
+    int *dev_error;  // device error word (tensor-core phases' bounded waits)
 };
 
 __host__ __device__ inline size_t ws_floats(int batch, int seqlen, int nheads, int headdim, int dstate,

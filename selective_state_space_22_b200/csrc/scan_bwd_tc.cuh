@@ -18,6 +18,7 @@
 #include <cuda_bf16.h>
 
 #include "scan_bwd_body.cuh"
+#include "scan_bwd_complex_body.cuh"
 #include "ssd_internal.cuh"
 #include "tc_ptx.cuh"
 
@@ -190,6 +191,171 @@ __global__ void __launch_bounds__(NTH) chunk_product_kernel(bwd::BwdArgs a) {
             tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + cb, r);
 #pragma unroll
             for (int i = 0; i < 32; ++i) out[(size_t)(cb + i) * ND] = __uint_as_float(r[i]);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 64);
+}
+
+// ------------------------------------------------------------ complex variant
+// The same two contractions for the complex head (head dim 64, 64 complex states,
+// 32-token chunks), as one real product each: with the complex weight folded into
+// the complex rows, S[p][n] = sum_s x_s[p] (w_s B_s[n]) and
+// R[p][n] = sum_l dy_l[p] conj(e_l C_l[n]) take M = the 128 interleaved (re, im)
+// values of n, N = p, K = the chunk's 32 tokens; TMEM lane k = 2n + (re, im) is
+// float k of row p of the interleaved result.
+constexpr int QCX = bwdc::QC;  // 32 tokens
+constexpr int NCX = 64;        // complex states of this path
+constexpr int C_AH = 0, C_AL = 8192, C_BH = 16384, C_BL = 20480, C_MISC = 24576;
+constexpr int CSMEM = C_MISC + 6 * QCX * 4 + 64 + 1024;
+
+template <bool READOUT>
+__global__ void __launch_bounds__(NTH) cplx_product_kernel(bwdc::BwdArgs a) {
+    using bwdc::c2;
+    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = bwdc::group_of(a, h), t0 = c * QCX, valid = min(QCX, a.seqlen - t0);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float *wgt = reinterpret_cast<float *>(sm + C_MISC);  // [QCX][2]: w_s, or e_l
+    uint64_t *bar = reinterpret_cast<uint64_t *>(wgt + 6 * QCX);
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(bar + 1);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tslot, 64);
+        tmem_relinquish();
+    }
+    // every row load in flight first: the complex rows [tokens][2N] (B or C) and
+    // the real rows [tokens][p] (x or dy)
+    const float *rows_n = READOUT ? a.C : a.B;
+    const float *rows_p = READOUT ? a.dy : a.x;
+    constexpr int IA = QCX * 32 / NTH, IB = QCX * 16 / NTH;  // 16-byte loads per thread
+    float4 ra[IA], rb[IB];
+#pragma unroll
+    for (int it = 0; it < IA; ++it) {
+        const int u = tid + it * NTH, r = u >> 5, q = u & 31;
+        ra[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < valid) ra[it] = __ldg(reinterpret_cast<const float4 *>(rows_n + 2 * bwdc::ix_bc(a, b, t0 + r, g, 0) + 4 * q));
+    }
+#pragma unroll
+    for (int it = 0; it < IB; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, q = u & 15;
+        rb[it] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < valid) rb[it] = __ldg(reinterpret_cast<const float4 *>(rows_p + bwdc::ix_x(a, b, t0 + r, h, 4 * q)));
+    }
+    const size_t bh = bwdc::ix_bh(a, b, h);
+    float *acs_g = a.acs + 2 * (bh * a.nchunks + c) * QCX;
+    if constexpr (!READOUT) {
+        // complex cumulative decay of the chunk (one warp), lam, w_s = exp(lam - acs_s) dt_s
+        if (warp == 0) {
+            const float d = lane < valid ? __ldg(a.dt + bwdc::ix_dt(a, b, t0 + lane, h)) : 0.f;
+            float vr = d * __ldg(a.A + 2 * h), vi = d * __ldg(a.A + 2 * h + 1);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float yr = __shfl_up_sync(0xffffffffu, vr, o), yi = __shfl_up_sync(0xffffffffu, vi, o);
+                if (lane >= o) vr += yr, vi += yi;
+            }
+            acs_g[2 * lane] = vr;
+            acs_g[2 * lane + 1] = vi;
+            const float lr = __shfl_sync(0xffffffffu, vr, 31), li = __shfl_sync(0xffffffffu, vi, 31);
+            if (lane == 0) {
+                a.lam[2 * (bh * a.nchunks + c)] = lr;
+                a.lam[2 * (bh * a.nchunks + c) + 1] = li;
+            }
+            const c2 wl = bwdc::cscale(bwdc::cexpc(c2{lr - vr, li - vi}), d);
+            wgt[2 * lane] = wl.re;
+            wgt[2 * lane + 1] = wl.im;
+        }
+    } else {
+        if (tid < QCX) {
+            const c2 e = bwdc::cexpc(c2{__ldg(acs_g + 2 * tid), __ldg(acs_g + 2 * tid + 1)});
+            wgt[2 * tid] = e.re;  // e_l; the weighted row is conjugated below
+            wgt[2 * tid + 1] = e.im;
+        }
+    }
+    __syncthreads();
+    // operands as bf16 hi/lo, 128-byte swizzled: the weighted complex rows (two
+    // 64-float halves) and the real rows
+#pragma unroll
+    for (int it = 0; it < IA; ++it) {
+        const int u = tid + it * NTH, r = u >> 5, q = u & 31;  // floats 4q .. 4q+3 = complex 2q, 2q+1
+        const c2 wr = c2{wgt[2 * r], wgt[2 * r + 1]};
+        const float4 v = ra[it];
+        c2 z0 = bwdc::cmul(wr, c2{v.x, v.y}), z1 = bwdc::cmul(wr, c2{v.z, v.w});
+        if (READOUT) z0 = bwdc::cconj(z0), z1 = bwdc::cconj(z1);  // conj(e_l C_l)
+        const float f4v[4] = {z0.re, z0.im, z1.re, z1.im};
+        // two 16-byte chunks (8 bf16) per 8 floats: this thread's 4 floats are half a chunk
+        const int ch = q >> 1, part = q & 1;
+        const uint32_t o = swz(r, ch, QCX * 128) + 8 * part;
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(f4v[2 * e], f4v[2 * e + 1]);
+            const float2 hf = __bfloat1622float2(hh);
+            const __nv_bfloat162 ll = __floats2bfloat162_rn(f4v[2 * e] - hf.x, f4v[2 * e + 1] - hf.y);
+            hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+            lw[e] = *reinterpret_cast<const uint32_t *>(&ll);
+        }
+        *reinterpret_cast<uint2 *>(sm + C_AH + o) = make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2 *>(sm + C_AL + o) = make_uint2(lw[0], lw[1]);
+    }
+#pragma unroll
+    for (int it = 0; it < IB; ++it) {
+        const int u = tid + it * NTH, r = u >> 4, q = u & 15;
+        const float4 v = rb[it];
+        const float f4v[4] = {v.x, v.y, v.z, v.w};
+        const int ch = q >> 1, part = q & 1;
+        const uint32_t o = swz(r, ch, QCX * 128) + 8 * part;
+        uint32_t hw[2], lw[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(f4v[2 * e], f4v[2 * e + 1]);
+            const float2 hf = __bfloat1622float2(hh);
+            const __nv_bfloat162 ll = __floats2bfloat162_rn(f4v[2 * e] - hf.x, f4v[2 * e + 1] - hf.y);
+            hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+            lw[e] = *reinterpret_cast<const uint32_t *>(&ll);
+        }
+        *reinterpret_cast<uint2 *>(sm + C_BH + o) = make_uint2(hw[0], hw[1]);
+        *reinterpret_cast<uint2 *>(sm + C_BL + o) = make_uint2(lw[0], lw[1]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tslot, sb = smem_u32(sm);
+    if (tid == 0) {
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {  // hi.hi + hi.lo + lo.hi
+            const uint32_t aA = sb + (pass == 2 ? C_AL : C_AH), aB = sb + (pass == 1 ? C_BL : C_BH);
+#pragma unroll 1
+            for (int kk = 0; kk < QCX / 16; ++kk)
+                mma_ss(tmem, smem_desc_sw128(aA + kk * 2048, QCX * 128, 1024),
+                       smem_desc_sw128(aB + kk * 2048, QCX * 128, 1024), IDESC, pass > 0 || kk > 0);
+        }
+        mma_commit(bar);
+    }
+    if (!mbar_try_wait(bar, 0)) {
+        const unsigned long long w0 = globaltimer_ns();
+        while (!mbar_try_wait(bar, 0))
+            if (globaltimer_ns() - w0 > WAIT_NS) {
+                atomicCAS(a.dev_error, 0, DEV_TIMEOUT);
+                break;
+            }
+    }
+    tc_fence_after();
+    {  // TMEM lane k = 2n + (re, im), columns p -> float k of row p of the [P][N] pairs
+        const int k = 32 * warp + lane;
+        float *out = a.st + 2 * bwdc::ix_pn(a, b, h, c) + k;
+#pragma unroll 1
+        for (int cb = 0; cb < PD; cb += 32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + ((uint32_t)(32 * warp) << 16) + cb, r);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) out[(size_t)(cb + i) * 2 * NCX] = __uint_as_float(r[i]);
         }
     }
     tc_fence_before();
