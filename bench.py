@@ -1160,8 +1160,8 @@ def bench_bwd(args, shape):
     t_call = statistics.median(per_step_ms) / 1e3
     roofline = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"], "traffic": None,
-                "kernel": ("ssd_scan_bwd_complex (7 CUDA-core launches, timed as one call)" if shape.complex
-                           else "ssd_scan_bwd (7 launches, two of them tcgen05, timed as one call)"),
+                "kernel": ("ssd_scan_bwd_complex" if shape.complex else "ssd_scan_bwd")
+                + " (7 launches, two of them tcgen05, timed as one call)",
                 "algorithmic_bytes_per_launch": abytes,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
                 if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",

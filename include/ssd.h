@@ -349,8 +349,9 @@ ssd_status ssd_scan_bwd(const float *x, const float *dt, const float *A, const f
  * float pairs), as are the outputs dA, dB, dC and dinit; x, dt, D, dy, dx, ddt
  * and dD are float32.  For a complex z = u + iv the gradient written is
  * dL/du + i dL/dv.  Limits: headdim <= 64 and dstate <= 64; the chunk is 32
- * tokens.  Workspace from ssd_scan_bwd_complex_workspace_size.  Everything else
- * as ssd_scan_bwd.
+ * tokens.  With headdim 64 and dstate 64 the chunk states and readout terms are
+ * tcgen05 products, as in ssd_scan_bwd.  Workspace from
+ * ssd_scan_bwd_complex_workspace_size.  Everything else as ssd_scan_bwd.
  */
 size_t ssd_scan_bwd_complex_workspace_size(int batch, int seqlen, int nheads, int headdim,
                                            int ngroups, int dstate);
