@@ -327,7 +327,9 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
  * caller-owned, 16-byte aligned, no initialisation needed) holds the chunk
  * states, the state gradients and per-head partial sums; it grows with
  * batch * nheads * ceil(seqlen / 64) * headdim * dstate * 12 bytes plus
- * batch * seqlen * nheads * dstate * 8 bytes.  SSD_ERR_WORKSPACE when it is NULL
+ * batch * seqlen * nheads * dstate * 8 bytes, plus, when the heads of a group
+ * share B and C (nheads / ngroups >= 2), each chunk's C B^T once per group:
+ * batch * ngroups * ceil(seqlen / 64) * 16 KB.  SSD_ERR_WORKSPACE when it is NULL
  * or too small.
  */
 size_t ssd_scan_bwd_workspace_size(int batch, int seqlen, int nheads, int headdim,

@@ -37,6 +37,15 @@ __global__ void __launch_bounds__(NT) bwd_chunk_state(BwdArgs a) {
     k1_state(a, c, h, b, tid, m);
 }
 
+__global__ void __launch_bounds__(NT) bwd_gram(BwdArgs a) {
+    extern __shared__ float sm[];
+    const Smem m = smem_map(sm);
+    const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
+    kg_load(a, c, g, b, tid, m);
+    __syncthreads();
+    kg_gram(a, c, g, b, tid, m);
+}
+
 __global__ void __launch_bounds__(NT) bwd_state_fwd(BwdArgs a) {
     k2_pass(a, blockIdx.x, blockIdx.y, blockIdx.z, threadIdx.x);
 }
@@ -229,9 +238,9 @@ bool bwd_supported(int headdim, int dstate) {
     return headdim >= 1 && headdim <= P_MAX && dstate >= 1 && dstate <= N_MAX;
 }
 
-size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate) {
+size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate) {
     const int nchunks = (seqlen + QB - 1) / QB;
-    return ws_floats(batch, seqlen, nheads, headdim, dstate, nchunks) * sizeof(float);
+    return ws_floats(batch, seqlen, nheads, headdim, ngroups, dstate, nchunks) * sizeof(float);
 }
 
 cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
@@ -260,7 +269,7 @@ cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
         void *ctx = current_context();
         if (!ctx || attr_ctx[dev] != ctx) {
             for (const void *f : {(const void *)bwd_chunk_state, (const void *)bwd_readout,
-                                  (const void *)bwd_chunk_grad}) {
+                                  (const void *)bwd_chunk_grad, (const void *)bwd_gram}) {
                 e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
                 if (e != cudaSuccess) return e;
             }
@@ -285,6 +294,7 @@ cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st) {
         else
             bwd_readout<<<gc, NT, SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwd_state_bwd<<<gh, NT, 0, st>>>(a);
+        if (a.gram) bwd_gram<<<dim3(a.nchunks, a.ngroups, a.batch), NT, SMEM_FLOATS_K3 * sizeof(float), st>>>(a);
         bwd_chunk_grad<<<gc, NT, SMEM_BYTES, st>>>(a);
         const size_t total = (size_t)a.batch * a.seqlen * a.ngroups * a.dstate;
         bwd_group_sum<<<(unsigned)((total + NT - 1) / NT), NT, 0, st>>>(a, total);

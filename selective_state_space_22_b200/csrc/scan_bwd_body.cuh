@@ -103,15 +103,20 @@ struct BwdArgs {
     float *dAp;   // [b][h][nchunks]
     float *dDp;   // [b][h][nchunks]
     int *dev_error;  // device error word (tensor-core phases' bounded waits)
+    float *gram;  // [b][g][nchunks][QB][QB]: C B^T of each chunk when the heads of a group share it, else null
 };
 
 // Workspace floats for one call (each region padded to 4 floats).
-__host__ __device__ inline size_t ws_floats(int batch, int seqlen, int nheads, int headdim, int dstate,
+// Whether the heads of a group share one C B^T per chunk (computed once, by the
+// group's own phase, and read by each head's per-chunk gradients).
+__host__ __device__ inline bool shared_gram(int nheads, int ngroups) { return nheads / ngroups >= 2; }
+__host__ __device__ inline size_t ws_floats(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate,
                                             int nchunks) {
     auto r4 = [](size_t v) { return (v + 3) / 4 * 4; };
     const size_t bh = (size_t)batch * nheads, pn = (size_t)headdim * dstate;
+    const size_t gram = shared_gram(nheads, ngroups) ? (size_t)batch * ngroups * nchunks * QB * QB : 0;
     return r4(bh * nchunks * QB) + r4(bh * nchunks) + 3 * r4(bh * nchunks * pn) +
-           2 * r4((size_t)batch * seqlen * nheads * dstate) + 2 * r4(bh * nchunks);
+           2 * r4((size_t)batch * seqlen * nheads * dstate) + 2 * r4(bh * nchunks) + r4(gram);
 }
 
 __host__ __device__ inline void carve(BwdArgs &a, float *ws) {
@@ -126,7 +131,8 @@ __host__ __device__ inline void carve(BwdArgs &a, float *ws) {
     a.dBh = p; p += r4((size_t)a.batch * a.seqlen * a.nheads * a.dstate);
     a.dCh = p; p += r4((size_t)a.batch * a.seqlen * a.nheads * a.dstate);
     a.dAp = p; p += r4(bh * a.nchunks);
-    a.dDp = p;
+    a.dDp = p; p += r4(bh * a.nchunks);
+    a.gram = shared_gram(a.nheads, a.ngroups) ? p : nullptr;
 }
 
 // ------------------------------------------------------------- indexing
@@ -475,6 +481,24 @@ __host__ __device__ inline void k4_pass(const BwdArgs &a, int blk, int h, int b,
     if (a.dinit) a.dinit[ix_bh(a, b, h) * pn + i] = gv;
 }
 
+// --------------------------- 5a: C B^T of a chunk, once per (batch, group)
+// When the heads of a group share B and C, G = C B^T of a chunk is the same for
+// all of them: it is formed here once and the per-chunk gradients read it.
+__host__ __device__ inline void kg_load(const BwdArgs &a, int c, int g, int b, int tid, const Smem &m) {
+    load_rows_n(a, a.B, c, g, b, tid, m.Bs);
+    load_rows_n(a, a.C, c, g, b, tid, m.Cs);
+    bwd_async_wait();
+}
+__host__ __device__ inline void kg_gram(const BwdArgs &a, int c, int g, int b, int tid, const Smem &m) {
+    const int r0 = 4 * (tid >> 4), tc = tid & 15;
+    float acc[4][4];
+    zero(acc);
+    mm_nt<4>(acc, m.Cs, NS, r0, m.Bs, NS, tc, 0, N_MAX);
+    float *dst = a.gram + (((size_t)b * a.ngroups + g) * a.nchunks + c) * QB * QB;
+    for (int i = 0; i < 4; ++i)
+        for (int j = 0; j < 4; ++j) dst[(r0 + i) * QB + tc + 16 * j] = acc[i][j];
+}
+
 // ------------------------------------------------ 5: gradients of one chunk
 __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, int tid, const Smem &m) {
     const int g = group_of(a, h);
@@ -497,17 +521,30 @@ __host__ __device__ inline void k5_load(const BwdArgs &a, int c, int h, int b, i
     load_rows_n(a, a.C, c, g, b, tid, m.Cs);
     load_pn(a, a.hin + ix_pn(a, b, h, c), tid, m.Hin);
     load_pn(a, a.gh + ix_pn(a, b, h, c), tid, m.Gh);
+    if (a.gram) {  // the group's C B^T of this chunk, into GL (k5_mats turns it into GL in place)
+        const float *gsrc = a.gram + (((size_t)b * a.ngroups + g) * a.nchunks + c) * QB * QB;
+#ifdef __CUDA_ARCH__
+        for (int i = tid; i < QB * QB / 4; i += NT)
+            bwd_cp16(m.GL + (i / (QB / 4)) * QS + 4 * (i % (QB / 4)), gsrc + 4 * i, true);
+#else
+        for (int i = tid; i < QB * QB; i += NT) m.GL[(i / QB) * QS + i % QB] = gsrc[i];
+#endif
+    }
     bwd_async_wait();
 }
 // GL = (C B^T) o L (causal), XY = dy x^T, K = L o dt_s o XY; thread tile rows
 // l = 4 tr + i, columns s = tc + 16 j.
 __host__ __device__ inline void k5_mats(const BwdArgs &a, int tid, const Smem &m) {
-    (void)a;
     const int r0 = 4 * (tid >> 4), tc = tid & 15;
     float g[4][4], xy[4][4];
     zero(g);
     zero(xy);
-    mm_nt<4>(g, m.Cs, NS, r0, m.Bs, NS, tc, 0, N_MAX);
+    if (a.gram) {  // the group's C B^T, loaded into GL
+        for (int i = 0; i < 4; ++i)
+            for (int j = 0; j < 4; ++j) g[i][j] = m.GL[(r0 + i) * QS + tc + 16 * j];
+    } else {
+        mm_nt<4>(g, m.Cs, NS, r0, m.Bs, NS, tc, 0, N_MAX);
+    }
     mm_nt<4>(xy, m.dY, PS, r0, m.X, PS, tc, 0, P_MAX);
     for (int i = 0; i < 4; ++i)
         for (int j = 0; j < 4; ++j) {

@@ -330,7 +330,7 @@ static ssd_status run_bwd(bool cplx, const float *x, const float *dt, const floa
     if ((unsigned long long)batch * seqlen * ngroups * dstate / 256 >= (1ULL << 31))
         return fail(SSD_ERR_UNSUPPORTED, "batch * seqlen * ngroups * dstate is beyond the supported grid");
     const size_t need = cplx ? ssd::bwd_complex_workspace_bytes(batch, seqlen, nheads, headdim, dstate)
-                             : ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
+                             : ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate);
     if (need > 0) {
         if (!workspace || workspace_bytes < need)
             return fail(SSD_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need,
@@ -503,7 +503,7 @@ size_t ssd_scan_bwd_workspace_size(int batch, int seqlen, int nheads, int headdi
     if (check_scan_dims(batch, seqlen, nheads, headdim, ngroups, dstate, 64) != SSD_OK)
         return SSD_WORKSPACE_INVALID;
     if (!ssd::bwd_supported(headdim, dstate)) return SSD_WORKSPACE_INVALID;
-    return ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, dstate);
+    return ssd::bwd_workspace_bytes(batch, seqlen, nheads, headdim, ngroups, dstate);
 }
 
 size_t ssd_scan_bwd_complex_workspace_size(int batch, int seqlen, int nheads, int headdim, int ngroups,

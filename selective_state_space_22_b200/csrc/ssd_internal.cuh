@@ -103,7 +103,7 @@ struct BwdCall {
     int *dev_error;  // device error word
 };
 bool bwd_supported(int headdim, int dstate);
-size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int dstate);
+size_t bwd_workspace_bytes(int batch, int seqlen, int nheads, int headdim, int ngroups, int dstate);
 cudaError_t launch_scan_bwd(const BwdCall &call, void *ws, cudaStream_t st);
 // Complex variant: A, B, C, init_state, dfinal and dA, dB, dC, dinit are float
 // pairs; headdim <= 64, dstate <= 64.

@@ -25,7 +25,7 @@ extern "C" int emulate_scan_bwd_real(const float *x, const float *dt, const floa
     a.batch = batch; a.seqlen = seqlen; a.nheads = nheads; a.headdim = headdim; a.ngroups = ngroups;
     a.dstate = dstate;
     a.nchunks = (seqlen + QB - 1) / QB;
-    std::vector<float> ws(ws_floats(batch, seqlen, nheads, headdim, dstate, a.nchunks) + 4,
+    std::vector<float> ws(ws_floats(batch, seqlen, nheads, headdim, ngroups, dstate, a.nchunks) + 4,
                           std::numeric_limits<float>::quiet_NaN());
     carve(a, ws.data());
     // Each chunk kernel gets exactly the shared memory its launch asks for, so
@@ -60,6 +60,14 @@ extern "C" int emulate_scan_bwd_real(const float *x, const float *dt, const floa
         for (int b = 0; b < batch; ++b)
             for (int h = 0; h < nheads; ++h)
                 for (int blk = 0; blk < pn_blocks; ++blk) each([&](int t) { k4_pass(a, blk, h, b, t); });
+        if (a.gram)
+            for (int b = 0; b < batch; ++b)
+                for (int g = 0; g < ngroups; ++g)
+                    for (int c = 0; c < a.nchunks; ++c) {
+                        fresh();
+                        each([&](int t) { kg_load(a, c, g, b, t, m3); });
+                        each([&](int t) { kg_gram(a, c, g, b, t, m3); });
+                    }
         for (int b = 0; b < batch; ++b)
             for (int h = 0; h < nheads; ++h)
                 for (int c = 0; c < a.nchunks; ++c) {
