@@ -1161,7 +1161,8 @@ def bench_bwd(args, shape):
     roofline = {"bound": "hbm", "achieved": abytes / t_call / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": abytes / t_call / 1e9 / peaks["hbm_gbs"], "traffic": None,
                 "kernel": ("ssd_scan_bwd_complex" if shape.complex else "ssd_scan_bwd")
-                + " (7 launches, two of them tcgen05, timed as one call)",
+                + (" (7 launches, two of them tcgen05, timed as one call)" if shape.complex
+                   or shape.nheads // shape.ngroups < 2 else " (8 launches, two of them tcgen05, timed as one call)"),
                 "algorithmic_bytes_per_launch": abytes,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
                 if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
@@ -1207,7 +1208,8 @@ def bench_bwd(args, shape):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic", "impl": "ours",
         "config": bwd_config(shape, world),
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": sampler.summary(t0, t1),
-        "gpu_launches": 7 * steps,
+        # seven phases, and an eighth (C B^T once per group) when heads share a group
+        "gpu_launches": (7 + (0 if shape.complex or shape.nheads // shape.ngroups < 2 else 1)) * steps,
         "step_ms_p10_p50_p90": [statistics.quantiles(per_step_ms, n=10)[0], statistics.median(per_step_ms),
                                 statistics.quantiles(per_step_ms, n=10)[-1]],
     }
