@@ -320,7 +320,8 @@ ssd_status ssd_state_update_complex(float *state, const float *x, const float *d
  *  gradient for D whether or not D was given.
  *
  * Limits: headdim <= 64 and dstate <= 128 (SSD_ERR_UNSUPPORTED otherwise).  Runs
- * in seven launches; with headdim 64 and dstate 128 the chunk states and the
+ * in seven launches (eight when heads share a group: C B^T once per group and
+ * chunk); with headdim 64 and dstate 128 the chunk states and the
  * readout terms are tcgen05 products (bf16 hi/lo, three products, float32
  * accumulation), the rest CUDA cores.  Sums are taken in a fixed order, so
  * repeated calls give identical bits.  The workspace (ssd_scan_bwd_workspace_size bytes,

@@ -1,7 +1,9 @@
-// scan_bwd.cu -- gradients of the real scan on CUDA cores (fp32), chunk by chunk.
+// scan_bwd.cu -- gradients of the real and complex scans (fp32), chunk by chunk.
 //
-// The arithmetic is in scan_bwd_body.cuh; this file only launches it.  Six
-// steps, seven launches, run on the caller's stream:
+// The arithmetic is in scan_bwd_body.cuh (and, for steps 1 and 3 at head dim 64,
+// in the tcgen05 kernels of scan_bwd_tc.cuh); this file only launches it.  Six
+// steps, seven launches (eight when the heads of a group share B and C: their
+// C B^T per chunk is formed once, before step 5), run on the caller's stream:
 //   1. chunk states S_c and the within-chunk cumulative decay      grid (chunks, heads, batch)
 //   2. the state entering each chunk, h_in (a forward pass over chunks)   grid (heads, batch)
 //   3. the readout terms R_c = sum_l exp(acs[l]) dy_l C_l^T         grid (chunks, heads, batch)
