@@ -69,6 +69,15 @@ def test_complex_mamba3lite_head_shape():
     check(1, 96, 4, 64, 4, 64, seed=3)
 
 
+@pytest.mark.parametrize("T", [1, 33, 70])
+def test_complex_tensor_core_phases_ragged(T):
+    """Head dim 64 and 64 complex states take the tcgen05 chunk-state and readout
+    kernels: ragged last chunks, one token, optional inputs absent."""
+    check(2, T, 4, 64, 4, 64, init=(T != 33), seed=40 + T)
+    got = check(1, T, 2, 64, 1, 64, init=False, use_D=False, use_dfinal=False, seed=50 + T)
+    assert got["dD"] is None
+
+
 def test_complex_optional_inputs_absent_and_empty():
     got = check(2, 50, 2, 4, 1, 8, init=False, use_D=False, use_dfinal=False, seed=4)
     assert got["dD"] is None

@@ -61,6 +61,24 @@ def test_mamba2_head_shape():
     check(1, 256, 8, 64, 2, 128, seed=3)
 
 
+@pytest.mark.parametrize("T", [1, 65, 200])
+def test_tensor_core_phases_ragged(T):
+    """Head dim 64 and d_state 128 take the tcgen05 chunk-state and readout
+    kernels (and, with heads sharing a group, the per-group C B^T): ragged last
+    chunks, one token, optional inputs absent."""
+    check(2, T, 4, 64, 2, 128, init=(T != 65), seed=40 + T)
+    got = check(1, T, 2, 64, 1, 128, init=False, use_D=False, use_dfinal=False, seed=50 + T)
+    assert got["dD"] is None
+
+
+def test_tensor_core_phases_bitwise_repeatable():
+    p, dy, dfinal = problem(1, 150, 4, 64, 1, 128, seed=8)
+    first = gpu_bwd(p, dy, dfinal)
+    again = gpu_bwd(p, dy, dfinal)
+    for k in NAMES:
+        assert np.array_equal(first[k], again[k]), k
+
+
 def test_optional_inputs_absent():
     got = check(2, 100, 2, 4, 1, 8, init=False, use_D=False, use_dfinal=False, seed=4)
     assert got["dD"] is None
