@@ -125,3 +125,22 @@ def test_slices_on_one_device(io, T, R):
     # the slice log-decay is A * sum(dt) over the slice
     lam0 = inp["A"].double()[None, :] * inp["dt"][:, cuts[0][0]:cuts[0][1]].double().sum(1)
     assert rel_err(lam[0].cpu().numpy(), lam0.numpy()) < 1e-6
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("b,T,H", [(1, 2048, 4), (2, 700, 8), (1, 128 * 37 + 5, 2)])
+def test_state_only_form_matches_the_full_scan_bitwise(b, T, H):
+    """The state-only form (its own kernel instance, W built by another warpgroup
+    into another buffer) forms the same bf16 W tiles and chunk-state products as
+    the full scan, in the same order: the final states agree bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import selective_state_space_22_b200 as ssd
+
+    shape = inputs.ScanShape("state-only-vs-full", b, T, H, 64, 1, 128, 128, "bf16", init_state=True, seed=T + H)
+    inp = inputs.scan_inputs(shape)
+    d = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    _, f_full = ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], chunk_size=128)
+    f_only, _ = ssd.ssd_scan_final_state(d["x"], d["dt"], d["A"], d["B"], d["init_state"], chunk_size=128)
+    ssd.ssd_get_device_status()
+    assert torch.equal(f_only, f_full)
