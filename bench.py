@@ -608,7 +608,8 @@ def bench_ours(args, shape):
     fn = ssd.ssd_scan_fwd_complex if cplx else ssd.ssd_scan_fwd
     launches = ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
                                             shape.ngroups, shape.dstate, shape.chunk, cplx, io)
-    tc_path = launches == 1 and not cplx and io == ssd.SSD_BF16
+    tc_path = (not cplx and io == ssd.SSD_BF16 and shape.headdim == 64 and shape.dstate == 128
+               and shape.seqlen >= 128)  # the tcgen05 kernel (1 launch; 3 for batch 1 cut in two)
     cplx_tc = cplx and shape.headdim == 64 and shape.dstate == 64  # the tcgen05 complex kernels
     kernel_chunk = 128 if (tc_path or cplx_tc) else shape.chunk  # the tensor-core kernels tile 128 tokens
 

@@ -103,8 +103,13 @@ int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int
  * seqlen may be 0 (then y is empty and final_state = init_state, or zeros) and
  * need not be a multiple of chunk_size.  io_dtype SSD_BF16 with headdim 64,
  * dstate 128 and seqlen >= 128 runs the tcgen05 tensor-core kernel: one launch,
- * no workspace, bitwise reproducible.  It evaluates 128-token chunks (its MMA
- * tile height) whatever chunk_size says.  Every other combination runs the
+ * no workspace, bitwise reproducible.  With batch 1 it takes a workspace of
+ * nheads * headdim * dstate * 4 bytes: when each sequence is cut in two (fewer
+ * sequences than SMs), the state between the halves is formed by a state-only
+ * launch on an internal second stream while the caller's stream scans the first
+ * half (three launches, joined back to the caller's stream before the call's work
+ * ends; the same bits as the one-launch form).  It evaluates 128-token chunks
+ * (its MMA tile height) whatever chunk_size says.  Every other combination runs the
  * float32 CUDA-core kernels (three launches, a workspace), which honour
  * chunk_size.  State and accumulation are float32 in both.
  */

@@ -751,35 +751,40 @@ bool tc_supported(int headdim, int dstate, int seqlen) {
     return headdim == PD && dstate == ND && seqlen >= QT;
 }
 
-size_t tc_workspace_bytes(int, int) { return 0; }
+// Batch 1: the state between the two halves of the split above, and room for a
+// copy of the initial state when the final state overwrites it.
+size_t tc_workspace_bytes(int batch, int nheads) {
+    return batch == 1 ? 2 * (size_t)nheads * PD * ND * sizeof(float) : 0;
+}
 
-int tc_kernel_launches() { return 1; }
-
-cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
-    cudaError_t e = get_encoder();
-    if (e != cudaSuccess) return e;
-    int dev = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    {
-        std::lock_guard<std::mutex> lk(g_dev_mu);
-        DevInfo &di = g_dev[dev];
-        void *ctx = current_context();
-        if (!di.init || di.ctx != ctx) {
-            di.init = false;
-            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          SMEM_ALLOC)) != cudaSuccess)
-                return e;
-            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                          SMEM_ALLOC)) != cudaSuccess)
-                return e;
-            if ((e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-            di.ctx = ctx;
-            di.init = true;
-        }
+namespace {
+int device_sms() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return 148;
     }
-    const DevInfo &di = g_dev[dev];
+    return sms;
+}
+// Batch 1 with two runs per sequence takes the split (three launches).
+bool batch1_split(int batch, int nheads, int seqlen, int sms) {
+    const int bH = batch * nheads, nchunks = (seqlen + QT - 1) / QT;
+    return batch == 1 && 4 * bH < 3 * sms && std::min({sms / bH, nchunks, MAX_RUNS}) == 2;
+}
+}  // namespace
 
+int tc_kernel_launches(int batch, int nheads, int seqlen) {
+    return batch1_split(batch, nheads, seqlen, device_sms()) ? 3 : 1;
+}
+
+namespace {
+
+// One launch for the problem in a.  first > 0: each sequence is scanned over its
+// first `first` chunks only, in full, as one run (no state-only prefix, no final
+// state).  whole: one run per sequence whatever the SM count.  Otherwise runs
+// are chosen as described at split_runs.
+cudaError_t launch_one(const ScanArgs &a, cudaStream_t st, int sms, int first, bool whole) {
+    cudaError_t e;
     CUtensorMap mx, mb, mc;
     if ((e = make_map(&mx, a.x, a.headdim, a.nheads, a.seqlen, a.batch)) != cudaSuccess) return e;
     if ((e = make_map(&mb, a.B, a.dstate, a.ngroups, a.seqlen, a.batch)) != cudaSuccess) return e;
@@ -803,8 +808,11 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     if (!a.y) {
         // State-only form (no C, no y): every tile of every sequence state-only.
         p.run_start[0] = p.run_start[1] = p.nchunks;
+    } else if (first > 0) {
+        p.run_start[0] = 0;
+        p.run_start[1] = first;
     } else {
-        if (4 * p.bH < 3 * di.sms) runs = std::max(1, std::min({di.sms / p.bH, p.nchunks, MAX_RUNS}));
+        if (!whole && 4 * p.bH < 3 * sms) runs = std::max(1, std::min({sms / p.bH, p.nchunks, MAX_RUNS}));
         split_runs(p.nchunks, runs, p.run_start);
     }
     p.runs = runs;
@@ -814,7 +822,7 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     p.withhold = g_withhold.load();
 
     const int items = p.bH * runs;
-    const int grid = std::min(items, di.sms);  // one CTA per SM
+    const int grid = std::min(items, sms);  // one CTA per SM
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(NTH);
@@ -822,6 +830,108 @@ cudaError_t launch_tc_scan(const ScanArgs &a, void *, cudaStream_t st) {
     cfg.stream = st;
     if (!a.y) return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel<true>, mx, mb, mc, p);
     return cudaLaunchKernelEx(&cfg, ssd_scan_tc_kernel<false>, mx, mb, mc, p);
+}
+
+// A second stream and two events per device for the batch-1 split below.
+struct SplitStream {
+    void *ctx = nullptr;
+    cudaStream_t s2 = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+SplitStream g_split[64];
+std::mutex g_split_mu;
+
+// Batch 1, two runs per sequence: instead of the second run replaying the first
+// run's chunks inside the launch (a state-only tile costs 0.65 of a full one
+// there), a second stream forms the state after the first `s` chunks with the
+// state-only form (its own kernel instance: 1.24 against 2.54 us per tile at 64
+// heads, alone) and then scans the rest from that state, while the first stream
+// scans the first `s` chunks in full.  Each is a launch of one CTA per sequence,
+// so the two streams run side by side.  s balances s full tiles against
+// ALPHA_SO s state-only and (nchunks - s) full ones; side by side the state-only
+// tiles cost more than alone, and 0.60 balanced best (T = 65536, 64 heads:
+// 868 us, against 877 at 0.54, 890 at 0.49 and 901 at 0.66).
+cudaError_t launch_batch1_split(const ScanArgs &a, float *h_split, cudaStream_t st, int sms, int dev) {
+    const double ALPHA_SO = 0.60;
+    const int nchunks = (a.seqlen + QT - 1) / QT;
+    const int s = std::min(nchunks - 1, std::max(1, (int)(nchunks / (2.0 - ALPHA_SO) + 0.5)));
+    cudaError_t e;
+    SplitStream &ss = g_split[dev];
+    void *ctx = current_context();
+    if (ss.ctx != ctx || !ss.s2) {
+        ss = SplitStream{};
+        if ((e = cudaStreamCreateWithFlags(&ss.s2, cudaStreamNonBlocking)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming)) != cudaSuccess) return e;
+        if ((e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming)) != cudaSuccess) return e;
+        ss.ctx = ctx;
+    }
+    // the second stream starts where the caller's stream is now
+    if ((e = cudaEventRecord(ss.fork, st)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(ss.s2, ss.fork, 0)) != cudaSuccess) return e;
+    ScanArgs first = a;  // chunks 0 .. s-1 in full
+    first.final_state = nullptr;
+    if ((e = launch_one(first, st, sms, s, false)) != cudaSuccess) return e;
+    ScanArgs prefix = a;  // the state after chunk s-1
+    prefix.y = nullptr;
+    prefix.seqlen = s * QT;
+    prefix.final_state = h_split;
+    if ((e = launch_one(prefix, ss.s2, sms, 0, false)) != cudaSuccess) return e;
+    const size_t t0 = (size_t)s * QT;  // the rest, from that state (batch 1: plain pointer offsets)
+    ScanArgs rest = a;
+    rest.x = static_cast<const __nv_bfloat16 *>(a.x) + t0 * a.nheads * a.headdim;
+    rest.dt = a.dt + t0 * a.nheads;
+    rest.B = static_cast<const __nv_bfloat16 *>(a.B) + t0 * a.ngroups * a.dstate;
+    rest.C = static_cast<const __nv_bfloat16 *>(a.C) + t0 * a.ngroups * a.dstate;
+    rest.y = static_cast<__nv_bfloat16 *>(a.y) + t0 * a.nheads * a.headdim;
+    rest.seqlen = a.seqlen - (int)t0;
+    rest.init_state = h_split;
+    if ((e = launch_one(rest, ss.s2, sms, 0, true)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ss.join, ss.s2)) != cudaSuccess) return e;
+    return cudaStreamWaitEvent(st, ss.join, 0);
+}
+
+}  // namespace
+
+cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st) {
+    cudaError_t e = get_encoder();
+    if (e != cudaSuccess) return e;
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(g_dev_mu);
+        DevInfo &di = g_dev[dev];
+        void *ctx = current_context();
+        if (!di.init || di.ctx != ctx) {
+            di.init = false;
+            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          SMEM_ALLOC)) != cudaSuccess)
+                return e;
+            if ((e = cudaFuncSetAttribute(ssd_scan_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          SMEM_ALLOC)) != cudaSuccess)
+                return e;
+            if ((e = cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+            di.ctx = ctx;
+            di.init = true;
+        }
+    }
+    const int sms = g_dev[dev].sms;
+    if (a.y && ws && batch1_split(a.batch, a.nheads, a.seqlen, sms)) {
+        // The second stream writes the final state while the first may still read
+        // the initial one: when they overlap, both read a copy in the workspace.
+        const size_t pn = (size_t)a.nheads * PD * ND;
+        float *h_split = static_cast<float *>(ws), *h_copy = h_split + pn;
+        ScanArgs b = a;
+        if (a.init_state && a.final_state && a.final_state < a.init_state + pn && a.init_state < a.final_state + pn) {
+            if ((e = cudaMemcpyAsync(h_copy, a.init_state, pn * sizeof(float), cudaMemcpyDeviceToDevice, st)) !=
+                cudaSuccess)
+                return e;
+            b.init_state = h_copy;
+        }
+        std::lock_guard<std::mutex> lk(g_split_mu);
+        return launch_batch1_split(b, h_split, st, sms, dev);
+    }
+    return launch_one(a, st, sms, 0, false);
 }
 
 }  // namespace ssd

@@ -106,7 +106,7 @@ Plan plan_scan(int batch, int seqlen, int nheads, int headdim, int ngroups, int 
     if (!cplx && bf16 && ssd::tc_supported(headdim, dstate, seqlen)) {
         p.tc = true;
         p.ws = ssd::tc_workspace_bytes(batch, nheads);
-        p.launches = ssd::tc_kernel_launches();
+        p.launches = ssd::tc_kernel_launches(batch, nheads, seqlen);
         return p;
     }
     if (cplx && ssd::cplx_tc_supported(headdim, dstate)) {  // tensor-core path: 128-token chunks

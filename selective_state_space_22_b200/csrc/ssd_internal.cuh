@@ -85,7 +85,7 @@ cudaError_t launch_generic_scan(const ScanArgs &a, bool cplx, bool bf16, void *w
 bool tc_supported(int headdim, int dstate, int seqlen);
 size_t tc_workspace_bytes(int batch, int nheads);
 cudaError_t launch_tc_scan(const ScanArgs &a, void *ws, cudaStream_t st);
-int tc_kernel_launches();
+int tc_kernel_launches(int batch, int nheads, int seqlen);
 // Test only: with withhold != 0 the tensor-core kernel's producer issues no load,
 // so every bounded wait runs out; wait_ns (0: the default) bounds each wait.
 void set_tc_fault_injection(int withhold, unsigned long long wait_ns);

@@ -140,9 +140,13 @@ def test_repeated_calls_are_bitwise_equal(io):
 
 
 def _tc(shape):
-    return ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
-                                        shape.ngroups, shape.dstate, shape.chunk, False,
-                                        ssd.SSD_BF16) == 1
+    """The shapes the tensor-core kernel takes (bf16, head dim 64, d_state 128, at
+    least one 128-token chunk): one launch, or three with batch 1 when each
+    sequence is cut in two."""
+    n = ssd.ssd_scan_kernel_launches(shape.batch, shape.seqlen, shape.nheads, shape.headdim,
+                                     shape.ngroups, shape.dstate, shape.chunk, False, ssd.SSD_BF16)
+    return (shape.headdim == 64 and shape.dstate == 128 and shape.seqlen >= 128
+            and (n == 1 or (n == 3 and shape.batch == 1)))
 
 
 @pytest.mark.parametrize("T", [128, 129, 256, 1000, 128 * 20 + 5])
@@ -153,6 +157,30 @@ def test_tcgen05_path(T, H, G):
     shape = small("tc", 2, T, H, 64, G, 128, 256, "bf16", init=(H != 1), seed=T + H)
     assert _tc(shape), "expected the tcgen05 kernel for this shape"
     check_full(shape, TOL_BF16)
+
+
+@pytest.mark.parametrize("T,H", [(300, 64), (128 * 9 + 17, 50), (256, 74)])
+def test_batch1_cut_in_two(T, H):
+    """Batch 1 with fewer sequences than SMs: the first part of each sequence on the
+    caller's stream, the state-only prefix and the rest on a second stream (three
+    launches); ragged tails, a nonzero initial state."""
+    shape = small("b1split", 1, T, H, 64, 1, 128, 256, "bf16", init=True, seed=T + H)
+    assert ssd.ssd_scan_kernel_launches(1, T, H, 64, 1, 128, 256, False, ssd.SSD_BF16) == 3
+    check_full(shape, TOL_BF16)
+
+
+def test_batch1_cut_in_two_final_state_aliases_initial_state():
+    """The second stream writes the final state while the first may still read the
+    initial one: with the two aliased, both halves start from a copy."""
+    shape = small("b1alias", 1, 700, 64, 64, 1, 128, 128, "bf16", init=True, seed=5)
+    inp = inputs.scan_inputs(shape)
+    y_ref, fs_ref = oracle_scan(inp)
+    d = to_dev(inp)
+    h = d["init_state"].clone()
+    y, fs = ssd.ssd_scan_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], h, final_state=h, chunk_size=128)
+    ssd.ssd_get_device_status()
+    assert rel_err(y.float().cpu().numpy(), y_ref) <= TOL_BF16
+    assert rel_err(h.cpu().numpy(), fs_ref) <= TOL_BF16
 
 
 @pytest.mark.parametrize("io", ["bf16", "f32"])
