@@ -681,7 +681,7 @@ def bench_ours(args, shape):
     traffic = lookup_traffic(kernel, src, shape.name)
     roofline = {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
                 "frac": achieved / peak, "traffic": traffic, "kernel": kernel,
-                "kernel_chunk": kernel_chunk,
+                "kernel_chunk": kernel_chunk, "launches_per_call": launches,
                 "algorithmic_bytes_per_launch": abytes, "algorithmic_flops_per_launch": aflops,
                 "peak_source": f"{peaks['source']} (MEASURED_PEAKS.json burst)"
                 if peaks["source"] == "measured" else "fallback (6.65 TB/s, 1.59 PFLOP/s)",
