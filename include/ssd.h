@@ -108,7 +108,8 @@ int ssd_scan_kernel_launches(int batch, int seqlen, int nheads, int headdim, int
  * sequences than SMs), the state between the halves is formed by a state-only
  * launch on an internal second stream while the caller's stream scans the first
  * half (three launches, joined back to the caller's stream before the call's work
- * ends; the same bits as the one-launch form).  It evaluates 128-token chunks
+ * ends; the same bits as the one-launch form).  The first such call on a device
+ * creates that stream and two events, so it should come before any stream capture.  It evaluates 128-token chunks
  * (its MMA tile height) whatever chunk_size says.  Every other combination runs the
  * float32 CUDA-core kernels (three launches, a workspace), which honour
  * chunk_size.  State and accumulation are float32 in both.
